@@ -138,6 +138,16 @@ static float load_elem(const void *x, int xdtype, int64_t i)
     return f;
 }
 
+/* max(m, v) where a NaN v (quiet or signalling) is ignored.  The amax and the
+ * history window skip NaN entries; libm fmaxf is not used because for a
+ * signalling NaN it returns NaN. */
+static float max_ignoring_nan(float m, float v)
+{
+    if (isnan(v)) return m;
+    if (isnan(m)) return v;
+    return v > m ? v : m;
+}
+
 /* fl32(x * scale): exact fp64 product, rounded once to fp32. */
 float orc_scaled(float x, float scale) { return (float)((double)x * (double)scale); }
 
@@ -165,7 +175,7 @@ void orc_cast_transpose_amax(const void *x, int xdtype, int64_t rows, int64_t co
             uint8_t q = encode_with_table(orc_scaled(v, scale), dec, top);
             if (y) y[i * cols + j] = q;
             if (yt) yt[j * rows + i] = q;
-            m = fmaxf(m, fabsf(v));
+            m = max_ignoring_nan(m, fabsf(v));
         }
     }
     if (amax) *amax = m;
@@ -198,7 +208,7 @@ void orc_update_scales(int64_t T, int H, float *hist, float *scale, float *scale
 {
     for (int64_t t = 0; t < T; ++t) {
         float a = hist[t];
-        for (int h = 1; h < H; ++h) a = fmaxf(a, hist[(int64_t)h * T + t]);
+        for (int h = 1; h < H; ++h) a = max_ignoring_nan(a, hist[(int64_t)h * T + t]);
         double fp8_max = orc_decode((uint8_t)max_finite_code(fmts[t]), fmts[t]);
         float s = scale[t];
         if (a > 0.0f && isfinite(a)) {

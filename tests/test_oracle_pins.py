@@ -217,6 +217,20 @@ def test_cast_transpose_amax_properties(fmt, dtype):
     assert am3 == np.float32(np.nanmax(np.abs(xn)))
 
 
+def test_amax_ignores_every_nan_pattern():
+    """Every bf16 bit pattern (quiet and signalling NaNs included): the amax is
+    numpy's nanmax of the absolute values."""
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    v = o.bf16_bits_to_f32(bits)
+    _, am, _ = o.quantize(bits, o.E4M3, 1.0)
+    assert am == np.nanmax(np.abs(v)) and np.isinf(am)
+    # a history window containing NaN entries ignores them as well
+    hist = np.zeros((4, 1), np.float32)
+    hist[:, 0] = [np.float32(2.0), np.uint32(0x7F810000).view(np.float32), np.nan, 1.0]
+    _, s2, _ = o.update_scales(hist, [1.0], [1.0], [0])
+    assert s2[0] == np.float32(224.0)
+
+
 def test_quantize_is_flat_cast():
     x = np.random.default_rng(1).standard_normal(1001).astype(np.float32)
     y, am, si = o.quantize(x, o.E4M3, 2.0)
