@@ -1,0 +1,212 @@
+"""Thin Python binding of libfp8ds.so (ctypes; argument marshalling only).
+
+Every function has the name of the C entry point it calls and the same
+argument order; tensors are torch CUDA tensors whose device pointers are
+passed through, the stream defaults to torch's current stream.  Nothing here
+computes: if the shared library is missing, importing this module raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8ds.so")
+
+E4M3 = 0
+E5M2 = 1
+F32 = 0
+BF16 = 1
+AMAX_MAX = 0
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_CUDA = 3
+ERR_TIMEOUT = 4
+
+_FMT_NAMES = {"e4m3": E4M3, "e5m2": E5M2, E4M3: E4M3, E5M2: E5M2}
+
+
+class Fp8dsError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("fp8ds status %d: %s" % (status, message))
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libfp8ds.so not found at %s; build it with "
+                      "`python -m fp8_delayed_scaling_cast_b200.build`" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_INT = ctypes.c_int
+
+
+class _Meta(ctypes.Structure):
+    _fields_ = [("amax_history", _P), ("scale", _P), ("scale_inv", _P), ("formats", _P),
+                ("num_tensors", _I64), ("hist_len", _I32)]
+
+
+class _Linear(ctypes.Structure):
+    _fields_ = [("w", _P), ("bias", _P), ("bias_dtype", _INT), ("in_features", _I64),
+                ("out_features", _I64), ("w8", _P), ("w8t", _P), ("w_scale_inv", _P),
+                ("meta_in", _I32), ("meta_w", _I32), ("meta_grad", _I32), ("cache_valid", _I32)]
+
+
+_SIGS = {
+    "fp8_quantize": [_P, _INT, _I64, _INT, _P, _P, _P, _P, _P],
+    "fp8_cast_transpose_amax": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
+    "fp8_update_scales": [_I64, _I32, _P, _P, _P, _P, _INT, _P],
+    "fp8_gemm": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
+    "fp8_linear_fwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _INT,
+                       _I32, _P, _P, _P, _P],
+    "fp8_linear_bwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P,
+                       _INT, _P, _P, _P, _P, _P],
+    "fp8ds_device_status": [ctypes.POINTER(_I32), _I32],
+}
+for _name, _args in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _INT
+_lib.fp8ds_last_error.restype = ctypes.c_char_p
+_lib.fp8ds_last_error.argtypes = []
+_lib.fp8ds_version.restype = ctypes.c_char_p
+_lib.fp8ds_version.argtypes = []
+
+
+def fp8ds_last_error():
+    return _lib.fp8ds_last_error().decode()
+
+
+def fp8ds_version():
+    return _lib.fp8ds_version().decode()
+
+
+def _check(status):
+    if status != OK:
+        raise Fp8dsError(status, fp8ds_last_error())
+
+
+def _ptr(t):
+    return None if t is None else _P(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _P(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype(t):
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("expected float32 or bfloat16 tensor, got %s" % t.dtype)
+
+
+def _fmt(f):
+    return _FMT_NAMES[f]
+
+
+def fp8_quantize(x, fmt, scale, y, amax=None, scale_inv=None, stream=None):
+    _check(_lib.fp8_quantize(_ptr(x), _dtype(x), x.numel(), _fmt(fmt), _ptr(scale), _ptr(y),
+                             _ptr(amax), _ptr(scale_inv), _stream(stream)))
+
+
+def fp8_cast_transpose_amax(x, fmt, scale, y, yt=None, amax=None, scale_inv=None, stream=None):
+    rows, cols = x.shape
+    _check(_lib.fp8_cast_transpose_amax(_ptr(x), _dtype(x), rows, cols, _fmt(fmt), _ptr(scale),
+                                        _ptr(y), _ptr(yt), _ptr(amax), _ptr(scale_inv),
+                                        _stream(stream)))
+
+
+def fp8_update_scales(amax_history, scale, scale_inv, formats, algo=AMAX_MAX, stream=None):
+    hist_len, num_tensors = amax_history.shape
+    _check(_lib.fp8_update_scales(num_tensors, hist_len, _ptr(amax_history), _ptr(scale),
+                                  _ptr(scale_inv), _ptr(formats), algo, _stream(stream)))
+
+
+def fp8_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, d, bias=None, stream=None):
+    m, k = a.shape
+    n = b.shape[0]
+    _check(_lib.fp8_gemm(_ptr(a), _fmt(a_fmt), _ptr(a_scale_inv), _ptr(b), _fmt(b_fmt),
+                         _ptr(b_scale_inv), _ptr(bias), F32 if bias is None else _dtype(bias),
+                         _ptr(d), _dtype(d), m, n, k, _stream(stream)))
+
+
+class Fp8Meta:
+    """Packed DelayedScaling state of T FP8 tensors (caller-owned device tensors)."""
+
+    def __init__(self, formats, hist_len=16, device="cuda"):
+        self.formats = torch.tensor([_fmt(f) for f in formats], dtype=torch.uint8, device=device)
+        T = self.formats.numel()
+        self.amax_history = torch.zeros(hist_len, T, dtype=torch.float32, device=device)
+        self.scale = torch.ones(T, dtype=torch.float32, device=device)
+        self.scale_inv = torch.ones(T, dtype=torch.float32, device=device)
+        self._c = _Meta(_ptr(self.amax_history), _ptr(self.scale), _ptr(self.scale_inv),
+                        _ptr(self.formats), T, hist_len)
+
+    @property
+    def num_tensors(self):
+        return self.formats.numel()
+
+    def update(self, stream=None):
+        fp8_update_scales(self.amax_history, self.scale, self.scale_inv, self.formats,
+                          stream=stream)
+
+
+class Fp8Linear:
+    """A linear layer's fp32 master weight, optional bias and FP8 weight cache."""
+
+    def __init__(self, w, bias, meta_in, meta_w, meta_grad):
+        out_f, in_f = w.shape
+        self.w = w
+        self.bias = bias
+        self.w8 = torch.empty(out_f, in_f, dtype=torch.uint8, device=w.device)
+        self.w8t = torch.empty(in_f, out_f, dtype=torch.uint8, device=w.device)
+        self.w_scale_inv = torch.ones(1, dtype=torch.float32, device=w.device)
+        self._c = _Linear(_ptr(w), _ptr(bias), F32 if bias is None else _dtype(bias), in_f, out_f,
+                          _ptr(self.w8), _ptr(self.w8t), _ptr(self.w_scale_inv),
+                          meta_in, meta_w, meta_grad, 0)
+
+    @property
+    def in_features(self):
+        return self._c.in_features
+
+    @property
+    def out_features(self):
+        return self._c.out_features
+
+    @property
+    def cache_valid(self):
+        return bool(self._c.cache_valid)
+
+    def invalidate_cache(self):
+        self._c.cache_valid = 0
+
+
+def fp8_linear_fwd(lin, meta, x, y, is_first_microbatch, x8, x8t=None, x_scale_inv=None,
+                   stream=None):
+    flag = -1 if is_first_microbatch is None else (1 if is_first_microbatch else 0)
+    _check(_lib.fp8_linear_fwd(ctypes.byref(lin._c), ctypes.byref(meta._c), _ptr(x), _dtype(x),
+                               x.shape[0], _ptr(y), _dtype(y), flag, _ptr(x8), _ptr(x8t),
+                               _ptr(x_scale_inv), _stream(stream)))
+
+
+def fp8_linear_bwd(lin, meta, dy, x8t, x_scale_inv, dw, dy8, dy8t, dy_scale_inv, dx=None,
+                   stream=None):
+    _check(_lib.fp8_linear_bwd(ctypes.byref(lin._c), ctypes.byref(meta._c), _ptr(dy), _dtype(dy),
+                               dy.shape[0], _ptr(x8t), _ptr(x_scale_inv), _ptr(dx),
+                               BF16 if dx is None else _dtype(dx), _ptr(dw), _ptr(dy8),
+                               _ptr(dy8t), _ptr(dy_scale_inv), _stream(stream)))
+
+
+def fp8ds_device_status(clear=True):
+    code = _I32(0)
+    _check(_lib.fp8ds_device_status(ctypes.byref(code), 1 if clear else 0))
+    return code.value

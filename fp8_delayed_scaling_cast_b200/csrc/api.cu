@@ -1,0 +1,228 @@
+// C ABI of libfp8ds.so: argument checks, error reporting and the FP8 linear
+// forward/backward glue.  Every numeric step runs in the kernels of cast.cu,
+// update.cu and gemm_sm100.cu; this file only validates and enqueues.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <mutex>
+
+#include "fp8ds_internal.h"
+
+namespace fp8ds {
+
+namespace {
+thread_local char g_msg[512] = "";
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_fmt(int f) { return f == FP8DS_E4M3 || f == FP8DS_E5M2; }
+bool valid_dtype(int d) { return d == FP8DS_F32 || d == FP8DS_BF16; }
+}  // namespace
+
+void set_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+}
+
+void clear_error() { g_msg[0] = '\0'; }
+
+int num_sms() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+static fp8ds_status cuda_status(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return FP8DS_OK;
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return FP8DS_ERR_CUDA;
+}
+
+static fp8ds_status invalid(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return FP8DS_ERR_INVALID_ARG;
+}
+
+// ------------------------------------------------------------------ checks --
+
+static fp8ds_status check_cast(const char *fn, const void *x, int x_dtype, int64_t a, int64_t b, int fmt,
+                               const float *scale, const uint8_t *y) {
+    if (a < 0 || b < 0) return invalid("%s: negative size", fn);
+    if (scale == nullptr) return invalid("%s: scale must not be NULL", fn);
+    if ((x == nullptr || y == nullptr) && a != 0 && b != 0)
+        return invalid("%s: x and y must not be NULL for a non-empty tensor", fn);
+    if (!valid_dtype(x_dtype)) return invalid("%s: unknown input dtype %d", fn, x_dtype);
+    if (!valid_fmt(fmt)) return invalid("%s: unknown FP8 format %d", fn, fmt);
+    return FP8DS_OK;
+}
+
+static fp8ds_status check_gemm(const uint8_t *a, int fa, const float *sa, const uint8_t *b, int fb,
+                               const float *sb, const void *bias, int bias_dtype, const void *d, int d_dtype,
+                               int64_t m, int64_t n, int64_t k) {
+    if (a == nullptr || b == nullptr || d == nullptr || sa == nullptr || sb == nullptr)
+        return invalid("fp8_gemm: a, b, d and the scale_inv pointers must not be NULL");
+    if (!valid_fmt(fa) || !valid_fmt(fb)) return invalid("fp8_gemm: unknown FP8 format");
+    if (!valid_dtype(d_dtype) || (bias != nullptr && !valid_dtype(bias_dtype)))
+        return invalid("fp8_gemm: unknown output or bias dtype");
+    if (m <= 0 || n <= 0 || k <= 0) return invalid("fp8_gemm: m, n, k must be positive");
+    if (m > 0x7FFFFFFF || n > 0x7FFFFFFF || k > 0x7FFFFFFF) return invalid("fp8_gemm: size exceeds 2^31-1");
+    if (k % 16 != 0) return invalid("fp8_gemm: k (%lld) must be a multiple of 16", (long long)k);
+    if (d_dtype == FP8DS_BF16 && n % 8 != 0) return invalid("fp8_gemm: n must be a multiple of 8 for bf16 output");
+    if (d_dtype == FP8DS_F32 && n % 4 != 0) return invalid("fp8_gemm: n must be a multiple of 4 for fp32 output");
+    if (!aligned16(a) || !aligned16(b) || !aligned16(d))
+        return invalid("fp8_gemm: a, b and d must be 16-byte aligned");
+    return FP8DS_OK;
+}
+
+static fp8ds_status check_meta(const char *fn, const fp8ds_meta *meta, int32_t idx) {
+    if (meta == nullptr || meta->amax_history == nullptr || meta->scale == nullptr || meta->scale_inv == nullptr)
+        return invalid("%s: incomplete meta", fn);
+    if (meta->hist_len < 1) return invalid("%s: hist_len must be >= 1", fn);
+    if (idx < 0 || idx >= meta->num_tensors) return invalid("%s: meta index %d out of range", fn, idx);
+    return FP8DS_OK;
+}
+
+}  // namespace fp8ds
+
+using namespace fp8ds;
+
+extern "C" {
+
+fp8ds_status fp8_quantize(const void *x, fp8ds_dtype x_dtype, int64_t n, fp8ds_format fmt, const float *scale,
+                          uint8_t *y, float *amax, float *scale_inv, fp8ds_stream stream) {
+    clear_error();
+    fp8ds_status st = check_cast("fp8_quantize", x, x_dtype, n, 1, fmt, scale, y);
+    if (st != FP8DS_OK) return st;
+    return cuda_status(launch_quantize(x, x_dtype, n, fmt, scale, y, amax, scale_inv, stream), "fp8_quantize");
+}
+
+fp8ds_status fp8_cast_transpose_amax(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
+                                     fp8ds_format fmt, const float *scale, uint8_t *y, uint8_t *yt, float *amax,
+                                     float *scale_inv, fp8ds_stream stream) {
+    clear_error();
+    fp8ds_status st = check_cast("fp8_cast_transpose_amax", x, x_dtype, rows, cols, fmt, scale, y);
+    if (st != FP8DS_OK) return st;
+    return cuda_status(launch_cast_transpose(x, x_dtype, rows, cols, fmt, scale, y, yt, amax, scale_inv, stream),
+                       "fp8_cast_transpose_amax");
+}
+
+fp8ds_status fp8_update_scales(int64_t num_tensors, int32_t hist_len, float *amax_history, float *scale,
+                               float *scale_inv, const uint8_t *formats, fp8ds_amax_algo algo,
+                               fp8ds_stream stream) {
+    clear_error();
+    if (num_tensors < 0) return invalid("fp8_update_scales: num_tensors < 0");
+    if (hist_len < 1) return invalid("fp8_update_scales: hist_len must be >= 1");
+    if (num_tensors > 0 && (amax_history == nullptr || scale == nullptr || scale_inv == nullptr || formats == nullptr))
+        return invalid("fp8_update_scales: NULL pointer");
+    if (algo != FP8DS_AMAX_MAX) {
+        set_error("fp8_update_scales: only amax_compute_algo=max is implemented");
+        return FP8DS_ERR_UNSUPPORTED;
+    }
+    return cuda_status(launch_update_scales(num_tensors, hist_len, amax_history, scale, scale_inv, formats, stream),
+                       "fp8_update_scales");
+}
+
+fp8ds_status fp8_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
+                      fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
+                      void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, fp8ds_stream stream) {
+    clear_error();
+    fp8ds_status st =
+        check_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k);
+    if (st != FP8DS_OK) return st;
+    return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k, stream);
+}
+
+fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x, fp8ds_dtype x_dtype,
+                            int64_t m, void *y, fp8ds_dtype y_dtype, int32_t is_first_microbatch, uint8_t *x8,
+                            uint8_t *x8t, float *x_scale_inv, fp8ds_stream stream) {
+    clear_error();
+    if (lin == nullptr || lin->w == nullptr || lin->w8 == nullptr || lin->w8t == nullptr ||
+        lin->w_scale_inv == nullptr)
+        return invalid("fp8_linear_fwd: incomplete linear handle");
+    if (x == nullptr || y == nullptr || x8 == nullptr || x_scale_inv == nullptr)
+        return invalid("fp8_linear_fwd: x, y, x8 and x_scale_inv must not be NULL");
+    if (is_first_microbatch < -1 || is_first_microbatch > 1)
+        return invalid("fp8_linear_fwd: is_first_microbatch must be -1, 0 or 1");
+    fp8ds_status st;
+    if ((st = check_meta("fp8_linear_fwd", meta, lin->meta_in)) != FP8DS_OK) return st;
+    if ((st = check_meta("fp8_linear_fwd", meta, lin->meta_w)) != FP8DS_OK) return st;
+    const int64_t K = lin->in_features, N = lin->out_features;
+    if ((st = check_cast("fp8_linear_fwd", x, x_dtype, m, K, FP8DS_E4M3, meta->scale, x8)) != FP8DS_OK) return st;
+    if ((st = check_gemm(x8, FP8DS_E4M3, x_scale_inv, lin->w8, FP8DS_E4M3, lin->w_scale_inv, lin->bias,
+                         lin->bias_dtype, y, y_dtype, m, N, K)) != FP8DS_OK)
+        return st;
+    cudaStream_t s = stream;
+    const int32_t hi = lin->meta_in, hw = lin->meta_w;
+    st = cuda_status(launch_cast_transpose(x, x_dtype, m, K, FP8DS_E4M3, meta->scale + hi, x8, x8t,
+                                           meta->amax_history + hi, x_scale_inv, s),
+                     "fp8_linear_fwd: input cast");
+    if (st != FP8DS_OK) return st;
+    const bool refresh = is_first_microbatch != 0 || !lin->cache_valid;
+    if (refresh) {
+        st = cuda_status(launch_cast_transpose(lin->w, FP8DS_F32, N, K, FP8DS_E4M3, meta->scale + hw, lin->w8,
+                                               lin->w8t, meta->amax_history + hw, lin->w_scale_inv, s),
+                         "fp8_linear_fwd: weight cast");
+        if (st != FP8DS_OK) return st;
+        lin->cache_valid = 1;
+    }
+    return launch_gemm(x8, FP8DS_E4M3, x_scale_inv, lin->w8, FP8DS_E4M3, lin->w_scale_inv, lin->bias,
+                       lin->bias_dtype, y, y_dtype, m, N, K, s);
+}
+
+fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy, fp8ds_dtype dy_dtype,
+                            int64_t m, const uint8_t *x8t, const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
+                            float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv, fp8ds_stream stream) {
+    clear_error();
+    if (lin == nullptr || lin->w8t == nullptr || lin->w_scale_inv == nullptr)
+        return invalid("fp8_linear_bwd: incomplete linear handle");
+    if (!lin->cache_valid) return invalid("fp8_linear_bwd: the weight cache is empty (run the forward first)");
+    if (dy == nullptr || x8t == nullptr || x_scale_inv == nullptr || dw == nullptr || dy8 == nullptr ||
+        dy8t == nullptr || dy_scale_inv == nullptr)
+        return invalid("fp8_linear_bwd: NULL pointer argument");
+    fp8ds_status st;
+    if ((st = check_meta("fp8_linear_bwd", meta, lin->meta_grad)) != FP8DS_OK) return st;
+    const int64_t K = lin->in_features, N = lin->out_features;
+    if ((st = check_cast("fp8_linear_bwd", dy, dy_dtype, m, N, FP8DS_E5M2, meta->scale, dy8)) != FP8DS_OK)
+        return st;
+    if (dx != nullptr && (st = check_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv,
+                                          nullptr, FP8DS_F32, dx, dx_dtype, m, K, N)) != FP8DS_OK)
+        return st;
+    if ((st = check_gemm(dy8t, FP8DS_E5M2, dy_scale_inv, x8t, FP8DS_E4M3, x_scale_inv, nullptr, FP8DS_F32, dw,
+                         FP8DS_F32, N, K, m)) != FP8DS_OK)
+        return st;
+    cudaStream_t s = stream;
+    const int32_t hg = lin->meta_grad;
+    st = cuda_status(launch_cast_transpose(dy, dy_dtype, m, N, FP8DS_E5M2, meta->scale + hg, dy8, dy8t,
+                                           meta->amax_history + hg, dy_scale_inv, s),
+                     "fp8_linear_bwd: grad cast");
+    if (st != FP8DS_OK) return st;
+    if (dx != nullptr) {
+        st = launch_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv, nullptr, FP8DS_F32,
+                         dx, dx_dtype, m, K, N, s);
+        if (st != FP8DS_OK) return st;
+    }
+    return launch_gemm(dy8t, FP8DS_E5M2, dy_scale_inv, x8t, FP8DS_E4M3, x_scale_inv, nullptr, FP8DS_F32, dw,
+                       FP8DS_F32, N, K, m, s);
+}
+
+const char *fp8ds_last_error(void) { return g_msg; }
+
+fp8ds_status fp8ds_device_status(int32_t *code_out, int32_t clear) {
+    clear_error();
+    if (code_out == nullptr) return invalid("fp8ds_device_status: code_out must not be NULL");
+    return cuda_status(read_device_error(code_out, clear != 0), "fp8ds_device_status");
+}
+
+const char *fp8ds_version(void) { return "fp8ds 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

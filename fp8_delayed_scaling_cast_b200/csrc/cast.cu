@@ -1,0 +1,356 @@
+// Per-tensor FP8 cast kernels for sm_100a: fp8_quantize (flat) and
+// fp8_cast_transpose_amax (2-D, with the FP8 transpose).
+//
+// What is computed ("Accelerating PyTorch Training Workloads with FP8 -- Part 2",
+// worked cast example; "[PyTorch] Refactor FP8 workspaces in linear modules",
+// Float8Tensor private scale-inverse):
+//   y = sat_rne_fp8(fl32(x * scale)),  yt = y^T,  amax = max(amax, max|x|),
+//   scale_inv = fl32(1 / scale).
+//
+// Both kernels are HBM-bound.  Design for B200:
+//   - every global access is a 16-byte vector (8-byte for the row-major FP8
+//     output of the transpose kernel), coalesced across the warp;
+//   - the transpose is done in two steps: a 4x4 byte transpose in registers
+//     (byte permutes) turns four input rows into column words, which go to a
+//     padded shared-memory tile; each thread then reads 16 consecutive rows
+//     of one column and writes them to yt as one 16-byte store;
+//   - amax is reduced with warp shuffles, then once per CTA, then one atomic
+//     max on the float's bit pattern (non-negative floats order like ints);
+//   - grids are sized to fill every SM with resident CTAs and loop over
+//     tiles (grid-stride), so the atomics are few.
+// The cast itself is the hardware conversion cvt.rn.satfinite.{e4m3,e5m2}x2,
+// which rounds to nearest-even and saturates finite overflow and infinities to
+// +-max; NaN inputs are rewritten to the canonical code 0x7F.
+#include <cuda_bf16.h>
+
+#include "fp8ds_internal.h"
+
+namespace fp8ds {
+namespace {
+
+// ---------------------------------------------------------------- elements --
+
+template <typename T>
+struct InElem;
+template <>
+struct InElem<float> {
+    static __device__ __forceinline__ float load(const float *p) { return __ldg(p); }
+};
+template <>
+struct InElem<uint16_t> {  // bf16 stored as raw bits; widening is exact
+    static __device__ __forceinline__ float load(const uint16_t *p) {
+        return __uint_as_float(static_cast<uint32_t>(__ldg(p)) << 16);
+    }
+};
+
+// Two FP8 codes packed in 16 bits: byte 0 = code(lo), byte 1 = code(hi).
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
+    uint16_t r;
+    if (FMT == FP8DS_E4M3) {
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    } else {
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    }
+    uint32_t v = r;
+    v = (lo != lo) ? ((v & 0xFF00u) | 0x007Fu) : v;
+    v = (hi != hi) ? ((v & 0x00FFu) | 0x7F00u) : v;
+    return v;
+}
+
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt1(float v) {
+    return cvt2<FMT>(v, 0.0f) & 0xFFu;
+}
+
+// Scale 4 values, cast, pack into one word (byte i = element i); fold |x| into m.
+template <int FMT>
+__device__ __forceinline__ uint32_t cast4(float a, float b, float c, float d, float s, float &m) {
+    m = fmaxf(m, fabsf(a));
+    m = fmaxf(m, fabsf(b));
+    m = fmaxf(m, fabsf(c));
+    m = fmaxf(m, fabsf(d));
+    return cvt2<FMT>(__fmul_rn(a, s), __fmul_rn(b, s)) |
+           (cvt2<FMT>(__fmul_rn(c, s), __fmul_rn(d, s)) << 16);
+}
+
+// Load 8 consecutive elements (16-byte aligned) and return them as two code
+// words (elements 0-3, 4-7).
+template <typename T, int FMT>
+struct Load8;
+template <int FMT>
+struct Load8<uint16_t, FMT> {
+    static __device__ __forceinline__ uint4 raw(const uint16_t *p) {
+        return __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    static __device__ __forceinline__ uint2 cast(const uint4 &v, float s, float &m) {
+        auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+        auto hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
+        uint2 r;
+        r.x = cast4<FMT>(lo(v.x), hi(v.x), lo(v.y), hi(v.y), s, m);
+        r.y = cast4<FMT>(lo(v.z), hi(v.z), lo(v.w), hi(v.w), s, m);
+        return r;
+    }
+};
+template <int FMT>
+struct Load8<float, FMT> {
+    struct Raw {
+        float4 a, b;
+    };
+    static __device__ __forceinline__ Raw raw(const float *p) {
+        Raw r;
+        r.a = __ldg(reinterpret_cast<const float4 *>(p));
+        r.b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+        return r;
+    }
+    static __device__ __forceinline__ uint2 cast(const Raw &v, float s, float &m) {
+        uint2 r;
+        r.x = cast4<FMT>(v.a.x, v.a.y, v.a.z, v.a.w, s, m);
+        r.y = cast4<FMT>(v.b.x, v.b.y, v.b.z, v.b.w, s, m);
+        return r;
+    }
+};
+
+__device__ __forceinline__ float warp_max(float m) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    return m;
+}
+
+// Block-wide max, then one atomic max into *amax (values are >= 0).
+template <int THREADS>
+__device__ __forceinline__ void block_amax_commit(float m, float *amax) {
+    __shared__ float red[THREADS / 32];
+    m = warp_max(m);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (warp == 0) {
+        m = lane < THREADS / 32 ? red[lane] : 0.0f;
+        m = warp_max(m);
+        if (lane == 0 && amax != nullptr && m > 0.0f)
+            atomicMax(reinterpret_cast<int *>(amax), __float_as_int(m));
+    }
+}
+
+// ------------------------------------------------------- cast + transpose --
+
+constexpr int CT_ROWS = 128;      // tile rows (x rows = yt columns)
+constexpr int CT_COLS = 64;       // tile columns
+constexpr int CT_THREADS = 256;
+constexpr int CT_TSTRIDE = 33;    // words per transposed row in shared memory (padded)
+
+// Vectorised path requirements (checked on the host): 16-byte aligned x, y,
+// yt; cols % 8 == 0; rows % 16 == 0.  Interior tiles take the vector path,
+// edge tiles the element path.  VEC = false forces the element path.
+template <typename T, int FMT, bool VEC, bool WRITE_T>
+__global__ void __launch_bounds__(CT_THREADS)
+cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
+                      const float *__restrict__ scale_ptr, uint8_t *__restrict__ y,
+                      uint8_t *__restrict__ yt, float *__restrict__ amax,
+                      float *__restrict__ scale_inv, int64_t tiles_c, int64_t num_tiles) {
+    __shared__ uint32_t tsm[CT_COLS * CT_TSTRIDE];
+    uint8_t *tsm8 = reinterpret_cast<uint8_t *>(tsm);
+    const float s = __ldg(scale_ptr);
+    const int tid = threadIdx.x;
+    float m = 0.0f;
+
+    if (blockIdx.x == 0 && tid == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
+
+    for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        const int64_t r0 = (tile / tiles_c) * CT_ROWS;
+        const int64_t c0 = (tile % tiles_c) * CT_COLS;
+        const bool full = VEC && (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
+        if (full) {
+            // Phase 1: thread = (column chunk cc of 8, row group rg of 4 rows).
+            const int cc = tid & 7, rg = tid >> 3;
+            const T *xp = x + (r0 + 4 * rg) * cols + c0 + 8 * cc;
+            decltype(Load8<T, FMT>::raw(xp)) raw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) raw[i] = Load8<T, FMT>::raw(xp + i * cols);
+            uint2 w[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = Load8<T, FMT>::cast(raw[i], s, m);
+            uint8_t *yp = y + (r0 + 4 * rg) * cols + c0 + 8 * cc;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) *reinterpret_cast<uint2 *>(yp + i * cols) = w[i];
+            if (WRITE_T) {
+                // 4 rows x 8 bytes -> 8 column words of 4 rows each.
+                uint32_t colw[8];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t a0 = h ? w[0].y : w[0].x, a1 = h ? w[1].y : w[1].x;
+                    const uint32_t a2 = h ? w[2].y : w[2].x, a3 = h ? w[3].y : w[3].x;
+                    const uint32_t p01l = __byte_perm(a0, a1, 0x5140);
+                    const uint32_t p01h = __byte_perm(a0, a1, 0x7362);
+                    const uint32_t p23l = __byte_perm(a2, a3, 0x5140);
+                    const uint32_t p23h = __byte_perm(a2, a3, 0x7362);
+                    colw[4 * h + 0] = __byte_perm(p01l, p23l, 0x5410);
+                    colw[4 * h + 1] = __byte_perm(p01l, p23l, 0x7632);
+                    colw[4 * h + 2] = __byte_perm(p01h, p23h, 0x5410);
+                    colw[4 * h + 3] = __byte_perm(p01h, p23h, 0x7632);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) tsm[(8 * cc + j) * CT_TSTRIDE + rg] = colw[j];
+                __syncthreads();
+                // Phase 2: 64 columns x 8 chunks of 16 rows; 2 chunks per thread.
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int idx = tid + CT_THREADS * k;
+                    const int c = idx >> 3, q = idx & 7;
+                    const uint32_t *src = tsm + c * CT_TSTRIDE + 4 * q;
+                    uint4 v = make_uint4(src[0], src[1], src[2], src[3]);
+                    *reinterpret_cast<uint4 *>(yt + (c0 + c) * rows + r0 + 16 * q) = v;
+                }
+                __syncthreads();
+            }
+        } else {
+            // Element path for edge tiles (and for unaligned tensors).
+            for (int i = 0; i < (CT_ROWS * CT_COLS) / CT_THREADS; ++i) {
+                const int e = tid + CT_THREADS * i;
+                const int r = e / CT_COLS, c = e % CT_COLS;
+                const int64_t gr = r0 + r, gc = c0 + c;
+                uint32_t code = 0;
+                if (gr < rows && gc < cols) {
+                    const float v = InElem<T>::load(x + gr * cols + gc);
+                    m = fmaxf(m, fabsf(v));
+                    code = cvt1<FMT>(__fmul_rn(v, s));
+                    y[gr * cols + gc] = static_cast<uint8_t>(code);
+                }
+                if (WRITE_T) tsm8[c * (CT_TSTRIDE * 4) + r] = static_cast<uint8_t>(code);
+            }
+            if (WRITE_T) {
+                __syncthreads();
+                for (int i = 0; i < (CT_ROWS * CT_COLS) / CT_THREADS; ++i) {
+                    const int e = tid + CT_THREADS * i;
+                    const int c = e / CT_ROWS, r = e % CT_ROWS;
+                    const int64_t gr = r0 + r, gc = c0 + c;
+                    if (gr < rows && gc < cols) yt[gc * rows + gr] = tsm8[c * (CT_TSTRIDE * 4) + r];
+                }
+                __syncthreads();
+            }
+        }
+    }
+    block_amax_commit<CT_THREADS>(m, amax);
+}
+
+// ---------------------------------------------------------------- quantize --
+
+constexpr int Q_THREADS = 256;
+
+// Each thread converts 16 elements per step: 16-byte loads, one 16-byte store.
+template <typename T, int FMT, bool VEC>
+__global__ void __launch_bounds__(Q_THREADS)
+quantize_kernel(const T *__restrict__ x, int64_t n, const float *__restrict__ scale_ptr,
+                uint8_t *__restrict__ y, float *__restrict__ amax, float *__restrict__ scale_inv) {
+    const float s = __ldg(scale_ptr);
+    float m = 0.0f;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * Q_THREADS + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * Q_THREADS;
+    if (tid == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
+    int64_t done = 0;
+    if (VEC) {
+        const int64_t n16 = n / 16;
+        for (int64_t i = tid; i < n16; i += stride) {
+            const T *xp = x + i * 16;
+            auto r0 = Load8<T, FMT>::raw(xp);
+            auto r1 = Load8<T, FMT>::raw(xp + 8);
+            const uint2 a = Load8<T, FMT>::cast(r0, s, m);
+            const uint2 b = Load8<T, FMT>::cast(r1, s, m);
+            *reinterpret_cast<uint4 *>(y + i * 16) = make_uint4(a.x, a.y, b.x, b.y);
+        }
+        done = n16 * 16;
+    }
+    for (int64_t i = done + tid; i < n; i += stride) {
+        const float v = InElem<T>::load(x + i);
+        m = fmaxf(m, fabsf(v));
+        y[i] = static_cast<uint8_t>(cvt1<FMT>(__fmul_rn(v, s)));
+    }
+    block_amax_commit<Q_THREADS>(m, amax);
+}
+
+// -------------------------------------------------------------- launchers --
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename K>
+int grid_for(K kernel, int threads, int64_t work_items) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm;
+    int64_t g = work_items < cap ? work_items : cap;
+    return static_cast<int>(g < 1 ? 1 : g);
+}
+
+template <typename T, int FMT, bool VEC, bool WRITE_T>
+cudaError_t ct_launch(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y,
+                      uint8_t *yt, float *amax, float *scale_inv, cudaStream_t stream) {
+    const int64_t tiles_c = (cols + CT_COLS - 1) / CT_COLS;
+    const int64_t tiles_r = (rows + CT_ROWS - 1) / CT_ROWS;
+    const int64_t num_tiles = tiles_c * tiles_r;
+    auto kernel = cast_transpose_kernel<T, FMT, VEC, WRITE_T>;
+    const int grid = grid_for(kernel, CT_THREADS, num_tiles);
+    kernel<<<grid, CT_THREADS, 0, stream>>>(static_cast<const T *>(x), rows, cols, scale, y, yt,
+                                            amax, scale_inv, tiles_c, num_tiles);
+    return cudaGetLastError();
+}
+
+template <typename T, int FMT>
+cudaError_t ct_dispatch(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y,
+                        uint8_t *yt, float *amax, float *scale_inv, cudaStream_t stream) {
+    const bool vec = aligned16(x) && aligned16(y) && (yt == nullptr || aligned16(yt)) &&
+                     (cols % 8 == 0) && (rows % 16 == 0);
+    if (yt != nullptr) {
+        return vec ? ct_launch<T, FMT, true, true>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
+                   : ct_launch<T, FMT, false, true>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+    }
+    return vec ? ct_launch<T, FMT, true, false>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
+               : ct_launch<T, FMT, false, false>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+}
+
+template <typename T, int FMT>
+cudaError_t q_dispatch(const void *x, int64_t n, const float *scale, uint8_t *y, float *amax,
+                       float *scale_inv, cudaStream_t stream) {
+    const bool vec = aligned16(x) && aligned16(y);
+    const int64_t items = vec ? (n / 16 > 0 ? n / 16 : 1) : (n > 0 ? n : 1);
+    if (vec) {
+        auto kernel = quantize_kernel<T, FMT, true>;
+        const int grid = grid_for(kernel, Q_THREADS, (items + Q_THREADS - 1) / Q_THREADS);
+        kernel<<<grid, Q_THREADS, 0, stream>>>(static_cast<const T *>(x), n, scale, y, amax, scale_inv);
+    } else {
+        auto kernel = quantize_kernel<T, FMT, false>;
+        const int grid = grid_for(kernel, Q_THREADS, (items + Q_THREADS - 1) / Q_THREADS);
+        kernel<<<grid, Q_THREADS, 0, stream>>>(static_cast<const T *>(x), n, scale, y, amax, scale_inv);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_cast_transpose(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
+                                  fp8ds_format fmt, const float *scale, uint8_t *y, uint8_t *yt,
+                                  float *amax, float *scale_inv, cudaStream_t stream) {
+    if (x_dtype == FP8DS_F32) {
+        return fmt == FP8DS_E4M3
+                   ? ct_dispatch<float, FP8DS_E4M3>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
+                   : ct_dispatch<float, FP8DS_E5M2>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+    }
+    return fmt == FP8DS_E4M3
+               ? ct_dispatch<uint16_t, FP8DS_E4M3>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
+               : ct_dispatch<uint16_t, FP8DS_E5M2>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+}
+
+cudaError_t launch_quantize(const void *x, fp8ds_dtype x_dtype, int64_t n, fp8ds_format fmt,
+                            const float *scale, uint8_t *y, float *amax, float *scale_inv,
+                            cudaStream_t stream) {
+    if (x_dtype == FP8DS_F32) {
+        return fmt == FP8DS_E4M3 ? q_dispatch<float, FP8DS_E4M3>(x, n, scale, y, amax, scale_inv, stream)
+                                 : q_dispatch<float, FP8DS_E5M2>(x, n, scale, y, amax, scale_inv, stream);
+    }
+    return fmt == FP8DS_E4M3 ? q_dispatch<uint16_t, FP8DS_E4M3>(x, n, scale, y, amax, scale_inv, stream)
+                             : q_dispatch<uint16_t, FP8DS_E5M2>(x, n, scale, y, amax, scale_inv, stream);
+}
+
+}  // namespace fp8ds

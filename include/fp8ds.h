@@ -1,0 +1,250 @@
+/*
+ * fp8ds.h -- C ABI of libfp8ds.so, the FP8 delayed-scaling linear hot path
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Sources of the method (web pages; cited by title and section):
+ *   [TE820]  "[PyTorch] Refactor FP8 workspaces in linear modules"
+ *            (TransformerEngine PR #820): one cached FP8 weight workspace per
+ *            linear; a Float8Tensor keeps a private scale-inverse that scale
+ *            updates do not touch until its data is rewritten; lazy transpose
+ *            cache; is_first_microbatch.
+ *   [TE761]  "CPU Overhead of te.Linear FP8 Layers" (TransformerEngine issue
+ *            #761): the DelayedScaling recipe (HYBRID format, amax history
+ *            length 16, amax_compute_algo "max"), the TEBlock workload, and
+ *            the per-linear launch overhead that motivates few launches.
+ *   [F8E312] "support delayed scaling of weight in float8 all-gather"
+ *            (float8_experimental PR #312): amax buffers of all linears
+ *            gathered into one tensor and synced once per step.
+ *   [PTFP8]  "Accelerating PyTorch Training Workloads with FP8 -- Part 2"
+ *            (PyTorch-native FP8 data types): float8_e4m3fn / float8_e5m2
+ *            finfo table, the worked cast example, torch._scaled_mm.
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers unless stated otherwise; the caller owns all
+ *     memory (tensors, weight cache, meta arrays).  The library allocates
+ *     nothing, keeps no device state between calls (except the error word read
+ *     by fp8ds_device_status) and never synchronises: every call only enqueues
+ *     work on `stream` (NULL = the legacy default stream).
+ *   - Scalars that the method updates on the device (scale, amax, scale_inv)
+ *     are passed as device pointers, so a sequence of calls can be captured
+ *     in a CUDA graph.
+ *   - Tensors are dense row-major.  FP8 data are raw bytes (uint8).
+ *   - Return value: FP8DS_OK, or an error detected on the host before any
+ *     launch (nothing is enqueued then), or FP8DS_ERR_CUDA if a launch failed.
+ *     fp8ds_last_error() gives a message for the calling thread.
+ */
+#ifndef FP8DS_H
+#define FP8DS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8DS_OK = 0,
+    FP8DS_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment */
+    FP8DS_ERR_UNSUPPORTED = 2,   /* valid but not implemented combination */
+    FP8DS_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+    FP8DS_ERR_TIMEOUT = 4        /* a bounded device wait gave up (device word) */
+} fp8ds_status;
+
+/* FP8 formats [PTFP8 finfo table]: E4M3FN (max 448, no inf) and E5M2 (max 57344). */
+typedef enum { FP8DS_E4M3 = 0, FP8DS_E5M2 = 1 } fp8ds_format;
+
+/* High-precision element types. */
+typedef enum { FP8DS_F32 = 0, FP8DS_BF16 = 1 } fp8ds_dtype;
+
+/* Amax reduction over the history window [TE761 recipe: amax_compute_algo]. */
+typedef enum { FP8DS_AMAX_MAX = 0 } fp8ds_amax_algo;
+
+/* A cudaStream_t. */
+typedef struct CUstream_st *fp8ds_stream;
+
+/*
+ * fp8_quantize -- per-tensor cast of a flat tensor [PTFP8 worked cast example;
+ * TE820 Float8Tensor scale-inverse].
+ *
+ *   y[i]       = sat_rne_fp8(fl32(x[i] * *scale))   for i < n
+ *   *amax      = max(*amax, max_i |x[i]|)           (unscaled input, NaN ignored)
+ *   *scale_inv = fl32(1 / *scale)                   (the tensor's private copy)
+ *
+ * sat_rne_fp8 rounds to nearest, ties to even, saturates to +-max (also +-inf),
+ * keeps the sign of zero and maps NaN to 0x7F.
+ *   x        [n] fp32 or bf16 (x_dtype).
+ *   scale    [1] fp32, read on the device.
+ *   y        [n] uint8 FP8 codes of format `fmt`.
+ *   amax     [1] fp32 or NULL.  Atomically max-ed into, so it must hold a
+ *            non-negative value (normally slot 0 of the tensor's amax history).
+ *   scale_inv[1] fp32 or NULL.
+ * Errors: FP8DS_ERR_INVALID_ARG if n < 0 or a required pointer is NULL.
+ * n == 0 enqueues only the scale_inv write.
+ */
+fp8ds_status fp8_quantize(const void *x, fp8ds_dtype x_dtype, int64_t n, fp8ds_format fmt,
+                          const float *scale, uint8_t *y, float *amax, float *scale_inv,
+                          fp8ds_stream stream);
+
+/*
+ * fp8_cast_transpose_amax -- fp8_quantize of a 2-D tensor that also writes the
+ * FP8 transpose [TE820: FP8 weight workspace and its transpose cache; the
+ * transposes feed the backward GEMMs].
+ *
+ *   y[r,c]  = sat_rne_fp8(fl32(x[r,c] * *scale))     y  [rows, cols]
+ *   yt[c,r] = y[r,c]                                  yt [cols, rows] (NULL: skipped)
+ *   amax, scale_inv as in fp8_quantize.
+ * Errors: FP8DS_ERR_INVALID_ARG for negative sizes or NULL x / scale / y.
+ * Any sizes are accepted; 16-byte aligned pointers with cols % 8 == 0 and
+ * rows % 16 == 0 take the vectorised path.
+ */
+fp8ds_status fp8_cast_transpose_amax(const void *x, fp8ds_dtype x_dtype, int64_t rows,
+                                     int64_t cols, fp8ds_format fmt, const float *scale,
+                                     uint8_t *y, uint8_t *yt, float *amax, float *scale_inv,
+                                     fp8ds_stream stream);
+
+/*
+ * fp8_update_scales -- the delayed-scaling recipe update of T FP8 meta tensors
+ * in ONE launch [TE820 "FP8 scale update kernel"; TE761 DelayedScaling(
+ * amax_history_len=16, amax_compute_algo="max"); F8E312 amax buffers of all
+ * linears handled together].  For every t < num_tensors:
+ *
+ *   a          = max_h amax_history[h, t]                (window of hist_len steps)
+ *   scale[t]   = fl32(fp8_max(formats[t]) / a)  if a > 0, a finite and the
+ *                quotient finite; otherwise scale[t] is kept
+ *   scale_inv[t] = fl32(1 / scale[t])                   (the meta's copy; FP8
+ *                tensors keep the private copy written by their cast)
+ *   amax_history[:, t] rolled by one: h <- h+1 (slot hist_len-1 receives the
+ *                current amax of slot 0), then slot 0 = 0 for the next step.
+ *
+ *   amax_history [hist_len, num_tensors] fp32, slot-major (row 0 = the amaxes
+ *                recorded in the current step; contiguous, so a cross-rank
+ *                max-reduction of row 0 is one contiguous buffer).
+ *   scale, scale_inv [num_tensors] fp32;  formats [num_tensors] uint8 (fp8ds_format).
+ * Errors: FP8DS_ERR_INVALID_ARG for num_tensors < 0, hist_len < 1 or NULL
+ * pointers; FP8DS_ERR_UNSUPPORTED for an algo other than FP8DS_AMAX_MAX.
+ */
+fp8ds_status fp8_update_scales(int64_t num_tensors, int32_t hist_len, float *amax_history,
+                               float *scale, float *scale_inv, const uint8_t *formats,
+                               fp8ds_amax_algo algo, fp8ds_stream stream);
+
+/*
+ * fp8_gemm -- scaled FP8 GEMM with a dequantising epilogue [PTFP8
+ * torch._scaled_mm: two FP8 operands, their scale factors, optional bias,
+ * chosen output dtype; TE761 HYBRID: e4m3 x e4m3 forward, e5m2 x e4m3 for
+ * gradients].
+ *
+ *   d[m,n] = (sum_k dec(a[m,k]) * dec(b[n,k])) * *a_scale_inv * *b_scale_inv
+ *            (+ bias[n])                       accumulated in fp32
+ *
+ *   a [m, k] uint8 FP8 (a_fmt), row-major (k contiguous)
+ *   b [n, k] uint8 FP8 (b_fmt), row-major (k contiguous): the "TN" layout of
+ *     torch._scaled_mm(a, b.t())
+ *   a_scale_inv, b_scale_inv [1] fp32 (normally the operands' private copies)
+ *   bias [n] (bias_dtype) or NULL
+ *   d [m, n] fp32 or bf16 (d_dtype)
+ * Requirements (TMA): k % 16 == 0, a/b/d 16-byte aligned, n % 8 == 0 for bf16
+ * and n % 4 == 0 for fp32 output.  m, n, k > 0.
+ * Errors: FP8DS_ERR_INVALID_ARG when a requirement fails; FP8DS_ERR_CUDA if
+ * the tensor maps cannot be encoded or the launch fails.  A device-side wait
+ * that exceeds its time limit aborts the kernel and sets the error word read
+ * by fp8ds_device_status (the output is then undefined).
+ */
+fp8ds_status fp8_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
+                      const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
+                      const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
+                      int64_t m, int64_t n, int64_t k, fp8ds_stream stream);
+
+/*
+ * Packed FP8 meta of T tensors (the DelayedScaling state [TE761; F8E312
+ * _amax_history_buffer / _scale_buffer]).  All arrays are caller-owned device
+ * memory; amax_history is [hist_len, num_tensors] slot-major, zero-filled and
+ * scale = 1 at initialisation (no amax-init pass).
+ */
+typedef struct {
+    float *amax_history;
+    float *scale;
+    float *scale_inv;
+    const uint8_t *formats;
+    int64_t num_tensors;
+    int32_t hist_len;
+} fp8ds_meta;
+
+/*
+ * One linear layer y = x . w^T + bias with its FP8 weight cache [TE820]:
+ * w8 / w8t hold the e4m3 weight and its transpose, w_scale_inv the private
+ * scale-inverse they were cast with.  meta_in / meta_w / meta_grad index the
+ * packed meta (input, weight, output-gradient tensors).  cache_valid is a host
+ * flag that fp8_linear_fwd sets once the cache holds a cast weight; set it to
+ * 0 to force the next forward to refresh the cache.
+ */
+typedef struct {
+    const float *w;            /* [out_features, in_features] fp32 master weight */
+    const void *bias;          /* [out_features] or NULL */
+    fp8ds_dtype bias_dtype;
+    int64_t in_features;
+    int64_t out_features;
+    uint8_t *w8;               /* [out_features, in_features] cached FP8 weight */
+    uint8_t *w8t;              /* [in_features, out_features] cached FP8 transpose */
+    float *w_scale_inv;        /* [1] private scale_inv of the cached weight */
+    int32_t meta_in, meta_w, meta_grad;
+    int32_t cache_valid;
+} fp8ds_linear;
+
+/*
+ * fp8_linear_fwd -- FP8 forward of one linear [TE820; TE761 HYBRID: e4m3]:
+ *   1. cast x -> x8 (and x8t if not NULL) with meta.scale[meta_in], amax into
+ *      amax_history[0, meta_in], private scale_inv into *x_scale_inv;
+ *   2. if is_first_microbatch is -1 (None: always), 1 (True: refresh and keep),
+ *      or 0 (False) with no valid cache: cast w -> w8 and w8t with
+ *      meta.scale[meta_w], amax into amax_history[0, meta_w], private
+ *      scale_inv into *w_scale_inv; sets cache_valid.  With 0 and a valid
+ *      cache the cached weight and its frozen scale_inv are reused;
+ *   3. y = fp8_gemm(x8, w8, *x_scale_inv, *w_scale_inv, bias).
+ *   x [m, in_features] (x_dtype); y [m, out_features] (y_dtype);
+ *   x8 [m, in_features], x8t [in_features, m] or NULL (needed by the backward).
+ * The delayed-scaling update is not part of the forward: call
+ * fp8_update_scales once per step over the whole meta.
+ * Errors: as the calls it makes; nothing is enqueued if the arguments fail.
+ */
+fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x,
+                            fp8ds_dtype x_dtype, int64_t m, void *y, fp8ds_dtype y_dtype,
+                            int32_t is_first_microbatch, uint8_t *x8, uint8_t *x8t,
+                            float *x_scale_inv, fp8ds_stream stream);
+
+/*
+ * fp8_linear_bwd -- FP8 backward of one linear [TE761 HYBRID: e5m2 gradients]:
+ *   1. cast dy -> e5m2 dy8 and dy8t with meta.scale[meta_grad], amax into
+ *      amax_history[0, meta_grad], private scale_inv into *dy_scale_inv;
+ *   2. dgrad (if dx != NULL): dx[m, in] = dy8 . (w8t)^T with
+ *      *dy_scale_inv * *w_scale_inv (the cached weight's private copy);
+ *   3. wgrad: dw[out, in] (fp32) = dy8t . (x8t)^T with *dy_scale_inv * *x_scale_inv.
+ *   dy [m, out_features] (dy_dtype); x8t [in_features, m] and x_scale_inv from
+ *   the forward; dy8 [m, out_features], dy8t [out_features, m] workspaces.
+ * Requires lin->cache_valid.  Errors: as the calls it makes.
+ */
+fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy,
+                            fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8t,
+                            const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
+                            float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv,
+                            fp8ds_stream stream);
+
+/* Message describing the last error returned on the calling thread ("" if none). */
+const char *fp8ds_last_error(void);
+
+/*
+ * fp8ds_device_status -- reads the device error word that kernels set when a
+ * bounded wait gives up (0 = none, otherwise FP8DS_ERR_TIMEOUT in the low byte
+ * and the site in the upper bytes).  Synchronises the current device.  If
+ * `clear` is non-zero the word is reset to 0.  Returns FP8DS_ERR_CUDA if the
+ * read fails.
+ */
+fp8ds_status fp8ds_device_status(int32_t *code_out, int32_t clear);
+
+/* Library version string. */
+const char *fp8ds_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8DS_H */

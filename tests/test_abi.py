@@ -1,0 +1,109 @@
+"""The C ABI library loads, exports every symbol the header declares, and
+rejects bad arguments on the host before any launch (no GPU needed: the
+argument checks run before the first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "fp8ds.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_delayed_scaling_cast_b200 import build
+    build.build()
+    from fp8_delayed_scaling_cast_b200 import binding
+    return binding
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(fp8\w*)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("fp8_quantize", "fp8_cast_transpose_amax", "fp8_update_scales", "fp8_gemm",
+              "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
+              "fp8ds_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in _declared_functions():
+        assert hasattr(raw, n), n
+
+
+def test_version(lib):
+    assert "sm_100a" in lib.fp8ds_version()
+
+
+P = ctypes.c_void_p
+FAKE = P(0x10000)          # never dereferenced: every call below fails its checks first
+FAKE_ODD = P(0x10001)
+
+
+def test_gemm_argument_checks(lib):
+    L = lib._lib
+    s = P(0)
+    ok_args = dict(a=FAKE, fa=0, sa=FAKE, b=FAKE, fb=0, sb=FAKE, bias=None, bt=0, d=FAKE, dt=1,
+                   m=128, n=256, k=128)
+
+    def call(**kw):
+        a = dict(ok_args)
+        a.update(kw)
+        return L.fp8_gemm(a["a"], a["fa"], a["sa"], a["b"], a["fb"], a["sb"], a["bias"], a["bt"],
+                          a["d"], a["dt"], a["m"], a["n"], a["k"], s)
+
+    assert call(k=120) == lib.ERR_INVALID_ARG and "multiple of 16" in lib.fp8ds_last_error()
+    assert call(a=None) == lib.ERR_INVALID_ARG
+    assert call(m=0) == lib.ERR_INVALID_ARG
+    assert call(n=12) == lib.ERR_INVALID_ARG           # bf16 output needs n % 8 == 0
+    assert call(a=FAKE_ODD) == lib.ERR_INVALID_ARG and "aligned" in lib.fp8ds_last_error()
+    assert call(fa=7) == lib.ERR_INVALID_ARG
+    assert call(m=1 << 31) == lib.ERR_INVALID_ARG
+
+
+def test_cast_and_update_argument_checks(lib):
+    L = lib._lib
+    s = P(0)
+    assert L.fp8_quantize(None, 0, 16, 0, FAKE, FAKE, None, None, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_quantize(FAKE, 0, -1, 0, FAKE, FAKE, None, None, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_quantize(FAKE, 0, 16, 3, FAKE, FAKE, None, None, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_quantize(FAKE, 5, 16, 0, FAKE, FAKE, None, None, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_cast_transpose_amax(FAKE, 0, 4, -4, 0, FAKE, FAKE, None, None, None, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_cast_transpose_amax(FAKE, 0, 4, 4, 0, None, FAKE, None, None, None, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_update_scales(-1, 16, FAKE, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_update_scales(4, 0, FAKE, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_update_scales(4, 16, None, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_update_scales(4, 16, FAKE, FAKE, FAKE, FAKE, 1, s) == lib.ERR_UNSUPPORTED
+    # zero tensors: nothing to do, nothing launched
+    assert L.fp8_update_scales(0, 16, None, None, None, None, 0, s) == lib.OK
+
+
+def test_linear_argument_checks(lib):
+    L = lib._lib
+    s = P(0)
+    meta = lib._Meta(FAKE, FAKE, FAKE, FAKE, 3, 16)
+    lin = lib._Linear(FAKE, None, 0, 256, 512, FAKE, FAKE, FAKE, 0, 1, 2, 0)
+    r = L.fp8_linear_fwd(ctypes.byref(lin), ctypes.byref(meta), FAKE, 0, 128, FAKE, 0, 2, FAKE,
+                         FAKE, FAKE, s)
+    assert r == lib.ERR_INVALID_ARG and "is_first_microbatch" in lib.fp8ds_last_error()
+    bad = lib._Linear(FAKE, None, 0, 256, 512, FAKE, FAKE, FAKE, 0, 7, 2, 0)
+    r = L.fp8_linear_fwd(ctypes.byref(bad), ctypes.byref(meta), FAKE, 0, 128, FAKE, 0, 1, FAKE,
+                         FAKE, FAKE, s)
+    assert r == lib.ERR_INVALID_ARG and "out of range" in lib.fp8ds_last_error()
+    r = L.fp8_linear_fwd(ctypes.byref(lin), ctypes.byref(meta), FAKE, 0, 128, FAKE, 0, 1, FAKE,
+                         FAKE, None, s)
+    assert r == lib.ERR_INVALID_ARG
+    # backward before any forward: the cache is empty
+    r = L.fp8_linear_bwd(ctypes.byref(lin), ctypes.byref(meta), FAKE, 1, 128, FAKE, FAKE, FAKE, 1,
+                         FAKE, FAKE, FAKE, FAKE, s)
+    assert r == lib.ERR_INVALID_ARG and "cache" in lib.fp8ds_last_error()
