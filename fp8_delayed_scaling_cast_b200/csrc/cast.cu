@@ -157,20 +157,36 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
 
     if (blockIdx.x == 0 && tid == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
 
+    // Vector path: thread = (column chunk cc of 8, row group rg of 4 rows).
+    // The next tile's loads are issued before the current tile is processed,
+    // so they stay in flight across its shared-memory transpose and barriers.
+    const int cc = tid & 7, rg = tid >> 3;
+    using Raw = decltype(Load8<T, FMT>::raw(x));
+    Raw cur[4], nxt[4];
+    auto tile_full = [&](int64_t tile) {
+        if (!VEC || tile >= num_tiles) return false;  // (tiles_c > 0 whenever num_tiles > 0)
+        const int64_t r0 = (tile / tiles_c) * CT_ROWS, c0 = (tile % tiles_c) * CT_COLS;
+        return (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
+    };
+    auto load_tile = [&](int64_t tile, Raw(&dst)[4]) {
+        const int64_t r0 = (tile / tiles_c) * CT_ROWS, c0 = (tile % tiles_c) * CT_COLS;
+        const T *xp = x + (r0 + 4 * rg) * cols + c0 + 8 * cc;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = Load8<T, FMT>::raw(xp + i * cols);
+    };
+    bool cur_full = tile_full(blockIdx.x);
+    if (cur_full) load_tile(blockIdx.x, cur);
+
     for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         const int64_t r0 = (tile / tiles_c) * CT_ROWS;
         const int64_t c0 = (tile % tiles_c) * CT_COLS;
-        const bool full = VEC && (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
-        if (full) {
-            // Phase 1: thread = (column chunk cc of 8, row group rg of 4 rows).
-            const int cc = tid & 7, rg = tid >> 3;
-            const T *xp = x + (r0 + 4 * rg) * cols + c0 + 8 * cc;
-            decltype(Load8<T, FMT>::raw(xp)) raw[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) raw[i] = Load8<T, FMT>::raw(xp + i * cols);
+        const int64_t next = tile + gridDim.x;
+        const bool next_full = tile_full(next);
+        if (next_full) load_tile(next, nxt);
+        if (cur_full) {
             uint2 w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = Load8<T, FMT>::cast(raw[i], s, m);
+            for (int i = 0; i < 4; ++i) w[i] = Load8<T, FMT>::cast(cur[i], s, m);
             uint8_t *yp = y + (r0 + 4 * rg) * cols + c0 + 8 * cc;
 #pragma unroll
             for (int i = 0; i < 4; ++i) *reinterpret_cast<uint2 *>(yp + i * cols) = w[i];
@@ -193,7 +209,7 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
 #pragma unroll
                 for (int j = 0; j < 8; ++j) tsm[(8 * cc + j) * CT_TSTRIDE + rg] = colw[j];
                 __syncthreads();
-                // Phase 2: 64 columns x 8 chunks of 16 rows; 2 chunks per thread.
+                // 64 columns x 8 chunks of 16 rows; 2 chunks per thread.
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     const int idx = tid + CT_THREADS * k;
@@ -230,6 +246,11 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
                 __syncthreads();
             }
         }
+        if (next_full) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
+        }
+        cur_full = next_full;
     }
     block_amax_commit<CT_THREADS>(m, amax);
 }

@@ -7,19 +7,32 @@
 // with A [M,K] and B [N,K] FP8, both contraction-major ("TN"), fp32
 // accumulation in tensor memory, fp32 or bf16 output.
 //
-// Kernel structure (one persistent CTA per SM, 6 warps):
-//   warp 0      TMA producer: 128x128-byte A and 256x128-byte B tiles into a
-//               4-stage shared-memory ring (128-byte swizzle), completion
-//               signalled on per-stage mbarriers (transaction bytes);
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
-//               issues tcgen05.mma.kind::f8f6f4 (M=128, N=256, K=32) from one
-//               thread; tcgen05.commit frees smem stages and publishes
-//               finished accumulators;
+// Two persistent warp-specialised kernels share one structure (6 warps):
+//   warp 0      TMA producer: A and B tiles (128-byte rows, 128-byte swizzle)
+//               into a shared-memory ring, completion on per-stage mbarriers
+//               (transaction bytes);
+//   warp 1      allocates 512 TMEM columns (two fp32 accumulators of 256
+//               columns) and issues tcgen05.mma.kind::f8f6f4 from one thread;
+//               tcgen05.commit frees ring stages and publishes accumulators;
 //   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, fp32 fma with the
 //               combined scale_inv and bias, conversion, 128-byte-swizzled
 //               staging in shared memory and TMA tensor stores.
-// Two accumulators let the epilogue of tile i overlap the main loop of tile
-// i+1.  No cluster multicast is used anywhere.
+// Two accumulators let the epilogue of tile i overlap the main loop of i+1.
+//
+//   fp8_gemm_1sm_kernel  one CTA per SM, tile 128 x 256, 4 stages of 48 KB
+//                        (used when M <= 128).
+//   fp8_gemm_2sm_kernel  CTA pairs (cluster of 2), tcgen05.mma.cta_group::2
+//                        with a 256 x 256 tile: each CTA loads its 128 rows of
+//                        A and its 128 rows of B (32 KB per stage, 6 stages),
+//                        the pair's MMA reads both CTAs' shared memory and
+//                        leaves rows 0-127 of D in CTA 0's TMEM and rows
+//                        128-255 in CTA 1's.  Per SM this halves the B bytes
+//                        moved per FLOP.  Both CTAs' loads signal CTA 0's
+//                        ring barriers; CTA 0's commits arrive on both CTAs'
+//                        barriers; both epilogues report to CTA 0.
+// Tiles are visited in groups of 8 row-tiles (column index slowest within a
+// group) so that concurrently running CTAs share A and B in L2.  No TMA load
+// uses cluster multicast.
 //
 // Every wait is bounded (wall-clock limit read from %globaltimer).  A wait
 // that gives up records FP8DS_ERR_TIMEOUT and its site in the device error
@@ -39,22 +52,37 @@ __device__ int32_t g_device_error = 0;
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 128;  // bytes == FP8 elements per k-block (one 128-byte swizzle row)
-constexpr int STAGES = 4;
-constexpr int UMMA_K = 32;
-constexpr int A_STAGE = BM * BK;
-constexpr int B_STAGE = BN * BK;
+constexpr int BK = 128;        // bytes == FP8 elements per k-block (one 128-byte swizzle row)
+constexpr int UMMA_K = 32;     // K of one kind::f8f6f4 MMA
+constexpr int ACC_N = 256;     // accumulator columns (tile N)
 constexpr int THREADS = 192;
 constexpr int EPI_WARP0 = 2;
-constexpr int TMEM_COLS = 512;
-constexpr int EPI_BOX_BYTES = 32 * 128;  // 32 rows x 128 bytes
+constexpr int TMEM_COLS = 512; // two accumulators
+constexpr int EPI_BOX_BYTES = 32 * 128;  // staging box: 32 rows x 128 bytes
 constexpr int EPI_BUFS = 2;
+constexpr int EPI_BYTES = 4 * EPI_BUFS * EPI_BOX_BYTES;
 constexpr int SMEM_ALIGN = 1024;
-constexpr int SMEM_BYTES = SMEM_ALIGN + STAGES * (A_STAGE + B_STAGE) + 4 * EPI_BUFS * EPI_BOX_BYTES + 256;
+constexpr int GROUP_M = 8;
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;  // 2 s
 constexpr unsigned long long DRAIN_NS = 200000000ull;     // 0.2 s
+
+// 1-SM kernel: tile 128 x 256, 4 stages of 16 KB (A) + 32 KB (B).
+constexpr int S1_BM = 128;
+constexpr int S1_STAGES = 4;
+constexpr int S1_A_STAGE = S1_BM * BK;
+constexpr int S1_B_STAGE = ACC_N * BK;
+constexpr int S1_SMEM = SMEM_ALIGN + S1_STAGES * (S1_A_STAGE + S1_B_STAGE) + EPI_BYTES + 256;
+
+// 2-SM kernel: pair tile 256 x 256; per CTA 128 rows of A and 128 rows of B
+// per stage (16 KB + 16 KB), 6 stages.
+constexpr int S2_BM = 128;           // rows of A (and of D) per CTA
+constexpr int S2_BN_HALF = 128;      // rows of B per CTA
+constexpr int S2_STAGES = 6;
+constexpr int S2_A_STAGE = S2_BM * BK;
+constexpr int S2_B_STAGE = S2_BN_HALF * BK;
+constexpr int S2_SMEM = SMEM_ALIGN + S2_STAGES * (S2_A_STAGE + S2_B_STAGE) + EPI_BYTES + 256;
+
+static_assert(S1_SMEM <= 232448 && S2_SMEM <= 232448, "shared memory per CTA exceeds 227 KB");
 
 enum Site : int32_t {
     SITE_PRODUCER_EMPTY = 1,
@@ -75,6 +103,23 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t cta_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(cta_addr), "r"(rank));
+    return r;
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
@@ -85,8 +130,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Arrive on a barrier given by its shared::cluster address (own CTA or peer).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
@@ -134,12 +180,25 @@ __device__ __noinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// TMA tile load into this CTA's shared memory, completion on a barrier of
+// this CTA.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,
                                             int32_t x, int32_t y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// TMA tile load into this CTA's shared memory whose completion is signalled
+// on a barrier of the pair's first CTA (bar_cluster_addr, shared::cluster).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_cluster_addr, void *dst,
+                                                 int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y)
         : "memory");
 }
 
@@ -203,8 +262,34 @@ __device__ __forceinline__ void umma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
+__device__ __forceinline__ void umma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// Commit of the pair's MMAs, arriving on the barrier at this offset in every
+// CTA of `cta_mask`.
+__device__ __forceinline__ void umma_commit_pair_to(uint64_t *bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
                  : "memory");
 }
@@ -224,14 +309,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Bias value for column n (0 when absent or out of range).
-__device__ __forceinline__ float bias_at(const void *bias, int bias_kind, int64_t n, int64_t N) {
-    if (bias_kind == 0 || n >= N) return 0.0f;
-    if (bias_kind == 1) return __ldg(static_cast<const float *>(bias) + n);
-    const uint16_t b = __ldg(static_cast<const uint16_t *>(bias) + n);
-    return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
 struct Params {
     const float *a_scale_inv;
     const float *b_scale_inv;
@@ -242,41 +319,181 @@ struct Params {
     uint32_t idesc;
 };
 
-// OUT_BF16: bf16 output (64 columns per 128-byte staging row), else fp32 (32).
+// Bias value for column n (0 when absent or out of range).
+__device__ __forceinline__ float bias_at(const Params &p, int64_t n) {
+    if (p.bias_kind == 0 || n >= p.N) return 0.0f;
+    if (p.bias_kind == 1) return __ldg(static_cast<const float *>(p.bias) + n);
+    const uint16_t b = __ldg(static_cast<const uint16_t *>(p.bias) + n);
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// Tile order: groups of GROUP_M row-tiles; inside a group the row index runs
+// fastest, so CTAs that run together share B columns and a band of A rows.
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &m_blk, int &n_blk) {
+    const int group_size = GROUP_M * tiles_n;
+    const int first_m = (tile / group_size) * GROUP_M;
+    const int rows = min(tiles_m - first_m, GROUP_M);
+    const int in_group = tile % group_size;
+    m_blk = first_m + in_group % rows;
+    n_blk = in_group / rows;
+}
+
+// Epilogue of one accumulator for one warp: 32 rows (this warp's TMEM lane
+// quarter) x 256 columns.  t_row addresses the warp's lanes at the
+// accumulator's first column; m_row0 is the global row of the warp's first
+// row.  After the last TMEM read the warp arrives (lane 0) on the
+// accumulator-empty barrier given by its shared::cluster address.
+template <bool OUT_BF16>
+__device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *bufs, int &buf,
+                                              const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
+                                              float sab, const Params &p, uint32_t empty_bar_cluster) {
+    constexpr int COLS_PER_BOX = OUT_BF16 ? 64 : 32;
+    constexpr int BOXES = ACC_N / COLS_PER_BOX;
+    for (int bx = 0; bx < BOXES; ++bx) {
+        uint32_t packed[32];
+        if (OUT_BF16) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(t_row + bx * 64, r0);
+            tmem_ld32(t_row + bx * 64 + 32, r1);
+            tmem_ld_wait();
+            if (bx == BOXES - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int64_t n = n_base + bx * 64 + 2 * j;
+                const float v0 = fmaf(__uint_as_float(r0[2 * j]), sab, bias_at(p, n));
+                const float v1 = fmaf(__uint_as_float(r0[2 * j + 1]), sab, bias_at(p, n + 1));
+                __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+                packed[j] = *reinterpret_cast<uint32_t *>(&h);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int64_t n = n_base + bx * 64 + 32 + 2 * j;
+                const float v0 = fmaf(__uint_as_float(r1[2 * j]), sab, bias_at(p, n));
+                const float v1 = fmaf(__uint_as_float(r1[2 * j + 1]), sab, bias_at(p, n + 1));
+                __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
+                packed[16 + j] = *reinterpret_cast<uint32_t *>(&h);
+            }
+        } else {
+            uint32_t r0[32];
+            tmem_ld32(t_row + bx * 32, r0);
+            tmem_ld_wait();
+            if (bx == BOXES - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int64_t n = n_base + bx * 32 + j;
+                packed[j] = __float_as_uint(fmaf(__uint_as_float(r0[j]), sab, bias_at(p, n)));
+            }
+        }
+        // Staging buffer reuse: the store issued from it two boxes ago must
+        // have finished reading shared memory.
+        if (lane == 0) tma_store_wait_read<EPI_BUFS - 1>();
+        __syncwarp();
+        uint8_t *box = bufs + buf * EPI_BOX_BYTES;
+        // Row `lane`, 16-byte chunk c goes to chunk c ^ (lane & 7) (the
+        // 128-byte swizzle the output tensor map expects).
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int pc = c ^ (lane & 7);
+            *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
+                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + bx * COLS_PER_BOX), m_row0);
+            tma_store_commit();
+        }
+        buf ^= 1;
+    }
+}
+
+// Shared-memory carve-up common to both kernels.
+struct Smem {
+    uint8_t *a, *b, *epi;
+    uint64_t *full, *empty, *tfull, *tempty, *drain;
+    uint32_t *tmem_slot;
+    volatile int *abort_flag;
+};
+
+template <int STAGES, int A_STAGE, int B_STAGE>
+__device__ __forceinline__ Smem carve(uint8_t *raw) {
+    Smem s;
+    uint8_t *base = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(raw) + SMEM_ALIGN - 1) & ~static_cast<uintptr_t>(SMEM_ALIGN - 1));
+    s.a = base;
+    s.b = s.a + STAGES * A_STAGE;
+    s.epi = s.b + STAGES * B_STAGE;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(s.epi + EPI_BYTES);
+    s.full = bars;
+    s.empty = bars + STAGES;
+    s.tfull = bars + 2 * STAGES;
+    s.tempty = bars + 2 * STAGES + 2;
+    s.drain = bars + 2 * STAGES + 4;
+    s.tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    s.abort_flag = reinterpret_cast<volatile int *>(s.tmem_slot + 1);
+    return s;
+}
+
+// Epilogue loop shared by both kernels.  rows_per_tile is the M extent of a
+// tile (128 for the 1-SM kernel, 256 for a pair) and row_offset this CTA's
+// first row inside it.
+template <bool OUT_BF16>
+__device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap *tmap_d, const Params &p,
+                                              uint32_t tmem_base, int warp, int lane, int first_tile,
+                                              int tile_stride, int rows_per_tile, int row_offset,
+                                              uint32_t tempty_rank) {
+    const int num_tiles = p.tiles_m * p.tiles_n;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint8_t *bufs = sm.epi + (warp - EPI_WARP0) * EPI_BUFS * EPI_BOX_BYTES;
+    const float sab = __fmul_rn(__ldg(p.a_scale_inv), __ldg(p.b_scale_inv));
+    int local = 0, buf = 0;
+    for (int tile = first_tile; tile < num_tiles; tile += tile_stride, ++local) {
+        int m_blk, n_blk;
+        tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
+        const int acc = local & 1;
+        const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+        if (!mbar_wait(&sm.tfull[acc], acc_phase, sm.abort_flag, SITE_EPI_TMEM_FULL)) break;
+        tc_fence_after();
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_N);
+        const uint32_t empty_addr = map_to_cta(smem_u32(&sm.tempty[acc]), tempty_rank);
+        epilogue_tile<OUT_BF16>(t_row, lane, bufs, buf, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
+                                m_blk * rows_per_tile + row_offset + q * 32, sab, p, empty_addr);
+    }
+    if (lane == 0) tma_store_wait_all();
+    __syncwarp();
+}
+
+// ------------------------------------------------------------ 1-SM kernel --
+
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(THREADS, 1)
-fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                const __grid_constant__ CUtensorMap tmap_d, const Params p) {
+fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_d, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + SMEM_ALIGN - 1) & ~static_cast<uintptr_t>(SMEM_ALIGN - 1));
-    uint8_t *smem_a = smem;
-    uint8_t *smem_b = smem_a + STAGES * A_STAGE;
-    uint8_t *smem_epi = smem_b + STAGES * B_STAGE;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_epi + 4 * EPI_BUFS * EPI_BOX_BYTES);
-    uint64_t *full_bar = bars;                   // [STAGES]
-    uint64_t *empty_bar = bars + STAGES;         // [STAGES]
-    uint64_t *tfull_bar = bars + 2 * STAGES;     // [2]
-    uint64_t *tempty_bar = bars + 2 * STAGES + 2;  // [2]
-    uint64_t *drain_bar = bars + 2 * STAGES + 4;   // [1]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-
+    const Smem sm = carve<S1_STAGES, S1_A_STAGE, S1_B_STAGE>(smem_raw);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int num_tiles = p.tiles_m * p.tiles_n;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], 1);
+        for (int s = 0; s < S1_STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], 4);
+            mbar_init(&sm.tfull[b], 1);
+            mbar_init(&sm.tempty[b], 4);
         }
-        mbar_init(drain_bar, 1);
-        *abort_flag = 0;
+        mbar_init(sm.drain, 1);
+        *sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         fence_async_smem();
         prefetch_tmap(&tmap_a);
@@ -285,7 +502,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(tmem_slot)),
+                         smem_u32(sm.tmem_slot)),
                      "r"(TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -293,28 +510,27 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    const uint32_t tmem_base = *sm.tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------ producer --
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int64_t issued = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int m_blk = tile % p.tiles_m;
-                const int n_blk = tile / p.tiles_m;
+                int m_blk, n_blk;
+                tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, SITE_PRODUCER_EMPTY)) {
+                    if (!mbar_wait(&sm.empty[stage], phase ^ 1u, sm.abort_flag, SITE_PRODUCER_EMPTY)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full_bar[stage], A_STAGE + B_STAGE);
-                    tma_load_2d(&tmap_a, &full_bar[stage], smem_a + stage * A_STAGE, kb * BK, m_blk * BM);
-                    tma_load_2d(&tmap_b, &full_bar[stage], smem_b + stage * B_STAGE, kb * BK, n_blk * BN);
+                    mbar_arrive_expect_tx(&sm.full[stage], S1_A_STAGE + S1_B_STAGE);
+                    tma_load_2d(&tmap_a, &sm.full[stage], sm.a + stage * S1_A_STAGE, kb * BK, m_blk * S1_BM);
+                    tma_load_2d(&tmap_b, &sm.full[stage], sm.b + stage * S1_B_STAGE, kb * BK, n_blk * ACC_N);
                     ++issued;
-                    if (++stage == STAGES) {
+                    if (++stage == S1_STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -322,15 +538,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
             }
             if (!ok) {
                 // Let every load already issued land before the CTA can exit.
-                for (int s = 0; s < STAGES; ++s) {
-                    const int64_t n_s = issued > s ? (issued - s + STAGES - 1) / STAGES : 0;
-                    if (n_s > 0) mbar_wait_drain(&full_bar[s], static_cast<uint32_t>((n_s - 1) & 1));
+                for (int s = 0; s < S1_STAGES; ++s) {
+                    const int64_t n_s = issued > s ? (issued - s + S1_STAGES - 1) / S1_STAGES : 0;
+                    if (n_s > 0) mbar_wait_drain(&sm.full[s], static_cast<uint32_t>((n_s - 1) & 1));
                 }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ----------------------------------------------------- MMA issuer --
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
@@ -339,125 +554,41 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
                 const int acc = local & 1;
                 const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
-                if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, SITE_MMA_TMEM_EMPTY)) {
+                if (!mbar_wait(&sm.tempty[acc], acc_phase ^ 1u, sm.abort_flag, SITE_MMA_TMEM_EMPTY)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_N);
                 for (int kb = 0; kb < p.num_kb; ++kb) {
-                    if (!mbar_wait(&full_bar[stage], phase, abort_flag, SITE_MMA_FULL)) {
+                    if (!mbar_wait(&sm.full[stage], phase, sm.abort_flag, SITE_MMA_FULL)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t a_desc = sw128_kmajor_desc(smem_u32(smem_a + stage * A_STAGE));
-                    const uint64_t b_desc = sw128_kmajor_desc(smem_u32(smem_b + stage * B_STAGE));
+                    const uint64_t a_desc = sw128_kmajor_desc(smem_u32(sm.a + stage * S1_A_STAGE));
+                    const uint64_t b_desc = sw128_kmajor_desc(smem_u32(sm.b + stage * S1_B_STAGE));
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // advance the start address by k * 32 bytes inside the swizzle row
                         const uint64_t adv = static_cast<uint64_t>((k * UMMA_K) >> 4);
                         umma_f8f6f4(d_tmem, a_desc + adv, b_desc + adv, p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
                     }
-                    umma_commit(&empty_bar[stage]);
-                    if (++stage == STAGES) {
+                    umma_commit(&sm.empty[stage]);
+                    if (++stage == S1_STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (ok) umma_commit(&tfull_bar[acc]);
+                if (ok) umma_commit(&sm.tfull[acc]);
             }
-            // Make sure every MMA issued has finished before TMEM can be freed.
-            umma_commit(drain_bar);
-            mbar_wait_drain(drain_bar, 0);
+            // Every MMA issued must have finished before TMEM can be freed.
+            umma_commit(sm.drain);
+            mbar_wait_drain(sm.drain, 0);
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------- epilogue --
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
-        const int row0 = q * 32;
-        uint8_t *bufs = smem_epi + (warp - EPI_WARP0) * EPI_BUFS * EPI_BOX_BYTES;
-        const float sab = __fmul_rn(__ldg(p.a_scale_inv), __ldg(p.b_scale_inv));
-        constexpr int COLS_PER_BOX = OUT_BF16 ? 64 : 32;
-        constexpr int BOXES = BN / COLS_PER_BOX;
-        int local = 0;
-        int buf = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
-            const int m_blk = tile % p.tiles_m;
-            const int n_blk = tile / p.tiles_m;
-            const int acc = local & 1;
-            const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
-            if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag, SITE_EPI_TMEM_FULL)) break;
-            tc_fence_after();
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(row0) << 16) + static_cast<uint32_t>(acc * BN);
-            const int64_t n_base = static_cast<int64_t>(n_blk) * BN;
-            for (int bx = 0; bx < BOXES; ++bx) {
-                uint32_t packed[32];
-                if (OUT_BF16) {
-                    uint32_t r0[32], r1[32];
-                    tmem_ld32(t_row + bx * 64, r0);
-                    tmem_ld32(t_row + bx * 64 + 32, r1);
-                    tmem_ld_wait();
-                    if (bx == BOXES - 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int64_t n = n_base + bx * 64 + 2 * j;
-                        const float v0 = fmaf(__uint_as_float(r0[2 * j]), sab, bias_at(p.bias, p.bias_kind, n, p.N));
-                        const float v1 = fmaf(__uint_as_float(r0[2 * j + 1]), sab, bias_at(p.bias, p.bias_kind, n + 1, p.N));
-                        __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-                        packed[j] = *reinterpret_cast<uint32_t *>(&h);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int64_t n = n_base + bx * 64 + 32 + 2 * j;
-                        const float v0 = fmaf(__uint_as_float(r1[2 * j]), sab, bias_at(p.bias, p.bias_kind, n, p.N));
-                        const float v1 = fmaf(__uint_as_float(r1[2 * j + 1]), sab, bias_at(p.bias, p.bias_kind, n + 1, p.N));
-                        __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-                        packed[16 + j] = *reinterpret_cast<uint32_t *>(&h);
-                    }
-                } else {
-                    uint32_t r0[32];
-                    tmem_ld32(t_row + bx * 32, r0);
-                    tmem_ld_wait();
-                    if (bx == BOXES - 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int64_t n = n_base + bx * 32 + j;
-                        packed[j] = __float_as_uint(fmaf(__uint_as_float(r0[j]), sab, bias_at(p.bias, p.bias_kind, n, p.N)));
-                    }
-                }
-                // Staging buffer reuse: the store issued from it two boxes ago
-                // must have finished reading shared memory.
-                if (lane == 0) tma_store_wait_read<EPI_BUFS - 1>();
-                __syncwarp();
-                uint8_t *box = bufs + buf * EPI_BOX_BYTES;
-                // Row `lane`, 16-byte chunk c goes to chunk c ^ (lane & 7).
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int pc = c ^ (lane & 7);
-                    *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
-                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmap_d, box, static_cast<int32_t>(n_base + bx * COLS_PER_BOX),
-                                 m_blk * BM + row0);
-                    tma_store_commit();
-                }
-                buf ^= 1;
-            }
-        }
-        if (lane == 0) tma_store_wait_all();
-        __syncwarp();
+        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, S1_BM, 0, 0u);
     }
 
     tc_fence_before();
@@ -465,6 +596,149 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constan
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------ 2-SM kernel --
+
+// Launched with clusters of 2 CTAs (gridDim.x even).  Cluster c handles pair
+// tiles c, c + clusters, ...; CTA rank r of the pair owns rows r*128..r*128+127
+// of each 256-row pair tile and loads rows r*128.. of the tile's 256 B rows.
+template <bool OUT_BF16>
+__global__ void __launch_bounds__(THREADS, 1)
+fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                    const __grid_constant__ CUtensorMap tmap_d, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    const Smem sm = carve<S2_STAGES, S2_A_STAGE, S2_B_STAGE>(smem_raw);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+    const int cluster_id = blockIdx.x >> 1;
+    const int num_clusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S2_STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.tfull[b], 1);
+            mbar_init(&sm.tempty[b], 8);  // 4 epilogue warps x 2 CTAs (the first CTA's is used)
+        }
+        mbar_init(sm.drain, 1);
+        *sm.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_async_smem();
+        prefetch_tmap(&tmap_a);
+        prefetch_tmap(&tmap_b);
+        prefetch_tmap(&tmap_d);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(sm.tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *sm.tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int64_t issued = 0;
+            bool ok = true;
+            for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+                int m_blk, n_blk;
+                tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
+                const int32_t a_row = m_blk * 2 * S2_BM + static_cast<int32_t>(rank) * S2_BM;
+                const int32_t b_row = n_blk * ACC_N + static_cast<int32_t>(rank) * S2_BN_HALF;
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(&sm.empty[stage], phase ^ 1u, sm.abort_flag, SITE_PRODUCER_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    // The pair's MMA waits on the first CTA's barrier for the
+                    // bytes of both CTAs.
+                    if (leader) mbar_arrive_expect_tx(&sm.full[stage], 2 * (S2_A_STAGE + S2_B_STAGE));
+                    const uint32_t full_leader = map_to_cta(smem_u32(&sm.full[stage]), 0u);
+                    tma_load_2d_pair(&tmap_a, full_leader, sm.a + stage * S2_A_STAGE, kb * BK, a_row);
+                    tma_load_2d_pair(&tmap_b, full_leader, sm.b + stage * S2_B_STAGE, kb * BK, b_row);
+                    ++issued;
+                    if (++stage == S2_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok && leader) {
+                for (int s = 0; s < S2_STAGES; ++s) {
+                    const int64_t n_s = issued > s ? (issued - s + S2_STAGES - 1) / S2_STAGES : 0;
+                    if (n_s > 0) mbar_wait_drain(&sm.full[s], static_cast<uint32_t>((n_s - 1) & 1));
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            int local = 0;
+            for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++local) {
+                const int acc = local & 1;
+                const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+                if (!mbar_wait(&sm.tempty[acc], acc_phase ^ 1u, sm.abort_flag, SITE_MMA_TMEM_EMPTY)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_N);
+                for (int kb = 0; kb < p.num_kb; ++kb) {
+                    if (!mbar_wait(&sm.full[stage], phase, sm.abort_flag, SITE_MMA_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t a_desc = sw128_kmajor_desc(smem_u32(sm.a + stage * S2_A_STAGE));
+                    const uint64_t b_desc = sw128_kmajor_desc(smem_u32(sm.b + stage * S2_B_STAGE));
+#pragma unroll
+                    for (int k = 0; k < BK / UMMA_K; ++k) {
+                        const uint64_t adv = static_cast<uint64_t>((k * UMMA_K) >> 4);
+                        umma_f8f6f4_pair(d_tmem, a_desc + adv, b_desc + adv, p.idesc,
+                                         (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit_pair_to(&sm.empty[stage], 0x3);
+                    if (++stage == S2_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) umma_commit_pair_to(&sm.tfull[acc], 0x3);
+            }
+            umma_commit_pair(sm.drain);
+            mbar_wait_drain(sm.drain, 0);
+        }
+        __syncwarp();
+    } else {
+        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, 2 * S2_BM,
+                                static_cast<int>(rank) * S2_BM, 0u);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // The peer's MMAs, loads and barrier arrivals target this CTA's memory
+    // until both CTAs are here.
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
                      : "memory");
     }
 }
@@ -504,26 +778,87 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint6
 // Instruction descriptor of tcgen05.mma.kind::f8f6f4 (dense, K-major A and B):
 // [4,6) D format (1 = fp32), [7,10) A format, [10,13) B format (0 = E4M3,
 // 1 = E5M2), [15] / [16] A / B major (0 = K), [17,23) N >> 3, [24,29) M >> 4.
-uint32_t make_idesc(fp8ds_format fa, fp8ds_format fb) {
+uint32_t make_idesc(fp8ds_format fa, fp8ds_format fb, int m, int n) {
     uint32_t d = 0;
     d |= 1u << 4;
     d |= static_cast<uint32_t>(fa == FP8DS_E5M2 ? 1 : 0) << 7;
     d |= static_cast<uint32_t>(fb == FP8DS_E5M2 ? 1 : 0) << 10;
-    d |= static_cast<uint32_t>(BN >> 3) << 17;
-    d |= static_cast<uint32_t>(BM >> 4) << 24;
+    d |= static_cast<uint32_t>(n >> 3) << 17;
+    d |= static_cast<uint32_t>(m >> 4) << 24;
     return d;
 }
 
-template <bool OUT_BF16>
-cudaError_t configure_once() {
-    static bool done[64] = {};
+template <typename K>
+cudaError_t set_smem_once(K kernel, int bytes, bool (&done)[64]) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-    e = cudaFuncSetAttribute(fp8_gemm_kernel<OUT_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
     return e;
+}
+
+// Number of CTA pairs of the 2-SM kernel that fit on the device at once.
+template <typename K>
+int max_pairs(K kernel) {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms() / 2;
+    if (cached[dev] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+        cfg.blockDim = dim3(THREADS, 1, 1);
+        cfg.dynamicSmemBytes = S2_SMEM;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) n = num_sms() / 2;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+template <bool OUT_BF16>
+cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
+                       cudaStream_t stream) {
+    static bool done[64] = {};
+    auto kernel = fp8_gemm_2sm_kernel<OUT_BF16>;
+    cudaError_t e = set_smem_once(kernel, S2_SMEM, done);
+    if (e != cudaSuccess) return e;
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int pairs = tiles < max_pairs(kernel) ? tiles : max_pairs(kernel);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = S2_SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, ta, tb, td, p);
+}
+
+template <bool OUT_BF16>
+cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
+                       cudaStream_t stream) {
+    static bool done[64] = {};
+    auto kernel = fp8_gemm_1sm_kernel<OUT_BF16>;
+    cudaError_t e = set_smem_once(kernel, S1_SMEM, done);
+    if (e != cudaSuccess) return e;
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    kernel<<<grid, THREADS, S1_SMEM, stream>>>(ta, tb, td, p);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -531,10 +866,11 @@ cudaError_t configure_once() {
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
                          fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
                          void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, cudaStream_t stream) {
-    CUtensorMap ta, tb, td;
     const bool out_bf16 = d_dtype == FP8DS_BF16;
-    bool ok = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, k, m, k, BK, BM) &&
-              encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, k, n, k, BK, BN) &&
+    const bool pair = m > S1_BM;
+    CUtensorMap ta, tb, td;
+    bool ok = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, k, m, k, BK, pair ? S2_BM : S1_BM) &&
+              encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, k, n, k, BK, pair ? S2_BN_HALF : ACC_N) &&
               (out_bf16 ? encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, n, m, n * 2, 64, 32)
                         : encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d, n, m, n * 4, 32, 32));
     if (!ok) {
@@ -550,20 +886,16 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.M = static_cast<int32_t>(m);
     p.N = static_cast<int32_t>(n);
     p.K = static_cast<int32_t>(k);
-    p.tiles_m = static_cast<int32_t>((m + BM - 1) / BM);
-    p.tiles_n = static_cast<int32_t>((n + BN - 1) / BN);
+    const int tile_m = pair ? 2 * S2_BM : S1_BM;
+    p.tiles_m = static_cast<int32_t>((m + tile_m - 1) / tile_m);
+    p.tiles_n = static_cast<int32_t>((n + ACC_N - 1) / ACC_N);
     p.num_kb = static_cast<int32_t>((k + BK - 1) / BK);
-    p.idesc = make_idesc(a_fmt, b_fmt);
-    const int tiles = p.tiles_m * p.tiles_n;
-    const int grid = tiles < num_sms() ? tiles : num_sms();
-    cudaError_t e = out_bf16 ? configure_once<true>() : configure_once<false>();
-    if (e == cudaSuccess) {
-        if (out_bf16)
-            fp8_gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, td, p);
-        else
-            fp8_gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, td, p);
-        e = cudaGetLastError();
-    }
+    p.idesc = make_idesc(a_fmt, b_fmt, tile_m, ACC_N);
+    cudaError_t e;
+    if (pair)
+        e = out_bf16 ? launch_2sm<true>(ta, tb, td, p, stream) : launch_2sm<false>(ta, tb, td, p, stream);
+    else
+        e = out_bf16 ? launch_1sm<true>(ta, tb, td, p, stream) : launch_1sm<false>(ta, tb, td, p, stream);
     if (e != cudaSuccess) {
         set_error("fp8_gemm: launch failed: %s", cudaGetErrorString(e));
         return FP8DS_ERR_CUDA;

@@ -82,8 +82,12 @@ def _compare(d, ref, rows, out_dtype, what, ops):
     return check_gemm_bf16(host_bits(got), ref, what, absdot=absdot, K=a.shape[1])
 
 
+# M <= 128 runs the 1-SM kernel, larger M the CTA-pair kernel (pair tile
+# 256 x 256): ragged M inside a pair, a second CTA with one row, B rows of the
+# second CTA entirely out of range (N <= 128), more tiles than SM pairs.
 SHAPES = [(128, 256, 128), (128, 512, 256), (300, 520, 272), (1, 8, 16), (129, 264, 144),
-          (256, 256, 1024), (4096, 2048, 256), (2048, 8192, 1024)]
+          (256, 256, 1024), (4096, 8, 256), (1000, 136, 528), (4096, 2048, 256),
+          (2048, 8192, 1024)]
 
 
 @pytest.mark.parametrize("shape", SHAPES)
