@@ -158,11 +158,13 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
     if (blockIdx.x == 0 && tid == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
 
     // Vector path: thread = (column chunk cc of 8, row group rg of 4 rows).
-    // The next tile's loads are issued before the current tile is processed,
-    // so they stay in flight across its shared-memory transpose and barriers.
+    // Two register buffers alternate between consecutive tiles of this CTA:
+    // the loads of tile i+1 are issued before tile i is processed, so they
+    // stay in flight across its shared-memory transpose and barriers (the
+    // loop is unrolled by two so that no register copy waits on them).
     const int cc = tid & 7, rg = tid >> 3;
     using Raw = decltype(Load8<T, FMT>::raw(x));
-    Raw cur[4], nxt[4];
+    Raw buf0[4], buf1[4];
     auto tile_full = [&](int64_t tile) {
         if (!VEC || tile >= num_tiles) return false;  // (tiles_c > 0 whenever num_tiles > 0)
         const int64_t r0 = (tile / tiles_c) * CT_ROWS, c0 = (tile % tiles_c) * CT_COLS;
@@ -174,19 +176,15 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
 #pragma unroll
         for (int i = 0; i < 4; ++i) dst[i] = Load8<T, FMT>::raw(xp + i * cols);
     };
-    bool cur_full = tile_full(blockIdx.x);
-    if (cur_full) load_tile(blockIdx.x, cur);
-
-    for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    // Cast, store y, transpose through shared memory and store yt for one
+    // tile whose input is in `src` (vector path) or in global memory.
+    auto process = [&](int64_t tile, bool full, const Raw(&src)[4]) {
         const int64_t r0 = (tile / tiles_c) * CT_ROWS;
         const int64_t c0 = (tile % tiles_c) * CT_COLS;
-        const int64_t next = tile + gridDim.x;
-        const bool next_full = tile_full(next);
-        if (next_full) load_tile(next, nxt);
-        if (cur_full) {
+        if (full) {
             uint2 w[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = Load8<T, FMT>::cast(cur[i], s, m);
+            for (int i = 0; i < 4; ++i) w[i] = Load8<T, FMT>::cast(src[i], s, m);
             uint8_t *yp = y + (r0 + 4 * rg) * cols + c0 + 8 * cc;
 #pragma unroll
             for (int i = 0; i < 4; ++i) *reinterpret_cast<uint2 *>(yp + i * cols) = w[i];
@@ -214,8 +212,8 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
                 for (int k = 0; k < 2; ++k) {
                     const int idx = tid + CT_THREADS * k;
                     const int c = idx >> 3, q = idx & 7;
-                    const uint32_t *src = tsm + c * CT_TSTRIDE + 4 * q;
-                    uint4 v = make_uint4(src[0], src[1], src[2], src[3]);
+                    const uint32_t *tp = tsm + c * CT_TSTRIDE + 4 * q;
+                    uint4 v = make_uint4(tp[0], tp[1], tp[2], tp[3]);
                     *reinterpret_cast<uint4 *>(yt + (c0 + c) * rows + r0 + 16 * q) = v;
                 }
                 __syncthreads();
@@ -246,11 +244,23 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
                 __syncthreads();
             }
         }
-        if (next_full) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) cur[i] = nxt[i];
-        }
-        cur_full = next_full;
+    };
+
+    const int64_t stride = gridDim.x;
+    int64_t tile = blockIdx.x;
+    bool full0 = tile_full(tile);
+    if (full0) load_tile(tile, buf0);
+    while (tile < num_tiles) {
+        const int64_t t1 = tile + stride;
+        const bool full1 = tile_full(t1);
+        if (full1) load_tile(t1, buf1);
+        process(tile, full0, buf0);
+        if (t1 >= num_tiles) break;
+        const int64_t t2 = t1 + stride;
+        full0 = tile_full(t2);
+        if (full0) load_tile(t2, buf0);
+        process(t1, full1, buf1);
+        tile = t2;
     }
     block_amax_commit<CT_THREADS>(m, amax);
 }

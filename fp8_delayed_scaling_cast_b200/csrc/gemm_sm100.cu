@@ -60,7 +60,8 @@ constexpr int EPI_WARP0 = 2;
 constexpr int TMEM_COLS = 512; // two accumulators
 constexpr int EPI_BOX_BYTES = 32 * 128;  // staging box: 32 rows x 128 bytes
 constexpr int EPI_BUFS = 2;
-constexpr int EPI_BYTES = 4 * EPI_BUFS * EPI_BOX_BYTES;
+constexpr int EPI_BYTES = 4 * EPI_BUFS * EPI_BOX_BYTES + 256 * 4;  // + the tile's bias (fp32 x 256)
+constexpr int EPI_THREADS = 128;
 constexpr int SMEM_ALIGN = 1024;
 constexpr int GROUP_M = 8;
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;  // 2 s
@@ -73,16 +74,24 @@ constexpr int S1_A_STAGE = S1_BM * BK;
 constexpr int S1_B_STAGE = ACC_N * BK;
 constexpr int S1_SMEM = SMEM_ALIGN + S1_STAGES * (S1_A_STAGE + S1_B_STAGE) + EPI_BYTES + 256;
 
-// 2-SM kernel: pair tile 256 x 256; per CTA 128 rows of A and 128 rows of B
-// per stage (16 KB + 16 KB), 6 stages.
-constexpr int S2_BM = 128;           // rows of A (and of D) per CTA
+// 2-SM kernel: pair tile (M_SUB x 256) x 256.  Per CTA and stage: M_SUB
+// boxes of 128 rows of A and 128 rows of B.  M_SUB = 1: 6 stages of 32 KB,
+// two accumulators (double-buffered).  M_SUB = 2: 4 stages of 48 KB, the two
+// M halves fill all 512 TMEM columns (one accumulator set, not overlapped
+// with the epilogue) in exchange for 25% fewer loaded bytes per FLOP.
+constexpr int S2_BM = 128;           // rows of A (and of D) per CTA and M half
 constexpr int S2_BN_HALF = 128;      // rows of B per CTA
-constexpr int S2_STAGES = 6;
-constexpr int S2_A_STAGE = S2_BM * BK;
 constexpr int S2_B_STAGE = S2_BN_HALF * BK;
-constexpr int S2_SMEM = SMEM_ALIGN + S2_STAGES * (S2_A_STAGE + S2_B_STAGE) + EPI_BYTES + 256;
+template <int M_SUB>
+struct Pair {
+    static constexpr int STAGES = M_SUB == 1 ? 6 : 4;
+    static constexpr int A_STAGE = M_SUB * S2_BM * BK;
+    static constexpr int ACC_BUFS = M_SUB == 1 ? 2 : 1;
+    static constexpr int SMEM = SMEM_ALIGN + STAGES * (A_STAGE + S2_B_STAGE) + EPI_BYTES + 256;
+};
 
-static_assert(S1_SMEM <= 232448 && S2_SMEM <= 232448, "shared memory per CTA exceeds 227 KB");
+static_assert(S1_SMEM <= 232448 && Pair<1>::SMEM <= 232448 && Pair<2>::SMEM <= 232448,
+              "shared memory per CTA exceeds 227 KB");
 
 enum Site : int32_t {
     SITE_PRODUCER_EMPTY = 1,
@@ -319,12 +328,43 @@ struct Params {
     uint32_t idesc;
 };
 
-// Bias value for column n (0 when absent or out of range).
-__device__ __forceinline__ float bias_at(const Params &p, int64_t n) {
-    if (p.bias_kind == 0 || n >= p.N) return 0.0f;
-    if (p.bias_kind == 1) return __ldg(static_cast<const float *>(p.bias) + n);
-    const uint16_t b = __ldg(static_cast<const uint16_t *>(p.bias) + n);
-    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+// Named barrier among the 4 epilogue warps.
+__device__ __forceinline__ void epilogue_bar() { asm volatile("bar.sync 1, %0;" ::"n"(EPI_THREADS) : "memory"); }
+
+// Named barrier among the 4 epilogue warps that also returns whether any of
+// their threads passed `v` true (so that all of them leave the loop together).
+__device__ __forceinline__ bool epilogue_any(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(v)), "n"(EPI_THREADS)
+        : "memory");
+    return r != 0;
+}
+
+// Stage bias[n_base .. n_base+255] (0 when absent or past N) as fp32 in
+// shared memory; called by all epilogue threads between epilogue_any() and
+// epilogue_bar().
+__device__ __forceinline__ void stage_bias(float *bias_s, const Params &p, int64_t n_base, int epi_tid) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int c = 2 * epi_tid + i;
+        const int64_t n = n_base + c;
+        float v = 0.0f;
+        if (p.bias_kind != 0 && n < p.N) {
+            if (p.bias_kind == 1) {
+                v = __ldg(static_cast<const float *>(p.bias) + n);
+            } else {
+                const uint16_t b = __ldg(static_cast<const uint16_t *>(p.bias) + n);
+                v = __uint_as_float(static_cast<uint32_t>(b) << 16);
+            }
+        }
+        bias_s[c] = v;
+    }
 }
 
 // Tile order: groups of GROUP_M row-tiles; inside a group the row index runs
@@ -346,7 +386,8 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
 template <bool OUT_BF16>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *bufs, int &buf,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
-                                              float sab, const Params &p, uint32_t empty_bar_cluster) {
+                                              float sab, const float *bias_s, uint32_t empty_bar_cluster,
+                                              bool arrive) {
     constexpr int COLS_PER_BOX = OUT_BF16 ? 64 : 32;
     constexpr int BOXES = ACC_N / COLS_PER_BOX;
     for (int bx = 0; bx < BOXES; ++bx) {
@@ -356,24 +397,25 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             tmem_ld32(t_row + bx * 64, r0);
             tmem_ld32(t_row + bx * 64 + 32, r1);
             tmem_ld_wait();
-            if (bx == BOXES - 1) {
+            if (arrive && bx == BOXES - 1) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
             }
+            const float2 *bs = reinterpret_cast<const float2 *>(bias_s + bx * 64);
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const int64_t n = n_base + bx * 64 + 2 * j;
-                const float v0 = fmaf(__uint_as_float(r0[2 * j]), sab, bias_at(p, n));
-                const float v1 = fmaf(__uint_as_float(r0[2 * j + 1]), sab, bias_at(p, n + 1));
+                const float2 b = bs[j];
+                const float v0 = fmaf(__uint_as_float(r0[2 * j]), sab, b.x);
+                const float v1 = fmaf(__uint_as_float(r0[2 * j + 1]), sab, b.y);
                 __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
                 packed[j] = *reinterpret_cast<uint32_t *>(&h);
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const int64_t n = n_base + bx * 64 + 32 + 2 * j;
-                const float v0 = fmaf(__uint_as_float(r1[2 * j]), sab, bias_at(p, n));
-                const float v1 = fmaf(__uint_as_float(r1[2 * j + 1]), sab, bias_at(p, n + 1));
+                const float2 b = bs[16 + j];
+                const float v0 = fmaf(__uint_as_float(r1[2 * j]), sab, b.x);
+                const float v1 = fmaf(__uint_as_float(r1[2 * j + 1]), sab, b.y);
                 __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
                 packed[16 + j] = *reinterpret_cast<uint32_t *>(&h);
             }
@@ -381,16 +423,14 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             uint32_t r0[32];
             tmem_ld32(t_row + bx * 32, r0);
             tmem_ld_wait();
-            if (bx == BOXES - 1) {
+            if (arrive && bx == BOXES - 1) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
             }
+            const float *bs = bias_s + bx * 32;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int64_t n = n_base + bx * 32 + j;
-                packed[j] = __float_as_uint(fmaf(__uint_as_float(r0[j]), sab, bias_at(p, n)));
-            }
+            for (int j = 0; j < 32; ++j) packed[j] = __float_as_uint(fmaf(__uint_as_float(r0[j]), sab, bs[j]));
         }
         // Staging buffer reuse: the store issued from it two boxes ago must
         // have finished reading shared memory.
@@ -442,30 +482,42 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     return s;
 }
 
-// Epilogue loop shared by both kernels.  rows_per_tile is the M extent of a
-// tile (128 for the 1-SM kernel, 256 for a pair) and row_offset this CTA's
-// first row inside it.
+// Epilogue loop shared by both kernels.  A tile spans m_sub row blocks of
+// rows_per_sub rows (row block h of the tile starts at row h * rows_per_sub,
+// and this CTA's rows at row_offset inside it); row block h sits at TMEM
+// column h * 256 of the accumulator.  acc_bufs accumulators alternate.
 template <bool OUT_BF16>
 __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap *tmap_d, const Params &p,
                                               uint32_t tmem_base, int warp, int lane, int first_tile,
-                                              int tile_stride, int rows_per_tile, int row_offset,
-                                              uint32_t tempty_rank) {
+                                              int tile_stride, int m_sub, int rows_per_sub, int row_offset,
+                                              int acc_bufs, uint32_t tempty_rank) {
     const int num_tiles = p.tiles_m * p.tiles_n;
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     uint8_t *bufs = sm.epi + (warp - EPI_WARP0) * EPI_BUFS * EPI_BOX_BYTES;
+    float *bias_s = reinterpret_cast<float *>(sm.epi + 4 * EPI_BUFS * EPI_BOX_BYTES);
+    const int epi_tid = (warp - EPI_WARP0) * 32 + lane;
     const float sab = __fmul_rn(__ldg(p.a_scale_inv), __ldg(p.b_scale_inv));
     int local = 0, buf = 0;
     for (int tile = first_tile; tile < num_tiles; tile += tile_stride, ++local) {
         int m_blk, n_blk;
         tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
-        const int acc = local & 1;
-        const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
-        if (!mbar_wait(&sm.tfull[acc], acc_phase, sm.abort_flag, SITE_EPI_TMEM_FULL)) break;
+        const int acc = acc_bufs == 2 ? (local & 1) : 0;
+        const uint32_t acc_phase = static_cast<uint32_t>(acc_bufs == 2 ? (local >> 1) : local) & 1u;
+        const bool ok = mbar_wait(&sm.tfull[acc], acc_phase, sm.abort_flag, SITE_EPI_TMEM_FULL);
+        // All epilogue warps meet here every tile: they leave together if any
+        // wait gave up, and none of them still reads the previous tile's bias.
+        if (epilogue_any(!ok)) break;
+        stage_bias(bias_s, p, static_cast<int64_t>(n_blk) * ACC_N, epi_tid);
+        epilogue_bar();
         tc_fence_after();
-        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_N);
         const uint32_t empty_addr = map_to_cta(smem_u32(&sm.tempty[acc]), tempty_rank);
-        epilogue_tile<OUT_BF16>(t_row, lane, bufs, buf, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
-                                m_blk * rows_per_tile + row_offset + q * 32, sab, p, empty_addr);
+        for (int h = 0; h < m_sub; ++h) {
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>((acc + h) * ACC_N);
+            epilogue_tile<OUT_BF16>(t_row, lane, bufs, buf, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
+                                    (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32, sab, bias_s,
+                                    empty_addr, h == m_sub - 1);
+        }
     }
     if (lane == 0) tma_store_wait_all();
     __syncwarp();
@@ -588,7 +640,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         __syncwarp();
     } else {
-        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, S1_BM, 0, 0u);
+        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u);
     }
 
     tc_fence_before();
@@ -603,14 +655,19 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
 // ------------------------------------------------------------ 2-SM kernel --
 
 // Launched with clusters of 2 CTAs (gridDim.x even).  Cluster c handles pair
-// tiles c, c + clusters, ...; CTA rank r of the pair owns rows r*128..r*128+127
-// of each 256-row pair tile and loads rows r*128.. of the tile's 256 B rows.
-template <bool OUT_BF16>
+// tiles c, c + clusters, ...; a pair tile has M_SUB row blocks of 256 rows
+// and 256 columns.  CTA rank r of the pair owns rows r*128..r*128+127 of each
+// row block and loads rows r*128.. of the tile's 256 B rows.
+template <bool OUT_BF16, int M_SUB>
 __global__ void __launch_bounds__(THREADS, 1)
 fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d, const Params p) {
+    using PC = Pair<M_SUB>;
+    constexpr int STAGES = PC::STAGES;
+    constexpr int A_STAGE = PC::A_STAGE;
+    constexpr int ACC_BUFS = PC::ACC_BUFS;
     extern __shared__ uint8_t smem_raw[];
-    const Smem sm = carve<S2_STAGES, S2_A_STAGE, S2_B_STAGE>(smem_raw);
+    const Smem sm = carve<STAGES, A_STAGE, S2_B_STAGE>(smem_raw);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -620,7 +677,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     const int num_clusters = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S2_STAGES; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
@@ -657,7 +714,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
                 int m_blk, n_blk;
                 tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
-                const int32_t a_row = m_blk * 2 * S2_BM + static_cast<int32_t>(rank) * S2_BM;
+                const int32_t a_row = m_blk * M_SUB * 2 * S2_BM + static_cast<int32_t>(rank) * S2_BM;
                 const int32_t b_row = n_blk * ACC_N + static_cast<int32_t>(rank) * S2_BN_HALF;
                 for (int kb = 0; kb < p.num_kb; ++kb) {
                     if (!mbar_wait(&sm.empty[stage], phase ^ 1u, sm.abort_flag, SITE_PRODUCER_EMPTY)) {
@@ -666,20 +723,23 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     }
                     // The pair's MMA waits on the first CTA's barrier for the
                     // bytes of both CTAs.
-                    if (leader) mbar_arrive_expect_tx(&sm.full[stage], 2 * (S2_A_STAGE + S2_B_STAGE));
+                    if (leader) mbar_arrive_expect_tx(&sm.full[stage], 2 * (A_STAGE + S2_B_STAGE));
                     const uint32_t full_leader = map_to_cta(smem_u32(&sm.full[stage]), 0u);
-                    tma_load_2d_pair(&tmap_a, full_leader, sm.a + stage * S2_A_STAGE, kb * BK, a_row);
+#pragma unroll
+                    for (int h = 0; h < M_SUB; ++h)
+                        tma_load_2d_pair(&tmap_a, full_leader, sm.a + stage * A_STAGE + h * S2_BM * BK, kb * BK,
+                                         a_row + h * 2 * S2_BM);
                     tma_load_2d_pair(&tmap_b, full_leader, sm.b + stage * S2_B_STAGE, kb * BK, b_row);
                     ++issued;
-                    if (++stage == S2_STAGES) {
+                    if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             if (!ok && leader) {
-                for (int s = 0; s < S2_STAGES; ++s) {
-                    const int64_t n_s = issued > s ? (issued - s + S2_STAGES - 1) / S2_STAGES : 0;
+                for (int s = 0; s < STAGES; ++s) {
+                    const int64_t n_s = issued > s ? (issued - s + STAGES - 1) / STAGES : 0;
                     if (n_s > 0) mbar_wait_drain(&sm.full[s], static_cast<uint32_t>((n_s - 1) & 1));
                 }
             }
@@ -692,30 +752,33 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             bool ok = true;
             int local = 0;
             for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++local) {
-                const int acc = local & 1;
-                const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+                const int acc = ACC_BUFS == 2 ? (local & 1) : 0;
+                const uint32_t acc_phase = static_cast<uint32_t>(ACC_BUFS == 2 ? (local >> 1) : local) & 1u;
                 if (!mbar_wait(&sm.tempty[acc], acc_phase ^ 1u, sm.abort_flag, SITE_MMA_TMEM_EMPTY)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_N);
                 for (int kb = 0; kb < p.num_kb; ++kb) {
                     if (!mbar_wait(&sm.full[stage], phase, sm.abort_flag, SITE_MMA_FULL)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t a_desc = sw128_kmajor_desc(smem_u32(sm.a + stage * S2_A_STAGE));
                     const uint64_t b_desc = sw128_kmajor_desc(smem_u32(sm.b + stage * S2_B_STAGE));
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         const uint64_t adv = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        umma_f8f6f4_pair(d_tmem, a_desc + adv, b_desc + adv, p.idesc,
-                                         (kb > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                        for (int h = 0; h < M_SUB; ++h) {
+                            const uint64_t a_desc =
+                                sw128_kmajor_desc(smem_u32(sm.a + stage * A_STAGE + h * S2_BM * BK));
+                            umma_f8f6f4_pair(tmem_base + static_cast<uint32_t>((acc + h) * ACC_N), a_desc + adv,
+                                             b_desc + adv, p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        }
                     }
                     umma_commit_pair_to(&sm.empty[stage], 0x3);
-                    if (++stage == S2_STAGES) {
+                    if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -727,8 +790,8 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         __syncwarp();
     } else {
-        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, 2 * S2_BM,
-                                static_cast<int>(rank) * S2_BM, 0u);
+        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, M_SUB,
+                                2 * S2_BM, static_cast<int>(rank) * S2_BM, ACC_BUFS, 0u);
     }
 
     tc_fence_before();
@@ -799,17 +862,16 @@ cudaError_t set_smem_once(K kernel, int bytes, bool (&done)[64]) {
     return e;
 }
 
-// Number of CTA pairs of the 2-SM kernel that fit on the device at once.
+// Number of CTA pairs of a 2-SM kernel that fit on the device at once.
 template <typename K>
-int max_pairs(K kernel) {
-    static int cached[64] = {};
+int max_pairs(K kernel, int smem_bytes, int (&cached)[64]) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms() / 2;
     if (cached[dev] == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
         cfg.blockDim = dim3(THREADS, 1, 1);
-        cfg.dynamicSmemBytes = S2_SMEM;
+        cfg.dynamicSmemBytes = smem_bytes;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -824,19 +886,22 @@ int max_pairs(K kernel) {
     return cached[dev];
 }
 
-template <bool OUT_BF16>
+template <bool OUT_BF16, int M_SUB>
 cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
                        cudaStream_t stream) {
     static bool done[64] = {};
-    auto kernel = fp8_gemm_2sm_kernel<OUT_BF16>;
-    cudaError_t e = set_smem_once(kernel, S2_SMEM, done);
+    static int cached_pairs[64] = {};
+    auto kernel = fp8_gemm_2sm_kernel<OUT_BF16, M_SUB>;
+    constexpr int smem = Pair<M_SUB>::SMEM;
+    cudaError_t e = set_smem_once(kernel, smem, done);
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
-    const int pairs = tiles < max_pairs(kernel) ? tiles : max_pairs(kernel);
+    const int cap = max_pairs(kernel, smem, cached_pairs);
+    const int pairs = tiles < cap ? tiles : cap;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * pairs, 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = S2_SMEM;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -868,6 +933,9 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
                          void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, cudaStream_t stream) {
     const bool out_bf16 = d_dtype == FP8DS_BF16;
     const bool pair = m > S1_BM;
+    // Long contractions amortise the non-overlapped epilogue of the 512-row
+    // pair tile; short ones keep the double-buffered 256-row tile.
+    const int m_sub = (pair && m > 2 * S2_BM && k >= 4096) ? 2 : 1;
     CUtensorMap ta, tb, td;
     bool ok = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, k, m, k, BK, pair ? S2_BM : S1_BM) &&
               encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, k, n, k, BK, pair ? S2_BN_HALF : ACC_N) &&
@@ -886,14 +954,16 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.M = static_cast<int32_t>(m);
     p.N = static_cast<int32_t>(n);
     p.K = static_cast<int32_t>(k);
-    const int tile_m = pair ? 2 * S2_BM : S1_BM;
+    const int tile_m = pair ? m_sub * 2 * S2_BM : S1_BM;
     p.tiles_m = static_cast<int32_t>((m + tile_m - 1) / tile_m);
     p.tiles_n = static_cast<int32_t>((n + ACC_N - 1) / ACC_N);
     p.num_kb = static_cast<int32_t>((k + BK - 1) / BK);
-    p.idesc = make_idesc(a_fmt, b_fmt, tile_m, ACC_N);
+    p.idesc = make_idesc(a_fmt, b_fmt, pair ? 2 * S2_BM : S1_BM, ACC_N);
     cudaError_t e;
-    if (pair)
-        e = out_bf16 ? launch_2sm<true>(ta, tb, td, p, stream) : launch_2sm<false>(ta, tb, td, p, stream);
+    if (pair && m_sub == 2)
+        e = out_bf16 ? launch_2sm<true, 2>(ta, tb, td, p, stream) : launch_2sm<false, 2>(ta, tb, td, p, stream);
+    else if (pair)
+        e = out_bf16 ? launch_2sm<true, 1>(ta, tb, td, p, stream) : launch_2sm<false, 1>(ta, tb, td, p, stream);
     else
         e = out_bf16 ? launch_1sm<true>(ta, tb, td, p, stream) : launch_1sm<false>(ta, tb, td, p, stream);
     if (e != cudaSuccess) {

@@ -82,12 +82,14 @@ def _compare(d, ref, rows, out_dtype, what, ops):
     return check_gemm_bf16(host_bits(got), ref, what, absdot=absdot, K=a.shape[1])
 
 
-# M <= 128 runs the 1-SM kernel, larger M the CTA-pair kernel (pair tile
-# 256 x 256): ragged M inside a pair, a second CTA with one row, B rows of the
-# second CTA entirely out of range (N <= 128), more tiles than SM pairs.
+# M <= 128 runs the 1-SM kernel, larger M the CTA-pair kernel: pair tile
+# 256 x 256, or 512 x 256 when M > 256 and K >= 4096.  Covered: ragged M
+# inside a pair and inside the 512-row tile, a second CTA with one row, B rows
+# of the second CTA entirely out of range (N <= 128), a partial last k-block,
+# more tiles than SM pairs.
 SHAPES = [(128, 256, 128), (128, 512, 256), (300, 520, 272), (1, 8, 16), (129, 264, 144),
           (256, 256, 1024), (4096, 8, 256), (1000, 136, 528), (4096, 2048, 256),
-          (2048, 8192, 1024)]
+          (2048, 8192, 1024), (600, 264, 4096), (1024, 512, 4112), (257, 136, 4096)]
 
 
 @pytest.mark.parametrize("shape", SHAPES)
@@ -104,7 +106,7 @@ def test_gemm_e4m3_realistic(fp8, shape, out_dtype):
 
 @pytest.mark.parametrize("fa,fb", [("e4m3", "e4m3"), ("e5m2", "e4m3"), ("e4m3", "e5m2"),
                                    ("e5m2", "e5m2")])
-@pytest.mark.parametrize("shape", [(200, 264, 160), (384, 512, 512)])
+@pytest.mark.parametrize("shape", [(200, 264, 160), (384, 512, 512), (640, 264, 4096)])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_gemm_format_pairs_random_codes(fp8, fa, fb, shape, out_dtype):
     M, N, K = shape
@@ -135,7 +137,8 @@ def _integer_codes(shape, fmt, seed):
 
 
 @pytest.mark.parametrize("fa,fb", [("e4m3", "e4m3"), ("e5m2", "e4m3")])
-@pytest.mark.parametrize("shape", [(128, 256, 128), (300, 520, 1040), (1024, 1024, 512)])
+@pytest.mark.parametrize("shape", [(128, 256, 128), (300, 520, 1040), (1024, 1024, 512),
+                                   (1100, 520, 4096)])
 def test_gemm_integer_exact(fp8, fa, fb, shape):
     M, N, K = shape
     a, av = _integer_codes((M, K), fa, 5)
