@@ -8,8 +8,12 @@
 //   scale_inv = fl32(1 / scale).
 //
 // Both kernels are HBM-bound.  Design for B200:
-//   - every global access is a 16-byte vector (8-byte for the row-major FP8
-//     output of the transpose kernel), coalesced across the warp;
+//   - the cast-transpose input arrives by TMA: 128-row x 64-column tiles
+//     (128-byte swizzle) stream into a 3- or 4-stage shared-memory ring per
+//     CTA, so load latency never sits between a tile's barriers; threads read
+//     their 4 rows x 8 columns conflict-free from the swizzled tile;
+//   - every other global access is a 16-byte vector (8-byte for the
+//     row-major FP8 output of the transpose kernel), coalesced;
 //   - the transpose is done in two steps: a 4x4 byte transpose in registers
 //     (byte permutes) turns four input rows into column words, which go to a
 //     padded shared-memory tile; each thread then reads 16 consecutive rows
@@ -19,13 +23,19 @@
 //   - grids are sized to fill every SM with resident CTAs and loop over
 //     tiles (grid-stride), so the atomics are few.
 // The cast itself is the hardware conversion cvt.rn.satfinite.{e4m3,e5m2}x2,
-// which rounds to nearest-even and saturates finite overflow and infinities to
-// +-max; NaN inputs are rewritten to the canonical code 0x7F.
+// which rounds to nearest-even, saturates finite overflow and infinities to
+// +-max, and turns every NaN (either sign, any payload) into 0x7F; the GPU
+// tests pin that behaviour for every bf16 pattern and every fp32 pattern in
+// the formats' range.
 #include <cuda_bf16.h>
 
 #include "fp8ds_internal.h"
+#include "ptx_sm100.cuh"
 
 namespace fp8ds {
+
+__device__ int32_t g_cast_error = 0;
+
 namespace {
 
 // ---------------------------------------------------------------- elements --
@@ -52,10 +62,7 @@ __device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
     } else {
         asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     }
-    uint32_t v = r;
-    v = (lo != lo) ? ((v & 0xFF00u) | 0x007Fu) : v;
-    v = (hi != hi) ? ((v & 0x00FFu) | 0x7F00u) : v;
-    return v;
+    return r;
 }
 
 template <int FMT>
@@ -265,6 +272,180 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
     block_amax_commit<CT_THREADS>(m, amax);
 }
 
+// -------------------------------------------- cast + transpose, TMA input --
+
+// Shared-memory ring of input tiles (one 128 x 64 tile per stage).
+template <typename T>
+struct TmaRing {
+    static constexpr int STAGES = sizeof(T) == 2 ? 4 : 2;   // 3 CTAs per SM fit either way
+    static constexpr int BOX_COLS = 128 / sizeof(T);             // one 128-byte swizzle row per box row
+    static constexpr int BOXES = CT_COLS / BOX_COLS;              // 1 (bf16) or 2 (fp32)
+    static constexpr int BOX_BYTES = CT_ROWS * 128;               // 16 KB
+    static constexpr int STAGE_BYTES = BOXES * BOX_BYTES;
+    static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES;      // + alignment slack
+};
+
+// 16 bytes of row r (tile-relative) starting at column 8*cc of a stage.
+template <typename T>
+__device__ __forceinline__ uint4 ring_read(const uint8_t *stage, int r, int granule) {
+    // granule: 16-byte unit index within the tile row (bf16: 0..7, fp32: 0..15)
+    const int box = granule >> 3, g = granule & 7;
+    return *reinterpret_cast<const uint4 *>(stage + box * TmaRing<T>::BOX_BYTES + r * 128 + ((g ^ (r & 7)) << 4));
+}
+
+template <typename T, int FMT>
+struct RingLoad8;
+template <int FMT>
+struct RingLoad8<uint16_t, FMT> {
+    static __device__ __forceinline__ uint2 cast(const uint8_t *stage, int r, int cc, float s, float &m) {
+        const uint4 v = ring_read<uint16_t>(stage, r, cc);
+        return Load8<uint16_t, FMT>::cast(v, s, m);
+    }
+};
+template <int FMT>
+struct RingLoad8<float, FMT> {
+    static __device__ __forceinline__ uint2 cast(const uint8_t *stage, int r, int cc, float s, float &m) {
+        typename Load8<float, FMT>::Raw v;
+        const uint4 a = ring_read<float>(stage, r, 2 * cc);
+        const uint4 b = ring_read<float>(stage, r, 2 * cc + 1);
+        v.a = make_float4(__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w));
+        v.b = make_float4(__uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w));
+        return Load8<float, FMT>::cast(v, s, m);
+    }
+};
+
+// Vectorised-path requirements (checked on the host): x 16-byte aligned
+// (TMA), cols % 8 == 0, rows % 16 == 0, y and yt 16-byte aligned.  Tiles
+// that reach past the tensor read zeros (TMA fill) and store element-wise.
+template <typename T, int FMT, bool WRITE_T>
+__global__ void __launch_bounds__(CT_THREADS, 3)
+cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t rows, int32_t cols,
+                          const float *__restrict__ scale_ptr, uint8_t *__restrict__ y, uint8_t *__restrict__ yt,
+                          float *__restrict__ amax, float *__restrict__ scale_inv, int32_t tiles_c,
+                          int32_t num_tiles) {
+    using R = TmaRing<T>;
+    constexpr int STAGES = R::STAGES;
+    extern __shared__ uint8_t dsm[];
+    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[STAGES];
+    __shared__ uint32_t tsm[CT_COLS * CT_TSTRIDE];
+    const float s = __ldg(scale_ptr);
+    const int tid = threadIdx.x;
+    const int cc = tid & 7, rg = tid >> 3;
+    float m = 0.0f;
+
+    if (tid == 0) {
+        if (blockIdx.x == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
+        for (int i = 0; i < STAGES; ++i) ptx::mbar_init(&full[i], 1);
+        ptx::fence_barrier_init();
+        ptx::fence_async_smem();
+        ptx::prefetch_tmap(&tmap_x);
+    }
+    __syncthreads();
+    // Thread 0 keeps up to STAGES tiles of this CTA in flight.
+    int issued = 0;
+    auto issue = [&](int tile, int stage) {
+        const int32_t r0 = (tile / tiles_c) * CT_ROWS;
+        const int32_t c0 = (tile % tiles_c) * CT_COLS;
+        ptx::mbar_arrive_expect_tx(&full[stage], R::STAGE_BYTES);
+#pragma unroll
+        for (int b = 0; b < R::BOXES; ++b)
+            ptx::tma_load_2d(&tmap_x, &full[stage], ring + stage * R::STAGE_BYTES + b * R::BOX_BYTES,
+                             c0 + b * R::BOX_COLS, r0);
+        ++issued;
+    };
+    if (tid == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            const int t = blockIdx.x + i * gridDim.x;
+            if (t < num_tiles) issue(t, i);
+        }
+    }
+
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+        const int stage = it % STAGES;
+        const uint32_t phase = static_cast<uint32_t>((it / STAGES) & 1);
+        const bool ok = ptx::mbar_wait_for(&full[stage], phase, ptx::TIMEOUT_NS);
+        // Every thread leaves together if the tile never arrived.
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicCAS(&g_cast_error, 0, (16 << 8) | FP8DS_ERR_TIMEOUT);
+            break;
+        }
+        const uint8_t *st = ring + stage * R::STAGE_BYTES;
+        const int32_t r0 = (tile / tiles_c) * CT_ROWS;
+        const int32_t c0 = (tile % tiles_c) * CT_COLS;
+        const bool full_tile = (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
+        uint2 w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = RingLoad8<T, FMT>::cast(st, 4 * rg + i, cc, s, m);
+        {
+            const int32_t gr0 = r0 + 4 * rg, gc0 = c0 + 8 * cc;
+            uint8_t *yp = y + static_cast<int64_t>(gr0) * cols + gc0;
+            if (full_tile) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) *reinterpret_cast<uint2 *>(yp + static_cast<int64_t>(i) * cols) = w[i];
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int b = 0; b < 8; ++b)
+                        if (gr0 + i < rows && gc0 + b < cols)
+                            yp[static_cast<int64_t>(i) * cols + b] =
+                                static_cast<uint8_t>(((b < 4 ? w[i].x : w[i].y) >> (8 * (b & 3))) & 0xFF);
+            }
+        }
+        if (WRITE_T) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t a0 = h ? w[0].y : w[0].x, a1 = h ? w[1].y : w[1].x;
+                const uint32_t a2 = h ? w[2].y : w[2].x, a3 = h ? w[3].y : w[3].x;
+                const uint32_t p01l = __byte_perm(a0, a1, 0x5140);
+                const uint32_t p01h = __byte_perm(a0, a1, 0x7362);
+                const uint32_t p23l = __byte_perm(a2, a3, 0x5140);
+                const uint32_t p23h = __byte_perm(a2, a3, 0x7362);
+                uint32_t *tw = tsm + (8 * cc + 4 * h) * CT_TSTRIDE + rg;
+                tw[0 * CT_TSTRIDE] = __byte_perm(p01l, p23l, 0x5410);
+                tw[1 * CT_TSTRIDE] = __byte_perm(p01l, p23l, 0x7632);
+                tw[2 * CT_TSTRIDE] = __byte_perm(p01h, p23h, 0x5410);
+                tw[3 * CT_TSTRIDE] = __byte_perm(p01h, p23h, 0x7632);
+            }
+        }
+        // The stage is fully read (and the transposed words written): refill it.
+        __syncthreads();
+        if (tid == 0) {
+            const int next = tile + STAGES * gridDim.x;
+            if (next < num_tiles) issue(next, stage);
+        }
+        if (WRITE_T) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int idx = tid + CT_THREADS * k;
+                const int c = idx >> 3, q = idx & 7;
+                const uint32_t *tp = tsm + c * CT_TSTRIDE + 4 * q;
+                const uint4 v = make_uint4(tp[0], tp[1], tp[2], tp[3]);
+                const int32_t gc = c0 + c, gr = r0 + 16 * q;
+                uint8_t *dst = yt + static_cast<int64_t>(gc) * rows + gr;
+                if (full_tile) {
+                    *reinterpret_cast<uint4 *>(dst) = v;
+                } else if (gc < cols) {
+                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int b = 0; b < 16; ++b)
+                        if (gr + b < rows) dst[b] = static_cast<uint8_t>((wv[b >> 2] >> (8 * (b & 3))) & 0xFF);
+                }
+            }
+        }
+        // (the next iteration's tsm writes come after its __syncthreads_or)
+    }
+    // Loads issued but never consumed (only after a timeout) must land before
+    // the CTA exits.
+    if (tid == 0) {
+        for (int j = it; j < issued; ++j)
+            ptx::mbar_wait_for(&full[j % STAGES], static_cast<uint32_t>((j / STAGES) & 1), ptx::DRAIN_NS);
+    }
+    block_amax_commit<CT_THREADS>(m, amax);
+}
+
 // ---------------------------------------------------------------- quantize --
 
 constexpr int Q_THREADS = 256;
@@ -315,30 +496,64 @@ int grid_for(K kernel, int threads, int64_t work_items) {
     return static_cast<int>(g < 1 ? 1 : g);
 }
 
-template <typename T, int FMT, bool VEC, bool WRITE_T>
-cudaError_t ct_launch(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y,
-                      uint8_t *yt, float *amax, float *scale_inv, cudaStream_t stream) {
+template <typename T, int FMT, bool WRITE_T>
+cudaError_t ct_launch_elem(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
+                           float *amax, float *scale_inv, cudaStream_t stream) {
     const int64_t tiles_c = (cols + CT_COLS - 1) / CT_COLS;
     const int64_t tiles_r = (rows + CT_ROWS - 1) / CT_ROWS;
     const int64_t num_tiles = tiles_c * tiles_r;
-    auto kernel = cast_transpose_kernel<T, FMT, VEC, WRITE_T>;
+    auto kernel = cast_transpose_kernel<T, FMT, false, WRITE_T>;
     const int grid = grid_for(kernel, CT_THREADS, num_tiles);
-    kernel<<<grid, CT_THREADS, 0, stream>>>(static_cast<const T *>(x), rows, cols, scale, y, yt,
-                                            amax, scale_inv, tiles_c, num_tiles);
+    kernel<<<grid, CT_THREADS, 0, stream>>>(static_cast<const T *>(x), rows, cols, scale, y, yt, amax, scale_inv,
+                                            tiles_c, num_tiles);
+    return cudaGetLastError();
+}
+
+template <typename T, int FMT, bool WRITE_T>
+cudaError_t ct_launch_tma(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
+                          float *amax, float *scale_inv, cudaStream_t stream) {
+    using R = TmaRing<T>;
+    const int64_t tiles_c = (cols + CT_COLS - 1) / CT_COLS;
+    const int64_t tiles_r = (rows + CT_ROWS - 1) / CT_ROWS;
+    const int64_t num_tiles = tiles_c * tiles_r;
+    CUtensorMap tm;
+    if (!encode_tmap_2d(&tm, sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x,
+                        static_cast<uint64_t>(cols), static_cast<uint64_t>(rows), static_cast<uint64_t>(cols) * sizeof(T),
+                        R::BOX_COLS, CT_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        return ct_launch_elem<T, FMT, WRITE_T>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+    auto kernel = cast_transpose_tma_kernel<T, FMT, WRITE_T>;
+    static bool configured[64] = {};
+    static int per_sm[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, R::SMEM);
+        if (e != cudaSuccess) return e;
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, CT_THREADS, R::SMEM) != cudaSuccess || n < 1) n = 1;
+        per_sm[dev] = n;
+        configured[dev] = true;
+    }
+    const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm[dev];
+    const int grid = static_cast<int>(num_tiles < cap ? (num_tiles > 0 ? num_tiles : 1) : cap);
+    kernel<<<grid, CT_THREADS, R::SMEM, stream>>>(tm, static_cast<int32_t>(rows), static_cast<int32_t>(cols), scale, y,
+                                                  yt, amax, scale_inv, static_cast<int32_t>(tiles_c),
+                                                  static_cast<int32_t>(num_tiles));
     return cudaGetLastError();
 }
 
 template <typename T, int FMT>
-cudaError_t ct_dispatch(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y,
-                        uint8_t *yt, float *amax, float *scale_inv, cudaStream_t stream) {
-    const bool vec = aligned16(x) && aligned16(y) && (yt == nullptr || aligned16(yt)) &&
-                     (cols % 8 == 0) && (rows % 16 == 0);
+cudaError_t ct_dispatch(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
+                        float *amax, float *scale_inv, cudaStream_t stream) {
+    const bool vec = rows > 0 && cols > 0 && aligned16(x) && aligned16(y) && (yt == nullptr || aligned16(yt)) &&
+                     (cols % 8 == 0) && (rows % 16 == 0) && rows < (int64_t(1) << 31) && cols < (int64_t(1) << 31);
     if (yt != nullptr) {
-        return vec ? ct_launch<T, FMT, true, true>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
-                   : ct_launch<T, FMT, false, true>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+        return vec ? ct_launch_tma<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
+                   : ct_launch_elem<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
     }
-    return vec ? ct_launch<T, FMT, true, false>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
-               : ct_launch<T, FMT, false, false>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+    return vec ? ct_launch_tma<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
+               : ct_launch_elem<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
 }
 
 template <typename T, int FMT>
@@ -359,6 +574,13 @@ cudaError_t q_dispatch(const void *x, int64_t n, const float *scale, uint8_t *y,
 }
 
 }  // namespace
+
+cudaError_t read_cast_error(int32_t *out, bool clear) {
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_cast_error, sizeof(int32_t));
+    if (e != cudaSuccess || !clear) return e;
+    const int32_t zero = 0;
+    return cudaMemcpyToSymbol(g_cast_error, &zero, sizeof(int32_t));
+}
 
 cudaError_t launch_cast_transpose(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
                                   fp8ds_format fmt, const float *scale, uint8_t *y, uint8_t *yt,

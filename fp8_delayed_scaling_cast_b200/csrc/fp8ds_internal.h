@@ -1,6 +1,7 @@
 // Internal declarations shared by the translation units of libfp8ds.so.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,7 +36,15 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
                          const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
                          int64_t m, int64_t n, int64_t k, cudaStream_t stream);
 
-// Device error word written by kernels whose bounded waits give up.
+// Device error words written by kernels whose bounded waits give up (one per
+// translation unit); read_device_error returns the first non-zero one.
 cudaError_t read_device_error(int32_t *out, bool clear);
+cudaError_t read_gemm_error(int32_t *out, bool clear);
+cudaError_t read_cast_error(int32_t *out, bool clear);
+
+// 2-D tiled tensor map (cuTensorMapEncodeTiled through the runtime's driver
+// entry point).  Returns false if the driver rejects the arguments.
+bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 }  // namespace fp8ds
