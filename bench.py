@@ -81,7 +81,7 @@ class ClockSampler:
             self.uuid = None
 
     def start(self):
-        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "100"]
+        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "20"]
         if self.uuid:
             cmd[1:1] = ["-i", self.uuid]
         try:
@@ -258,15 +258,14 @@ def time_cast_workload(fp8, device, reps=40):
     for fmt in ("e4m3", "e5m2"):
         for i in range(5):
             fp8.fp8_cast_transpose_amax(xs[i % 8], fmt, s, y, yt, am, si)
-        log = EventLog()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
+        e0.record()
         for i in range(reps):
-            done = log("cast", fmt)
             fp8.fp8_cast_transpose_amax(xs[i % 8], fmt, s, y, yt, am, si)
-            done()
+        e1.record()
         torch.cuda.synchronize()
-        ts = [t for _, t in log.summary()["cast"]]
-        res[fmt] = {"us_median": 1e3 * statistics.median(ts), "us_mean": 1e3 * statistics.mean(ts)}
+        res[fmt] = {"us_mean": 1e3 * e0.elapsed_time(e1) / reps}
     return res
 
 
@@ -281,15 +280,14 @@ def time_headline_gemm(fp8, device, reps=30):
         d = torch.empty(M, N, dtype=torch.bfloat16, device=device)
         for _ in range(5):
             fp8.fp8_gemm(a, "e4m3", sa, b, "e4m3", sa, d)
-        log = EventLog()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
+        e0.record()
         for _ in range(reps):
-            done = log("gemm", "h")
             fp8.fp8_gemm(a, "e4m3", sa, b, "e4m3", sa, d)
-            done()
+        e1.record()
         torch.cuda.synchronize()
-        ts = [t for _, t in log.summary()["gemm"]]
-        us = 1e3 * statistics.median(ts)
+        us = 1e3 * e0.elapsed_time(e1) / reps
         out["%dx%dx%d" % (M, N, K)] = {"us_median": us, "tflops": 2.0 * M * N * K / (us * 1e-6) / 1e12}
     return out
 
@@ -399,13 +397,15 @@ def single_kernel(args):
         run = lambda: fp8.fp8_gemm(a, "e4m3", sa, b, "e4m3", sa, d)  # noqa: E731
         work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     else:
-        x = inputs.spiky_bf16().to(dev)
+        base = inputs.spiky_bf16().to(dev)
+        xs = [base] + [base.roll(i * 17, dims=1).contiguous() for i in range(1, 8)]
         y = torch.empty(C2_ROWS, C2_COLS, dtype=torch.uint8, device=dev)
         yt = torch.empty(C2_COLS, C2_ROWS, dtype=torch.uint8, device=dev)
         s = torch.ones(1, device=dev)
         am = torch.zeros(1, device=dev)
         si = torch.zeros(1, device=dev)
-        run = lambda: fp8.fp8_cast_transpose_amax(x, args.fmt, s, y, yt, am, si)  # noqa: E731
+        it = iter(range(1 << 30))
+        run = lambda: fp8.fp8_cast_transpose_amax(xs[next(it) % 8], args.fmt, s, y, yt, am, si)  # noqa: E731
         work, unit = C2_BYTES / 1e9, "GB/s"
     for _ in range(2):
         run()
@@ -495,27 +495,34 @@ def main():
 
     # warm-up
     for i in range(args.warmup):
-        step.run_kernels(i, sync_amax=sync)
+        step.run_linear_api(i, sync_amax=sync)
     barrier_sync(world)
 
-    # timed region: K steps, every kernel bracketed by events on its stream
+    # timed region: K steps through the public linear API, launched back to
+    # back (no host sync, no events between kernels)
     clocks = ClockSampler(device) if rank == 0 else None
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    log = EventLog()
     barrier_sync(world)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record()
     for i in range(args.steps):
-        step.run_kernels(i, ev=log, sync_amax=sync)
+        step.run_linear_api(i, sync_amax=sync)
     t_end.record()
     barrier_sync(world)
     clock_info = clocks.stop() if clocks else None
     ms_local = t_start.elapsed_time(t_end) / args.steps
     ms = max_over_ranks(ms_local, world, device)
     status = fp8.fp8ds_device_status()
+
+    # per-kernel durations: the same launches, one C call per kernel, each
+    # bracketed by CUDA events on the launching stream (K more steps)
+    log = EventLog()
+    for i in range(args.steps):
+        step.run_kernels(i, ev=log, sync_amax=sync)
+    barrier_sync(world)
 
     per = log.summary()
     gemm_ms = [t for _, t in per["gemm"]]
@@ -528,6 +535,7 @@ def main():
     fp8_peak = 2.0 * pk["bf16"]                       # nominal fp8:bf16 ratio 4.5 / 2.25
     fp8_peak_sus = 2.0 * pk["bf16_sus"]
     cast_total_ms = sum(sum(v) for v in cast_ms.values()) / args.steps
+    kernel_ms = (sum(gemm_ms) + sum(upd_ms)) / args.steps + cast_total_ms
     cast_gbs_step = STEP_CAST_BYTES / (cast_total_ms * 1e-3) / 1e9
     value = world * STEP_FLOP / (ms * 1e-3) / 1e12
 
@@ -584,6 +592,7 @@ def main():
             "peak_note": "fp8 dense = 2 x measured bf16 burst (%s); sustained: %.1f TFLOP/s, frac %.3f" % (
                 pk["src"], fp8_peak_sus, gemm_tflops / fp8_peak_sus),
             "flop_per_launch": GEMM_FLOP, "launch_us": 1e3 * gemm_avg,
+            "timing": "mean CUDA-event duration of the step's 6 GEMM launches, each bracketed by events",
         },
         "cast_transpose_amax": {
             "workload": "bf16 [8192, 2048] (0.1%% spikes x1000) -> FP8 + transpose + amax, 8 rotating inputs",
@@ -593,6 +602,7 @@ def main():
             "in_step_gbs": cast_gbs_step, "in_step_frac": cast_gbs_step / pk["hbm"],
         },
         "update_scales_us": 1e3 * statistics.mean(upd_ms),
+        "kernels_sum_ms_per_step": kernel_ms,
         "gemm_alone": heads,
         "step_roofline_frac": ((STEP_FLOP / (fp8_peak * 1e12)) + (STEP_CAST_BYTES / (pk["hbm"] * 1e9))) /
                               (ms * 1e-3),
@@ -600,6 +610,7 @@ def main():
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "fp8_linear_fwd/bwd + fp8_update_scales, pinned host X/dY, double-buffered copies"},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "launch_mode": "programmatic dependent launch (griddepcontrol) on every kernel",
         "device_status": status,
         "clocks": clock_info,
         "cpu_baseline": cpu,

@@ -9,9 +9,11 @@
 //
 // Both kernels are HBM-bound.  Design for B200:
 //   - the cast-transpose input arrives by TMA: 128-row x 64-column tiles
-//     (128-byte swizzle) stream into a 3- or 4-stage shared-memory ring per
+//     (128-byte swizzle) stream into a 2- or 3-stage shared-memory ring per
 //     CTA, so load latency never sits between a tile's barriers; threads read
-//     their 4 rows x 8 columns conflict-free from the swizzled tile;
+//     their 4 rows x 8 columns conflict-free from the swizzled tile; one block
+//     barrier per tile (the transposed tile is double-buffered and each
+//     tile's yt stores run in the next tile's iteration);
 //   - every other global access is a 16-byte vector (8-byte for the
 //     row-major FP8 output of the transpose kernel), coalesced;
 //   - the transpose is done in two steps: a 4x4 byte transpose in registers
@@ -158,6 +160,8 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
                       float *__restrict__ scale_inv, int64_t tiles_c, int64_t num_tiles) {
     __shared__ uint32_t tsm[CT_COLS * CT_TSTRIDE];
     uint8_t *tsm8 = reinterpret_cast<uint8_t *>(tsm);
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
     const float s = __ldg(scale_ptr);
     const int tid = threadIdx.x;
     float m = 0.0f;
@@ -277,7 +281,7 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
 // Shared-memory ring of input tiles (one 128 x 64 tile per stage).
 template <typename T>
 struct TmaRing {
-    static constexpr int STAGES = sizeof(T) == 2 ? 4 : 2;   // 3 CTAs per SM fit either way
+    static constexpr int STAGES = sizeof(T) == 2 ? 3 : 2;   // bf16: 3 CTAs per SM; fp32: 2
     static constexpr int BOX_COLS = 128 / sizeof(T);             // one 128-byte swizzle row per box row
     static constexpr int BOXES = CT_COLS / BOX_COLS;              // 1 (bf16) or 2 (fp32)
     static constexpr int BOX_BYTES = CT_ROWS * 128;               // 16 KB
@@ -328,19 +332,23 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
     extern __shared__ uint8_t dsm[];
     uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[STAGES];
-    __shared__ uint32_t tsm[CT_COLS * CT_TSTRIDE];
-    const float s = __ldg(scale_ptr);
+    // Transposed words of two consecutive tiles: tile i writes buffer i & 1
+    // while the yt stores of tile i-1 read the other one.
+    __shared__ uint32_t tsm[2][CT_COLS * CT_TSTRIDE];
     const int tid = threadIdx.x;
     const int cc = tid & 7, rg = tid >> 3;
     float m = 0.0f;
 
     if (tid == 0) {
-        if (blockIdx.x == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
         for (int i = 0; i < STAGES; ++i) ptx::mbar_init(&full[i], 1);
         ptx::fence_barrier_init();
         ptx::fence_async_smem();
         ptx::prefetch_tmap(&tmap_x);
     }
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    const float s = __ldg(scale_ptr);
+    if (tid == 0 && blockIdx.x == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
     __syncthreads();
     // Thread 0 keeps up to STAGES tiles of this CTA in flight.
     int issued = 0;
@@ -361,7 +369,36 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
         }
     }
 
+    // yt stores of a tile whose transposed words are in tsm[buf].
+    auto store_yt = [&](int tile, int buf) {
+        const int32_t r0 = (tile / tiles_c) * CT_ROWS;
+        const int32_t c0 = (tile % tiles_c) * CT_COLS;
+        const bool full_tile = (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int idx = tid + CT_THREADS * k;
+            const int c = idx >> 3, q = idx & 7;
+            const uint32_t *tp = tsm[buf] + c * CT_TSTRIDE + 4 * q;
+            const uint4 v = make_uint4(tp[0], tp[1], tp[2], tp[3]);
+            const int32_t gc = c0 + c, gr = r0 + 16 * q;
+            uint8_t *dst = yt + static_cast<int64_t>(gc) * rows + gr;
+            if (full_tile) {
+                *reinterpret_cast<uint4 *>(dst) = v;
+            } else if (gc < cols) {
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int b = 0; b < 16; ++b)
+                    if (gr + b < rows) dst[b] = static_cast<uint8_t>((wv[b >> 2] >> (8 * (b & 3))) & 0xFF);
+            }
+        }
+    };
+
+    // One block barrier per tile.  Iteration i: wait for tile i; barrier
+    // (all threads are past tile i-1: its stage can be refilled and its
+    // transposed words are complete); refill; cast tile i into y and
+    // tsm[i & 1]; write yt of tile i-1 from tsm[(i-1) & 1].
     int it = 0;
+    int prev = -1;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
         const int stage = it % STAGES;
         const uint32_t phase = static_cast<uint32_t>((it / STAGES) & 1);
@@ -369,7 +406,12 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
         // Every thread leaves together if the tile never arrived.
         if (__syncthreads_or(!ok)) {
             if (tid == 0) atomicCAS(&g_cast_error, 0, (16 << 8) | FP8DS_ERR_TIMEOUT);
+            prev = -1;
             break;
+        }
+        if (tid == 0 && it > 0) {
+            const int next = prev + STAGES * gridDim.x;  // the stage tile i-1 used
+            if (next < num_tiles) issue(next, (it - 1) % STAGES);
         }
         const uint8_t *st = ring + stage * R::STAGE_BYTES;
         const int32_t r0 = (tile / tiles_c) * CT_ROWS;
@@ -403,40 +445,19 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
                 const uint32_t p01h = __byte_perm(a0, a1, 0x7362);
                 const uint32_t p23l = __byte_perm(a2, a3, 0x5140);
                 const uint32_t p23h = __byte_perm(a2, a3, 0x7362);
-                uint32_t *tw = tsm + (8 * cc + 4 * h) * CT_TSTRIDE + rg;
+                uint32_t *tw = tsm[it & 1] + (8 * cc + 4 * h) * CT_TSTRIDE + rg;
                 tw[0 * CT_TSTRIDE] = __byte_perm(p01l, p23l, 0x5410);
                 tw[1 * CT_TSTRIDE] = __byte_perm(p01l, p23l, 0x7632);
                 tw[2 * CT_TSTRIDE] = __byte_perm(p01h, p23h, 0x5410);
                 tw[3 * CT_TSTRIDE] = __byte_perm(p01h, p23h, 0x7632);
             }
+            if (prev >= 0) store_yt(prev, (it - 1) & 1);
         }
-        // The stage is fully read (and the transposed words written): refill it.
-        __syncthreads();
-        if (tid == 0) {
-            const int next = tile + STAGES * gridDim.x;
-            if (next < num_tiles) issue(next, stage);
-        }
-        if (WRITE_T) {
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int idx = tid + CT_THREADS * k;
-                const int c = idx >> 3, q = idx & 7;
-                const uint32_t *tp = tsm + c * CT_TSTRIDE + 4 * q;
-                const uint4 v = make_uint4(tp[0], tp[1], tp[2], tp[3]);
-                const int32_t gc = c0 + c, gr = r0 + 16 * q;
-                uint8_t *dst = yt + static_cast<int64_t>(gc) * rows + gr;
-                if (full_tile) {
-                    *reinterpret_cast<uint4 *>(dst) = v;
-                } else if (gc < cols) {
-                    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int b = 0; b < 16; ++b)
-                        if (gr + b < rows) dst[b] = static_cast<uint8_t>((wv[b >> 2] >> (8 * (b & 3))) & 0xFF);
-                }
-            }
-        }
-        // (the next iteration's tsm writes come after its __syncthreads_or)
+        prev = tile;
     }
+    // The last tile's transposed words: one more barrier, then its yt.
+    __syncthreads();
+    if (WRITE_T && prev >= 0) store_yt(prev, (it - 1) & 1);
     // Loads issued but never consumed (only after a timeout) must land before
     // the CTA exits.
     if (tid == 0) {
@@ -455,6 +476,8 @@ template <typename T, int FMT, bool VEC>
 __global__ void __launch_bounds__(Q_THREADS)
 quantize_kernel(const T *__restrict__ x, int64_t n, const float *__restrict__ scale_ptr,
                 uint8_t *__restrict__ y, float *__restrict__ amax, float *__restrict__ scale_inv) {
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
     const float s = __ldg(scale_ptr);
     float m = 0.0f;
     const int64_t tid = static_cast<int64_t>(blockIdx.x) * Q_THREADS + threadIdx.x;
@@ -504,9 +527,8 @@ cudaError_t ct_launch_elem(const void *x, int64_t rows, int64_t cols, const floa
     const int64_t num_tiles = tiles_c * tiles_r;
     auto kernel = cast_transpose_kernel<T, FMT, false, WRITE_T>;
     const int grid = grid_for(kernel, CT_THREADS, num_tiles);
-    kernel<<<grid, CT_THREADS, 0, stream>>>(static_cast<const T *>(x), rows, cols, scale, y, yt, amax, scale_inv,
-                                            tiles_c, num_tiles);
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), 0, stream, 1, static_cast<const T *>(x), rows, cols,
+                      scale, y, yt, amax, scale_inv, tiles_c, num_tiles);
 }
 
 template <typename T, int FMT, bool WRITE_T>
@@ -537,10 +559,9 @@ cudaError_t ct_launch_tma(const void *x, int64_t rows, int64_t cols, const float
     }
     const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm[dev];
     const int grid = static_cast<int>(num_tiles < cap ? (num_tiles > 0 ? num_tiles : 1) : cap);
-    kernel<<<grid, CT_THREADS, R::SMEM, stream>>>(tm, static_cast<int32_t>(rows), static_cast<int32_t>(cols), scale, y,
-                                                  yt, amax, scale_inv, static_cast<int32_t>(tiles_c),
-                                                  static_cast<int32_t>(num_tiles));
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), R::SMEM, stream, 1, tm, static_cast<int32_t>(rows),
+                      static_cast<int32_t>(cols), scale, y, yt, amax, scale_inv, static_cast<int32_t>(tiles_c),
+                      static_cast<int32_t>(num_tiles));
 }
 
 template <typename T, int FMT>
@@ -564,13 +585,14 @@ cudaError_t q_dispatch(const void *x, int64_t n, const float *scale, uint8_t *y,
     if (vec) {
         auto kernel = quantize_kernel<T, FMT, true>;
         const int grid = grid_for(kernel, Q_THREADS, (items + Q_THREADS - 1) / Q_THREADS);
-        kernel<<<grid, Q_THREADS, 0, stream>>>(static_cast<const T *>(x), n, scale, y, amax, scale_inv);
+        return launch_pdl(kernel, dim3(grid), dim3(Q_THREADS), 0, stream, 1, static_cast<const T *>(x), n, scale, y,
+                          amax, scale_inv);
     } else {
         auto kernel = quantize_kernel<T, FMT, false>;
         const int grid = grid_for(kernel, Q_THREADS, (items + Q_THREADS - 1) / Q_THREADS);
-        kernel<<<grid, Q_THREADS, 0, stream>>>(static_cast<const T *>(x), n, scale, y, amax, scale_inv);
+        return launch_pdl(kernel, dim3(grid), dim3(Q_THREADS), 0, stream, 1, static_cast<const T *>(x), n, scale, y,
+                          amax, scale_inv);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace

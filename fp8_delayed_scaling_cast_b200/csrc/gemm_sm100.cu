@@ -14,9 +14,11 @@
 //   warp 1      allocates 512 TMEM columns (two fp32 accumulators of 256
 //               columns) and issues tcgen05.mma.kind::f8f6f4 from one thread;
 //               tcgen05.commit frees ring stages and publishes accumulators;
-//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, fp32 fma with the
-//               combined scale_inv and bias, conversion, 128-byte-swizzled
-//               staging in shared memory and TMA tensor stores.
+//   warps 2..9  epilogue: each reads 32 TMEM lanes (its lane quarter) of half
+//               of the accumulator columns with tcgen05.ld, fp32 fma with the
+//               combined scale_inv and the tile's bias (staged once in shared
+//               memory), conversion, 128-byte-swizzled staging in shared memory
+//               and TMA tensor stores.
 // Two accumulators let the epilogue of tile i overlap the main loop of i+1.
 //
 //   fp8_gemm_1sm_kernel  one CTA per SM, tile 128 x 256, 4 stages of 48 KB
@@ -55,13 +57,13 @@ namespace {
 constexpr int BK = 128;        // bytes == FP8 elements per k-block (one 128-byte swizzle row)
 constexpr int UMMA_K = 32;     // K of one kind::f8f6f4 MMA
 constexpr int ACC_N = 256;     // accumulator columns (tile N)
-constexpr int THREADS = 192;
+constexpr int EPI_WARPS = 8;               // two per TMEM lane quarter
+constexpr int THREADS = 64 + 32 * EPI_WARPS; // producer warp, MMA warp, epilogue warps
 constexpr int EPI_WARP0 = 2;
 constexpr int TMEM_COLS = 512; // two accumulators
 constexpr int EPI_BOX_BYTES = 32 * 128;  // staging box: 32 rows x 128 bytes
-constexpr int EPI_BUFS = 2;
-constexpr int EPI_BYTES = 4 * EPI_BUFS * EPI_BOX_BYTES + 256 * 4;  // + the tile's bias (fp32 x 256)
-constexpr int EPI_THREADS = 128;
+constexpr int EPI_BYTES = EPI_WARPS * EPI_BOX_BYTES + 256 * 4;  // + the tile's bias (fp32 x 256)
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int SMEM_ALIGN = 1024;
 constexpr int GROUP_M = 8;
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;  // 2 s
@@ -351,8 +353,8 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
 // epilogue_bar().
 __device__ __forceinline__ void stage_bias(float *bias_s, const Params &p, int64_t n_base, int epi_tid) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int c = 2 * epi_tid + i;
+    for (int i = 0; i < ACC_N / EPI_THREADS; ++i) {
+        const int c = epi_tid + i * EPI_THREADS;
         const int64_t n = n_base + c;
         float v = 0.0f;
         if (p.bias_kind != 0 && n < p.N) {
@@ -384,20 +386,21 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
 // row.  After the last TMEM read the warp arrives (lane 0) on the
 // accumulator-empty barrier given by its shared::cluster address.
 template <bool OUT_BF16>
-__device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *bufs, int &buf,
+__device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *box, int half,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                               float sab, const float *bias_s, uint32_t empty_bar_cluster,
                                               bool arrive) {
     constexpr int COLS_PER_BOX = OUT_BF16 ? 64 : 32;
     constexpr int BOXES = ACC_N / COLS_PER_BOX;
-    for (int bx = 0; bx < BOXES; ++bx) {
+    constexpr int HALF = BOXES / 2;
+    for (int bx = half * HALF; bx < (half + 1) * HALF; ++bx) {
         uint32_t packed[32];
         if (OUT_BF16) {
             uint32_t r0[32], r1[32];
             tmem_ld32(t_row + bx * 64, r0);
             tmem_ld32(t_row + bx * 64 + 32, r1);
             tmem_ld_wait();
-            if (arrive && bx == BOXES - 1) {
+            if (arrive && bx == (half + 1) * HALF - 1) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
@@ -423,7 +426,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             uint32_t r0[32];
             tmem_ld32(t_row + bx * 32, r0);
             tmem_ld_wait();
-            if (arrive && bx == BOXES - 1) {
+            if (arrive && bx == (half + 1) * HALF - 1) {
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
@@ -432,11 +435,10 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
 #pragma unroll
             for (int j = 0; j < 32; ++j) packed[j] = __float_as_uint(fmaf(__uint_as_float(r0[j]), sab, bs[j]));
         }
-        // Staging buffer reuse: the store issued from it two boxes ago must
-        // have finished reading shared memory.
-        if (lane == 0) tma_store_wait_read<EPI_BUFS - 1>();
+        // Staging buffer reuse: the previous store from it must have finished
+        // reading shared memory.
+        if (lane == 0) tma_store_wait_read<0>();
         __syncwarp();
-        uint8_t *box = bufs + buf * EPI_BOX_BYTES;
         // Row `lane`, 16-byte chunk c goes to chunk c ^ (lane & 7) (the
         // 128-byte swizzle the output tensor map expects).
 #pragma unroll
@@ -451,7 +453,6 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + bx * COLS_PER_BOX), m_row0);
             tma_store_commit();
         }
-        buf ^= 1;
     }
 }
 
@@ -492,12 +493,13 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
                                               int tile_stride, int m_sub, int rows_per_sub, int row_offset,
                                               int acc_bufs, uint32_t tempty_rank) {
     const int num_tiles = p.tiles_m * p.tiles_n;
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint8_t *bufs = sm.epi + (warp - EPI_WARP0) * EPI_BUFS * EPI_BOX_BYTES;
-    float *bias_s = reinterpret_cast<float *>(sm.epi + 4 * EPI_BUFS * EPI_BOX_BYTES);
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int half = (warp - EPI_WARP0) >> 2;  // which half of the accumulator columns
+    uint8_t *box = sm.epi + (warp - EPI_WARP0) * EPI_BOX_BYTES;
+    float *bias_s = reinterpret_cast<float *>(sm.epi + EPI_WARPS * EPI_BOX_BYTES);
     const int epi_tid = (warp - EPI_WARP0) * 32 + lane;
     const float sab = __fmul_rn(__ldg(p.a_scale_inv), __ldg(p.b_scale_inv));
-    int local = 0, buf = 0;
+    int local = 0;
     for (int tile = first_tile; tile < num_tiles; tile += tile_stride, ++local) {
         int m_blk, n_blk;
         tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
@@ -514,7 +516,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
         for (int h = 0; h < m_sub; ++h) {
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>((acc + h) * ACC_N);
-            epilogue_tile<OUT_BF16>(t_row, lane, bufs, buf, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
+            epilogue_tile<OUT_BF16>(t_row, lane, box, half, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
                                     (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32, sab, bias_s,
                                     empty_addr, h == m_sub - 1);
         }
@@ -542,7 +544,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.tfull[b], 1);
-            mbar_init(&sm.tempty[b], 4);
+            mbar_init(&sm.tempty[b], EPI_WARPS);
         }
         mbar_init(sm.drain, 1);
         *sm.abort_flag = 0;
@@ -563,6 +565,10 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *sm.tmem_slot;
+    // Everything above touched only this CTA; global memory waits for the
+    // previous kernel in the stream.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -683,7 +689,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.tfull[b], 1);
-            mbar_init(&sm.tempty[b], 8);  // 4 epilogue warps x 2 CTAs (the first CTA's is used)
+            mbar_init(&sm.tempty[b], 2 * EPI_WARPS);  // epilogue warps of both CTAs (the first CTA's is used)
         }
         mbar_init(sm.drain, 1);
         *sm.abort_flag = 0;
@@ -704,6 +710,8 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *sm.tmem_slot;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == 0) {
         if (lane == 0) {
@@ -873,19 +881,7 @@ cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
     const int tiles = p.tiles_m * p.tiles_n;
     const int cap = max_pairs(kernel, smem, cached_pairs);
     const int pairs = tiles < cap ? tiles : cap;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * pairs, 1, 1);
-    cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, ta, tb, td, p);
+    return launch_pdl(kernel, dim3(2 * pairs), dim3(THREADS), smem, stream, 2, ta, tb, td, p);
 }
 
 template <bool OUT_BF16>
@@ -897,8 +893,7 @@ cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    kernel<<<grid, THREADS, S1_SMEM, stream>>>(ta, tb, td, p);
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3(grid), dim3(THREADS), S1_SMEM, stream, 1, ta, tb, td, p);
 }
 
 }  // namespace

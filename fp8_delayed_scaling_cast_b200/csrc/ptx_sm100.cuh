@@ -46,7 +46,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 }
 
 // Wait for the phase of `bar` with the given parity for at most `limit_ns`.
-__device__ __noinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
+static __device__ __noinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, unsigned long long limit_ns) {
     const uint32_t addr = smem_u32(bar);
     if (mbar_try_wait(addr, parity)) return true;
     const uint64_t t0 = globaltimer();
@@ -56,6 +56,18 @@ __device__ __noinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity, unsig
             if (mbar_try_wait(addr, parity)) return true;
         if (globaltimer() - t0 > limit_ns) return false;
     }
+}
+
+// Programmatic dependent launch: kernels are launched so that they may start
+// while the previous kernel in the stream is still running.  pdl_wait()
+// blocks until that kernel has completed and its memory is visible; every
+// kernel calls it before its first global-memory access.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel in the stream be scheduled early (it still waits in
+// pdl_wait() for this kernel's completion before touching memory).
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void fence_barrier_init() {

@@ -16,6 +16,7 @@
 // (coalesced).  The work is a few tens of KB: the kernel is launch-latency
 // bound, which is why all T tensors share one launch.
 #include "fp8ds_internal.h"
+#include "ptx_sm100.cuh"
 
 namespace fp8ds {
 namespace {
@@ -25,6 +26,8 @@ constexpr int U_THREADS = 128;
 __global__ void __launch_bounds__(U_THREADS)
 update_scales_kernel(int64_t T, int H, float *__restrict__ hist, float *__restrict__ scale,
                      float *__restrict__ scale_inv, const uint8_t *__restrict__ formats) {
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
     const int64_t t = static_cast<int64_t>(blockIdx.x) * U_THREADS + threadIdx.x;
     if (t >= T) return;
     const float first = hist[t];
@@ -51,9 +54,8 @@ cudaError_t launch_update_scales(int64_t num_tensors, int32_t hist_len, float *a
                                  cudaStream_t stream) {
     if (num_tensors == 0) return cudaSuccess;
     const int64_t blocks = (num_tensors + U_THREADS - 1) / U_THREADS;
-    update_scales_kernel<<<static_cast<unsigned>(blocks), U_THREADS, 0, stream>>>(
-        num_tensors, hist_len, amax_history, scale, scale_inv, formats);
-    return cudaGetLastError();
+    return launch_pdl(update_scales_kernel, dim3(static_cast<unsigned>(blocks)), dim3(U_THREADS), 0, stream, 1,
+                      num_tensors, static_cast<int>(hist_len), amax_history, scale, scale_inv, formats);
 }
 
 }  // namespace fp8ds
