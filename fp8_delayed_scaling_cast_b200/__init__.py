@@ -7,7 +7,8 @@ generators) can be imported on machines without the built library.
 """
 
 __all__ = [
-    "fp8_quantize", "fp8_cast_transpose_amax", "fp8_update_scales", "fp8_gemm",
+    "fp8_quantize", "fp8_cast_transpose_amax", "fp8_update_scales", "fp8_gemm", "fp8_gemm_ex",
+    "fp8_gemm_workspace_size", "gemm_workspace",
     "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
     "fp8ds_version", "Fp8Meta", "Fp8Linear", "Fp8dsError", "E4M3", "E5M2",
 ]

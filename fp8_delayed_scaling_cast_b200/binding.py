@@ -54,7 +54,8 @@ class _Meta(ctypes.Structure):
 class _Linear(ctypes.Structure):
     _fields_ = [("w", _P), ("bias", _P), ("bias_dtype", _INT), ("in_features", _I64),
                 ("out_features", _I64), ("w8", _P), ("w8t", _P), ("w_scale_inv", _P),
-                ("meta_in", _I32), ("meta_w", _I32), ("meta_grad", _I32), ("cache_valid", _I32)]
+                ("meta_in", _I32), ("meta_w", _I32), ("meta_grad", _I32), ("cache_valid", _I32),
+                ("workspace", _P), ("workspace_bytes", ctypes.c_size_t)]
 
 
 _SIGS = {
@@ -62,6 +63,9 @@ _SIGS = {
     "fp8_cast_transpose_amax": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
     "fp8_update_scales": [_I64, _I32, _P, _P, _P, _P, _INT, _P],
     "fp8_gemm": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
+    "fp8_gemm_ex": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P,
+                    ctypes.c_size_t, _P],
+    "fp8_gemm_workspace_size": [ctypes.POINTER(ctypes.c_size_t)],
     "fp8_linear_fwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _INT,
                        _I32, _P, _P, _P, _P],
     "fp8_linear_bwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P,
@@ -139,6 +143,27 @@ def fp8_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, d, bias=None, stream=
                          _ptr(d), _dtype(d), m, n, k, _stream(stream)))
 
 
+def fp8_gemm_ex(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, d, bias=None, workspace=None,
+                stream=None):
+    m, k = a.shape
+    n = b.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.fp8_gemm_ex(_ptr(a), _fmt(a_fmt), _ptr(a_scale_inv), _ptr(b), _fmt(b_fmt),
+                            _ptr(b_scale_inv), _ptr(bias), F32 if bias is None else _dtype(bias),
+                            _ptr(d), _dtype(d), m, n, k, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def fp8_gemm_workspace_size():
+    n = ctypes.c_size_t(0)
+    _check(_lib.fp8_gemm_workspace_size(ctypes.byref(n)))
+    return n.value
+
+
+def gemm_workspace(device="cuda"):
+    """A zero-filled workspace of fp8_gemm_workspace_size() bytes (uint8 tensor)."""
+    return torch.zeros(fp8_gemm_workspace_size(), dtype=torch.uint8, device=device)
+
+
 class Fp8Meta:
     """Packed DelayedScaling state of T FP8 tensors (caller-owned device tensors)."""
 
@@ -163,16 +188,18 @@ class Fp8Meta:
 class Fp8Linear:
     """A linear layer's fp32 master weight, optional bias and FP8 weight cache."""
 
-    def __init__(self, w, bias, meta_in, meta_w, meta_grad):
+    def __init__(self, w, bias, meta_in, meta_w, meta_grad, workspace=None):
         out_f, in_f = w.shape
         self.w = w
         self.bias = bias
+        self.workspace = workspace
         self.w8 = torch.empty(out_f, in_f, dtype=torch.uint8, device=w.device)
         self.w8t = torch.empty(in_f, out_f, dtype=torch.uint8, device=w.device)
         self.w_scale_inv = torch.ones(1, dtype=torch.float32, device=w.device)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
         self._c = _Linear(_ptr(w), _ptr(bias), F32 if bias is None else _dtype(bias), in_f, out_f,
                           _ptr(self.w8), _ptr(self.w8t), _ptr(self.w_scale_inv),
-                          meta_in, meta_w, meta_grad, 0)
+                          meta_in, meta_w, meta_grad, 0, _ptr(workspace), ws_bytes)
 
     @property
     def in_features(self):

@@ -180,7 +180,28 @@ fp8ds_status fp8_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale
     fp8ds_status st =
         check_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k);
     if (st != FP8DS_OK) return st;
-    return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k, stream);
+    return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k, nullptr,
+                       0, stream);
+}
+
+fp8ds_status fp8_gemm_workspace_size(size_t *bytes) {
+    clear_error();
+    if (bytes == nullptr) return invalid("fp8_gemm_workspace_size: bytes must not be NULL");
+    *bytes = gemm_workspace_bytes();
+    return FP8DS_OK;
+}
+
+fp8ds_status fp8_gemm_ex(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
+                         fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
+                         void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, void *workspace,
+                         size_t workspace_bytes, fp8ds_stream stream) {
+    clear_error();
+    fp8ds_status st =
+        check_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k);
+    if (st != FP8DS_OK) return st;
+    if (workspace != nullptr && !aligned16(workspace)) return invalid("fp8_gemm_ex: workspace must be 16-byte aligned");
+    return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k, workspace,
+                       workspace_bytes, stream);
 }
 
 fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x, fp8ds_dtype x_dtype,
@@ -217,7 +238,7 @@ fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const voi
         lin->cache_valid = 1;
     }
     return launch_gemm(x8, FP8DS_E4M3, x_scale_inv, lin->w8, FP8DS_E4M3, lin->w_scale_inv, lin->bias,
-                       lin->bias_dtype, y, y_dtype, m, N, K, s);
+                       lin->bias_dtype, y, y_dtype, m, N, K, lin->workspace, lin->workspace_bytes, s);
 }
 
 fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy, fp8ds_dtype dy_dtype,
@@ -249,11 +270,11 @@ fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, con
     if (st != FP8DS_OK) return st;
     if (dx != nullptr) {
         st = launch_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv, nullptr, FP8DS_F32,
-                         dx, dx_dtype, m, K, N, s);
+                         dx, dx_dtype, m, K, N, lin->workspace, lin->workspace_bytes, s);
         if (st != FP8DS_OK) return st;
     }
     return launch_gemm(dy8t, FP8DS_E5M2, dy_scale_inv, x8t, FP8DS_E4M3, x_scale_inv, nullptr, FP8DS_F32, dw,
-                       FP8DS_F32, N, K, m, s);
+                       FP8DS_F32, N, K, m, lin->workspace, lin->workspace_bytes, s);
 }
 
 const char *fp8ds_last_error(void) { return g_msg; }

@@ -33,10 +33,16 @@ cudaError_t launch_update_scales(int64_t num_tensors, int32_t hist_len, float *a
                                  cudaStream_t stream);
 
 // Returns FP8DS_OK or an error (message set) for tensor-map or launch failures.
+// workspace (may be NULL) enables the stream-K schedule when it holds at
+// least gemm_workspace_bytes().
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
                          const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
                          const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
-                         int64_t m, int64_t n, int64_t k, cudaStream_t stream);
+                         int64_t m, int64_t n, int64_t k, void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+// Workspace bytes the stream-K schedule needs on the current device.
+size_t gemm_workspace_bytes();
 
 // Device error words written by kernels whose bounded waits give up (one per
 // translation unit); read_device_error returns the first non-zero one.

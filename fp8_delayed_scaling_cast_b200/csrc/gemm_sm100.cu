@@ -44,6 +44,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "fp8ds_internal.h"
@@ -100,6 +101,7 @@ enum Site : int32_t {
     SITE_MMA_FULL = 2,
     SITE_MMA_TMEM_EMPTY = 3,
     SITE_EPI_TMEM_FULL = 4,
+    SITE_EPI_PARTIAL = 5,
 };
 
 // ------------------------------------------------------------ PTX helpers --
@@ -328,6 +330,54 @@ struct Params {
     int32_t M, N, K;
     int32_t tiles_m, tiles_n, num_kb;
     uint32_t idesc;
+    // stream-K (pair kernel only): 0 = whole tiles per cluster
+    int32_t stream_k;
+    uint32_t epoch;       // non-zero per launch; partials are published with it
+    int32_t *flags;       // [clusters][2] publication words
+    float *partials;      // [clusters][2 CTAs][2 row blocks][128 x 256] fp32
+};
+
+// Workspace of the stream-K schedule: publication words, then one partial
+// accumulator slot per cluster (a pair's two CTAs, up to two row blocks each).
+constexpr size_t WS_FLAG_BYTES = 4096;  // room for 1024 clusters
+constexpr size_t WS_SLOT_FLOATS = 2 * 2 * 128 * 256;
+
+// Work assignment of a cluster (or CTA).  Stream-K: cluster c of C owns the
+// units [c*U/C, (c+1)*U/C) of the U = tiles * num_kb (tile, k-block) units in
+// tile order, as segments (tile, kb0, kb1); requires tiles >= C so that a
+// tile is split between at most two clusters.  Otherwise whole tiles c,
+// c + C, ...
+struct Sched {
+    int64_t u, u1;
+    int t, stride, num_tiles, num_kb;
+    bool sk;
+    __device__ __forceinline__ Sched(const Params &p, int c, int C) {
+        num_tiles = p.tiles_m * p.tiles_n;
+        num_kb = p.num_kb;
+        sk = p.stream_k != 0;
+        const int64_t U = static_cast<int64_t>(num_tiles) * num_kb;
+        u = U * c / C;
+        u1 = U * (c + 1) / C;
+        t = c;
+        stride = C;
+    }
+    __device__ __forceinline__ bool next(int &tile, int &kb0, int &kb1) {
+        if (sk) {
+            if (u >= u1) return false;
+            tile = static_cast<int>(u / num_kb);
+            kb0 = static_cast<int>(u % num_kb);
+            const int64_t left = u1 - u;
+            kb1 = left < num_kb - kb0 ? kb0 + static_cast<int>(left) : num_kb;
+            u += kb1 - kb0;
+            return true;
+        }
+        if (t >= num_tiles) return false;
+        tile = t;
+        kb0 = 0;
+        kb1 = num_kb;
+        t += stride;
+        return true;
+    }
 };
 
 // Named barrier among the 4 epilogue warps.
@@ -385,68 +435,97 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
 // accumulator's first column; m_row0 is the global row of the warp's first
 // row.  After the last TMEM read the warp arrives (lane 0) on the
 // accumulator-empty barrier given by its shared::cluster address.
+// Partial accumulators of a stream-K split tile, lane-major so that a warp's
+// access of 4 consecutive columns of its 32 rows is 512 contiguous bytes:
+// element (row block h, lane quarter q, column c, lane l) at
+// (((h * 4 + q) * 64 + c / 4) * 32 + l) * 4 + c % 4.
+__device__ __forceinline__ float4 *partial_at(float *slot, int h, int q, int col, int lane) {
+    return reinterpret_cast<float4 *>(slot) + ((h * 4 + q) * 64 + col / 4) * 32 + lane;
+}
+
+// Store (mode 1) or add (mode 2) the partial accumulator of 32 columns.
+__device__ __forceinline__ void partial_io(int mode, uint32_t (&r)[32], float *slot, int h, int q, int col0,
+                                           int lane) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float4 *ptr = partial_at(slot, h, q, col0 + 4 * i, lane);
+        if (mode == 1) {
+            *ptr = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+        } else {
+            const float4 v = __ldcg(ptr);
+            r[4 * i] = __float_as_uint(__uint_as_float(r[4 * i]) + v.x);
+            r[4 * i + 1] = __float_as_uint(__uint_as_float(r[4 * i + 1]) + v.y);
+            r[4 * i + 2] = __float_as_uint(__uint_as_float(r[4 * i + 2]) + v.z);
+            r[4 * i + 3] = __float_as_uint(__uint_as_float(r[4 * i + 3]) + v.w);
+        }
+    }
+}
+
+// mode 0: convert and store D; mode 1: store the raw partial (no D); mode 2:
+// add the partial of the other cluster, then convert and store D.
 template <bool OUT_BF16>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *box, int half,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                               float sab, const float *bias_s, uint32_t empty_bar_cluster,
-                                              bool arrive) {
+                                              bool arrive, int mode, float *slot, int h, int q) {
     constexpr int COLS_PER_BOX = OUT_BF16 ? 64 : 32;
     constexpr int BOXES = ACC_N / COLS_PER_BOX;
     constexpr int HALF = BOXES / 2;
+    // 32 accumulator columns per TMEM load (fp32: a whole 128-byte staging
+    // row; bf16: half of one), which keeps the live registers within the
+    // 168 that 10 warps per SM allow.
+    constexpr int LOADS_PER_BOX = OUT_BF16 ? 2 : 1;
     for (int bx = half * HALF; bx < (half + 1) * HALF; ++bx) {
-        uint32_t packed[32];
-        if (OUT_BF16) {
-            uint32_t r0[32], r1[32];
-            tmem_ld32(t_row + bx * 64, r0);
-            tmem_ld32(t_row + bx * 64 + 32, r1);
-            tmem_ld_wait();
-            if (arrive && bx == (half + 1) * HALF - 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
-            }
-            const float2 *bs = reinterpret_cast<const float2 *>(bias_s + bx * 64);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float2 b = bs[j];
-                const float v0 = fmaf(__uint_as_float(r0[2 * j]), sab, b.x);
-                const float v1 = fmaf(__uint_as_float(r0[2 * j + 1]), sab, b.y);
-                __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-                packed[j] = *reinterpret_cast<uint32_t *>(&h);
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float2 b = bs[16 + j];
-                const float v0 = fmaf(__uint_as_float(r1[2 * j]), sab, b.x);
-                const float v1 = fmaf(__uint_as_float(r1[2 * j + 1]), sab, b.y);
-                __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-                packed[16 + j] = *reinterpret_cast<uint32_t *>(&h);
-            }
-        } else {
-            uint32_t r0[32];
-            tmem_ld32(t_row + bx * 32, r0);
-            tmem_ld_wait();
-            if (arrive && bx == (half + 1) * HALF - 1) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
-            }
-            const float *bs = bias_s + bx * 32;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) packed[j] = __float_as_uint(fmaf(__uint_as_float(r0[j]), sab, bs[j]));
-        }
         // Staging buffer reuse: the previous store from it must have finished
         // reading shared memory.
         if (lane == 0) tma_store_wait_read<0>();
         __syncwarp();
-        // Row `lane`, 16-byte chunk c goes to chunk c ^ (lane & 7) (the
-        // 128-byte swizzle the output tensor map expects).
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const int pc = c ^ (lane & 7);
-            *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
-                make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        for (int hh = 0; hh < LOADS_PER_BOX; ++hh) {
+            const int col0 = bx * COLS_PER_BOX + hh * 32;
+            uint32_t r[32];
+            tmem_ld32(t_row + col0, r);
+            tmem_ld_wait();
+            if (arrive && bx == (half + 1) * HALF - 1 && hh == LOADS_PER_BOX - 1) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
+            }
+            if (mode != 0) partial_io(mode, r, slot, h, q, col0, lane);
+            if (mode == 1) continue;
+            const float *bs = bias_s + col0;
+            // 32 columns -> 128 bytes (fp32) or 64 bytes (bf16) of row `lane`;
+            // 16-byte chunk c of the row goes to chunk c ^ (lane & 7) (the
+            // 128-byte swizzle the output tensor map expects).
+            if (OUT_BF16) {
+                uint32_t packed[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float v0 = fmaf(__uint_as_float(r[2 * j]), sab, bs[2 * j]);
+                    const float v1 = fmaf(__uint_as_float(r[2 * j + 1]), sab, bs[2 * j + 1]);
+                    __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
+                    packed[j] = *reinterpret_cast<uint32_t *>(&hv);
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int pc = (hh * 4 + c) ^ (lane & 7);
+                    *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
+                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int pc = c ^ (lane & 7);
+                    *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
+                        make_uint4(__float_as_uint(fmaf(__uint_as_float(r[4 * c]), sab, bs[4 * c])),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * c + 1]), sab, bs[4 * c + 1])),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * c + 2]), sab, bs[4 * c + 2])),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * c + 3]), sab, bs[4 * c + 3])));
+                }
+            }
         }
+        if (mode == 1) continue;
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -483,29 +562,63 @@ __device__ __forceinline__ Smem carve(uint8_t *raw) {
     return s;
 }
 
+__device__ __forceinline__ int32_t ld_acquire(const int32_t *p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(int32_t *p, int32_t v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Epilogue loop shared by both kernels.  A tile spans m_sub row blocks of
 // rows_per_sub rows (row block h of the tile starts at row h * rows_per_sub,
 // and this CTA's rows at row_offset inside it); row block h sits at TMEM
 // column h * 256 of the accumulator.  acc_bufs accumulators alternate.
+// Stream-K segments: a tail (kb0 > 0, the first segment of this cluster)
+// publishes its partial in slot `cluster`; a head (kb0 == 0, kb1 < num_kb,
+// the last segment) adds the partial of slot cluster + 1 before storing D.
 template <bool OUT_BF16>
 __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap *tmap_d, const Params &p,
-                                              uint32_t tmem_base, int warp, int lane, int first_tile,
-                                              int tile_stride, int m_sub, int rows_per_sub, int row_offset,
-                                              int acc_bufs, uint32_t tempty_rank) {
-    const int num_tiles = p.tiles_m * p.tiles_n;
+                                              uint32_t tmem_base, int warp, int lane, int cluster, int clusters,
+                                              int m_sub, int rows_per_sub, int row_offset, int acc_bufs,
+                                              uint32_t tempty_rank, int rank) {
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - EPI_WARP0) >> 2;  // which half of the accumulator columns
     uint8_t *box = sm.epi + (warp - EPI_WARP0) * EPI_BOX_BYTES;
     float *bias_s = reinterpret_cast<float *>(sm.epi + EPI_WARPS * EPI_BOX_BYTES);
     const int epi_tid = (warp - EPI_WARP0) * 32 + lane;
     const float sab = __fmul_rn(__ldg(p.a_scale_inv), __ldg(p.b_scale_inv));
-    int local = 0;
-    for (int tile = first_tile; tile < num_tiles; tile += tile_stride, ++local) {
+    Sched sched(p, cluster, clusters);
+    int local = 0, tile, kb0, kb1;
+    while (sched.next(tile, kb0, kb1)) {
         int m_blk, n_blk;
         tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
         const int acc = acc_bufs == 2 ? (local & 1) : 0;
         const uint32_t acc_phase = static_cast<uint32_t>(acc_bufs == 2 ? (local >> 1) : local) & 1u;
-        const bool ok = mbar_wait(&sm.tfull[acc], acc_phase, sm.abort_flag, SITE_EPI_TMEM_FULL);
+        ++local;
+        const int mode = kb0 > 0 ? 1 : (kb1 < p.num_kb ? 2 : 0);
+        bool ok = mbar_wait(&sm.tfull[acc], acc_phase, sm.abort_flag, SITE_EPI_TMEM_FULL);
+        float *slot = nullptr;
+        int32_t *flag = nullptr;
+        if (mode != 0) {
+            const int s = mode == 1 ? cluster : cluster + 1;
+            slot = p.partials + (static_cast<size_t>(s) * 2 + rank) * WS_SLOT_FLOATS;
+            flag = p.flags + s * 2 + rank;
+        }
+        if (mode == 2 && ok && epi_tid == 0) {
+            // The other cluster wrote this partial at the start of its range.
+            const uint64_t t0 = globaltimer();
+            while (ld_acquire(flag) != static_cast<int32_t>(p.epoch)) {
+                if (*sm.abort_flag || globaltimer() - t0 > TIMEOUT_NS) {
+                    *sm.abort_flag = 1;
+                    record_error(SITE_EPI_PARTIAL);
+                    ok = false;
+                    break;
+                }
+            }
+        }
         // All epilogue warps meet here every tile: they leave together if any
         // wait gave up, and none of them still reads the previous tile's bias.
         if (epilogue_any(!ok)) break;
@@ -518,7 +631,18 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
                                    static_cast<uint32_t>((acc + h) * ACC_N);
             epilogue_tile<OUT_BF16>(t_row, lane, box, half, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
                                     (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32, sab, bias_s,
-                                    empty_addr, h == m_sub - 1);
+                                    empty_addr, h == m_sub - 1, mode, slot, h, q);
+        }
+        if (mode == 1) {
+            // Publish: every epilogue thread's partial stores precede the flag.
+            epilogue_bar();
+            if (epi_tid == 0) {
+                __threadfence();
+                st_release(flag, static_cast<int32_t>(p.epoch));
+            }
+        } else if (mode == 2) {
+            epilogue_bar();
+            if (epi_tid == 0) *flag = 0;  // consumed; the slot is free for the next launch
         }
     }
     if (lane == 0) tma_store_wait_all();
@@ -535,8 +659,6 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     const Smem sm = carve<S1_STAGES, S1_A_STAGE, S1_B_STAGE>(smem_raw);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_tiles = p.tiles_m * p.tiles_n;
-
     if (threadIdx.x == 0) {
         for (int s = 0; s < S1_STAGES; ++s) {
             mbar_init(&sm.full[s], 1);
@@ -576,10 +698,12 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             uint32_t phase = 0;
             int64_t issued = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            Sched sched(p, blockIdx.x, gridDim.x);
+            int tile, kb0, kb1;
+            while (ok && sched.next(tile, kb0, kb1)) {
                 int m_blk, n_blk;
                 tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&sm.empty[stage], phase ^ 1u, sm.abort_flag, SITE_PRODUCER_EMPTY)) {
                         ok = false;
                         break;
@@ -609,16 +733,19 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             uint32_t phase = 0;
             bool ok = true;
             int local = 0;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++local) {
+            Sched sched(p, blockIdx.x, gridDim.x);
+            int tile, kb0, kb1;
+            while (ok && sched.next(tile, kb0, kb1)) {
                 const int acc = local & 1;
                 const uint32_t acc_phase = static_cast<uint32_t>(local >> 1) & 1u;
+                ++local;
                 if (!mbar_wait(&sm.tempty[acc], acc_phase ^ 1u, sm.abort_flag, SITE_MMA_TMEM_EMPTY)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_N);
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&sm.full[stage], phase, sm.abort_flag, SITE_MMA_FULL)) {
                         ok = false;
                         break;
@@ -630,7 +757,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // advance the start address by k * 32 bytes inside the swizzle row
                         const uint64_t adv = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        umma_f8f6f4(d_tmem, a_desc + adv, b_desc + adv, p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                        umma_f8f6f4(d_tmem, a_desc + adv, b_desc + adv, p.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit(&sm.empty[stage]);
                     if (++stage == S1_STAGES) {
@@ -646,7 +773,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         __syncwarp();
     } else {
-        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u);
+        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u, 0);
     }
 
     tc_fence_before();
@@ -678,7 +805,6 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     const int lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    const int num_tiles = p.tiles_m * p.tiles_n;
     const int cluster_id = blockIdx.x >> 1;
     const int num_clusters = gridDim.x >> 1;
 
@@ -719,12 +845,14 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             uint32_t phase = 0;
             int64_t issued = 0;
             bool ok = true;
-            for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+            Sched sched(p, cluster_id, num_clusters);
+            int tile, kb0, kb1;
+            while (ok && sched.next(tile, kb0, kb1)) {
                 int m_blk, n_blk;
                 tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
                 const int32_t a_row = m_blk * M_SUB * 2 * S2_BM + static_cast<int32_t>(rank) * S2_BM;
                 const int32_t b_row = n_blk * ACC_N + static_cast<int32_t>(rank) * S2_BN_HALF;
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&sm.empty[stage], phase ^ 1u, sm.abort_flag, SITE_PRODUCER_EMPTY)) {
                         ok = false;
                         break;
@@ -759,15 +887,18 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             uint32_t phase = 0;
             bool ok = true;
             int local = 0;
-            for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters, ++local) {
+            Sched sched(p, cluster_id, num_clusters);
+            int tile, kb0, kb1;
+            while (ok && sched.next(tile, kb0, kb1)) {
                 const int acc = ACC_BUFS == 2 ? (local & 1) : 0;
                 const uint32_t acc_phase = static_cast<uint32_t>(ACC_BUFS == 2 ? (local >> 1) : local) & 1u;
+                ++local;
                 if (!mbar_wait(&sm.tempty[acc], acc_phase ^ 1u, sm.abort_flag, SITE_MMA_TMEM_EMPTY)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb < p.num_kb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&sm.full[stage], phase, sm.abort_flag, SITE_MMA_FULL)) {
                         ok = false;
                         break;
@@ -782,7 +913,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                             const uint64_t a_desc =
                                 sw128_kmajor_desc(smem_u32(sm.a + stage * A_STAGE + h * S2_BM * BK));
                             umma_f8f6f4_pair(tmem_base + static_cast<uint32_t>((acc + h) * ACC_N), a_desc + adv,
-                                             b_desc + adv, p.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                                             b_desc + adv, p.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
                         }
                     }
                     umma_commit_pair_to(&sm.empty[stage], 0x3);
@@ -799,7 +930,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         __syncwarp();
     } else {
         epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, M_SUB,
-                                2 * S2_BM, static_cast<int>(rank) * S2_BM, ACC_BUFS, 0u);
+                                2 * S2_BM, static_cast<int>(rank) * S2_BM, ACC_BUFS, 0u, static_cast<int>(rank));
     }
 
     tc_fence_before();
@@ -898,9 +1029,16 @@ cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
 
 }  // namespace
 
+size_t gemm_workspace_bytes() {
+    static int cached[64] = {};
+    const int pairs = max_pairs(fp8_gemm_2sm_kernel<true, 1>, Pair<1>::SMEM, cached);
+    return WS_FLAG_BYTES + static_cast<size_t>(pairs) * 2 * WS_SLOT_FLOATS * sizeof(float);
+}
+
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
                          fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
-                         void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, cudaStream_t stream) {
+                         void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, void *workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
     const bool out_bf16 = d_dtype == FP8DS_BF16;
     const bool pair = m > S1_BM;
     // Long contractions amortise the non-overlapped epilogue of the 512-row
@@ -929,6 +1067,26 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.tiles_n = static_cast<int32_t>((n + ACC_N - 1) / ACC_N);
     p.num_kb = static_cast<int32_t>((k + BK - 1) / BK);
     p.idesc = make_idesc(a_fmt, b_fmt, pair ? 2 * S2_BM : S1_BM, ACC_N);
+    p.stream_k = 0;
+    p.epoch = 0;
+    p.flags = nullptr;
+    p.partials = nullptr;
+    if (pair && workspace != nullptr && workspace_bytes >= gemm_workspace_bytes()) {
+        // Stream-K when whole tiles would leave a ragged last wave: at least
+        // one tile per pair, fewer than 8 waves, not a whole number of waves.
+        static int cached[64] = {};
+        const int cap = max_pairs(fp8_gemm_2sm_kernel<true, 1>, Pair<1>::SMEM, cached);
+        const int tiles = p.tiles_m * p.tiles_n;
+        if (tiles >= cap && tiles % cap != 0 && tiles < 8 * cap && cap <= static_cast<int>(WS_FLAG_BYTES / 8)) {
+            static std::atomic<uint32_t> launches{0};
+            uint32_t e = ++launches;
+            if (e == 0) e = ++launches;
+            p.stream_k = 1;
+            p.epoch = e;
+            p.flags = static_cast<int32_t *>(workspace);
+            p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + WS_FLAG_BYTES);
+        }
+    }
     cudaError_t e;
     if (pair && m_sub == 2)
         e = out_bf16 ? launch_2sm<true, 2>(ta, tb, td, p, stream) : launch_2sm<false, 2>(ta, tb, td, p, stream);

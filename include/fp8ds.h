@@ -36,6 +36,7 @@
 #ifndef FP8DS_H
 #define FP8DS_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -155,6 +156,38 @@ fp8ds_status fp8_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale
                       int64_t m, int64_t n, int64_t k, fp8ds_stream stream);
 
 /*
+ * fp8_gemm_workspace_size -- bytes of workspace that let fp8_gemm_ex use the
+ * stream-K schedule on the current device (a few tens of MB on B200).  Host
+ * only; no device work.
+ */
+fp8ds_status fp8_gemm_workspace_size(size_t *bytes);
+
+/*
+ * fp8_gemm_ex -- fp8_gemm with a caller-owned device workspace.  When the
+ * tile count would leave a ragged last wave of CTA pairs, every pair then
+ * takes an equal share of the (tile, k-block) work ("stream-K"); a tile split
+ * between two pairs is combined through the workspace: one pair stores its
+ * fp32 partial accumulator there and publishes it, the other adds it before
+ * the epilogue.  The result satisfies the same bounds as fp8_gemm (the two
+ * partials are added in fp32).  On B200 under the 1 kW power cap the
+ * whole-tile schedule of fp8_gemm measured faster for 8192 x 2048 x 8192
+ * class shapes (idle SMs in the last wave let the busy ones clock higher);
+ * the stream-K schedule is for cases where a profile shows the ragged last
+ * wave dominating.
+ *   workspace  16-byte aligned device memory of at least
+ *              fp8_gemm_workspace_size() bytes, ZERO-FILLED before its first
+ *              use; the library leaves its publication words at zero after
+ *              every completed call.  NULL (or fewer bytes) means fp8_gemm.
+ *              Calls that may run concurrently must not share a workspace.
+ * Errors: as fp8_gemm; FP8DS_ERR_INVALID_ARG for an unaligned workspace.
+ */
+fp8ds_status fp8_gemm_ex(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
+                         const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
+                         const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
+                         int64_t m, int64_t n, int64_t k, void *workspace, size_t workspace_bytes,
+                         fp8ds_stream stream);
+
+/*
  * Packed FP8 meta of T tensors (the DelayedScaling state [TE761; F8E312
  * _amax_history_buffer / _scale_buffer]).  All arrays are caller-owned device
  * memory; amax_history is [hist_len, num_tensors] slot-major, zero-filled and
@@ -188,6 +221,8 @@ typedef struct {
     float *w_scale_inv;        /* [1] private scale_inv of the cached weight */
     int32_t meta_in, meta_w, meta_grad;
     int32_t cache_valid;
+    void *workspace;           /* NULL or the GEMM workspace of fp8_gemm_ex */
+    size_t workspace_bytes;
 } fp8ds_linear;
 
 /*

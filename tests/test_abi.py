@@ -30,6 +30,7 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("fp8_quantize", "fp8_cast_transpose_amax", "fp8_update_scales", "fp8_gemm",
+              "fp8_gemm_ex", "fp8_gemm_workspace_size",
               "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
               "fp8ds_version"):
         assert n in names
@@ -69,6 +70,11 @@ def test_gemm_argument_checks(lib):
     assert call(a=FAKE_ODD) == lib.ERR_INVALID_ARG and "aligned" in lib.fp8ds_last_error()
     assert call(fa=7) == lib.ERR_INVALID_ARG
     assert call(m=1 << 31) == lib.ERR_INVALID_ARG
+    # the workspace variant checks the same arguments plus the workspace alignment
+    assert L.fp8_gemm_ex(FAKE, 0, FAKE, FAKE, 0, FAKE, None, 0, FAKE, 1, 128, 256, 120, FAKE, 64, s) == \
+        lib.ERR_INVALID_ARG
+    assert L.fp8_gemm_ex(FAKE, 0, FAKE, FAKE, 0, FAKE, None, 0, FAKE, 1, 128, 256, 128, FAKE_ODD, 64, s) == \
+        lib.ERR_INVALID_ARG and "workspace" in lib.fp8ds_last_error()
 
 
 def test_cast_and_update_argument_checks(lib):
@@ -92,11 +98,11 @@ def test_linear_argument_checks(lib):
     L = lib._lib
     s = P(0)
     meta = lib._Meta(FAKE, FAKE, FAKE, FAKE, 3, 16)
-    lin = lib._Linear(FAKE, None, 0, 256, 512, FAKE, FAKE, FAKE, 0, 1, 2, 0)
+    lin = lib._Linear(FAKE, None, 0, 256, 512, FAKE, FAKE, FAKE, 0, 1, 2, 0, None, 0)
     r = L.fp8_linear_fwd(ctypes.byref(lin), ctypes.byref(meta), FAKE, 0, 128, FAKE, 0, 2, FAKE,
                          FAKE, FAKE, s)
     assert r == lib.ERR_INVALID_ARG and "is_first_microbatch" in lib.fp8ds_last_error()
-    bad = lib._Linear(FAKE, None, 0, 256, 512, FAKE, FAKE, FAKE, 0, 7, 2, 0)
+    bad = lib._Linear(FAKE, None, 0, 256, 512, FAKE, FAKE, FAKE, 0, 7, 2, 0, None, 0)
     r = L.fp8_linear_fwd(ctypes.byref(bad), ctypes.byref(meta), FAKE, 0, 128, FAKE, 0, 1, FAKE,
                          FAKE, FAKE, s)
     assert r == lib.ERR_INVALID_ARG and "out of range" in lib.fp8ds_last_error()

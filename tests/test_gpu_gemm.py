@@ -170,3 +170,70 @@ def test_gemm_repeatable(fp8):
     d1 = _run(fp8, a, "e4m3", sa, b, "e4m3", sb, torch.float32)
     d2 = _run(fp8, a, "e4m3", sa, b, "e4m3", sb, torch.float32)
     assert torch.equal(d1.view(torch.int32), d2.view(torch.int32))
+
+
+# ------------------------------------------------------------------ stream-K --
+# With a workspace, shapes whose pair tiles would leave a ragged last wave run
+# the stream-K schedule: every pair takes an equal share of the (tile,
+# k-block) work and tiles split between two pairs are combined through the
+# workspace.  (4096, 2048, 256): 128 tiles of 256x256; (4608, 2304, 4096):
+# 81 tiles of 512x256; both have more tiles than the 74 pairs of a B200 and
+# are not whole waves.
+
+@pytest.fixture(scope="module")
+def ws(fp8):
+    return fp8.gemm_workspace()
+
+
+def _flags_clear(ws):
+    return int(ws[:4096].view(torch.int32).abs().sum().item()) == 0
+
+
+@pytest.mark.parametrize("shape", [(4096, 2048, 256), (4608, 2304, 4096)])
+@pytest.mark.parametrize("fa,fb", [("e4m3", "e4m3"), ("e5m2", "e4m3")])
+def test_gemm_stream_k_integer_exact(fp8, ws, shape, fa, fb):
+    """Integer operands: every partial sum, and the sum of two partials, is
+    exact in fp32, so the split tiles must reproduce the exact product."""
+    M, N, K = shape
+    a, av = _integer_codes((M, K), fa, 15)
+    b, bv = _integer_codes((N, K), fb, 16)
+    d = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    fp8.fp8_gemm_ex(dev(a), fa, torch.tensor([0.5], device="cuda"), dev(b), fb,
+                    torch.tensor([4.0], device="cuda"), d, workspace=ws)
+    torch.cuda.synchronize()
+    assert fp8.fp8ds_device_status() == 0
+    ref = (torch.from_numpy(av).double() @ torch.from_numpy(bv).double().T) * 2.0
+    got = d.cpu().double()
+    bad = torch.nonzero(got != ref)
+    assert bad.shape[0] == 0, "mismatches at %s" % bad[:5].tolist()
+    assert _flags_clear(ws)
+
+
+@pytest.mark.parametrize("shape", [(8192, 2048, 8192), (2048, 8192, 8192), (4096, 2048, 256)])
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_gemm_stream_k_realistic(fp8, ws, shape, out_dtype):
+    M, N, K = shape
+    a, b, sa, sb = _realistic_operands(M, N, K, "e4m3", "e4m3", seed=21)
+    rows = _rows_for(M, N, K)
+    ref = o.gemm(a, o.E4M3, b, o.E4M3, sa, sb, rows=rows)
+    d = torch.full((M, N), float("nan"), dtype=out_dtype, device="cuda")
+    fp8.fp8_gemm_ex(dev(a), "e4m3", torch.tensor([sa], device="cuda"), dev(b), "e4m3",
+                    torch.tensor([sb], device="cuda"), d, workspace=ws)
+    torch.cuda.synchronize()
+    assert fp8.fp8ds_device_status() == 0
+    _compare(d, ref, rows, out_dtype, "stream-K %s" % (shape,), (a, "e4m3", b, "e4m3", sa, sb))
+    assert _flags_clear(ws)
+
+
+def test_gemm_stream_k_repeatable(fp8, ws):
+    """The split tiles are combined in a fixed order: same bits every run."""
+    a, b, sa, sb = _realistic_operands(4096, 2048, 256, "e4m3", "e4m3", seed=22)
+    outs = []
+    for _ in range(3):
+        d = torch.empty(4096, 2048, dtype=torch.float32, device="cuda")
+        fp8.fp8_gemm_ex(dev(a), "e4m3", torch.tensor([sa], device="cuda"), dev(b), "e4m3",
+                        torch.tensor([sb], device="cuda"), d, workspace=ws)
+        outs.append(d)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0].view(torch.int32), outs[1].view(torch.int32))
+    assert torch.equal(outs[0].view(torch.int32), outs[2].view(torch.int32))
