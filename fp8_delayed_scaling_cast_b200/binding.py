@@ -66,6 +66,7 @@ _SIGS = {
     "fp8_gemm_ex": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P,
                     ctypes.c_size_t, _P],
     "fp8_gemm_workspace_size": [ctypes.POINTER(ctypes.c_size_t)],
+    "fp8_gemm_noalloc": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
     "fp8_linear_fwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _INT,
                        _I32, _P, _P, _P, _P],
     "fp8_linear_bwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P,
@@ -151,6 +152,14 @@ def fp8_gemm_ex(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, d, bias=None, work
     _check(_lib.fp8_gemm_ex(_ptr(a), _fmt(a_fmt), _ptr(a_scale_inv), _ptr(b), _fmt(b_fmt),
                             _ptr(b_scale_inv), _ptr(bias), F32 if bias is None else _dtype(bias),
                             _ptr(d), _dtype(d), m, n, k, _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def fp8_gemm_noalloc(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, d, bias=None, stream=None):
+    m, k = a.shape
+    n = b.shape[0]
+    _check(_lib.fp8_gemm_noalloc(_ptr(a), _fmt(a_fmt), _ptr(a_scale_inv), _ptr(b), _fmt(b_fmt),
+                                 _ptr(b_scale_inv), _ptr(bias), F32 if bias is None else _dtype(bias),
+                                 _ptr(d), _dtype(d), m, n, k, _stream(stream)))
 
 
 def fp8_gemm_workspace_size():

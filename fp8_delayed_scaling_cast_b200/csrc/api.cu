@@ -204,6 +204,17 @@ fp8ds_status fp8_gemm_ex(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
                        workspace_bytes, stream);
 }
 
+fp8ds_status fp8_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
+                              fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
+                              void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, fp8ds_stream stream) {
+    clear_error();
+    fp8ds_status st =
+        check_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k);
+    if (st != FP8DS_OK) return st;
+    return launch_gemm_noalloc(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k,
+                               stream);
+}
+
 fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x, fp8ds_dtype x_dtype,
                             int64_t m, void *y, fp8ds_dtype y_dtype, int32_t is_first_microbatch, uint8_t *x8,
                             uint8_t *x8t, float *x_scale_inv, fp8ds_stream stream) {

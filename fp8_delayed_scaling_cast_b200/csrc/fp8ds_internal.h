@@ -44,6 +44,12 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
 // Workspace bytes the stream-K schedule needs on the current device.
 size_t gemm_workspace_bytes();
 
+// launch_gemm with the library's static device scratch as the workspace.
+fp8ds_status launch_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
+                                 const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
+                                 const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
+                                 int64_t m, int64_t n, int64_t k, cudaStream_t stream);
+
 // Device error words written by kernels whose bounded waits give up (one per
 // translation unit); read_device_error returns the first non-zero one.
 cudaError_t read_device_error(int32_t *out, bool clear);

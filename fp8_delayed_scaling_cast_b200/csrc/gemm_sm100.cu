@@ -1101,6 +1101,64 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     return FP8DS_OK;
 }
 
+// ------------------------------------------- allocation-free GEMM variant --
+
+// Scratch of fp8_gemm_noalloc: the stream-K workspace (publication words and
+// partial-accumulator slots) as a file-scope device array, so that callers
+// that may not allocate device memory still get the split-tile schedule.
+// Every device that loads the library holds these bytes until the process
+// exits.  80 MiB covers the 74 CTA pairs of a B200 (4 KiB of words + 1 MiB
+// per pair).
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(80) << 20;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+fp8ds_status launch_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
+                                 fp8ds_format b_fmt, const float *b_scale_inv, const void *bias,
+                                 fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k,
+                                 cudaStream_t stream) {
+    // Device address of the scratch, looked up once per device with that
+    // device current (host code cannot use the array's name as an address).
+    static void *scratch[64] = {};
+    static std::mutex lock;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        set_error("fp8_gemm_noalloc: no usable current device (%s)", cudaGetErrorString(e));
+        return FP8DS_ERR_CUDA;
+    }
+    void *ws = nullptr;
+    {
+        std::lock_guard<std::mutex> g(lock);
+        if (scratch[dev] == nullptr) {
+            void *ptr = nullptr;
+            e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+            if (e != cudaSuccess || ptr == nullptr) {
+                set_error("fp8_gemm_noalloc: cudaGetSymbolAddress of the static scratch failed: %s",
+                          cudaGetErrorString(e));
+                return FP8DS_ERR_CUDA;
+            }
+            scratch[dev] = ptr;
+        }
+        ws = scratch[dev];
+    }
+    const size_t need = gemm_workspace_bytes();
+    if (need > NOALLOC_SCRATCH_BYTES) {
+        set_error("fp8_gemm_noalloc: this device needs %zu bytes of stream-K scratch, more than the %zu-byte static "
+                  "scratch (use fp8_gemm_ex with a workspace)",
+                  need, NOALLOC_SCRATCH_BYTES);
+        return FP8DS_ERR_INVALID_ARG;
+    }
+    // The array keeps whatever the previous call left: the publication words
+    // must start at zero.
+    e = cudaMemsetAsync(ws, 0, WS_FLAG_BYTES, stream);
+    if (e != cudaSuccess) {
+        set_error("fp8_gemm_noalloc: clearing the scratch failed: %s", cudaGetErrorString(e));
+        return FP8DS_ERR_CUDA;
+    }
+    return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k, ws,
+                       NOALLOC_SCRATCH_BYTES, stream);
+}
+
 cudaError_t read_gemm_error(int32_t *out, bool clear) {
     cudaError_t e = cudaMemcpyFromSymbol(out, g_device_error, sizeof(int32_t));
     if (e != cudaSuccess || !clear) return e;

@@ -188,6 +188,32 @@ fp8ds_status fp8_gemm_ex(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
                          fp8ds_stream stream);
 
 /*
+ * fp8_gemm_noalloc -- fp8_gemm_ex for callers that cannot allocate device
+ * memory: the stream-K scratch is an 80 MiB array inside the library (held by
+ * every device that loads it until the process exits) instead of a workspace
+ * argument.  The pages have no counterpart; it exists because some callers
+ * must not call cudaMalloc -- for example a program whose device memory is
+ * all handed to a framework's caching allocator or reserved by a serving
+ * engine at start-up, or C code that only receives tensor pointers and owns
+ * no allocator -- yet want the same GEMM.
+ *   Arguments, layouts and results as fp8_gemm.  Calls no allocator (no
+ *   cudaMalloc/cudaFree, no library routine that allocates); it only enqueues
+ *   a 4 KiB memset of the scratch's publication words and the GEMM on
+ *   `stream`.
+ *   The first call on a device looks up the scratch's device address (a
+ *   runtime query, done once per device with that device current); make that
+ *   first call before any stream capture on the device.
+ *   All calls share the one scratch: calls that may overlap on the GPU (other
+ *   streams, other threads) race and must be ordered by the caller.
+ * Errors: as fp8_gemm; FP8DS_ERR_INVALID_ARG if the device needs more
+ * stream-K scratch than the 80 MiB array holds (more than 79 CTA pairs).
+ */
+fp8ds_status fp8_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
+                              const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
+                              const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
+                              int64_t m, int64_t n, int64_t k, fp8ds_stream stream);
+
+/*
  * Packed FP8 meta of T tensors (the DelayedScaling state [TE761; F8E312
  * _amax_history_buffer / _scale_buffer]).  All arrays are caller-owned device
  * memory; amax_history is [hist_len, num_tensors] slot-major, zero-filled and

@@ -70,6 +70,9 @@ def test_gemm_argument_checks(lib):
     assert call(a=FAKE_ODD) == lib.ERR_INVALID_ARG and "aligned" in lib.fp8ds_last_error()
     assert call(fa=7) == lib.ERR_INVALID_ARG
     assert call(m=1 << 31) == lib.ERR_INVALID_ARG
+    # the allocation-free variant checks the same arguments before anything else
+    assert L.fp8_gemm_noalloc(FAKE, 0, FAKE, FAKE, 0, FAKE, None, 0, FAKE, 1, 128, 256, 120, s) == \
+        lib.ERR_INVALID_ARG and "multiple of 16" in lib.fp8ds_last_error()
     # the workspace variant checks the same arguments plus the workspace alignment
     assert L.fp8_gemm_ex(FAKE, 0, FAKE, FAKE, 0, FAKE, None, 0, FAKE, 1, 128, 256, 120, FAKE, 64, s) == \
         lib.ERR_INVALID_ARG
