@@ -44,6 +44,7 @@ def lib():
         L.orc_cast_transpose_amax.argtypes = [P, ctypes.c_int, i64, i64, ctypes.c_int, f32,
                                               P, P, P, P]
         L.orc_quantize.argtypes = [P, ctypes.c_int, i64, ctypes.c_int, f32, P, P, P]
+        L.orc_amax.argtypes = [P, ctypes.c_int, i64, P]
         L.orc_update_scales.argtypes = [i64, ctypes.c_int, P, P, P, P]
         L.orc_gemm_rows.argtypes = [P, ctypes.c_int, P, ctypes.c_int, f32, f32, P,
                                     i64, i64, i64, P, i64, P]
@@ -126,6 +127,14 @@ def quantize(x, fmt, scale, amax=0.0):
     si = np.zeros(1, np.float32)
     lib().orc_quantize(_ptr(x), tag, x.size, fmt, float(scale), _ptr(y), _ptr(am), _ptr(si))
     return y, am[0], si[0]
+
+
+def amax(x, amax=0.0):
+    """max(amax, max|x|) over the unscaled input, NaN ignored (float32)."""
+    x, tag = _as_input(x)
+    am = np.array([amax], np.float32)
+    lib().orc_amax(_ptr(x), tag, x.size, _ptr(am))
+    return am[0]
 
 
 def update_scales(hist, scale, scale_inv, fmts):

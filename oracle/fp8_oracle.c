@@ -189,6 +189,18 @@ void orc_quantize(const void *x, int xdtype, int64_t n, int fmt, float scale, ui
     orc_cast_transpose_amax(x, xdtype, 1, n, fmt, scale, y, NULL, amax, scale_inv_out);
 }
 
+/*
+ * The amax alone: *amax = max(*amax, max |x|) over n elements, NaN ignored --
+ * the reduction the cast above records, without producing codes.  Full-size
+ * checks use it for tensors whose complete cast would take minutes here.
+ */
+void orc_amax(const void *x, int xdtype, int64_t n, float *amax)
+{
+    float m = *amax;
+    for (int64_t i = 0; i < n; ++i) m = max_ignoring_nan(m, fabsf(load_elem(x, xdtype, i)));
+    *amax = m;
+}
+
 /* --------------------------------------------------------------- update -- */
 
 /*

@@ -224,11 +224,33 @@ def test_amax_ignores_every_nan_pattern():
     v = o.bf16_bits_to_f32(bits)
     _, am, _ = o.quantize(bits, o.E4M3, 1.0)
     assert am == np.nanmax(np.abs(v)) and np.isinf(am)
+    # the amax-only reduction over the same patterns, and over the finite ones
+    assert o.amax(bits) == am
+    finite = bits[np.isfinite(v)]
+    assert o.amax(finite) == np.float32(np.abs(o.bf16_bits_to_f32(finite)).max()) == np.float32(3.3895314e38)
     # a history window containing NaN entries ignores them as well
     hist = np.zeros((4, 1), np.float32)
     hist[:, 0] = [np.float32(2.0), np.uint32(0x7F810000).view(np.float32), np.nan, 1.0]
     _, s2, _ = o.update_scales(hist, [1.0], [1.0], [0])
     assert s2[0] == np.float32(224.0)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_amax_alone(dtype):
+    """max|x| of the unscaled input (numpy), a running value kept when larger,
+    NaN skipped wherever it sits (first element included), empty input."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((301, 7)) * 4).astype(np.float32)
+    x[100, 3] = -768.0
+    xin = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16) if dtype == "bf16" else x
+    xf = o.bf16_bits_to_f32(xin) if dtype == "bf16" else x
+    assert o.amax(xin) == np.float32(np.abs(xf).max()) == np.float32(768.0)
+    assert o.amax(xin, amax=1000.0) == np.float32(1000.0)
+    xn = np.array(xin, copy=True)
+    xn.flat[0] = np.uint16(0x7FC1) if dtype == "bf16" else np.float32(np.nan)
+    xn.flat[-1] = np.uint16(0xFF81) if dtype == "bf16" else np.float32(-np.nan)
+    assert o.amax(xn) == np.float32(768.0)
+    assert o.amax(xin[:0]) == np.float32(0.0)
 
 
 def test_quantize_is_flat_cast():
