@@ -66,59 +66,125 @@ def peaks():
 # ------------------------------------------------------------------ clocks --
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """SM clock and clock-event reasons sampled during the timed region.
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NVML is polled every 2 ms on a host thread; only the samples taken between
+    mark_start() and mark_end() (host times around the timed launches and the
+    synchronize that ends them) count.  Without NVML it falls back to
+    `nvidia-smi -lms 20` over the same window.
+    """
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device):
-        self.proc = None
-        self.out = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        import threading
+        self.samples = []           # (host time, sm MHz, set of reason names)
+        self.t0 = self.t1 = None
+        self.max_mhz = None
+        self.src = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
         try:
-            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
         except Exception:
-            self.uuid = None
+            uuid = None
+        self.uuid = uuid
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.src = "nvml"
+        except Exception:
+            self.nv = None
+
+    def _poll_nvml(self):
+        nv = self.nv
+        bits = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+        while not self._stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, {n for n, b in bits if r & b}))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def start(self):
-        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits", "-lms", "20"]
+        import threading
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self._thread.start()
+            return
+        cmd = ["nvidia-smi", "--query-gpu=" + self.SMI_FIELDS, "--format=csv,noheader,nounits", "-lms", "20"]
         if self.uuid:
             cmd[1:1] = ["-i", self.uuid]
         try:
-            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+            self._out = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+            self._proc = subprocess.Popen(cmd, stdout=self._out, stderr=subprocess.DEVNULL)
+            self._proc_t0 = time.perf_counter()
+            self.src = "nvidia-smi"
         except Exception:
-            self.proc = None
+            self._proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
-        self.proc.terminate()
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
+    def _read_smi(self):
+        # nvidia-smi lines carry no host time: spread them evenly over the
+        # sampler's lifetime and keep those inside the window
+        self._proc.terminate()
         try:
-            self.proc.wait(timeout=5)
+            self._proc.wait(timeout=5)
         except Exception:
-            self.proc.kill()
-        self.out.flush()
-        self.out.seek(0)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.out.read().splitlines():
+            self._proc.kill()
+        t_end = time.perf_counter()
+        self._out.flush()
+        self._out.seek(0)
+        lines = [ln for ln in self._out.read().splitlines() if ln.count(",") >= 5]
+        os.unlink(self._out.name)
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for idx, line in enumerate(lines):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 8:
-                continue
             try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
+                mhz, mx = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
-            for name, val in zip(names, parts[4:8]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        os.unlink(self.out.name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+            self.max_mhz = mx if self.max_mhz is None else max(self.max_mhz, mx)
+            t = self._proc_t0 + (t_end - self._proc_t0) * (idx + 0.5) / len(lines)
+            self.samples.append((t, mhz, {n for n, v in zip(names, parts[2:6]) if v.lower().startswith("active")}))
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=5)
+        elif self._proc is not None:
+            self._read_smi()
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock source"]}
+        inside = [(m, r) for t, m, r in self.samples
+                  if self.t0 is not None and self.t1 is not None and self.t0 <= t <= self.t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples in the timed region"],
+                    "source": self.src}
+        reasons = set()
+        for _, r in inside:
+            reasons |= r
+        return {"sm_mhz": statistics.median(m for m, _ in inside), "sm_min_mhz": min(m for m, _ in inside),
+                "sm_max_mhz": self.max_mhz, "samples": len(inside), "reasons": sorted(reasons),
+                "source": self.src}
 
 
 # --------------------------------------------------------------- the step --
@@ -503,15 +569,19 @@ def main():
     clocks = ClockSampler(device) if rank == 0 else None
     if clocks:
         clocks.start()
-        time.sleep(0.3)
+        time.sleep(0.1)
     barrier_sync(world)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    if clocks:
+        clocks.mark_start()
     t_start.record()
     for i in range(args.steps):
         step.run_linear_api(i, sync_amax=sync)
     t_end.record()
     barrier_sync(world)
+    if clocks:
+        clocks.mark_end()
     clock_info = clocks.stop() if clocks else None
     ms_local = t_start.elapsed_time(t_end) / args.steps
     ms = max_over_ranks(ms_local, world, device)

@@ -63,20 +63,41 @@ def spiky_bf16(rows=TOKENS, cols=HIDDEN, seed=0, spike_frac=1e-3, spike_mult=100
     return x.to(torch.bfloat16)
 
 
-def teblock_weights(seed=0, blocks=1, scale=1):
-    """fp32 master weights [out, in] and biases of `blocks` TEBlocks, block-major.
+def iter_teblock_weights(seed=0, blocks=1, scale=1):
+    """Yield (fp32 master weight [out, in], bias or None) of `blocks` TEBlocks,
+    block-major, one linear at a time (so a large model need not sit on the
+    host all at once).
 
     `scale` divides every feature size (tests use it to shrink the block while
     keeping its structure).  Biases come from a second generator (seed + 1).
     """
     g = gen(seed)
     gb = gen(seed + 1)
-    ws, bs = [], []
     for _ in range(blocks):
         for out_f, in_f, has_bias in TEBLOCK_LINEARS:
-            ws.append(normal((out_f // scale, in_f // scale), g, 0.02))
-            bs.append(normal((out_f // scale,), gb, 0.02) if has_bias else None)
+            w = normal((out_f // scale, in_f // scale), g, 0.02)
+            yield w, (normal((out_f // scale,), gb, 0.02) if has_bias else None)
+
+
+def teblock_weights(seed=0, blocks=1, scale=1):
+    """Lists (weights, biases) of iter_teblock_weights (same bytes)."""
+    ws, bs = [], []
+    for w, b in iter_teblock_weights(seed, blocks, scale):
+        ws.append(w)
+        bs.append(b)
     return ws, bs
+
+
+def teblock_microbatch(mb, seed=0, tokens=TOKENS, hidden=HIDDEN):
+    """TEBlock input of microbatch `mb`: X ~ U[0,1) fp32 [tokens, hidden] from
+    generator 2000 + mb + seed (each microbatch can be regenerated alone)."""
+    return uniform((tokens, hidden), gen(2000 + mb + seed))
+
+
+def toy_step_input(step, seed=0, tokens=TOKENS, hidden=HIDDEN):
+    """Input of forward step `step` of the 32-block model: X ~ U[0,1) fp32
+    [tokens, hidden] from generator 3000 + step + seed."""
+    return uniform((tokens, hidden), gen(3000 + step + seed))
 
 
 def mlp_pair(seed=0, tokens=TOKENS, hidden=HIDDEN, ratio=MLP_RATIO):

@@ -30,8 +30,8 @@ def f32(t):
 
 
 def assert_bytes_equal(got, want, what):
-    got = np.asarray(got)
-    want = np.asarray(want)
+    got = np.atleast_1d(np.asarray(got))
+    want = np.atleast_1d(np.asarray(want))
     assert got.shape == want.shape, (what, got.shape, want.shape)
     bad = np.nonzero(got != want)
     if bad[0].size:
