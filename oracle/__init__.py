@@ -46,6 +46,7 @@ def lib():
         L.orc_quantize.argtypes = [P, ctypes.c_int, i64, ctypes.c_int, f32, P, P, P]
         L.orc_amax.argtypes = [P, ctypes.c_int, i64, P]
         L.orc_update_scales.argtypes = [i64, ctypes.c_int, P, P, P, P]
+        L.orc_update_scales_algo.argtypes = [i64, ctypes.c_int, P, P, P, P, ctypes.c_int]
         L.orc_gemm_rows.argtypes = [P, ctypes.c_int, P, ctypes.c_int, f32, f32, P,
                                     i64, i64, i64, P, i64, P]
         L.orc_round_bf16.restype = ctypes.c_uint16
@@ -137,14 +138,20 @@ def amax(x, amax=0.0):
     return am[0]
 
 
-def update_scales(hist, scale, scale_inv, fmts):
-    """One delayed-scaling update over T metas; returns new (hist, scale, scale_inv)."""
+AMAX_MAX = 0
+AMAX_MOST_RECENT = 1
+
+
+def update_scales(hist, scale, scale_inv, fmts, algo=AMAX_MAX):
+    """One delayed-scaling update over T metas; returns new (hist, scale, scale_inv).
+    algo: AMAX_MAX (max over the history window) or AMAX_MOST_RECENT (the
+    current step's amax)."""
     hist = np.array(hist, np.float32, copy=True, order="C")
     scale = np.array(scale, np.float32, copy=True)
     scale_inv = np.array(scale_inv, np.float32, copy=True)
     fmts = np.ascontiguousarray(fmts, dtype=np.uint8)
     H, T = hist.shape
-    lib().orc_update_scales(T, H, _ptr(hist), _ptr(scale), _ptr(scale_inv), _ptr(fmts))
+    lib().orc_update_scales_algo(T, H, _ptr(hist), _ptr(scale), _ptr(scale_inv), _ptr(fmts), int(algo))
     return hist, scale, scale_inv
 
 

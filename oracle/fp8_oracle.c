@@ -204,10 +204,12 @@ void orc_amax(const void *x, int xdtype, int64_t n, float *amax)
 /* --------------------------------------------------------------- update -- */
 
 /*
- * Delayed-scaling update of T meta tensors, amax_compute_algo = "max".
+ * Delayed-scaling update of T meta tensors.
  * History layout: hist[h * T + t], h = 0..H-1 (slot 0 holds the amax recorded
  * in the current step).  Per tensor t:
- *   a      = max_h hist[h][t]
+ *   a      = max_h hist[h][t]            amax_compute_algo = "max" (algo 0)
+ *            hist[0][t]                   "most_recent" (algo 1): the current
+ *                                         step's amax alone
  *   scale' = fl32(fp8_max / a)  if a > 0, a finite and the quotient finite;
  *            otherwise the previous scale is kept
  *   scale_inv = fl32(1 / scale')
@@ -215,12 +217,13 @@ void orc_amax(const void *x, int xdtype, int64_t n, float *amax)
  * After the roll slot H-1 holds the current amax and slot 0 is clear for the
  * next step, so each max is over exactly the last H recorded amaxes.
  */
-void orc_update_scales(int64_t T, int H, float *hist, float *scale, float *scale_inv,
-                       const uint8_t *fmts)
+void orc_update_scales_algo(int64_t T, int H, float *hist, float *scale, float *scale_inv,
+                            const uint8_t *fmts, int algo)
 {
     for (int64_t t = 0; t < T; ++t) {
         float a = hist[t];
-        for (int h = 1; h < H; ++h) a = max_ignoring_nan(a, hist[(int64_t)h * T + t]);
+        if (algo == 0)
+            for (int h = 1; h < H; ++h) a = max_ignoring_nan(a, hist[(int64_t)h * T + t]);
         double fp8_max = orc_decode((uint8_t)max_finite_code(fmts[t]), fmts[t]);
         float s = scale[t];
         if (a > 0.0f && isfinite(a)) {
@@ -234,6 +237,12 @@ void orc_update_scales(int64_t T, int H, float *hist, float *scale, float *scale
         hist[(int64_t)(H - 1) * T + t] = first;
         hist[t] = 0.0f;
     }
+}
+
+void orc_update_scales(int64_t T, int H, float *hist, float *scale, float *scale_inv,
+                       const uint8_t *fmts)
+{
+    orc_update_scales_algo(T, H, hist, scale, scale_inv, fmts, 0);
 }
 
 /* ----------------------------------------------------------- bf16 output -- */

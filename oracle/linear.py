@@ -36,9 +36,9 @@ class OracleMeta:
     def record(self, t, amax):
         self.hist[0, t] = amax
 
-    def update(self):
+    def update(self, algo=0):
         self.hist, self.scale, self.scale_inv = update_scales(
-            self.hist, self.scale, self.scale_inv, self.fmts)
+            self.hist, self.scale, self.scale_inv, self.fmts, algo)
 
 
 class OracleLinear:

@@ -308,6 +308,41 @@ def test_update_matches_brute_force_window():
     assert got[3 + H, 0] != np.float32(448.0) / np.float32(1000.0)
 
 
+def test_update_most_recent_is_a_window_of_one():
+    """amax_compute_algo "most_recent": the scale follows the current step's
+    amax alone (the brute-force window of length 1), zero amaxes keep the
+    scale, a spike is forgotten the very next step; the history rolls exactly
+    as with "max"."""
+    rng = np.random.default_rng(9)
+    H, T, steps = 16, 3, 30
+    fmts = np.array([0, 1, 0], np.uint8)
+    amax_seq = rng.uniform(0.01, 5.0, size=(steps, T)).astype(np.float32)
+    amax_seq[4, 0] = 1000.0
+    amax_seq[7:12, 2] = 0.0
+    amax_seq[20, 1] = np.inf
+    recent = o.OracleMeta(fmts, H)
+    window = o.OracleMeta(fmts, H)
+    got = []
+    for k in range(steps):
+        for t in range(T):
+            recent.record(t, amax_seq[k, t])
+            window.record(t, amax_seq[k, t])
+        recent.update(algo=o.AMAX_MOST_RECENT)
+        window.update()
+        got.append(recent.scale.copy())
+        assert np.array_equal(recent.hist.view(np.uint32), window.hist.view(np.uint32))
+        assert np.array_equal(recent.scale_inv, np.float32(1.0) / recent.scale)
+    got = np.array(got)
+    for t in range(T):
+        fmax = 448.0 if fmts[t] == 0 else 57344.0
+        ref = _brute_force_trajectory(amax_seq[:, t], fmax, 1)
+        assert np.array_equal(got[:, t], np.array(ref, np.float32)), t
+    assert got[4, 0] == np.float32(448.0) / np.float32(1000.0)
+    assert got[5, 0] == np.float32(448.0) / amax_seq[5, 0]
+    assert np.all(got[7:12, 2] == got[6, 2])          # zero amax: scale kept
+    assert got[20, 1] == got[19, 1]                   # infinite amax: scale kept
+
+
 def test_update_history_layout_closed_form():
     """After k < H steps, slots H-k..H-1 hold the k recorded amaxes oldest first
     and slot 0 is zero."""
