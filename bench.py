@@ -4,9 +4,14 @@ One step = one pass of the whole path over one batch: the forward and
 backward of the MLP pair 2048 -> 8192 -> 2048 at 8192 tokens (batch 8 x seq
 1024) with the HYBRID recipe (e4m3 forward tensors, e5m2 gradients), weights
 recast into the FP8 cache every step (is_first_microbatch=True), and one
-multi-tensor delayed-scaling update of all 6 metas (history 16).  Per step:
-6 cast+transpose+amax launches, 6 FP8 GEMMs (fwd, dgrad, wgrad of both
-linears; 1.649 TFLOP), 1 update launch.  Under torchrun every rank runs its
+multi-tensor delayed-scaling update of all 6 metas (history 16).  H (fc1's
+output) and dH (fc2's dgrad) are handed to the next GEMM in FP8: the GEMM
+epilogue casts them with the consumer's delayed scale, writes the transpose
+and records the amax (fp8_linear_fwd_ex / fp8_linear_bwd_ex), with results
+identical to the unfused calls.  Per step: 4 cast+transpose+amax launches
+(X, W1, W2, dY), 6 FP8 GEMMs (fwd, dgrad, wgrad of both linears; 1.649
+TFLOP), 1 update launch.  The unfused step (6 casts) is timed beside it and
+reported as "unfused_step".  Under torchrun every rank runs its
 own batch (data parallel, weak scaling) and the ranks max-reduce the current
 amaxes over NCCL before the update (the amax sync of delayed scaling).
 
@@ -46,6 +51,11 @@ CAST_BYTES = {
     "w2": HIDDEN * FFN * (4 + 2), "dy": TOKENS * HIDDEN * (2 + 2), "dh": TOKENS * FFN * (2 + 2),
 }
 STEP_CAST_BYTES = sum(CAST_BYTES.values())
+# With the FP8 hand-over, H and dH are cast inside the GEMM epilogues (fc1
+# forward, fc2 dgrad), which write FP8 codes + transpose (2 B per element)
+# instead of bf16 (2 B): the separate H and dH casts disappear.
+FUSED_CASTS = ("x", "w1", "w2", "dy")
+STEP_CAST_BYTES_FUSED = sum(CAST_BYTES[k] for k in FUSED_CASTS)
 C2_ROWS, C2_COLS = TOKENS, HIDDEN                  # cast-transpose-amax workload
 C2_BYTES = C2_ROWS * C2_COLS * (2 + 1 + 1)
 META_NAMES = ["fc1.in", "fc1.w", "fc1.grad", "fc2.in", "fc2.w", "fc2.grad"]
@@ -216,10 +226,26 @@ class MlpStep:
         self.dw2 = e(HIDDEN, FFN, dt=f32)
         self.si = e(4, dt=f32)  # private scale_invs of x8, h8, dy8, dh8
 
-    def run_linear_api(self, i, sync_amax=None):
-        """The step through the public linear API (what a user calls)."""
+    def run_linear_api(self, i, sync_amax=None, fused=True):
+        """The step through the public linear API (what a user calls).  fused:
+        H and dH pass between the linears in FP8, cast in the GEMM epilogues
+        (fp8_linear_fwd_ex / fp8_linear_bwd_ex); otherwise each linear casts
+        its own input and gradient (fp8_linear_fwd / fp8_linear_bwd)."""
         fp8, m = self.fp8, self.meta
         x, dy = self.xs[i % len(self.xs)], self.dys[i % len(self.dys)]
+        if fused:
+            fp8.fp8_linear_fwd_ex(self.fc1, m, x, None, True, self.x8, self.x8t, self.si[0:1], out_meta=3,
+                                  out8=self.h8, out8t=self.h8t, out_scale_inv=self.si[1:2])
+            fp8.fp8_linear_fwd_ex(self.fc2, m, None, self.y, True, self.h8, self.h8t, self.si[1:2], in_cast=True)
+            fp8.fp8_linear_bwd_ex(self.fc2, m, dy, self.h8t, self.si[1:2], self.dw2, self.dy8, self.dy8t,
+                                  self.si[2:3], out_meta=2, out8=self.dh8, out8t=self.dh8t,
+                                  out_scale_inv=self.si[3:4])
+            fp8.fp8_linear_bwd_ex(self.fc1, m, None, self.x8t, self.si[0:1], self.dw1, self.dh8, self.dh8t,
+                                  self.si[3:4], dx=self.dx, in_cast=True)
+            if sync_amax is not None:
+                sync_amax(m.amax_history[0])
+            m.update()
+            return
         fp8.fp8_linear_fwd(self.fc1, m, x, self.h, True, self.x8, self.x8t, self.si[0:1])
         fp8.fp8_linear_fwd(self.fc2, m, self.h, self.y, True, self.h8, self.h8t, self.si[1:2])
         fp8.fp8_linear_bwd(self.fc2, m, dy, self.h8t, self.si[1:2], self.dw2, self.dy8, self.dy8t,
@@ -230,7 +256,7 @@ class MlpStep:
             sync_amax(m.amax_history[0])
         m.update()
 
-    def run_kernels(self, i, ev=None, sync_amax=None):
+    def run_kernels(self, i, ev=None, sync_amax=None, fused=True):
         """The same launches as run_linear_api, issued one C call per kernel so
         that CUDA events can bracket each one.  ev(kind, key) returns a callable
         recorded after the launch, or None."""
@@ -250,17 +276,33 @@ class MlpStep:
             if h0:
                 h0()
 
+        def gemm_cast(key, a, fa, sa, b, fb, sb, out_fmt, t, d8, d8t, si, bias=None):
+            h0 = mark("gemm", key)
+            fp8.fp8_gemm_cast(a, fa, sa, b, fb, sb, out_fmt, m.scale[t:t + 1], d8, d8t,
+                              m.amax_history[0, t:t + 1], si, bias=bias)
+            if h0:
+                h0()
+
         fc1, fc2 = self.fc1, self.fc2
         ct("x", x, "e4m3", 0, self.x8, self.x8t, self.si[0:1])
         ct("w1", fc1.w, "e4m3", 1, fc1.w8, fc1.w8t, fc1.w_scale_inv)
-        gemm("fc1.fwd", self.x8, "e4m3", self.si[0:1], fc1.w8, "e4m3", fc1.w_scale_inv, self.h, fc1.bias)
-        ct("h", self.h, "e4m3", 3, self.h8, self.h8t, self.si[1:2])
+        if fused:
+            gemm_cast("fc1.fwd", self.x8, "e4m3", self.si[0:1], fc1.w8, "e4m3", fc1.w_scale_inv, "e4m3", 3,
+                      self.h8, self.h8t, self.si[1:2], fc1.bias)
+        else:
+            gemm("fc1.fwd", self.x8, "e4m3", self.si[0:1], fc1.w8, "e4m3", fc1.w_scale_inv, self.h, fc1.bias)
+            ct("h", self.h, "e4m3", 3, self.h8, self.h8t, self.si[1:2])
         ct("w2", fc2.w, "e4m3", 4, fc2.w8, fc2.w8t, fc2.w_scale_inv)
         gemm("fc2.fwd", self.h8, "e4m3", self.si[1:2], fc2.w8, "e4m3", fc2.w_scale_inv, self.y, fc2.bias)
         ct("dy", dy, "e5m2", 5, self.dy8, self.dy8t, self.si[2:3])
-        gemm("fc2.dgrad", self.dy8, "e5m2", self.si[2:3], fc2.w8t, "e4m3", fc2.w_scale_inv, self.dh)
+        if fused:
+            gemm_cast("fc2.dgrad", self.dy8, "e5m2", self.si[2:3], fc2.w8t, "e4m3", fc2.w_scale_inv, "e5m2", 2,
+                      self.dh8, self.dh8t, self.si[3:4])
+        else:
+            gemm("fc2.dgrad", self.dy8, "e5m2", self.si[2:3], fc2.w8t, "e4m3", fc2.w_scale_inv, self.dh)
         gemm("fc2.wgrad", self.dy8t, "e5m2", self.si[2:3], self.h8t, "e4m3", self.si[1:2], self.dw2)
-        ct("dh", self.dh, "e5m2", 2, self.dh8, self.dh8t, self.si[3:4])
+        if not fused:
+            ct("dh", self.dh, "e5m2", 2, self.dh8, self.dh8t, self.si[3:4])
         gemm("fc1.dgrad", self.dh8, "e5m2", self.si[3:4], fc1.w8t, "e4m3", fc1.w_scale_inv, self.dx)
         gemm("fc1.wgrad", self.dh8t, "e5m2", self.si[3:4], self.x8t, "e4m3", self.si[0:1], self.dw1)
         if sync_amax is not None:
@@ -271,7 +313,8 @@ class MlpStep:
             h0()
 
 
-LAUNCHES_PER_STEP = 6 + 6 + 1
+LAUNCHES_PER_STEP = 4 + 6 + 1           # fused step: 4 casts, 6 GEMMs, 1 update
+LAUNCHES_PER_STEP_UNFUSED = 6 + 6 + 1
 
 
 class EventLog:
@@ -310,7 +353,7 @@ def max_over_ranks(v, world, device):
 
 # ---------------------------------------------------------- measurements --
 
-def time_cast_workload(fp8, device, reps=40):
+def time_cast_workload(fp8, device, reps=100):
     """bf16 [8192, 2048] (0.1% spikes) -> e4m3 and e5m2 with transpose and amax,
     over 8 rotating input buffers (268 MB > L2); per-launch CUDA-event times."""
     base = inputs.spiky_bf16().to(device)
@@ -332,11 +375,26 @@ def time_cast_workload(fp8, device, reps=40):
         e1.record()
         torch.cuda.synchronize()
         res[fmt] = {"us_mean": 1e3 * e0.elapsed_time(e1) / reps}
+    # dynamic scaling of the same tensors (amax pass, scale, cast: the input
+    # is read twice) for comparison with the delayed cast above
+    sd = torch.ones(1, device=device)
+    for i in range(5):
+        fp8.fp8_cast_transpose_amax_dynamic(xs[i % 8], "e4m3", sd, y, yt, am, si)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(reps):
+        fp8.fp8_cast_transpose_amax_dynamic(xs[i % 8], "e4m3", sd, y, yt, am, si)
+    e1.record()
+    torch.cuda.synchronize()
+    res["dynamic_e4m3"] = {"us_mean": 1e3 * e0.elapsed_time(e1) / reps}
     return res
 
 
-def time_headline_gemm(fp8, device, reps=30):
-    """8192x2048x8192 and 8192x8192x2048 e4m3 GEMMs (bf16 out), timed alone."""
+def time_headline_gemm(fp8, device, reps=50, warmup=10):
+    """8192x2048x8192 and 8192x8192x2048 e4m3 GEMMs (bf16 out), timed alone:
+    10 warm-up and 50 timed launches.  torch._scaled_mm (a library GEMM) is
+    timed on the same operands as context only; it is not part of the path."""
     out = {}
     for (M, N, K) in [(8192, 2048, 8192), (8192, 8192, 2048)]:
         g = torch.Generator(device="cpu").manual_seed(3)
@@ -344,17 +402,30 @@ def time_headline_gemm(fp8, device, reps=30):
         b = torch.randint(0, 0x7F, (N, K), generator=g, dtype=torch.uint8).to(device)
         sa = torch.full((1,), 2.0 ** -10, device=device)
         d = torch.empty(M, N, dtype=torch.bfloat16, device=device)
-        for _ in range(5):
-            fp8.fp8_gemm(a, "e4m3", sa, b, "e4m3", sa, d)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record()
-        for _ in range(reps):
-            fp8.fp8_gemm(a, "e4m3", sa, b, "e4m3", sa, d)
-        e1.record()
-        torch.cuda.synchronize()
-        us = 1e3 * e0.elapsed_time(e1) / reps
-        out["%dx%dx%d" % (M, N, K)] = {"us_median": us, "tflops": 2.0 * M * N * K / (us * 1e-6) / 1e12}
+
+        def timed(fn):
+            for _ in range(warmup):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            return 1e3 * e0.elapsed_time(e1) / reps
+
+        us = timed(lambda: fp8.fp8_gemm(a, "e4m3", sa, b, "e4m3", sa, d))
+        row = {"us_mean": us, "tflops": 2.0 * M * N * K / (us * 1e-6) / 1e12}
+        try:
+            a8, b8 = a.view(torch.float8_e4m3fn), b.view(torch.float8_e4m3fn)
+            s0 = sa.reshape(())
+            us_lib = timed(lambda: torch._scaled_mm(a8, b8.t(), scale_a=s0, scale_b=s0, out_dtype=torch.bfloat16))
+            row["context_torch_scaled_mm"] = {"us_mean": us_lib,
+                                              "tflops": 2.0 * M * N * K / (us_lib * 1e-6) / 1e12}
+        except Exception as exc:  # context only
+            row["context_torch_scaled_mm"] = {"unavailable": str(exc)[:120]}
+        out["%dx%dx%d" % (M, N, K)] = row
     return out
 
 
@@ -448,19 +519,57 @@ def e2e_linear_api(fp8, step, device, steps, warmup):
     return ms, h2d, d2h
 
 
+def time_graph_step(step, steps):
+    """The fused step captured once in a CUDA graph and replayed `steps` times
+    (no host work per step beyond the replay call).  The graph reads the
+    first input set; returns device ms per step and host us per replay."""
+    saved = step.xs, step.dys
+    step.xs, step.dys = saved[0][:1], saved[1][:1]
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step.run_linear_api(0)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    h0 = time.perf_counter()
+    s.record()
+    for _ in range(steps):
+        graph.replay()
+    e.record()
+    host_s = time.perf_counter() - h0
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    step.xs, step.dys = saved
+    del graph
+    return {"ms_per_step": ms, "value": STEP_FLOP / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "host_us_per_step": 1e6 * host_s / steps}
+
+
 def single_kernel(args):
     """One kernel alone on its workload: 2 warm-up launches then --reps timed
     ones (used under ncu with -s 2)."""
     from fp8_delayed_scaling_cast_b200 import binding as fp8
     dev = torch.device("cuda", 0)
-    if args.kernel == "gemm":
+    if args.kernel in ("gemm", "gemmcast"):
         M, N, K = (int(v) for v in args.shape.split("x"))
         g = torch.Generator(device="cpu").manual_seed(3)
         a = torch.randint(0, 0x7F, (M, K), generator=g, dtype=torch.uint8).to(dev)
         b = torch.randint(0, 0x7F, (N, K), generator=g, dtype=torch.uint8).to(dev)
         sa = torch.full((1,), 2.0 ** -10, device=dev)
-        d = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        run = lambda: fp8.fp8_gemm(a, "e4m3", sa, b, "e4m3", sa, d)  # noqa: E731
+        if args.kernel == "gemm":
+            d = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            run = lambda: fp8.fp8_gemm(a, "e4m3", sa, b, "e4m3", sa, d)  # noqa: E731
+        else:
+            # FP8 output with transpose and amax (the fused hand-over epilogue)
+            d8 = torch.empty(M, N, dtype=torch.uint8, device=dev)
+            d8t = torch.empty(N, M, dtype=torch.uint8, device=dev)
+            so = torch.full((1,), 0.5, device=dev)
+            am = torch.zeros(1, device=dev)
+            si = torch.zeros(1, device=dev)
+            run = lambda: fp8.fp8_gemm_cast(a, "e4m3", sa, b, "e4m3", sa, "e4m3", so, d8, d8t, am, si)  # noqa: E731
         work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     else:
         base = inputs.spiky_bf16().to(dev)
@@ -498,7 +607,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=None,
                     help="tokens of the oracle's sample (default 128; 8 per step for --impl reference)")
-    ap.add_argument("--kernel", choices=["gemm", "cast"], default=None,
+    ap.add_argument("--kernel", choices=["gemm", "gemmcast", "cast"], default=None,
                     help="run one kernel alone (2 warm-up + --reps launches), for profilers")
     ap.add_argument("--shape", default="8192x2048x8192", help="MxNxK for --kernel gemm")
     ap.add_argument("--fmt", default="e4m3", help="FP8 format for --kernel cast")
@@ -559,7 +668,9 @@ def main():
 
     sync = sync_amax if world > 1 else None
 
-    # warm-up
+    # warm-up (both variants of the step)
+    for i in range(args.warmup):
+        step.run_linear_api(i, sync_amax=sync, fused=False)
     for i in range(args.warmup):
         step.run_linear_api(i, sync_amax=sync)
     barrier_sync(world)
@@ -576,8 +687,10 @@ def main():
     if clocks:
         clocks.mark_start()
     t_start.record()
+    h0 = time.perf_counter()
     for i in range(args.steps):
         step.run_linear_api(i, sync_amax=sync)
+    host_us = 1e6 * (time.perf_counter() - h0) / args.steps
     t_end.record()
     barrier_sync(world)
     if clocks:
@@ -586,6 +699,19 @@ def main():
     ms_local = t_start.elapsed_time(t_end) / args.steps
     ms = max_over_ranks(ms_local, world, device)
     status = fp8.fp8ds_device_status()
+
+    # the same step with each linear casting its own input and gradient
+    barrier_sync(world)
+    t_start.record()
+    for i in range(args.steps):
+        step.run_linear_api(i, sync_amax=sync, fused=False)
+    t_end.record()
+    barrier_sync(world)
+    ms_unfused = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, device)
+
+    # the fused step replayed from a CUDA graph (one GPU: the amax sync of
+    # several ranks is not captured)
+    graph_info = time_graph_step(step, args.steps) if world == 1 else None
 
     # per-kernel durations: the same launches, one C call per kernel, each
     # bracketed by CUDA events on the launching stream (K more steps)
@@ -596,6 +722,9 @@ def main():
 
     per = log.summary()
     gemm_ms = [t for _, t in per["gemm"]]
+    gemm_by_key = {}
+    for key, t in per["gemm"]:
+        gemm_by_key.setdefault(key, []).append(t)
     cast_ms = {}
     for key, t in per["cast"]:
         cast_ms.setdefault(key, []).append(t)
@@ -606,7 +735,7 @@ def main():
     fp8_peak_sus = 2.0 * pk["bf16_sus"]
     cast_total_ms = sum(sum(v) for v in cast_ms.values()) / args.steps
     kernel_ms = (sum(gemm_ms) + sum(upd_ms)) / args.steps + cast_total_ms
-    cast_gbs_step = STEP_CAST_BYTES / (cast_total_ms * 1e-3) / 1e9
+    cast_gbs_step = STEP_CAST_BYTES_FUSED / (cast_total_ms * 1e-3) / 1e9
     value = world * STEP_FLOP / (ms * 1e-3) / 1e12
 
     # standalone: cast-transpose-amax workload and the headline GEMM shapes
@@ -650,13 +779,14 @@ def main():
         "data": "synthetic",
         "config": {
             "workload": "MLP pair 2048->8192->2048 fwd+bwd at 8192 tokens (batch 8 x seq 1024), "
-                        "HYBRID delayed scaling, amax history 16, weights recast every step",
+                        "HYBRID delayed scaling, amax history 16, weights recast every step, "
+                        "H and dH handed over in FP8 from the GEMM epilogues",
             "tokens": TOKENS, "hidden": HIDDEN, "ffn": FFN, "gemms_per_step": STEP_GEMMS,
             "parallelism": "dp%d" % world,
             "l2": "inputs larger than L2: about 1.5 GB touched per step, X/dY rotate over 2 sets",
         },
         "roofline": {
-            "kernel": "fp8_gemm_kernel (tcgen05, bf16/fp32 out)",
+            "kernel": "fp8_gemm_2sm_kernel (tcgen05 CTA pairs; bf16 / fp32 / FP8 out)",
             "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
             "frac": gemm_tflops / fp8_peak, "traffic": None,
             "peak_note": "fp8 dense = 2 x measured bf16 burst (%s); sustained: %.1f TFLOP/s, frac %.3f" % (
@@ -670,16 +800,26 @@ def main():
             "bytes_per_launch": C2_BYTES, "achieved": c2_gbs, "peak": pk["hbm"], "unit": "GB/s",
             "frac": c2_gbs / pk["hbm"], "bound": "hbm",
             "in_step_gbs": cast_gbs_step, "in_step_frac": cast_gbs_step / pk["hbm"],
+            "dynamic_scaling_e4m3_us": c2["dynamic_e4m3"]["us_mean"],
+            "dynamic_note": "amax pass + scale + cast (input read twice) vs the delayed cast's one read",
         },
         "update_scales_us": 1e3 * statistics.mean(upd_ms),
+        "gemm_us": {k: 1e3 * statistics.mean(v) for k, v in gemm_by_key.items()},
+        "cast_us": {k: 1e3 * statistics.mean(v) for k, v in cast_ms.items()},
         "kernels_sum_ms_per_step": kernel_ms,
         "gemm_alone": heads,
-        "step_roofline_frac": ((STEP_FLOP / (fp8_peak * 1e12)) + (STEP_CAST_BYTES / (pk["hbm"] * 1e9))) /
+        "step_roofline_frac": ((STEP_FLOP / (fp8_peak * 1e12)) + (STEP_CAST_BYTES_FUSED / (pk["hbm"] * 1e9))) /
                               (ms * 1e-3),
+        "host_us_per_step": host_us,
+        "graph_step": graph_info,
+        "unfused_step": {"ms_per_step": ms_unfused, "value": world * STEP_FLOP / (ms_unfused * 1e-3) / 1e12,
+                         "unit": "TFLOP/s", "gpu_launches_per_step": LAUNCHES_PER_STEP_UNFUSED,
+                         "api": "fp8_linear_fwd/bwd: every linear casts its own input and gradient"},
         "e2e": {"value": world * STEP_FLOP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "fp8_linear_fwd/bwd + fp8_update_scales, pinned host X/dY, double-buffered copies"},
+                "api": "fp8_linear_fwd_ex/bwd_ex + fp8_update_scales, pinned host X/dY, double-buffered copies"},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches_per_step": LAUNCHES_PER_STEP,
         "launch_mode": "programmatic dependent launch (griddepcontrol) on every kernel",
         "device_status": status,
         "clocks": clock_info,

@@ -18,6 +18,7 @@ E5M2 = 1
 F32 = 0
 BF16 = 1
 AMAX_MAX = 0
+AMAX_MOST_RECENT = 1
 
 OK = 0
 ERR_INVALID_ARG = 1
@@ -55,20 +56,31 @@ class _Linear(ctypes.Structure):
     _fields_ = [("w", _P), ("bias", _P), ("bias_dtype", _INT), ("in_features", _I64),
                 ("out_features", _I64), ("w8", _P), ("w8t", _P), ("w_scale_inv", _P),
                 ("meta_in", _I32), ("meta_w", _I32), ("meta_grad", _I32), ("cache_valid", _I32),
-                ("workspace", _P), ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace", _P), ("workspace_bytes", ctypes.c_size_t), ("w_noop_flag", _P)]
+
+
+class _Fp8Io(ctypes.Structure):
+    _fields_ = [("in_cast", _I32), ("out_meta", _I32), ("out8", _P), ("out8t", _P), ("out_scale_inv", _P)]
 
 
 _SIGS = {
     "fp8_quantize": [_P, _INT, _I64, _INT, _P, _P, _P, _P, _P],
     "fp8_cast_transpose_amax": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
+    "fp8_cast_transpose_amax_noop": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P, _P],
+    "fp8_cast_transpose_amax_dynamic": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
     "fp8_update_scales": [_I64, _I32, _P, _P, _P, _P, _INT, _P],
     "fp8_gemm": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
     "fp8_gemm_ex": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P,
                     ctypes.c_size_t, _P],
     "fp8_gemm_workspace_size": [ctypes.POINTER(ctypes.c_size_t)],
     "fp8_gemm_noalloc": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
+    "fp8_gemm_cast": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _I64, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
     "fp8_linear_fwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _INT,
                        _I32, _P, _P, _P, _P],
+    "fp8_linear_fwd_ex": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _INT,
+                          _I32, _P, _P, _P, ctypes.POINTER(_Fp8Io), _P],
+    "fp8_linear_bwd_ex": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P,
+                          _INT, _P, _P, _P, _P, ctypes.POINTER(_Fp8Io), _P],
     "fp8_linear_bwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P,
                        _INT, _P, _P, _P, _P, _P],
     "fp8ds_device_status": [ctypes.POINTER(_I32), _I32],
@@ -130,6 +142,20 @@ def fp8_cast_transpose_amax(x, fmt, scale, y, yt=None, amax=None, scale_inv=None
                                         _stream(stream)))
 
 
+def fp8_cast_transpose_amax_noop(x, fmt, scale, y, yt, amax, scale_inv, noop_flag, stream=None):
+    rows, cols = x.shape
+    _check(_lib.fp8_cast_transpose_amax_noop(_ptr(x), _dtype(x), rows, cols, _fmt(fmt), _ptr(scale), _ptr(y),
+                                             _ptr(yt), _ptr(amax), _ptr(scale_inv), _ptr(noop_flag),
+                                             _stream(stream)))
+
+
+def fp8_cast_transpose_amax_dynamic(x, fmt, scale, y, yt=None, amax=None, scale_inv=None, stream=None):
+    """Dynamic scaling: amax of x, scale = fp8_max / amax (scale is in/out), cast."""
+    rows, cols = x.shape
+    _check(_lib.fp8_cast_transpose_amax_dynamic(_ptr(x), _dtype(x), rows, cols, _fmt(fmt), _ptr(scale), _ptr(y),
+                                                _ptr(yt), _ptr(amax), _ptr(scale_inv), _stream(stream)))
+
+
 def fp8_update_scales(amax_history, scale, scale_inv, formats, algo=AMAX_MAX, stream=None):
     hist_len, num_tensors = amax_history.shape
     _check(_lib.fp8_update_scales(num_tensors, hist_len, _ptr(amax_history), _ptr(scale),
@@ -162,6 +188,16 @@ def fp8_gemm_noalloc(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, d, bias=None,
                                  _ptr(d), _dtype(d), m, n, k, _stream(stream)))
 
 
+def fp8_gemm_cast(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, out_fmt, out_scale, d8, d8t=None,
+                  out_amax=None, out_scale_inv=None, bias=None, stream=None):
+    m, k = a.shape
+    n = b.shape[0]
+    _check(_lib.fp8_gemm_cast(_ptr(a), _fmt(a_fmt), _ptr(a_scale_inv), _ptr(b), _fmt(b_fmt),
+                              _ptr(b_scale_inv), _ptr(bias), F32 if bias is None else _dtype(bias), m, n, k,
+                              _fmt(out_fmt), _ptr(out_scale), _ptr(d8), _ptr(d8t), _ptr(out_amax),
+                              _ptr(out_scale_inv), _stream(stream)))
+
+
 def fp8_gemm_workspace_size():
     n = ctypes.c_size_t(0)
     _check(_lib.fp8_gemm_workspace_size(ctypes.byref(n)))
@@ -189,26 +225,30 @@ class Fp8Meta:
     def num_tensors(self):
         return self.formats.numel()
 
-    def update(self, stream=None):
-        fp8_update_scales(self.amax_history, self.scale, self.scale_inv, self.formats,
+    def update(self, algo=AMAX_MAX, stream=None):
+        fp8_update_scales(self.amax_history, self.scale, self.scale_inv, self.formats, algo=algo,
                           stream=stream)
 
 
 class Fp8Linear:
     """A linear layer's fp32 master weight, optional bias and FP8 weight cache."""
 
-    def __init__(self, w, bias, meta_in, meta_w, meta_grad, workspace=None):
+    def __init__(self, w, bias, meta_in, meta_w, meta_grad, workspace=None, w_noop_flag=None):
+        """w_noop_flag: optional device int32 tensor; when given, the forward
+        always enqueues the weight cast and the GPU skips it while the flag is
+        non-zero (graph-capturable weight caching)."""
         out_f, in_f = w.shape
         self.w = w
         self.bias = bias
         self.workspace = workspace
+        self.w_noop_flag = w_noop_flag
         self.w8 = torch.empty(out_f, in_f, dtype=torch.uint8, device=w.device)
         self.w8t = torch.empty(in_f, out_f, dtype=torch.uint8, device=w.device)
         self.w_scale_inv = torch.ones(1, dtype=torch.float32, device=w.device)
         ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
         self._c = _Linear(_ptr(w), _ptr(bias), F32 if bias is None else _dtype(bias), in_f, out_f,
                           _ptr(self.w8), _ptr(self.w8t), _ptr(self.w_scale_inv),
-                          meta_in, meta_w, meta_grad, 0, _ptr(workspace), ws_bytes)
+                          meta_in, meta_w, meta_grad, 0, _ptr(workspace), ws_bytes, _ptr(w_noop_flag))
 
     @property
     def in_features(self):
@@ -240,6 +280,36 @@ def fp8_linear_bwd(lin, meta, dy, x8t, x_scale_inv, dw, dy8, dy8t, dy_scale_inv,
                                dy.shape[0], _ptr(x8t), _ptr(x_scale_inv), _ptr(dx),
                                BF16 if dx is None else _dtype(dx), _ptr(dw), _ptr(dy8),
                                _ptr(dy8t), _ptr(dy_scale_inv), _stream(stream)))
+
+
+def _io(in_cast, out_meta, out8, out8t, out_scale_inv):
+    return _Fp8Io(1 if in_cast else 0, -1 if out_meta is None else int(out_meta), _ptr(out8), _ptr(out8t),
+                  _ptr(out_scale_inv))
+
+
+def fp8_linear_fwd_ex(lin, meta, x, y, is_first_microbatch, x8, x8t=None, x_scale_inv=None, in_cast=False,
+                      out_meta=None, out8=None, out8t=None, out_scale_inv=None, stream=None):
+    """fp8_linear_fwd with FP8 hand-over: in_cast -> x8/x8t/x_scale_inv already
+    hold the cast input (x may be None); out_meta -> the output is cast in the
+    GEMM epilogue into out8/out8t/out_scale_inv (y may be None)."""
+    flag = -1 if is_first_microbatch is None else (1 if is_first_microbatch else 0)
+    io = _io(in_cast, out_meta, out8, out8t, out_scale_inv)
+    _check(_lib.fp8_linear_fwd_ex(ctypes.byref(lin._c), ctypes.byref(meta._c), _ptr(x),
+                                  F32 if x is None else _dtype(x), x8.shape[0], _ptr(y),
+                                  BF16 if y is None else _dtype(y), flag, _ptr(x8), _ptr(x8t),
+                                  _ptr(x_scale_inv), ctypes.byref(io), _stream(stream)))
+
+
+def fp8_linear_bwd_ex(lin, meta, dy, x8t, x_scale_inv, dw, dy8, dy8t, dy_scale_inv, dx=None, in_cast=False,
+                      out_meta=None, out8=None, out8t=None, out_scale_inv=None, stream=None):
+    """fp8_linear_bwd with FP8 hand-over: in_cast -> dy8/dy8t/dy_scale_inv
+    already hold the cast gradient (dy may be None); out_meta -> the dgrad is
+    cast in the GEMM epilogue into out8/out8t/out_scale_inv."""
+    io = _io(in_cast, out_meta, out8, out8t, out_scale_inv)
+    _check(_lib.fp8_linear_bwd_ex(ctypes.byref(lin._c), ctypes.byref(meta._c), _ptr(dy),
+                                  BF16 if dy is None else _dtype(dy), dy8.shape[0], _ptr(x8t),
+                                  _ptr(x_scale_inv), _ptr(dx), BF16 if dx is None else _dtype(dx), _ptr(dw),
+                                  _ptr(dy8), _ptr(dy8t), _ptr(dy_scale_inv), ctypes.byref(io), _stream(stream)))
 
 
 def fp8ds_device_status(clear=True):

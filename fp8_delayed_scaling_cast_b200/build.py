@@ -28,7 +28,8 @@ def _nvcc():
 
 def _inputs():
     files = [os.path.join(CSRC, s) for s in SOURCES]
-    files += [os.path.join(CSRC, "fp8ds_internal.h"), os.path.join(INCLUDE, "fp8ds.h")]
+    files += [os.path.join(CSRC, "fp8ds_internal.h"), os.path.join(CSRC, "ptx_sm100.cuh"),
+              os.path.join(INCLUDE, "fp8ds.h")]
     return files
 
 

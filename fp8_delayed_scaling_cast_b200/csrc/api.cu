@@ -125,6 +125,19 @@ static fp8ds_status check_gemm(const uint8_t *a, int fa, const float *sa, const 
     return FP8DS_OK;
 }
 
+// Extra conditions of a GEMM whose output is FP8 codes (row pitch n bytes,
+// transposed pitch m bytes: both multiples of 16 for the tensor maps).
+static fp8ds_status check_cast_out(const char *fn, const uint8_t *d8, const uint8_t *d8t, const float *scale,
+                                   int64_t m, int64_t n) {
+    if (d8 == nullptr || scale == nullptr) return invalid("%s: the FP8 output and its scale must not be NULL", fn);
+    if (n % 16 != 0) return invalid("%s: n (%lld) must be a multiple of 16 for FP8 output", fn, (long long)n);
+    if (d8t != nullptr && m % 16 != 0)
+        return invalid("%s: m (%lld) must be a multiple of 16 for the transposed FP8 output", fn, (long long)m);
+    if (!aligned16(d8) || (d8t != nullptr && !aligned16(d8t)))
+        return invalid("%s: the FP8 outputs must be 16-byte aligned", fn);
+    return FP8DS_OK;
+}
+
 static fp8ds_status check_meta(const char *fn, const fp8ds_meta *meta, int32_t idx) {
     if (meta == nullptr || meta->amax_history == nullptr || meta->scale == nullptr || meta->scale_inv == nullptr)
         return invalid("%s: incomplete meta", fn);
@@ -157,6 +170,31 @@ fp8ds_status fp8_cast_transpose_amax(const void *x, fp8ds_dtype x_dtype, int64_t
                        "fp8_cast_transpose_amax");
 }
 
+fp8ds_status fp8_cast_transpose_amax_noop(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
+                                          fp8ds_format fmt, const float *scale, uint8_t *y, uint8_t *yt,
+                                          float *amax, float *scale_inv, const int32_t *noop_flag,
+                                          fp8ds_stream stream) {
+    clear_error();
+    fp8ds_status st = check_cast("fp8_cast_transpose_amax_noop", x, x_dtype, rows, cols, fmt, scale, y);
+    if (st != FP8DS_OK) return st;
+    if (noop_flag == nullptr) return invalid("fp8_cast_transpose_amax_noop: noop_flag must not be NULL");
+    return cuda_status(
+        launch_cast_transpose(x, x_dtype, rows, cols, fmt, scale, y, yt, amax, scale_inv, stream, noop_flag),
+        "fp8_cast_transpose_amax_noop");
+}
+
+fp8ds_status fp8_cast_transpose_amax_dynamic(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
+                                             fp8ds_format fmt, float *scale, uint8_t *y, uint8_t *yt, float *amax,
+                                             float *scale_inv, fp8ds_stream stream) {
+    clear_error();
+    fp8ds_status st = check_cast("fp8_cast_transpose_amax_dynamic", x, x_dtype, rows, cols, fmt, scale, y);
+    if (st != FP8DS_OK) return st;
+    if (amax == nullptr) return invalid("fp8_cast_transpose_amax_dynamic: amax must not be NULL");
+    return cuda_status(
+        launch_cast_transpose_dynamic(x, x_dtype, rows, cols, fmt, scale, y, yt, amax, scale_inv, stream),
+        "fp8_cast_transpose_amax_dynamic");
+}
+
 fp8ds_status fp8_update_scales(int64_t num_tensors, int32_t hist_len, float *amax_history, float *scale,
                                float *scale_inv, const uint8_t *formats, fp8ds_amax_algo algo,
                                fp8ds_stream stream) {
@@ -165,12 +203,13 @@ fp8ds_status fp8_update_scales(int64_t num_tensors, int32_t hist_len, float *ama
     if (hist_len < 1) return invalid("fp8_update_scales: hist_len must be >= 1");
     if (num_tensors > 0 && (amax_history == nullptr || scale == nullptr || scale_inv == nullptr || formats == nullptr))
         return invalid("fp8_update_scales: NULL pointer");
-    if (algo != FP8DS_AMAX_MAX) {
-        set_error("fp8_update_scales: only amax_compute_algo=max is implemented");
+    if (algo != FP8DS_AMAX_MAX && algo != FP8DS_AMAX_MOST_RECENT) {
+        set_error("fp8_update_scales: unknown amax_compute_algo %d", static_cast<int>(algo));
         return FP8DS_ERR_UNSUPPORTED;
     }
-    return cuda_status(launch_update_scales(num_tensors, hist_len, amax_history, scale, scale_inv, formats, stream),
-                       "fp8_update_scales");
+    return cuda_status(
+        launch_update_scales(num_tensors, hist_len, amax_history, scale, scale_inv, formats, algo, stream),
+        "fp8_update_scales");
 }
 
 fp8ds_status fp8_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
@@ -215,77 +254,162 @@ fp8ds_status fp8_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float 
                                stream);
 }
 
-fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x, fp8ds_dtype x_dtype,
-                            int64_t m, void *y, fp8ds_dtype y_dtype, int32_t is_first_microbatch, uint8_t *x8,
-                            uint8_t *x8t, float *x_scale_inv, fp8ds_stream stream) {
+fp8ds_status fp8_gemm_cast(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
+                           fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
+                           int64_t m, int64_t n, int64_t k, fp8ds_format out_fmt, const float *out_scale,
+                           uint8_t *d8, uint8_t *d8t, float *out_amax, float *out_scale_inv, fp8ds_stream stream) {
     clear_error();
+    fp8ds_status st =
+        check_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d8, FP8DS_BF16, m, n, k);
+    if (st != FP8DS_OK) return st;
+    if (!valid_fmt(out_fmt)) return invalid("fp8_gemm_cast: unknown output FP8 format %d", out_fmt);
+    if ((st = check_cast_out("fp8_gemm_cast", d8, d8t, out_scale, m, n)) != FP8DS_OK) return st;
+    const GemmCastOut cast{out_fmt, out_scale, d8t, out_amax, out_scale_inv};
+    return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d8, FP8DS_BF16, m, n, k,
+                       nullptr, 0, stream, &cast);
+}
+
+// The linear forward and backward, with the options of the _ex forms (NULL:
+// none).  io->in_cast: the input (gradient) already sits in x8 / x8t /
+// x_scale_inv (dy8 / dy8t / dy_scale_inv).  io->out_meta >= 0: the output
+// (dgrad) is cast in the GEMM epilogue with that meta's scale.
+static fp8ds_status linear_fwd(const char *fn, fp8ds_linear *lin, const fp8ds_meta *meta, const void *x,
+                               fp8ds_dtype x_dtype, int64_t m, void *y, fp8ds_dtype y_dtype,
+                               int32_t is_first_microbatch, uint8_t *x8, uint8_t *x8t, float *x_scale_inv,
+                               const fp8ds_fp8_io *io, cudaStream_t s) {
     if (lin == nullptr || lin->w == nullptr || lin->w8 == nullptr || lin->w8t == nullptr ||
         lin->w_scale_inv == nullptr)
-        return invalid("fp8_linear_fwd: incomplete linear handle");
-    if (x == nullptr || y == nullptr || x8 == nullptr || x_scale_inv == nullptr)
-        return invalid("fp8_linear_fwd: x, y, x8 and x_scale_inv must not be NULL");
+        return invalid("%s: incomplete linear handle", fn);
+    const bool in_cast = io != nullptr && io->in_cast != 0;
+    const bool out_cast = io != nullptr && io->out_meta >= 0;
+    if ((!in_cast && x == nullptr) || (!out_cast && y == nullptr) || x8 == nullptr || x_scale_inv == nullptr)
+        return invalid("%s: x, y, x8 and x_scale_inv must not be NULL", fn);
     if (is_first_microbatch < -1 || is_first_microbatch > 1)
-        return invalid("fp8_linear_fwd: is_first_microbatch must be -1, 0 or 1");
+        return invalid("%s: is_first_microbatch must be -1, 0 or 1", fn);
     fp8ds_status st;
-    if ((st = check_meta("fp8_linear_fwd", meta, lin->meta_in)) != FP8DS_OK) return st;
-    if ((st = check_meta("fp8_linear_fwd", meta, lin->meta_w)) != FP8DS_OK) return st;
+    if ((st = check_meta(fn, meta, lin->meta_in)) != FP8DS_OK) return st;
+    if ((st = check_meta(fn, meta, lin->meta_w)) != FP8DS_OK) return st;
+    if (out_cast && (st = check_meta(fn, meta, io->out_meta)) != FP8DS_OK) return st;
     const int64_t K = lin->in_features, N = lin->out_features;
-    if ((st = check_cast("fp8_linear_fwd", x, x_dtype, m, K, FP8DS_E4M3, meta->scale, x8)) != FP8DS_OK) return st;
+    if (!in_cast && (st = check_cast(fn, x, x_dtype, m, K, FP8DS_E4M3, meta->scale, x8)) != FP8DS_OK) return st;
     if ((st = check_gemm(x8, FP8DS_E4M3, x_scale_inv, lin->w8, FP8DS_E4M3, lin->w_scale_inv, lin->bias,
-                         lin->bias_dtype, y, y_dtype, m, N, K)) != FP8DS_OK)
+                         lin->bias_dtype, out_cast ? static_cast<void *>(io->out8) : y,
+                         out_cast ? FP8DS_BF16 : y_dtype, m, N, K)) != FP8DS_OK)
         return st;
-    cudaStream_t s = stream;
+    if (out_cast && (st = check_cast_out(fn, io->out8, io->out8t, meta->scale, m, N)) != FP8DS_OK) return st;
     const int32_t hi = lin->meta_in, hw = lin->meta_w;
-    st = cuda_status(launch_cast_transpose(x, x_dtype, m, K, FP8DS_E4M3, meta->scale + hi, x8, x8t,
-                                           meta->amax_history + hi, x_scale_inv, s),
-                     "fp8_linear_fwd: input cast");
-    if (st != FP8DS_OK) return st;
-    const bool refresh = is_first_microbatch != 0 || !lin->cache_valid;
+    if (!in_cast) {
+        st = cuda_status(launch_cast_transpose(x, x_dtype, m, K, FP8DS_E4M3, meta->scale + hi, x8, x8t,
+                                               meta->amax_history + hi, x_scale_inv, s),
+                         "fp8_linear_fwd: input cast");
+        if (st != FP8DS_OK) return st;
+    }
+    // With a device-side flag the weight cast is always enqueued and the GPU
+    // decides (a captured graph then serves every microbatch); otherwise the
+    // host decides from is_first_microbatch and the cache state.
+    const bool refresh = lin->w_noop_flag != nullptr || is_first_microbatch != 0 || !lin->cache_valid;
     if (refresh) {
         st = cuda_status(launch_cast_transpose(lin->w, FP8DS_F32, N, K, FP8DS_E4M3, meta->scale + hw, lin->w8,
-                                               lin->w8t, meta->amax_history + hw, lin->w_scale_inv, s),
+                                               lin->w8t, meta->amax_history + hw, lin->w_scale_inv, s,
+                                               lin->w_noop_flag),
                          "fp8_linear_fwd: weight cast");
         if (st != FP8DS_OK) return st;
         lin->cache_valid = 1;
+    }
+    if (out_cast) {
+        const int32_t ho = io->out_meta;
+        const GemmCastOut cast{FP8DS_E4M3, meta->scale + ho, io->out8t, meta->amax_history + ho, io->out_scale_inv};
+        return launch_gemm(x8, FP8DS_E4M3, x_scale_inv, lin->w8, FP8DS_E4M3, lin->w_scale_inv, lin->bias,
+                           lin->bias_dtype, io->out8, FP8DS_BF16, m, N, K, lin->workspace, lin->workspace_bytes, s,
+                           &cast);
     }
     return launch_gemm(x8, FP8DS_E4M3, x_scale_inv, lin->w8, FP8DS_E4M3, lin->w_scale_inv, lin->bias,
                        lin->bias_dtype, y, y_dtype, m, N, K, lin->workspace, lin->workspace_bytes, s);
 }
 
-fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy, fp8ds_dtype dy_dtype,
-                            int64_t m, const uint8_t *x8t, const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
-                            float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv, fp8ds_stream stream) {
-    clear_error();
+static fp8ds_status linear_bwd(const char *fn, const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy,
+                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8t, const float *x_scale_inv,
+                               void *dx, fp8ds_dtype dx_dtype, float *dw, uint8_t *dy8, uint8_t *dy8t,
+                               float *dy_scale_inv, const fp8ds_fp8_io *io, cudaStream_t s) {
     if (lin == nullptr || lin->w8t == nullptr || lin->w_scale_inv == nullptr)
-        return invalid("fp8_linear_bwd: incomplete linear handle");
-    if (!lin->cache_valid) return invalid("fp8_linear_bwd: the weight cache is empty (run the forward first)");
-    if (dy == nullptr || x8t == nullptr || x_scale_inv == nullptr || dw == nullptr || dy8 == nullptr ||
-        dy8t == nullptr || dy_scale_inv == nullptr)
-        return invalid("fp8_linear_bwd: NULL pointer argument");
+        return invalid("%s: incomplete linear handle", fn);
+    if (!lin->cache_valid) return invalid("%s: the weight cache is empty (run the forward first)", fn);
+    const bool in_cast = io != nullptr && io->in_cast != 0;
+    const bool out_cast = io != nullptr && io->out_meta >= 0;
+    if ((!in_cast && dy == nullptr) || x8t == nullptr || x_scale_inv == nullptr || dw == nullptr ||
+        dy8 == nullptr || dy8t == nullptr || dy_scale_inv == nullptr)
+        return invalid("%s: NULL pointer argument", fn);
     fp8ds_status st;
-    if ((st = check_meta("fp8_linear_bwd", meta, lin->meta_grad)) != FP8DS_OK) return st;
+    if ((st = check_meta(fn, meta, lin->meta_grad)) != FP8DS_OK) return st;
+    if (out_cast && (st = check_meta(fn, meta, io->out_meta)) != FP8DS_OK) return st;
     const int64_t K = lin->in_features, N = lin->out_features;
-    if ((st = check_cast("fp8_linear_bwd", dy, dy_dtype, m, N, FP8DS_E5M2, meta->scale, dy8)) != FP8DS_OK)
+    if (!in_cast && (st = check_cast(fn, dy, dy_dtype, m, N, FP8DS_E5M2, meta->scale, dy8)) != FP8DS_OK) return st;
+    if (out_cast) {
+        if ((st = check_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv, nullptr,
+                             FP8DS_F32, io->out8, FP8DS_BF16, m, K, N)) != FP8DS_OK)
+            return st;
+        if ((st = check_cast_out(fn, io->out8, io->out8t, meta->scale, m, K)) != FP8DS_OK) return st;
+    } else if (dx != nullptr && (st = check_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3,
+                                                 lin->w_scale_inv, nullptr, FP8DS_F32, dx, dx_dtype, m, K, N)) !=
+                                    FP8DS_OK) {
         return st;
-    if (dx != nullptr && (st = check_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv,
-                                          nullptr, FP8DS_F32, dx, dx_dtype, m, K, N)) != FP8DS_OK)
-        return st;
+    }
     if ((st = check_gemm(dy8t, FP8DS_E5M2, dy_scale_inv, x8t, FP8DS_E4M3, x_scale_inv, nullptr, FP8DS_F32, dw,
                          FP8DS_F32, N, K, m)) != FP8DS_OK)
         return st;
-    cudaStream_t s = stream;
     const int32_t hg = lin->meta_grad;
-    st = cuda_status(launch_cast_transpose(dy, dy_dtype, m, N, FP8DS_E5M2, meta->scale + hg, dy8, dy8t,
-                                           meta->amax_history + hg, dy_scale_inv, s),
-                     "fp8_linear_bwd: grad cast");
-    if (st != FP8DS_OK) return st;
-    if (dx != nullptr) {
+    if (!in_cast) {
+        st = cuda_status(launch_cast_transpose(dy, dy_dtype, m, N, FP8DS_E5M2, meta->scale + hg, dy8, dy8t,
+                                               meta->amax_history + hg, dy_scale_inv, s),
+                         "fp8_linear_bwd: grad cast");
+        if (st != FP8DS_OK) return st;
+    }
+    if (out_cast) {
+        const int32_t ho = io->out_meta;
+        const GemmCastOut cast{FP8DS_E5M2, meta->scale + ho, io->out8t, meta->amax_history + ho, io->out_scale_inv};
+        st = launch_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv, nullptr, FP8DS_F32,
+                         io->out8, FP8DS_BF16, m, K, N, lin->workspace, lin->workspace_bytes, s, &cast);
+        if (st != FP8DS_OK) return st;
+    } else if (dx != nullptr) {
         st = launch_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv, nullptr, FP8DS_F32,
                          dx, dx_dtype, m, K, N, lin->workspace, lin->workspace_bytes, s);
         if (st != FP8DS_OK) return st;
     }
     return launch_gemm(dy8t, FP8DS_E5M2, dy_scale_inv, x8t, FP8DS_E4M3, x_scale_inv, nullptr, FP8DS_F32, dw,
                        FP8DS_F32, N, K, m, lin->workspace, lin->workspace_bytes, s);
+}
+
+fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x, fp8ds_dtype x_dtype,
+                            int64_t m, void *y, fp8ds_dtype y_dtype, int32_t is_first_microbatch, uint8_t *x8,
+                            uint8_t *x8t, float *x_scale_inv, fp8ds_stream stream) {
+    clear_error();
+    return linear_fwd("fp8_linear_fwd", lin, meta, x, x_dtype, m, y, y_dtype, is_first_microbatch, x8, x8t,
+                      x_scale_inv, nullptr, stream);
+}
+
+fp8ds_status fp8_linear_fwd_ex(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x, fp8ds_dtype x_dtype,
+                               int64_t m, void *y, fp8ds_dtype y_dtype, int32_t is_first_microbatch, uint8_t *x8,
+                               uint8_t *x8t, float *x_scale_inv, const fp8ds_fp8_io *io, fp8ds_stream stream) {
+    clear_error();
+    return linear_fwd("fp8_linear_fwd_ex", lin, meta, x, x_dtype, m, y, y_dtype, is_first_microbatch, x8, x8t,
+                      x_scale_inv, io, stream);
+}
+
+fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy, fp8ds_dtype dy_dtype,
+                            int64_t m, const uint8_t *x8t, const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
+                            float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv, fp8ds_stream stream) {
+    clear_error();
+    return linear_bwd("fp8_linear_bwd", lin, meta, dy, dy_dtype, m, x8t, x_scale_inv, dx, dx_dtype, dw, dy8, dy8t,
+                      dy_scale_inv, nullptr, stream);
+}
+
+fp8ds_status fp8_linear_bwd_ex(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy,
+                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8t, const float *x_scale_inv,
+                               void *dx, fp8ds_dtype dx_dtype, float *dw, uint8_t *dy8, uint8_t *dy8t,
+                               float *dy_scale_inv, const fp8ds_fp8_io *io, fp8ds_stream stream) {
+    clear_error();
+    return linear_bwd("fp8_linear_bwd_ex", lin, meta, dy, dy_dtype, m, x8t, x_scale_inv, dx, dx_dtype, dw, dy8, dy8t,
+                      dy_scale_inv, io, stream);
 }
 
 const char *fp8ds_last_error(void) { return g_msg; }

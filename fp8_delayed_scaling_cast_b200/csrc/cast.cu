@@ -157,11 +157,13 @@ __global__ void __launch_bounds__(CT_THREADS)
 cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
                       const float *__restrict__ scale_ptr, uint8_t *__restrict__ y,
                       uint8_t *__restrict__ yt, float *__restrict__ amax,
-                      float *__restrict__ scale_inv, int64_t tiles_c, int64_t num_tiles) {
+                      float *__restrict__ scale_inv, int64_t tiles_c, int64_t num_tiles,
+                      const int32_t *__restrict__ noop) {
     __shared__ uint32_t tsm[CT_COLS * CT_TSTRIDE];
     uint8_t *tsm8 = reinterpret_cast<uint8_t *>(tsm);
     ptx::pdl_wait();
     ptx::pdl_launch_dependents();
+    if (noop != nullptr && __ldg(noop) != 0) return;  // device-side skip (whole grid)
     const float s = __ldg(scale_ptr);
     const int tid = threadIdx.x;
     float m = 0.0f;
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(CT_THREADS, 3)
 cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t rows, int32_t cols,
                           const float *__restrict__ scale_ptr, uint8_t *__restrict__ y, uint8_t *__restrict__ yt,
                           float *__restrict__ amax, float *__restrict__ scale_inv, int32_t tiles_c,
-                          int32_t num_tiles) {
+                          int32_t num_tiles, const int32_t *__restrict__ noop) {
     using R = TmaRing<T>;
     constexpr int STAGES = R::STAGES;
     extern __shared__ uint8_t dsm[];
@@ -347,6 +349,8 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
     }
     ptx::pdl_wait();
     ptx::pdl_launch_dependents();
+    // device-side skip (whole grid), before any load is issued
+    if (noop != nullptr && __ldg(noop) != 0) return;
     const float s = __ldg(scale_ptr);
     if (tid == 0 && blockIdx.x == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
     __syncthreads();
@@ -521,19 +525,19 @@ int grid_for(K kernel, int threads, int64_t work_items) {
 
 template <typename T, int FMT, bool WRITE_T>
 cudaError_t ct_launch_elem(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
-                           float *amax, float *scale_inv, cudaStream_t stream) {
+                           float *amax, float *scale_inv, const int32_t *noop, cudaStream_t stream) {
     const int64_t tiles_c = (cols + CT_COLS - 1) / CT_COLS;
     const int64_t tiles_r = (rows + CT_ROWS - 1) / CT_ROWS;
     const int64_t num_tiles = tiles_c * tiles_r;
     auto kernel = cast_transpose_kernel<T, FMT, false, WRITE_T>;
     const int grid = grid_for(kernel, CT_THREADS, num_tiles);
     return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), 0, stream, 1, static_cast<const T *>(x), rows, cols,
-                      scale, y, yt, amax, scale_inv, tiles_c, num_tiles);
+                      scale, y, yt, amax, scale_inv, tiles_c, num_tiles, noop);
 }
 
 template <typename T, int FMT, bool WRITE_T>
 cudaError_t ct_launch_tma(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
-                          float *amax, float *scale_inv, cudaStream_t stream) {
+                          float *amax, float *scale_inv, const int32_t *noop, cudaStream_t stream) {
     using R = TmaRing<T>;
     const int64_t tiles_c = (cols + CT_COLS - 1) / CT_COLS;
     const int64_t tiles_r = (rows + CT_ROWS - 1) / CT_ROWS;
@@ -542,7 +546,7 @@ cudaError_t ct_launch_tma(const void *x, int64_t rows, int64_t cols, const float
     if (!encode_tmap_2d(&tm, sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x,
                         static_cast<uint64_t>(cols), static_cast<uint64_t>(rows), static_cast<uint64_t>(cols) * sizeof(T),
                         R::BOX_COLS, CT_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
-        return ct_launch_elem<T, FMT, WRITE_T>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+        return ct_launch_elem<T, FMT, WRITE_T>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
     auto kernel = cast_transpose_tma_kernel<T, FMT, WRITE_T>;
     static bool configured[64] = {};
     static int per_sm[64] = {};
@@ -561,20 +565,20 @@ cudaError_t ct_launch_tma(const void *x, int64_t rows, int64_t cols, const float
     const int grid = static_cast<int>(num_tiles < cap ? (num_tiles > 0 ? num_tiles : 1) : cap);
     return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), R::SMEM, stream, 1, tm, static_cast<int32_t>(rows),
                       static_cast<int32_t>(cols), scale, y, yt, amax, scale_inv, static_cast<int32_t>(tiles_c),
-                      static_cast<int32_t>(num_tiles));
+                      static_cast<int32_t>(num_tiles), noop);
 }
 
 template <typename T, int FMT>
 cudaError_t ct_dispatch(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
-                        float *amax, float *scale_inv, cudaStream_t stream) {
+                        float *amax, float *scale_inv, const int32_t *noop, cudaStream_t stream) {
     const bool vec = rows > 0 && cols > 0 && aligned16(x) && aligned16(y) && (yt == nullptr || aligned16(yt)) &&
                      (cols % 8 == 0) && (rows % 16 == 0) && rows < (int64_t(1) << 31) && cols < (int64_t(1) << 31);
     if (yt != nullptr) {
-        return vec ? ct_launch_tma<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
-                   : ct_launch_elem<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+        return vec ? ct_launch_tma<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
+                   : ct_launch_elem<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
     }
-    return vec ? ct_launch_tma<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
-               : ct_launch_elem<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+    return vec ? ct_launch_tma<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
+               : ct_launch_elem<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
 }
 
 template <typename T, int FMT>
@@ -595,7 +599,90 @@ cudaError_t q_dispatch(const void *x, int64_t n, const float *scale, uint8_t *y,
     }
 }
 
+// -------------------------------------------------------- dynamic scaling --
+
+// The first pass of dynamic scaling: amax of a tensor alone.  16-byte loads
+// (grid-stride), warp shuffles, one atomic max per CTA on the float's bits.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(Q_THREADS)
+amax_kernel(const T *__restrict__ x, int64_t n, float *__restrict__ amax) {
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    constexpr int PER16 = 16 / sizeof(T);
+    float m = 0.0f;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * Q_THREADS + threadIdx.x;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * Q_THREADS;
+    int64_t done = 0;
+    if (VEC) {
+        const int64_t nv = n / PER16;
+        const uint4 *xv = reinterpret_cast<const uint4 *>(x);
+        for (int64_t i = tid; i < nv; i += stride) {
+            const uint4 v = __ldg(xv + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (sizeof(T) == 2) {
+                    m = fmaxf(m, fabsf(__uint_as_float(w[j] << 16)));
+                    m = fmaxf(m, fabsf(__uint_as_float(w[j] & 0xFFFF0000u)));
+                } else {
+                    m = fmaxf(m, fabsf(__uint_as_float(w[j])));
+                }
+            }
+        }
+        done = nv * PER16;
+    }
+    for (int64_t i = done + tid; i < n; i += stride) m = fmaxf(m, fabsf(InElem<T>::load(x + i)));
+    block_amax_commit<Q_THREADS>(m, amax);
+}
+
+// scale = fl32(fp8_max / amax) when amax > 0, finite and the quotient finite,
+// else the given scale is kept; scale_inv = fl32(1 / scale).  One thread.
+__global__ void scale_from_amax_kernel(const float *__restrict__ amax, float *__restrict__ scale,
+                                       float *__restrict__ scale_inv, float fp8_max) {
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    if (threadIdx.x != 0 || blockIdx.x != 0) return;
+    const float a = *amax;
+    float s = *scale;
+    if (a > 0.0f && isfinite(a)) {
+        const float q = __fdiv_rn(fp8_max, a);
+        if (isfinite(q)) s = q;
+    }
+    *scale = s;
+    if (scale_inv != nullptr) *scale_inv = __frcp_rn(s);
+}
+
+template <typename T>
+cudaError_t amax_dispatch(const void *x, int64_t n, float *amax, cudaStream_t stream) {
+    const bool vec = aligned16(x);
+    const int64_t items = vec ? n / (16 / static_cast<int64_t>(sizeof(T))) : n;
+    const int64_t blocks = (items + Q_THREADS - 1) / Q_THREADS;
+    if (vec) {
+        auto kernel = amax_kernel<T, true>;
+        return launch_pdl(kernel, dim3(grid_for(kernel, Q_THREADS, blocks > 0 ? blocks : 1)), dim3(Q_THREADS), 0,
+                          stream, 1, static_cast<const T *>(x), n, amax);
+    }
+    auto kernel = amax_kernel<T, false>;
+    return launch_pdl(kernel, dim3(grid_for(kernel, Q_THREADS, blocks > 0 ? blocks : 1)), dim3(Q_THREADS), 0,
+                      stream, 1, static_cast<const T *>(x), n, amax);
+}
+
 }  // namespace
+
+cudaError_t launch_cast_transpose_dynamic(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
+                                          fp8ds_format fmt, float *scale, uint8_t *y, uint8_t *yt, float *amax,
+                                          float *scale_inv, cudaStream_t stream) {
+    cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    const int64_t n = rows * cols;
+    e = x_dtype == FP8DS_F32 ? amax_dispatch<float>(x, n, amax, stream) : amax_dispatch<uint16_t>(x, n, amax, stream);
+    if (e != cudaSuccess) return e;
+    const float fp8_max = fmt == FP8DS_E4M3 ? 448.0f : 57344.0f;
+    e = launch_pdl(scale_from_amax_kernel, dim3(1), dim3(32), 0, stream, 1, static_cast<const float *>(amax), scale,
+                   scale_inv, fp8_max);
+    if (e != cudaSuccess) return e;
+    return launch_cast_transpose(x, x_dtype, rows, cols, fmt, scale, y, yt, nullptr, nullptr, stream);
+}
 
 cudaError_t read_cast_error(int32_t *out, bool clear) {
     cudaError_t e = cudaMemcpyFromSymbol(out, g_cast_error, sizeof(int32_t));
@@ -606,15 +693,15 @@ cudaError_t read_cast_error(int32_t *out, bool clear) {
 
 cudaError_t launch_cast_transpose(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
                                   fp8ds_format fmt, const float *scale, uint8_t *y, uint8_t *yt,
-                                  float *amax, float *scale_inv, cudaStream_t stream) {
+                                  float *amax, float *scale_inv, cudaStream_t stream, const int32_t *noop) {
     if (x_dtype == FP8DS_F32) {
         return fmt == FP8DS_E4M3
-                   ? ct_dispatch<float, FP8DS_E4M3>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
-                   : ct_dispatch<float, FP8DS_E5M2>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+                   ? ct_dispatch<float, FP8DS_E4M3>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
+                   : ct_dispatch<float, FP8DS_E5M2>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
     }
     return fmt == FP8DS_E4M3
-               ? ct_dispatch<uint16_t, FP8DS_E4M3>(x, rows, cols, scale, y, yt, amax, scale_inv, stream)
-               : ct_dispatch<uint16_t, FP8DS_E5M2>(x, rows, cols, scale, y, yt, amax, scale_inv, stream);
+               ? ct_dispatch<uint16_t, FP8DS_E4M3>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
+               : ct_dispatch<uint16_t, FP8DS_E5M2>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
 }
 
 cudaError_t launch_quantize(const void *x, fp8ds_dtype x_dtype, int64_t n, fp8ds_format fmt,

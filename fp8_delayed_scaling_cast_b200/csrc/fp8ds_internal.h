@@ -24,22 +24,45 @@ cudaError_t launch_quantize(const void *x, fp8ds_dtype x_dtype, int64_t n, fp8ds
                             const float *scale, uint8_t *y, float *amax, float *scale_inv,
                             cudaStream_t stream);
 
+// noop (may be NULL): a device int32; when it holds non-zero at run time the
+// kernel returns before touching anything (outputs keep their values).
 cudaError_t launch_cast_transpose(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
                                   fp8ds_format fmt, const float *scale, uint8_t *y, uint8_t *yt,
-                                  float *amax, float *scale_inv, cudaStream_t stream);
+                                  float *amax, float *scale_inv, cudaStream_t stream,
+                                  const int32_t *noop = nullptr);
+
+// Dynamic scaling: amax = max |x| (written, not accumulated), then
+// scale = fp8_max / amax (kept when that is not finite and positive),
+// scale_inv = 1 / scale, then the cast with that scale.
+cudaError_t launch_cast_transpose_dynamic(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
+                                          fp8ds_format fmt, float *scale, uint8_t *y, uint8_t *yt, float *amax,
+                                          float *scale_inv, cudaStream_t stream);
 
 cudaError_t launch_update_scales(int64_t num_tensors, int32_t hist_len, float *amax_history,
                                  float *scale, float *scale_inv, const uint8_t *formats,
-                                 cudaStream_t stream);
+                                 fp8ds_amax_algo algo, cudaStream_t stream);
+
+// FP8 output of launch_gemm: the bf16-rounded result cast with the delayed
+// scale `*scale` into d (codes [m, n]) and, when d8t is not NULL, its
+// transpose [n, m]; amax (may be NULL) receives max |bf16 result|, scale_inv
+// (may be NULL) fl32(1 / *scale).
+struct GemmCastOut {
+    fp8ds_format fmt;
+    const float *scale;
+    uint8_t *d8t;
+    float *amax;
+    float *scale_inv;
+};
 
 // Returns FP8DS_OK or an error (message set) for tensor-map or launch failures.
 // workspace (may be NULL) enables the stream-K schedule when it holds at
-// least gemm_workspace_bytes().
+// least gemm_workspace_bytes().  With `cast`, d receives FP8 codes and
+// d_dtype is ignored.
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
                          const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
                          const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
                          int64_t m, int64_t n, int64_t k, void *workspace, size_t workspace_bytes,
-                         cudaStream_t stream);
+                         cudaStream_t stream, const GemmCastOut *cast = nullptr);
 
 // Workspace bytes the stream-K schedule needs on the current device.
 size_t gemm_workspace_bytes();

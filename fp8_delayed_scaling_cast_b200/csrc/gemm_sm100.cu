@@ -7,7 +7,7 @@
 // with A [M,K] and B [N,K] FP8, both contraction-major ("TN"), fp32
 // accumulation in tensor memory, fp32 or bf16 output.
 //
-// Two persistent warp-specialised kernels share one structure (6 warps):
+// Two persistent warp-specialised kernels share one structure (10 warps):
 //   warp 0      TMA producer: A and B tiles (128-byte rows, 128-byte swizzle)
 //               into a shared-memory ring, completion on per-stage mbarriers
 //               (transaction bytes);
@@ -32,9 +32,14 @@
 //                        moved per FLOP.  Both CTAs' loads signal CTA 0's
 //                        ring barriers; CTA 0's commits arrive on both CTAs'
 //                        barriers; both epilogues report to CTA 0.
+// The pair kernel has a second tile mode for long contractions (K >= 4096):
+// a 512 x 256 pair tile (each CTA loads two 128-row boxes of A per stage)
+// that fills all 512 TMEM columns with one accumulator set.
 // Tiles are visited in groups of 8 row-tiles (column index slowest within a
-// group) so that concurrently running CTAs share A and B in L2.  No TMA load
-// uses cluster multicast.
+// group) so that concurrently running CTAs share A and B in L2.  With a
+// workspace (fp8_gemm_ex, fp8_gemm_noalloc) a ragged last wave is replaced by
+// a stream-K split of (tile, k-block) units; partial sums of a split tile go
+// through the workspace.  No TMA load uses cluster multicast.
 //
 // Every wait is bounded (wall-clock limit read from %globaltimer).  A wait
 // that gives up records FP8DS_ERR_TIMEOUT and its site in the device error
@@ -67,6 +72,15 @@ constexpr int EPI_BYTES = EPI_WARPS * EPI_BOX_BYTES + 256 * 4;  // + the tile's 
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int SMEM_ALIGN = 1024;
 constexpr int GROUP_M = 8;
+// Smallest K for which the pair kernel takes the 512-row tile (compile-time
+// setting; 4096 measured best on B200 for the MLP shapes).
+#ifndef FP8DS_MSUB2_MIN_K
+#define FP8DS_MSUB2_MIN_K 4096
+#endif
+// Output kinds of the epilogue.
+constexpr int OUT_F32 = 0;
+constexpr int OUT_BF16 = 1;
+constexpr int OUT_FP8 = 2;   // bf16-rounded D cast to FP8 with a delayed scale (+ transpose, amax)
 constexpr unsigned long long TIMEOUT_NS = 2000000000ull;  // 2 s
 constexpr unsigned long long DRAIN_NS = 200000000ull;     // 0.2 s
 
@@ -335,6 +349,13 @@ struct Params {
     uint32_t epoch;       // non-zero per launch; partials are published with it
     int32_t *flags;       // [clusters][2] publication words
     float *partials;      // [clusters][2 CTAs][2 row blocks][128 x 256] fp32
+    // OUT_FP8: codes = cast(fl32(bf16(D) * out_scale)), amax of bf16(D)
+    const float *out_scale;
+    float *out_amax;       // NULL or atomic-max target
+    float *out_scale_inv;  // NULL or fl32(1 / out_scale)
+    uint8_t *out_d8;       // [M, N] codes
+    uint8_t *out_d8t;      // [N, M] codes or NULL
+    int32_t out_fmt;
 };
 
 // Workspace of the stream-K schedule: publication words, then one partial
@@ -535,6 +556,102 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
     }
 }
 
+// Two FP8 codes (saturating, round to nearest even) packed in 16 bits:
+// byte 0 = code(lo), byte 1 = code(hi); NaN becomes 0x7F.
+__device__ __forceinline__ uint32_t cvt_fp8x2(float lo, float hi, int fmt) {
+    uint16_t r;
+    if (fmt == FP8DS_E4M3)
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    else
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// FP8-output epilogue of one accumulator for one warp: 32 rows (its TMEM
+// lane quarter) x this warp's 128 columns, in chunks of 32 columns.  Each
+// value is first rounded to bf16 exactly as the bf16 output would be, then
+// cast like fp8_cast_transpose_amax: code = cvt(fl32(h * s_out)), amax over
+// |h|.  Lane r holds row r's 32 codes of a chunk and stores them straight to
+// global memory (32 contiguous bytes, whole sectors).  For the transpose it
+// also writes them into a shared 32 x 32-byte tile whose rows are 48 bytes
+// apart (so that both these 16-byte row writes and the byte gathers below are
+// free of bank conflicts); lane c then gathers column c (one byte per row)
+// and stores it as 32 contiguous bytes of row n0 + c of the transpose.  Two
+// tiles per warp alternate between chunks, so one __syncwarp per chunk
+// orders the writes and the gathers.  N and M are multiples of 16, so a
+// chunk's row (column) segment is whole, half or wholly outside.
+constexpr int FP8_TSTRIDE = 48;
+constexpr int FP8_TILE_BYTES = 32 * FP8_TSTRIDE;
+static_assert(2 * FP8_TILE_BYTES <= EPI_BOX_BYTES, "transpose tiles exceed the warp's staging box");
+
+__device__ __forceinline__ void store_segment(uint8_t *dst, int64_t left, const uint32_t (&w)[8]) {
+    if (left >= 32) {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(dst + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+    } else if (left >= 16) {
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+__device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint8_t *box, int half, uint8_t *d8,
+                                                  uint8_t *d8t, int64_t n_base, int32_t m_row0, float sab,
+                                                  const float *bias_s, uint32_t empty_bar_cluster, bool arrive,
+                                                  int mode, float *slot, int h, int q, float s_out, int fmt,
+                                                  int32_t m_total, int32_t n_total, float &amax) {
+    constexpr int CHUNKS = ACC_N / 32 / 2;
+    const int32_t m = m_row0 + lane;
+    for (int c = 0; c < CHUNKS; ++c) {
+        const int col0 = (half * CHUNKS + c) * 32;
+        uint32_t r[32];
+        tmem_ld32(t_row + col0, r);
+        tmem_ld_wait();
+        if (arrive && c == CHUNKS - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
+        }
+        if (mode != 0) partial_io(mode, r, slot, h, q, col0, lane);
+        if (mode == 1) continue;
+        const float *bs = bias_s + col0;
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float hv[4];
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                const float v0 = fmaf(__uint_as_float(r[4 * j + e]), sab, bs[4 * j + e]);
+                const float v1 = fmaf(__uint_as_float(r[4 * j + e + 1]), sab, bs[4 * j + e + 1]);
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+                hv[e] = __low2float(b2);
+                hv[e + 1] = __high2float(b2);
+            }
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
+            const uint32_t lo = cvt_fp8x2(__fmul_rn(hv[0], s_out), __fmul_rn(hv[1], s_out), fmt);
+            const uint32_t hi = cvt_fp8x2(__fmul_rn(hv[2], s_out), __fmul_rn(hv[3], s_out), fmt);
+            w[j] = lo | (hi << 16);
+        }
+        const int64_t n0 = n_base + col0;
+        if (m < m_total && n0 < n_total) store_segment(d8 + static_cast<int64_t>(m) * n_total + n0, n_total - n0, w);
+        if (d8t != nullptr) {
+            uint8_t *tile = box + (c & 1) * FP8_TILE_BYTES;
+            *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+            __syncwarp();
+            uint32_t t[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                t[i] = static_cast<uint32_t>(tile[(4 * i) * FP8_TSTRIDE + lane]) |
+                       (static_cast<uint32_t>(tile[(4 * i + 1) * FP8_TSTRIDE + lane]) << 8) |
+                       (static_cast<uint32_t>(tile[(4 * i + 2) * FP8_TSTRIDE + lane]) << 16) |
+                       (static_cast<uint32_t>(tile[(4 * i + 3) * FP8_TSTRIDE + lane]) << 24);
+            }
+            const int64_t n = n0 + lane;
+            if (n < n_total && m_row0 < m_total)
+                store_segment(d8t + n * m_total + m_row0, static_cast<int64_t>(m_total) - m_row0, t);
+        }
+    }
+}
+
 // Shared-memory carve-up common to both kernels.
 struct Smem {
     uint8_t *a, *b, *epi;
@@ -579,7 +696,7 @@ __device__ __forceinline__ void st_release(int32_t *p, int32_t v) {
 // Stream-K segments: a tail (kb0 > 0, the first segment of this cluster)
 // publishes its partial in slot `cluster`; a head (kb0 == 0, kb1 < num_kb,
 // the last segment) adds the partial of slot cluster + 1 before storing D.
-template <bool OUT_BF16>
+template <int OUT>
 __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap *tmap_d, const Params &p,
                                               uint32_t tmem_base, int warp, int lane, int cluster, int clusters,
                                               int m_sub, int rows_per_sub, int row_offset, int acc_bufs,
@@ -590,6 +707,8 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
     float *bias_s = reinterpret_cast<float *>(sm.epi + EPI_WARPS * EPI_BOX_BYTES);
     const int epi_tid = (warp - EPI_WARP0) * 32 + lane;
     const float sab = __fmul_rn(__ldg(p.a_scale_inv), __ldg(p.b_scale_inv));
+    const float s_out = OUT == OUT_FP8 ? __ldg(p.out_scale) : 0.0f;
+    float amax = 0.0f;
     Sched sched(p, cluster, clusters);
     int local = 0, tile, kb0, kb1;
     while (sched.next(tile, kb0, kb1)) {
@@ -629,9 +748,14 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
         for (int h = 0; h < m_sub; ++h) {
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>((acc + h) * ACC_N);
-            epilogue_tile<OUT_BF16>(t_row, lane, box, half, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
-                                    (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32, sab, bias_s,
-                                    empty_addr, h == m_sub - 1, mode, slot, h, q);
+            const int32_t m_row0 = (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32;
+            if constexpr (OUT == OUT_FP8)
+                epilogue_tile_fp8(t_row, lane, box, half, p.out_d8, p.out_d8t, static_cast<int64_t>(n_blk) * ACC_N,
+                                  m_row0, sab, bias_s, empty_addr, h == m_sub - 1, mode, slot, h, q, s_out,
+                                  p.out_fmt, p.M, p.N, amax);
+            else
+                epilogue_tile<OUT == OUT_BF16>(t_row, lane, box, half, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
+                                               m_row0, sab, bias_s, empty_addr, h == m_sub - 1, mode, slot, h, q);
         }
         if (mode == 1) {
             // Publish: every epilogue thread's partial stores precede the flag.
@@ -645,13 +769,22 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             if (epi_tid == 0) *flag = 0;  // consumed; the slot is free for the next launch
         }
     }
+    if constexpr (OUT == OUT_FP8) {
+        // amax of this warp's outputs: one atomic max per warp on the float's
+        // bits (non-negative floats order like integers)
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0 && p.out_amax != nullptr && amax > 0.0f)
+            atomicMax(reinterpret_cast<int *>(p.out_amax), __float_as_int(amax));
+        if (p.out_scale_inv != nullptr && blockIdx.x == 0 && epi_tid == 0) *p.out_scale_inv = __frcp_rn(s_out);
+    }
     if (lane == 0) tma_store_wait_all();
     __syncwarp();
 }
 
 // ------------------------------------------------------------ 1-SM kernel --
 
-template <bool OUT_BF16>
+template <int OUT>
 __global__ void __launch_bounds__(THREADS, 1)
 fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d, const Params p) {
@@ -773,7 +906,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         __syncwarp();
     } else {
-        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u, 0);
+        epilogue_loop<OUT>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u, 0);
     }
 
     tc_fence_before();
@@ -791,7 +924,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
 // tiles c, c + clusters, ...; a pair tile has M_SUB row blocks of 256 rows
 // and 256 columns.  CTA rank r of the pair owns rows r*128..r*128+127 of each
 // row block and loads rows r*128.. of the tile's 256 B rows.
-template <bool OUT_BF16, int M_SUB>
+template <int OUT, int M_SUB>
 __global__ void __launch_bounds__(THREADS, 1)
 fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d, const Params p) {
@@ -929,8 +1062,8 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         __syncwarp();
     } else {
-        epilogue_loop<OUT_BF16>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, M_SUB,
-                                2 * S2_BM, static_cast<int>(rank) * S2_BM, ACC_BUFS, 0u, static_cast<int>(rank));
+        epilogue_loop<OUT>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, M_SUB, 2 * S2_BM,
+                           static_cast<int>(rank) * S2_BM, ACC_BUFS, 0u, static_cast<int>(rank));
     }
 
     tc_fence_before();
@@ -1000,12 +1133,12 @@ int max_pairs(K kernel, int smem_bytes, int (&cached)[64]) {
     return cached[dev];
 }
 
-template <bool OUT_BF16, int M_SUB>
+template <int OUT, int M_SUB>
 cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
                        cudaStream_t stream) {
     static bool done[64] = {};
     static int cached_pairs[64] = {};
-    auto kernel = fp8_gemm_2sm_kernel<OUT_BF16, M_SUB>;
+    auto kernel = fp8_gemm_2sm_kernel<OUT, M_SUB>;
     constexpr int smem = Pair<M_SUB>::SMEM;
     cudaError_t e = set_smem_once(kernel, smem, done);
     if (e != cudaSuccess) return e;
@@ -1015,11 +1148,11 @@ cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
     return launch_pdl(kernel, dim3(2 * pairs), dim3(THREADS), smem, stream, 2, ta, tb, td, p);
 }
 
-template <bool OUT_BF16>
+template <int OUT>
 cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
                        cudaStream_t stream) {
     static bool done[64] = {};
-    auto kernel = fp8_gemm_1sm_kernel<OUT_BF16>;
+    auto kernel = fp8_gemm_1sm_kernel<OUT>;
     cudaError_t e = set_smem_once(kernel, S1_SMEM, done);
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
@@ -1031,24 +1164,30 @@ cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
 
 size_t gemm_workspace_bytes() {
     static int cached[64] = {};
-    const int pairs = max_pairs(fp8_gemm_2sm_kernel<true, 1>, Pair<1>::SMEM, cached);
+    const int pairs = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached);
     return WS_FLAG_BYTES + static_cast<size_t>(pairs) * 2 * WS_SLOT_FLOATS * sizeof(float);
 }
 
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
                          fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
                          void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, void *workspace,
-                         size_t workspace_bytes, cudaStream_t stream) {
-    const bool out_bf16 = d_dtype == FP8DS_BF16;
+                         size_t workspace_bytes, cudaStream_t stream, const GemmCastOut *cast) {
+    const int out = cast != nullptr ? OUT_FP8 : (d_dtype == FP8DS_BF16 ? OUT_BF16 : OUT_F32);
     const bool pair = m > S1_BM;
     // Long contractions amortise the non-overlapped epilogue of the 512-row
     // pair tile; short ones keep the double-buffered 256-row tile.
-    const int m_sub = (pair && m > 2 * S2_BM && k >= 4096) ? 2 : 1;
+    const int m_sub = (pair && m > 2 * S2_BM && k >= FP8DS_MSUB2_MIN_K) ? 2 : 1;
     CUtensorMap ta, tb, td;
     bool ok = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, k, m, k, BK, pair ? S2_BM : S1_BM) &&
-              encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, k, n, k, BK, pair ? S2_BN_HALF : ACC_N) &&
-              (out_bf16 ? encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, n, m, n * 2, 64, 32)
-                        : encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d, n, m, n * 4, 32, 32));
+              encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, k, n, k, BK, pair ? S2_BN_HALF : ACC_N);
+    if (out == OUT_FP8) {
+        // the FP8 epilogue stores with plain global stores; the map stays a
+        // valid description of the codes (it is only prefetched)
+        ok = ok && encode_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT8, d, n, m, n, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    } else {
+        ok = ok && (out == OUT_BF16 ? encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, n, m, n * 2, 64, 32)
+                                    : encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d, n, m, n * 4, 32, 32));
+    }
     if (!ok) {
         set_error("fp8_gemm: cuTensorMapEncodeTiled failed (m=%lld n=%lld k=%lld)", (long long)m, (long long)n,
                   (long long)k);
@@ -1071,11 +1210,17 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.epoch = 0;
     p.flags = nullptr;
     p.partials = nullptr;
+    p.out_scale = cast != nullptr ? cast->scale : nullptr;
+    p.out_amax = cast != nullptr ? cast->amax : nullptr;
+    p.out_scale_inv = cast != nullptr ? cast->scale_inv : nullptr;
+    p.out_fmt = cast != nullptr ? static_cast<int32_t>(cast->fmt) : 0;
+    p.out_d8 = cast != nullptr ? static_cast<uint8_t *>(d) : nullptr;
+    p.out_d8t = cast != nullptr ? cast->d8t : nullptr;
     if (pair && workspace != nullptr && workspace_bytes >= gemm_workspace_bytes()) {
         // Stream-K when whole tiles would leave a ragged last wave: at least
         // one tile per pair, fewer than 8 waves, not a whole number of waves.
         static int cached[64] = {};
-        const int cap = max_pairs(fp8_gemm_2sm_kernel<true, 1>, Pair<1>::SMEM, cached);
+        const int cap = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached);
         const int tiles = p.tiles_m * p.tiles_n;
         if (tiles >= cap && tiles % cap != 0 && tiles < 8 * cap && cap <= static_cast<int>(WS_FLAG_BYTES / 8)) {
             static std::atomic<uint32_t> launches{0};
@@ -1088,12 +1233,19 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
         }
     }
     cudaError_t e;
-    if (pair && m_sub == 2)
-        e = out_bf16 ? launch_2sm<true, 2>(ta, tb, td, p, stream) : launch_2sm<false, 2>(ta, tb, td, p, stream);
-    else if (pair)
-        e = out_bf16 ? launch_2sm<true, 1>(ta, tb, td, p, stream) : launch_2sm<false, 1>(ta, tb, td, p, stream);
-    else
-        e = out_bf16 ? launch_1sm<true>(ta, tb, td, p, stream) : launch_1sm<false>(ta, tb, td, p, stream);
+    if (pair && m_sub == 2) {
+        e = out == OUT_FP8    ? launch_2sm<OUT_FP8, 2>(ta, tb, td, p, stream)
+            : out == OUT_BF16 ? launch_2sm<OUT_BF16, 2>(ta, tb, td, p, stream)
+                              : launch_2sm<OUT_F32, 2>(ta, tb, td, p, stream);
+    } else if (pair) {
+        e = out == OUT_FP8    ? launch_2sm<OUT_FP8, 1>(ta, tb, td, p, stream)
+            : out == OUT_BF16 ? launch_2sm<OUT_BF16, 1>(ta, tb, td, p, stream)
+                              : launch_2sm<OUT_F32, 1>(ta, tb, td, p, stream);
+    } else {
+        e = out == OUT_FP8    ? launch_1sm<OUT_FP8>(ta, tb, td, p, stream)
+            : out == OUT_BF16 ? launch_1sm<OUT_BF16>(ta, tb, td, p, stream)
+                              : launch_1sm<OUT_F32>(ta, tb, td, p, stream);
+    }
     if (e != cudaSuccess) {
         set_error("fp8_gemm: launch failed: %s", cudaGetErrorString(e));
         return FP8DS_ERR_CUDA;

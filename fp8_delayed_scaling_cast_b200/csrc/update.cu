@@ -6,8 +6,9 @@
 // "FP8 scale update kernel" of "[PyTorch] Refactor FP8 workspaces in linear
 // modules"; all linears' amax buffers handled together as in "support delayed
 // scaling of weight in float8 all-gather"):
-//   a = max over the history window; scale = fp8_max / a when a > 0, a finite
-//   and the quotient finite, else the scale is kept; scale_inv = 1 / scale;
+//   a = max over the history window (amax_compute_algo "max"), or the
+//   current step's amax alone ("most_recent"); scale = fp8_max / a when a > 0,
+//   a finite and the quotient finite, else the scale is kept; scale_inv = 1 / scale;
 //   the history rolls by one slot (slot 0 moves to the end) and slot 0 is
 //   cleared for the next step's amax.
 //
@@ -25,14 +26,15 @@ constexpr int U_THREADS = 128;
 
 __global__ void __launch_bounds__(U_THREADS)
 update_scales_kernel(int64_t T, int H, float *__restrict__ hist, float *__restrict__ scale,
-                     float *__restrict__ scale_inv, const uint8_t *__restrict__ formats) {
+                     float *__restrict__ scale_inv, const uint8_t *__restrict__ formats, int most_recent) {
     ptx::pdl_wait();
     ptx::pdl_launch_dependents();
     const int64_t t = static_cast<int64_t>(blockIdx.x) * U_THREADS + threadIdx.x;
     if (t >= T) return;
     const float first = hist[t];
     float a = first;
-    for (int h = 1; h < H; ++h) a = fmaxf(a, hist[static_cast<int64_t>(h) * T + t]);
+    if (!most_recent)
+        for (int h = 1; h < H; ++h) a = fmaxf(a, hist[static_cast<int64_t>(h) * T + t]);
     const float fp8_max = formats[t] == FP8DS_E4M3 ? 448.0f : 57344.0f;
     float s = scale[t];
     if (a > 0.0f && isfinite(a)) {
@@ -51,11 +53,12 @@ update_scales_kernel(int64_t T, int H, float *__restrict__ hist, float *__restri
 
 cudaError_t launch_update_scales(int64_t num_tensors, int32_t hist_len, float *amax_history,
                                  float *scale, float *scale_inv, const uint8_t *formats,
-                                 cudaStream_t stream) {
+                                 fp8ds_amax_algo algo, cudaStream_t stream) {
     if (num_tensors == 0) return cudaSuccess;
     const int64_t blocks = (num_tensors + U_THREADS - 1) / U_THREADS;
     return launch_pdl(update_scales_kernel, dim3(static_cast<unsigned>(blocks)), dim3(U_THREADS), 0, stream, 1,
-                      num_tensors, static_cast<int>(hist_len), amax_history, scale, scale_inv, formats);
+                      num_tensors, static_cast<int>(hist_len), amax_history, scale, scale_inv, formats,
+                      algo == FP8DS_AMAX_MOST_RECENT ? 1 : 0);
 }
 
 }  // namespace fp8ds

@@ -57,8 +57,12 @@ typedef enum { FP8DS_E4M3 = 0, FP8DS_E5M2 = 1 } fp8ds_format;
 /* High-precision element types. */
 typedef enum { FP8DS_F32 = 0, FP8DS_BF16 = 1 } fp8ds_dtype;
 
-/* Amax reduction over the history window [TE761 recipe: amax_compute_algo]. */
-typedef enum { FP8DS_AMAX_MAX = 0 } fp8ds_amax_algo;
+/*
+ * Amax used by the update [TE761 recipe: amax_compute_algo, "max" in the
+ * repro]: MAX = the max over the history window; MOST_RECENT = the amax
+ * recorded in the current step alone (the recipe parameter's other choice).
+ */
+typedef enum { FP8DS_AMAX_MAX = 0, FP8DS_AMAX_MOST_RECENT = 1 } fp8ds_amax_algo;
 
 /* A cudaStream_t. */
 typedef struct CUstream_st *fp8ds_stream;
@@ -104,12 +108,47 @@ fp8ds_status fp8_cast_transpose_amax(const void *x, fp8ds_dtype x_dtype, int64_t
                                      fp8ds_stream stream);
 
 /*
+ * fp8_cast_transpose_amax_noop -- fp8_cast_transpose_amax with a device-side
+ * skip flag (TE's noop flag) [TE820: with CUDA graphs the choice of casting or
+ * reusing the cached weight must be made on the GPU at replay time].
+ *   noop_flag  device int32, read by the kernel when it runs: non-zero ->
+ *              nothing is written (y, yt, amax, scale_inv keep their values);
+ *              zero -> exactly fp8_cast_transpose_amax.
+ * Errors: as fp8_cast_transpose_amax; FP8DS_ERR_INVALID_ARG for a NULL flag.
+ */
+fp8ds_status fp8_cast_transpose_amax_noop(const void *x, fp8ds_dtype x_dtype, int64_t rows,
+                                          int64_t cols, fp8ds_format fmt, const float *scale,
+                                          uint8_t *y, uint8_t *yt, float *amax, float *scale_inv,
+                                          const int32_t *noop_flag, fp8ds_stream stream);
+
+/*
+ * fp8_cast_transpose_amax_dynamic -- dynamic scaling, for comparison with the
+ * delayed recipe [F8E312: delayed vs dynamic scaling; "delayed scaling is
+ * theoretically faster than dynamic scaling (less memory reads)" is the
+ * page's claim this measures].  The scale comes from the tensor itself, so
+ * the input is read twice:
+ *   *amax      = max |x|                         (overwritten; NaN ignored)
+ *   *scale     = fl32(fp8_max / *amax) if that amax is > 0 and finite and the
+ *                quotient finite; otherwise the value passed in is kept
+ *   *scale_inv = fl32(1 / *scale)                (if not NULL)
+ *   y, yt      = fp8_cast_transpose_amax(x, fmt, scale) (no amax accumulation)
+ * Arguments and layouts as fp8_cast_transpose_amax; scale is in/out, amax
+ * required.  Enqueues a 4-byte memset and three kernels on `stream`.
+ * Errors: as fp8_cast_transpose_amax; FP8DS_ERR_INVALID_ARG for NULL amax.
+ */
+fp8ds_status fp8_cast_transpose_amax_dynamic(const void *x, fp8ds_dtype x_dtype, int64_t rows,
+                                             int64_t cols, fp8ds_format fmt, float *scale,
+                                             uint8_t *y, uint8_t *yt, float *amax,
+                                             float *scale_inv, fp8ds_stream stream);
+
+/*
  * fp8_update_scales -- the delayed-scaling recipe update of T FP8 meta tensors
  * in ONE launch [TE820 "FP8 scale update kernel"; TE761 DelayedScaling(
  * amax_history_len=16, amax_compute_algo="max"); F8E312 amax buffers of all
  * linears handled together].  For every t < num_tensors:
  *
- *   a          = max_h amax_history[h, t]                (window of hist_len steps)
+ *   a          = max_h amax_history[h, t]   (algo MAX: window of hist_len steps)
+ *                amax_history[0, t]          (algo MOST_RECENT: this step's amax)
  *   scale[t]   = fl32(fp8_max(formats[t]) / a)  if a > 0, a finite and the
  *                quotient finite; otherwise scale[t] is kept
  *   scale_inv[t] = fl32(1 / scale[t])                   (the meta's copy; FP8
@@ -122,7 +161,7 @@ fp8ds_status fp8_cast_transpose_amax(const void *x, fp8ds_dtype x_dtype, int64_t
  *                max-reduction of row 0 is one contiguous buffer).
  *   scale, scale_inv [num_tensors] fp32;  formats [num_tensors] uint8 (fp8ds_format).
  * Errors: FP8DS_ERR_INVALID_ARG for num_tensors < 0, hist_len < 1 or NULL
- * pointers; FP8DS_ERR_UNSUPPORTED for an algo other than FP8DS_AMAX_MAX.
+ * pointers; FP8DS_ERR_UNSUPPORTED for an unknown algo.
  */
 fp8ds_status fp8_update_scales(int64_t num_tensors, int32_t hist_len, float *amax_history,
                                float *scale, float *scale_inv, const uint8_t *formats,
@@ -214,6 +253,33 @@ fp8ds_status fp8_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float 
                               int64_t m, int64_t n, int64_t k, fp8ds_stream stream);
 
 /*
+ * fp8_gemm_cast -- the GEMM with an FP8 output for the next layer [PTFP8
+ * torch._scaled_mm with out_dtype=float8_e4m3fn, returning the output and its
+ * amax].  Reading used here: the FP8 output is the cast that the next layer
+ * would apply to this GEMM's bf16 output, done inside the epilogue, so fusing
+ * changes no result:
+ *   h[m,n]   = bf16_rne((sum_k dec(a[m,k]) dec(b[n,k])) * *a_scale_inv
+ *              * *b_scale_inv (+ bias[n]))      exactly fp8_gemm's bf16 output
+ *   d8[m,n]  = sat_rne_fp8(fl32(h[m,n] * *out_scale))  (out_fmt)
+ *   d8t[n,m] = d8[m,n]                              (if d8t is not NULL)
+ *   *out_amax = max(*out_amax, max |h|)             (if not NULL; NaN ignored)
+ *   *out_scale_inv = fl32(1 / *out_scale)           (if not NULL)
+ * i.e. fp8_cast_transpose_amax(h, out_fmt, out_scale, d8, d8t, out_amax,
+ * out_scale_inv) without h ever reaching memory.  out_scale is normally the
+ * next layer's delayed scale (meta.scale[t]) and out_amax its history slot 0
+ * (amax_history[0, t]).
+ *   a, b, bias, m, n, k, formats: as fp8_gemm.
+ *   d8 [m, n] uint8, d8t [n, m] uint8 or NULL; out_scale [1] fp32.
+ * Requirements: as fp8_gemm, plus n % 16 == 0, m % 16 == 0 when d8t is not
+ * NULL, d8 / d8t 16-byte aligned.  Errors: as fp8_gemm.
+ */
+fp8ds_status fp8_gemm_cast(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
+                           const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
+                           const void *bias, fp8ds_dtype bias_dtype, int64_t m, int64_t n, int64_t k,
+                           fp8ds_format out_fmt, const float *out_scale, uint8_t *d8, uint8_t *d8t,
+                           float *out_amax, float *out_scale_inv, fp8ds_stream stream);
+
+/*
  * Packed FP8 meta of T tensors (the DelayedScaling state [TE761; F8E312
  * _amax_history_buffer / _scale_buffer]).  All arrays are caller-owned device
  * memory; amax_history is [hist_len, num_tensors] slot-major, zero-filled and
@@ -249,6 +315,7 @@ typedef struct {
     int32_t cache_valid;
     void *workspace;           /* NULL or the GEMM workspace of fp8_gemm_ex */
     size_t workspace_bytes;
+    const int32_t *w_noop_flag; /* NULL or a device int32: see fp8_linear_fwd */
 } fp8ds_linear;
 
 /*
@@ -261,6 +328,12 @@ typedef struct {
  *      scale_inv into *w_scale_inv; sets cache_valid.  With 0 and a valid
  *      cache the cached weight and its frozen scale_inv are reused;
  *   3. y = fp8_gemm(x8, w8, *x_scale_inv, *w_scale_inv, bias).
+ * With lin->w_noop_flag set, step 2 is decided on the device instead [TE820:
+ * a CUDA graph captured around the forward must not bake in the weight-cache
+ * decision]: the weight cast is always enqueued and skips itself while
+ * *w_noop_flag != 0 at run time (the cache and its frozen scale_inv stay);
+ * is_first_microbatch is then ignored for the weight.  Write 0 to the flag
+ * for a microbatch that must refresh the cache, 1 for the others.
  *   x [m, in_features] (x_dtype); y [m, out_features] (y_dtype);
  *   x8 [m, in_features], x8t [in_features, m] or NULL (needed by the backward).
  * The delayed-scaling update is not part of the forward: call
@@ -288,6 +361,48 @@ fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, con
                             const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
                             float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv,
                             fp8ds_stream stream);
+
+/*
+ * Options of fp8_linear_fwd_ex / fp8_linear_bwd_ex: how the FP8 tensors pass
+ * between consecutive linears without a separate cast (zero-initialise, set
+ * out_meta = -1 for "no FP8 output").
+ *   in_cast   non-zero: the input (forward) or output gradient (backward) is
+ *             already cast -- x8 / x8t / x_scale_inv (dy8 / dy8t /
+ *             dy_scale_inv) hold it, written by the neighbouring layer's
+ *             fused epilogue, which also recorded its amax -- so x (dy) may be
+ *             NULL and no cast is enqueued.
+ *   out_meta  >= 0: the forward output (backward dgrad) is cast in the GEMM
+ *             epilogue as fp8_gemm_cast does, with meta.scale[out_meta]
+ *             (format e4m3 forward, e5m2 backward: HYBRID), its amax recorded
+ *             in amax_history[0, out_meta]; y (dx) is not written.  -1: none.
+ *   out8      [m, out_features] forward / [m, in_features] backward codes.
+ *   out8t     their transpose, or NULL.
+ *   out_scale_inv  [1] private scale_inv of out8 (fl32(1 / scale)).
+ * With both, an MLP hands H and dH from GEMM to GEMM in FP8: fc1's forward
+ * writes fc2's x8 / x8t (out_meta = fc2's meta_in) and fc2's backward writes
+ * fc1's dy8 / dy8t (out_meta = fc1's meta_grad).  The results are those of
+ * the unfused calls: the same bytes, amaxes and scales.
+ */
+typedef struct {
+    int32_t in_cast;
+    int32_t out_meta;
+    uint8_t *out8;
+    uint8_t *out8t;
+    float *out_scale_inv;
+} fp8ds_fp8_io;
+
+/* fp8_linear_fwd with the options above (io may be NULL: same as fp8_linear_fwd). */
+fp8ds_status fp8_linear_fwd_ex(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x,
+                               fp8ds_dtype x_dtype, int64_t m, void *y, fp8ds_dtype y_dtype,
+                               int32_t is_first_microbatch, uint8_t *x8, uint8_t *x8t,
+                               float *x_scale_inv, const fp8ds_fp8_io *io, fp8ds_stream stream);
+
+/* fp8_linear_bwd with the options above (io may be NULL: same as fp8_linear_bwd). */
+fp8ds_status fp8_linear_bwd_ex(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy,
+                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8t,
+                               const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
+                               float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv,
+                               const fp8ds_fp8_io *io, fp8ds_stream stream);
 
 /* Message describing the last error returned on the calling thread ("" if none). */
 const char *fp8ds_last_error(void);

@@ -30,7 +30,9 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ("fp8_quantize", "fp8_cast_transpose_amax", "fp8_update_scales", "fp8_gemm",
-              "fp8_gemm_ex", "fp8_gemm_workspace_size",
+              "fp8_gemm_ex", "fp8_gemm_workspace_size", "fp8_gemm_noalloc", "fp8_gemm_cast",
+              "fp8_linear_fwd_ex", "fp8_linear_bwd_ex", "fp8_cast_transpose_amax_noop",
+              "fp8_cast_transpose_amax_dynamic",
               "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
               "fp8ds_version"):
         assert n in names
@@ -92,7 +94,7 @@ def test_cast_and_update_argument_checks(lib):
     assert L.fp8_update_scales(-1, 16, FAKE, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG
     assert L.fp8_update_scales(4, 0, FAKE, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG
     assert L.fp8_update_scales(4, 16, None, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG
-    assert L.fp8_update_scales(4, 16, FAKE, FAKE, FAKE, FAKE, 1, s) == lib.ERR_UNSUPPORTED
+    assert L.fp8_update_scales(4, 16, FAKE, FAKE, FAKE, FAKE, 2, s) == lib.ERR_UNSUPPORTED
     # zero tensors: nothing to do, nothing launched
     assert L.fp8_update_scales(0, 16, None, None, None, None, 0, s) == lib.OK
 
@@ -116,3 +118,59 @@ def test_linear_argument_checks(lib):
     r = L.fp8_linear_bwd(ctypes.byref(lin), ctypes.byref(meta), FAKE, 1, 128, FAKE, FAKE, FAKE, 1,
                          FAKE, FAKE, FAKE, FAKE, s)
     assert r == lib.ERR_INVALID_ARG and "cache" in lib.fp8ds_last_error()
+
+
+def test_gemm_cast_argument_checks(lib):
+    """The FP8-output GEMM: codes need n % 16 (row pitch) and, with the
+    transpose, m % 16; the output format must be known; the scale and the
+    output must not be NULL.  Every call below fails a check (no launch)."""
+    L = lib._lib
+    s = P(0)
+
+    def call(m=128, n=256, k=128, fmt=0, scale=FAKE, d8=FAKE, d8t=None):
+        return L.fp8_gemm_cast(FAKE, 0, FAKE, FAKE, 0, FAKE, None, 0, m, n, k, fmt, scale, d8, d8t, None, None, s)
+
+    assert call(n=264) == lib.ERR_INVALID_ARG and "multiple of 16" in lib.fp8ds_last_error()
+    assert call(m=120, d8t=FAKE) == lib.ERR_INVALID_ARG and "transposed" in lib.fp8ds_last_error()
+    assert call(fmt=5) == lib.ERR_INVALID_ARG and "format" in lib.fp8ds_last_error()
+    assert call(scale=None) == lib.ERR_INVALID_ARG
+    assert call(d8=None) == lib.ERR_INVALID_ARG
+    assert call(d8t=FAKE_ODD) == lib.ERR_INVALID_ARG and "aligned" in lib.fp8ds_last_error()
+    assert call(k=120) == lib.ERR_INVALID_ARG
+
+
+def test_linear_ex_argument_checks(lib):
+    """FP8 hand-over options of the _ex linear calls (every call fails a check)."""
+    L = lib._lib
+    s = P(0)
+    meta = lib._Meta(FAKE, FAKE, FAKE, FAKE, 4, 16)
+    lin = lib._Linear(FAKE, None, 0, 256, 520, FAKE, FAKE, FAKE, 0, 1, 2, 0, None, 0)
+
+    def fwd(io, x=FAKE, y=FAKE, lin_=lin):
+        return L.fp8_linear_fwd_ex(ctypes.byref(lin_), ctypes.byref(meta), x, 0, 128, y, 1, 1, FAKE, FAKE, FAKE,
+                                   ctypes.byref(io), s)
+
+    # output meta out of range
+    assert fwd(lib._Fp8Io(0, 9, FAKE, FAKE, FAKE)) == lib.ERR_INVALID_ARG and "out of range" in lib.fp8ds_last_error()
+    # without in_cast the input must be given
+    assert fwd(lib._Fp8Io(0, -1, None, None, None), x=None) == lib.ERR_INVALID_ARG
+    # FP8 output requested but no buffer for it
+    assert fwd(lib._Fp8Io(0, 3, None, None, None)) == lib.ERR_INVALID_ARG
+    # 520 output features: bf16 is fine (n % 8) but FP8 codes need n % 16
+    assert fwd(lib._Fp8Io(1, 3, FAKE, None, FAKE), x=None, y=None) == lib.ERR_INVALID_ARG and \
+        "multiple of 16" in lib.fp8ds_last_error()
+
+    def bwd(io, lin_, dy=FAKE, m=128):
+        return L.fp8_linear_bwd_ex(ctypes.byref(lin_), ctypes.byref(meta), dy, 1, m, FAKE, FAKE, FAKE, 1, FAKE,
+                                   FAKE, FAKE, FAKE, ctypes.byref(io), s)
+
+    assert bwd(lib._Fp8Io(0, -1, None, None, None), lin) == lib.ERR_INVALID_ARG and \
+        "cache" in lib.fp8ds_last_error()
+    cached = lib._Linear(FAKE, None, 0, 256, 512, FAKE, FAKE, FAKE, 0, 1, 2, 1, None, 0)
+    # without in_cast the gradient must be given
+    assert bwd(lib._Fp8Io(0, -1, None, None, None), cached, dy=None) == lib.ERR_INVALID_ARG
+    # transposed FP8 dgrad needs m % 16
+    assert bwd(lib._Fp8Io(1, 3, FAKE, FAKE, FAKE), cached, dy=None, m=120) == lib.ERR_INVALID_ARG and \
+        "transposed" in lib.fp8ds_last_error()
+    assert bwd(lib._Fp8Io(1, 11, FAKE, FAKE, FAKE), cached, dy=None) == lib.ERR_INVALID_ARG and \
+        "out of range" in lib.fp8ds_last_error()

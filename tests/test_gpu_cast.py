@@ -216,3 +216,54 @@ def test_amax_accumulates_across_calls(fp8):
         _, _, ref, _ = o.cast_transpose_amax(x.numpy(), o.E4M3, 1.0, ref, transpose=False)
     torch.cuda.synchronize()
     assert_f32_bits_equal(am.cpu().numpy(), [ref], "amax")
+
+
+def _oracle_dynamic(x_host, fmt, scale_in):
+    """Dynamic scaling from oracle pieces: the tensor's amax, the update with a
+    window of one on it (scale kept when the amax is not positive and finite),
+    then the cast with that scale."""
+    am = o.amax(x_host)
+    _, s, si = o.update_scales(np.array([[am]], np.float32), [scale_in], [1.0], [FMT[fmt]], o.AMAX_MOST_RECENT)
+    y, yt, _, si2 = o.cast_transpose_amax(x_host, FMT[fmt], s[0])
+    assert si2 == si[0]
+    return y, yt, am, s[0], si[0]
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("dtype,rows,cols", [("bf16", 8192, 2048), ("bf16", 100, 36), ("f32", 256, 192),
+                                             ("f32", 37, 53)])
+def test_dynamic_scaling_cast(fp8, fmt, dtype, rows, cols):
+    x = inputs.normal((rows, cols), inputs.gen(rows + cols), 2.0)
+    x[rows // 3, cols // 2] = -300.0
+    if dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    xh = host_bits(x)
+    xd = x.cuda()
+    y = torch.full((rows, cols), 0xAA, dtype=torch.uint8, device="cuda")
+    yt = torch.full((cols, rows), 0xAA, dtype=torch.uint8, device="cuda")
+    s = torch.tensor([3.0], device="cuda")
+    am = torch.tensor([12345.0], device="cuda")       # overwritten, not accumulated
+    si = torch.zeros(1, device="cuda")
+    fp8.fp8_cast_transpose_amax_dynamic(xd, fmt, s, y, yt, am, si)
+    ry, ryt, ram, rs, rsi = _oracle_dynamic(xh, fmt, np.float32(3.0))
+    torch.cuda.synchronize()
+    assert_bytes_equal(u8(y), ry, "y")
+    assert_bytes_equal(u8(yt), ryt, "yt")
+    assert_f32_bits_equal(am.cpu().numpy(), [ram], "amax")
+    assert_f32_bits_equal(s.cpu().numpy(), [rs], "scale")
+    assert_f32_bits_equal(si.cpu().numpy(), [rsi], "scale_inv")
+    # the largest magnitude lands exactly on the format's max
+    assert (ry.reshape(-1)[np.argmax(np.abs(o.bf16_bits_to_f32(xh) if dtype == "bf16" else xh))] & 0x7F) == \
+        (0x7E if fmt == "e4m3" else 0x7B)
+
+
+def test_dynamic_scaling_all_zero_keeps_scale(fp8):
+    x = torch.zeros(64, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((64, 64), 0xAA, dtype=torch.uint8, device="cuda")
+    s = torch.tensor([5.0], device="cuda")
+    am = torch.tensor([7.0], device="cuda")
+    si = torch.zeros(1, device="cuda")
+    fp8.fp8_cast_transpose_amax_dynamic(x, "e4m3", s, y, None, am, si)
+    torch.cuda.synchronize()
+    assert am.item() == 0.0 and s.item() == 5.0 and si.item() == np.float32(0.2)
+    assert bool((y == 0).all())

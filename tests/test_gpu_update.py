@@ -17,9 +17,10 @@ def fp8():
     return binding
 
 
+@pytest.mark.parametrize("algo", [o.AMAX_MAX, o.AMAX_MOST_RECENT])
 @pytest.mark.parametrize("T,H", [(1, 16), (2, 16), (18, 16), (576, 16), (1000, 16), (7, 1),
                                  (130, 3), (33, 1024)])
-def test_update_trajectory(fp8, T, H):
+def test_update_trajectory(fp8, T, H, algo):
     rng = np.random.default_rng(T * 31 + H)
     fmts = rng.integers(0, 2, T).astype(np.uint8)
     hist = np.zeros((H, T), np.float32)
@@ -34,8 +35,8 @@ def test_update_trajectory(fp8, T, H):
             am[-1] = np.float32(1e-44)
         hist[0] = am
         dh[0].copy_(torch.from_numpy(am))
-        hist, scale, scale_inv = o.update_scales(hist, scale, scale_inv, fmts)
-        fp8.fp8_update_scales(dh, ds, dsi, df)
+        hist, scale, scale_inv = o.update_scales(hist, scale, scale_inv, fmts, algo)
+        fp8.fp8_update_scales(dh, ds, dsi, df, algo=algo)
         torch.cuda.synchronize()
         assert_f32_bits_equal(dh.cpu().numpy(), hist, "history step %d" % step)
         assert_f32_bits_equal(ds.cpu().numpy(), scale, "scale step %d" % step)
