@@ -485,39 +485,44 @@ __device__ __forceinline__ void partial_io(int mode, uint32_t (&r)[32], float *s
 
 // mode 0: convert and store D; mode 1: store the raw partial (no D); mode 2:
 // add the partial of the other cluster, then convert and store D.
+// The warp reads its 128 columns as four 32-column TMEM loads (which keeps
+// the live registers within the 168 that 10 warps per SM allow).  The load
+// of chunk c + 1 is issued as soon as chunk c has been converted, into the
+// same registers, so its latency overlaps chunk c's staging and store; the
+// loop is fully unrolled so that every load has its own registers.
 template <bool OUT_BF16>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *box, int half,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                               float sab, const float *bias_s, uint32_t empty_bar_cluster,
                                               bool arrive, int mode, float *slot, int h, int q) {
     constexpr int COLS_PER_BOX = OUT_BF16 ? 64 : 32;
-    constexpr int BOXES = ACC_N / COLS_PER_BOX;
-    constexpr int HALF = BOXES / 2;
-    // 32 accumulator columns per TMEM load (fp32: a whole 128-byte staging
-    // row; bf16: half of one), which keeps the live registers within the
-    // 168 that 10 warps per SM allow.
     constexpr int LOADS_PER_BOX = OUT_BF16 ? 2 : 1;
-    for (int bx = half * HALF; bx < (half + 1) * HALF; ++bx) {
-        // Staging buffer reuse: the previous store from it must have finished
-        // reading shared memory.
-        if (lane == 0) tma_store_wait_read<0>();
-        __syncwarp();
+    constexpr int CHUNKS = ACC_N / 32 / 2;
+    uint32_t r[32];
+    tmem_ld32(t_row + half * CHUNKS * 32, r);
+    tmem_ld_wait();
 #pragma unroll
-        for (int hh = 0; hh < LOADS_PER_BOX; ++hh) {
-            const int col0 = bx * COLS_PER_BOX + hh * 32;
-            uint32_t r[32];
-            tmem_ld32(t_row + col0, r);
-            tmem_ld_wait();
-            if (arrive && bx == (half + 1) * HALF - 1 && hh == LOADS_PER_BOX - 1) {
-                tc_fence_before();
+    for (int c = 0; c < CHUNKS; ++c) {
+        const int col0 = (half * CHUNKS + c) * 32;
+        const int hh = c % LOADS_PER_BOX;
+        const int bx = col0 / COLS_PER_BOX;
+        if (arrive && c == CHUNKS - 1) {
+            // every TMEM load of this accumulator has completed
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
+        }
+        if (mode != 0) partial_io(mode, r, slot, h, q, col0, lane);
+        if (mode != 1) {
+            if (hh == 0) {
+                // Staging buffer reuse: the previous store from it must have
+                // finished reading shared memory.
+                if (lane == 0) tma_store_wait_read<0>();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
             }
-            if (mode != 0) partial_io(mode, r, slot, h, q, col0, lane);
-            if (mode == 1) continue;
             const float *bs = bias_s + col0;
             // 32 columns -> 128 bytes (fp32) or 64 bytes (bf16) of row `lane`;
-            // 16-byte chunk c of the row goes to chunk c ^ (lane & 7) (the
+            // 16-byte chunk k of the row goes to chunk k ^ (lane & 7) (the
             // 128-byte swizzle the output tensor map expects).
             if (OUT_BF16) {
                 uint32_t packed[16];
@@ -529,31 +534,52 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
                     packed[j] = *reinterpret_cast<uint32_t *>(&hv);
                 }
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int pc = (hh * 4 + c) ^ (lane & 7);
+                for (int k = 0; k < 4; ++k) {
+                    const int pc = (hh * 4 + k) ^ (lane & 7);
                     *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
-                        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+                        make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
                 }
             } else {
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int pc = c ^ (lane & 7);
+                for (int k = 0; k < 8; ++k) {
+                    const int pc = k ^ (lane & 7);
                     *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
-                        make_uint4(__float_as_uint(fmaf(__uint_as_float(r[4 * c]), sab, bs[4 * c])),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * c + 1]), sab, bs[4 * c + 1])),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * c + 2]), sab, bs[4 * c + 2])),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * c + 3]), sab, bs[4 * c + 3])));
+                        make_uint4(__float_as_uint(fmaf(__uint_as_float(r[4 * k]), sab, bs[4 * k])),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 1]), sab, bs[4 * k + 1])),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 2]), sab, bs[4 * k + 2])),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 3]), sab, bs[4 * k + 3])));
                 }
             }
         }
-        if (mode == 1) continue;
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + bx * COLS_PER_BOX), m_row0);
-            tma_store_commit();
+        if (c + 1 < CHUNKS) tmem_ld32(t_row + col0 + 32, r);
+        if (mode != 1 && hh == LOADS_PER_BOX - 1) {
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + bx * COLS_PER_BOX), m_row0);
+                tma_store_commit();
+            }
         }
+        if (c + 1 < CHUNKS) tmem_ld_wait();
     }
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic; each lane rounds exactly as
+// the scalar fmaf / __fmul_rn).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
 }
 
 // Two FP8 codes (saturating, round to nearest even) packed in 16 bits:
@@ -600,55 +626,66 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
                                                   int32_t m_total, int32_t n_total, float &amax) {
     constexpr int CHUNKS = ACC_N / 32 / 2;
     const int32_t m = m_row0 + lane;
+    const uint64_t sab2 = pack_f32x2(sab, sab);
+    const uint64_t s2 = pack_f32x2(s_out, s_out);
+    uint32_t r[32];
+    tmem_ld32(t_row + half * CHUNKS * 32, r);
+    tmem_ld_wait();
+#pragma unroll
     for (int c = 0; c < CHUNKS; ++c) {
         const int col0 = (half * CHUNKS + c) * 32;
-        uint32_t r[32];
-        tmem_ld32(t_row + col0, r);
-        tmem_ld_wait();
         if (arrive && c == CHUNKS - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
         }
         if (mode != 0) partial_io(mode, r, slot, h, q, col0, lane);
-        if (mode == 1) continue;
-        const float *bs = bias_s + col0;
         uint32_t w[8];
+        if (mode != 1) {
+            const float *bs = bias_s + col0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float hv[4];
-#pragma unroll
-            for (int e = 0; e < 4; e += 2) {
-                const float v0 = fmaf(__uint_as_float(r[4 * j + e]), sab, bs[4 * j + e]);
-                const float v1 = fmaf(__uint_as_float(r[4 * j + e + 1]), sab, bs[4 * j + e + 1]);
-                const __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
-                hv[e] = __low2float(b2);
-                hv[e + 1] = __high2float(b2);
+            for (int j = 0; j < 8; ++j) {
+                const float4 b = *reinterpret_cast<const float4 *>(bs + 4 * j);
+                const uint64_t v01 = fma_f32x2(pack_f32x2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])),
+                                               sab2, pack_f32x2(b.x, b.y));
+                const uint64_t v23 = fma_f32x2(
+                    pack_f32x2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), sab2,
+                    pack_f32x2(b.z, b.w));
+                const __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
+                const __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
+                const float h0 = __low2float(ha), h1 = __high2float(ha);
+                const float h2 = __low2float(hb), h3 = __high2float(hb);
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+                const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
+                const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
+                w[j] = cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) | (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
             }
-            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(hv[0]), fabsf(hv[1])), fmaxf(fabsf(hv[2]), fabsf(hv[3]))));
-            const uint32_t lo = cvt_fp8x2(__fmul_rn(hv[0], s_out), __fmul_rn(hv[1], s_out), fmt);
-            const uint32_t hi = cvt_fp8x2(__fmul_rn(hv[2], s_out), __fmul_rn(hv[3], s_out), fmt);
-            w[j] = lo | (hi << 16);
         }
-        const int64_t n0 = n_base + col0;
-        if (m < m_total && n0 < n_total) store_segment(d8 + static_cast<int64_t>(m) * n_total + n0, n_total - n0, w);
-        if (d8t != nullptr) {
-            uint8_t *tile = box + (c & 1) * FP8_TILE_BYTES;
-            *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE) = make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE + 16) = make_uint4(w[4], w[5], w[6], w[7]);
-            __syncwarp();
-            uint32_t t[8];
+        // the registers of r are free: start the next chunk's TMEM load
+        if (c + 1 < CHUNKS) tmem_ld32(t_row + col0 + 32, r);
+        if (mode != 1) {
+            const int64_t n0 = n_base + col0;
+            if (m < m_total && n0 < n_total)
+                store_segment(d8 + static_cast<int64_t>(m) * n_total + n0, n_total - n0, w);
+            if (d8t != nullptr) {
+                uint8_t *tile = box + (c & 1) * FP8_TILE_BYTES;
+                *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                __syncwarp();
+                uint32_t t[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                t[i] = static_cast<uint32_t>(tile[(4 * i) * FP8_TSTRIDE + lane]) |
-                       (static_cast<uint32_t>(tile[(4 * i + 1) * FP8_TSTRIDE + lane]) << 8) |
-                       (static_cast<uint32_t>(tile[(4 * i + 2) * FP8_TSTRIDE + lane]) << 16) |
-                       (static_cast<uint32_t>(tile[(4 * i + 3) * FP8_TSTRIDE + lane]) << 24);
+                for (int i = 0; i < 8; ++i) {
+                    t[i] = static_cast<uint32_t>(tile[(4 * i) * FP8_TSTRIDE + lane]) |
+                           (static_cast<uint32_t>(tile[(4 * i + 1) * FP8_TSTRIDE + lane]) << 8) |
+                           (static_cast<uint32_t>(tile[(4 * i + 2) * FP8_TSTRIDE + lane]) << 16) |
+                           (static_cast<uint32_t>(tile[(4 * i + 3) * FP8_TSTRIDE + lane]) << 24);
+                }
+                const int64_t n = n0 + lane;
+                if (n < n_total && m_row0 < m_total)
+                    store_segment(d8t + n * m_total + m_row0, static_cast<int64_t>(m_total) - m_row0, t);
             }
-            const int64_t n = n0 + lane;
-            if (n < n_total && m_row0 < m_total)
-                store_segment(d8t + n * m_total + m_row0, static_cast<int64_t>(m_total) - m_row0, t);
         }
+        if (c + 1 < CHUNKS) tmem_ld_wait();
     }
 }
 
