@@ -45,6 +45,19 @@ TOKENS, HIDDEN, FFN = inputs.TOKENS, inputs.HIDDEN, inputs.MLP_RATIO * inputs.HI
 GEMM_FLOP = 2.0 * TOKENS * FFN * HIDDEN          # every GEMM of the step has this size
 STEP_GEMMS = 6
 STEP_FLOP = STEP_GEMMS * GEMM_FLOP
+# Algorithmic DRAM bytes of the step's six GEMM launches: both FP8 operands
+# read once (1 B per element) and the output written once -- FP8 codes +
+# transpose (2 B) for fc1 fwd and fc2 dgrad, bf16 (2 B) for fc2 fwd and fc1
+# dgrad, fp32 (4 B) for the wgrads.  Mean per launch.
+_T, _H, _F = TOKENS, HIDDEN, FFN
+GEMM_ALG_BYTES = (
+    (_T * _H + _F * _H + 2 * _T * _F)          # fc1 fwd:   X8, W1_8 -> H8, H8^T
+    + (_T * _F + _H * _F + 2 * _T * _H)        # fc2 fwd:   H8, W2_8 -> Y bf16
+    + (_T * _H + _F * _H + 2 * _T * _F)        # fc2 dgrad: dY8, W2_8^T -> dH8, dH8^T
+    + (_H * _T + _F * _T + 4 * _H * _F)        # fc2 wgrad: dY8^T, H8^T -> dW2 fp32
+    + (_T * _F + _H * _F + 2 * _T * _H)        # fc1 dgrad: dH8, W1_8^T -> dX bf16
+    + (_F * _T + _H * _T + 4 * _F * _H)        # fc1 wgrad: dH8^T, X8^T -> dW1 fp32
+) / 6.0
 # cast+transpose+amax algorithmic bytes: read input + write y + write yt
 CAST_BYTES = {
     "x": TOKENS * HIDDEN * (4 + 2), "w1": FFN * HIDDEN * (4 + 2), "h": TOKENS * FFN * (2 + 2),
@@ -243,7 +256,7 @@ class MlpStep:
             fp8.fp8_linear_bwd_ex(self.fc1, m, None, self.x8t, self.si[0:1], self.dw1, self.dh8, self.dh8t,
                                   self.si[3:4], dx=self.dx, in_cast=True)
             if sync_amax is not None:
-                sync_amax(m.amax_history[0])
+                sync_amax(m)
             m.update()
             return
         fp8.fp8_linear_fwd(self.fc1, m, x, self.h, True, self.x8, self.x8t, self.si[0:1])
@@ -253,7 +266,7 @@ class MlpStep:
         fp8.fp8_linear_bwd(self.fc1, m, self.dh, self.x8t, self.si[0:1], self.dw1, self.dh8, self.dh8t,
                            self.si[3:4], dx=self.dx)
         if sync_amax is not None:
-            sync_amax(m.amax_history[0])
+            sync_amax(m)
         m.update()
 
     def run_kernels(self, i, ev=None, sync_amax=None, fused=True):
@@ -306,7 +319,7 @@ class MlpStep:
         gemm("fc1.dgrad", self.dh8, "e5m2", self.si[3:4], fc1.w8t, "e4m3", fc1.w_scale_inv, self.dx)
         gemm("fc1.wgrad", self.dh8t, "e5m2", self.si[3:4], self.x8t, "e4m3", self.si[0:1], self.dw1)
         if sync_amax is not None:
-            sync_amax(m.amax_history[0])
+            sync_amax(m)
         h0 = mark("update", "update")
         m.update()
         if h0:
@@ -519,6 +532,31 @@ def e2e_linear_api(fp8, step, device, steps, warmup):
     return ms, h2d, d2h
 
 
+TRAFFIC_PROFILE = os.path.join("profiles", "gemm_traffic_mlp_pair_step.md")
+GEMM_SOURCE = os.path.join("fp8_delayed_scaling_cast_b200", "csrc", "gemm_sm100.cu")
+
+
+def committed_gemm_traffic(root):
+    """Mean DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per GEMM
+    launch of the step, from the committed ncu summary -- only if that capture
+    was taken on the current GEMM source (its SHA-256 is recorded beside the
+    number); otherwise None and the reason."""
+    import hashlib
+    try:
+        text = open(os.path.join(root, TRAFFIC_PROFILE)).read()
+        sha = hashlib.sha256(open(os.path.join(root, GEMM_SOURCE), "rb").read()).hexdigest()
+    except OSError:
+        return None, "no capture"
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.split(":", 1)[0] in ("gemm_source_sha256", "traffic_bytes_per_launch"):
+            k, v = line.split(":", 1)
+            fields[k] = v.strip()
+    if fields.get("gemm_source_sha256") != sha:
+        return None, "GEMM source changed since the ncu capture"
+    return float(fields["traffic_bytes_per_launch"]), "ncu capture of the step's 6 GEMM launches (%s)" % TRAFFIC_PROFILE
+
+
 def time_graph_step(step, steps):
     """The fused step captured once in a CUDA graph and replayed `steps` times
     (no host work per step beyond the replay call).  The graph reads the
@@ -663,9 +701,7 @@ def main():
     pk = peaks()
     step = MlpStep(fp8, device)
 
-    def sync_amax(row):
-        torch.distributed.all_reduce(row, op=torch.distributed.ReduceOp.MAX)
-
+    from fp8_delayed_scaling_cast_b200.dist import sync_amax
     sync = sync_amax if world > 1 else None
 
     # warm-up (both variants of the step)
@@ -755,6 +791,7 @@ def main():
     if rank != 0:
         return
 
+    traffic, traffic_note = committed_gemm_traffic(os.path.dirname(os.path.abspath(__file__)))
     cpu = None
     args.cpu_tokens = args.cpu_tokens or 128
     if not args.no_cpu_baseline and world == 1:
@@ -788,7 +825,8 @@ def main():
         "roofline": {
             "kernel": "fp8_gemm_2sm_kernel (tcgen05 CTA pairs; bf16 / fp32 / FP8 out)",
             "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
-            "frac": gemm_tflops / fp8_peak, "traffic": None,
+            "frac": gemm_tflops / fp8_peak, "traffic": traffic, "traffic_unit": "bytes per launch",
+            "traffic_note": traffic_note, "algorithmic_bytes_per_launch": GEMM_ALG_BYTES,
             "peak_note": "fp8 dense = 2 x measured bf16 burst (%s); sustained: %.1f TFLOP/s, frac %.3f" % (
                 pk["src"], fp8_peak_sus, gemm_tflops / fp8_peak_sus),
             "flop_per_launch": GEMM_FLOP, "launch_us": 1e3 * gemm_avg,

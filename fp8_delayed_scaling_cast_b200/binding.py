@@ -68,6 +68,7 @@ _SIGS = {
     "fp8_cast_transpose_amax": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
     "fp8_cast_transpose_amax_noop": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P, _P],
     "fp8_cast_transpose_amax_dynamic": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
+    "fp8_transpose": [_P, _I64, _I64, _P, _P],
     "fp8_update_scales": [_I64, _I32, _P, _P, _P, _P, _INT, _P],
     "fp8_gemm": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
     "fp8_gemm_ex": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P,
@@ -109,7 +110,13 @@ def _check(status):
 
 
 def _ptr(t):
-    return None if t is None else _P(t.data_ptr())
+    """Device pointer of a CUDA tensor (None -> NULL).  Host tensors are
+    refused here: every pointer the library takes is a device pointer."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libfp8ds takes CUDA tensors; got a %s tensor on %s" % (t.dtype, t.device))
+    return _P(t.data_ptr())
 
 
 def _stream(stream):
@@ -154,6 +161,11 @@ def fp8_cast_transpose_amax_dynamic(x, fmt, scale, y, yt=None, amax=None, scale_
     rows, cols = x.shape
     _check(_lib.fp8_cast_transpose_amax_dynamic(_ptr(x), _dtype(x), rows, cols, _fmt(fmt), _ptr(scale), _ptr(y),
                                                 _ptr(yt), _ptr(amax), _ptr(scale_inv), _stream(stream)))
+
+
+def fp8_transpose(y, yt, stream=None):
+    rows, cols = y.shape
+    _check(_lib.fp8_transpose(_ptr(y), rows, cols, _ptr(yt), _stream(stream)))
 
 
 def fp8_update_scales(amax_history, scale, scale_inv, formats, algo=AMAX_MAX, stream=None):
@@ -210,7 +222,7 @@ def gemm_workspace(device="cuda"):
 
 
 class Fp8Meta:
-    """Packed DelayedScaling state of T FP8 tensors (caller-owned device tensors)."""
+    """Packed DelayedScaling state of T FP8 tensors (caller-owned CUDA tensors)."""
 
     def __init__(self, formats, hist_len=16, device="cuda"):
         self.formats = torch.tensor([_fmt(f) for f in formats], dtype=torch.uint8, device=device)

@@ -195,6 +195,15 @@ fp8ds_status fp8_cast_transpose_amax_dynamic(const void *x, fp8ds_dtype x_dtype,
         "fp8_cast_transpose_amax_dynamic");
 }
 
+fp8ds_status fp8_transpose(const uint8_t *y, int64_t rows, int64_t cols, uint8_t *yt, fp8ds_stream stream) {
+    clear_error();
+    if (rows < 0 || cols < 0) return invalid("fp8_transpose: negative size");
+    if ((y == nullptr || yt == nullptr) && rows != 0 && cols != 0)
+        return invalid("fp8_transpose: y and yt must not be NULL for a non-empty tensor");
+    if (y == yt && rows != 0 && cols != 0) return invalid("fp8_transpose: y and yt must not alias");
+    return cuda_status(launch_transpose_u8(y, rows, cols, yt, stream), "fp8_transpose");
+}
+
 fp8ds_status fp8_update_scales(int64_t num_tensors, int32_t hist_len, float *amax_history, float *scale,
                                float *scale_inv, const uint8_t *formats, fp8ds_amax_algo algo,
                                fp8ds_stream stream) {

@@ -667,6 +667,56 @@ cudaError_t amax_dispatch(const void *x, int64_t n, float *amax, cudaStream_t st
                       stream, 1, static_cast<const T *>(x), n, amax);
 }
 
+// ------------------------------------------------------------ transpose --
+
+// Byte transpose yt[c, r] = y[r, c] of an FP8 tensor (the transpose cache of
+// a weight that arrived already cast).  64 x 64-byte tiles, 256 threads:
+// thread t loads 16 bytes of row t / 4 (one 16-byte load) into a shared tile;
+// then thread t gathers column t % 64 of rows (t / 64) * 16 .. + 15 (a warp
+// reads 32 consecutive bytes of one row per step: no bank conflict) and
+// stores them as one 16-byte segment of transposed row t % 64.
+constexpr int TR_TILE = 64;
+constexpr int TR_THREADS = 256;
+
+template <bool VEC>
+__global__ void __launch_bounds__(TR_THREADS)
+transpose_u8_kernel(const uint8_t *__restrict__ y, int64_t rows, int64_t cols, uint8_t *__restrict__ yt,
+                    int64_t tiles_c, int64_t num_tiles) {
+    __shared__ __align__(16) uint8_t tile[TR_TILE * TR_TILE];
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    const int t = threadIdx.x;
+    for (int64_t tl = blockIdx.x; tl < num_tiles; tl += gridDim.x) {
+        const int64_t r0 = (tl / tiles_c) * TR_TILE, c0 = (tl % tiles_c) * TR_TILE;
+        if (VEC) {
+            // rows % 16 == 0 and cols % 16 == 0: a 16-byte segment is wholly in or out
+            const int lr = t / 4, lc = (t % 4) * 16;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r0 + lr < rows && c0 + lc < cols)
+                v = __ldg(reinterpret_cast<const uint4 *>(y + (r0 + lr) * cols + c0 + lc));
+            *reinterpret_cast<uint4 *>(tile + lr * TR_TILE + lc) = v;
+            __syncthreads();
+            const int oc = t % TR_TILE, rg = (t / TR_TILE) * 16;
+            uint32_t w[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                w[k] = static_cast<uint32_t>(tile[(rg + 4 * k) * TR_TILE + oc]) |
+                       (static_cast<uint32_t>(tile[(rg + 4 * k + 1) * TR_TILE + oc]) << 8) |
+                       (static_cast<uint32_t>(tile[(rg + 4 * k + 2) * TR_TILE + oc]) << 16) |
+                       (static_cast<uint32_t>(tile[(rg + 4 * k + 3) * TR_TILE + oc]) << 24);
+            }
+            if (c0 + oc < cols && r0 + rg < rows)
+                *reinterpret_cast<uint4 *>(yt + (c0 + oc) * rows + r0 + rg) = make_uint4(w[0], w[1], w[2], w[3]);
+            __syncthreads();
+        } else {
+            for (int i = t; i < TR_TILE * TR_TILE; i += TR_THREADS) {
+                const int64_t r = r0 + i / TR_TILE, c = c0 + i % TR_TILE;
+                if (r < rows && c < cols) yt[c * rows + r] = y[r * cols + c];
+            }
+        }
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_cast_transpose_dynamic(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
@@ -682,6 +732,21 @@ cudaError_t launch_cast_transpose_dynamic(const void *x, fp8ds_dtype x_dtype, in
                    scale_inv, fp8_max);
     if (e != cudaSuccess) return e;
     return launch_cast_transpose(x, x_dtype, rows, cols, fmt, scale, y, yt, nullptr, nullptr, stream);
+}
+
+cudaError_t launch_transpose_u8(const uint8_t *y, int64_t rows, int64_t cols, uint8_t *yt, cudaStream_t stream) {
+    if (rows == 0 || cols == 0) return cudaSuccess;
+    const int64_t tiles_c = (cols + TR_TILE - 1) / TR_TILE;
+    const int64_t num_tiles = tiles_c * ((rows + TR_TILE - 1) / TR_TILE);
+    const bool vec = aligned16(y) && aligned16(yt) && rows % 16 == 0 && cols % 16 == 0;
+    if (vec) {
+        auto kernel = transpose_u8_kernel<true>;
+        return launch_pdl(kernel, dim3(grid_for(kernel, TR_THREADS, num_tiles)), dim3(TR_THREADS), 0, stream, 1, y,
+                          rows, cols, yt, tiles_c, num_tiles);
+    }
+    auto kernel = transpose_u8_kernel<false>;
+    return launch_pdl(kernel, dim3(grid_for(kernel, TR_THREADS, num_tiles)), dim3(TR_THREADS), 0, stream, 1, y, rows,
+                      cols, yt, tiles_c, num_tiles);
 }
 
 cudaError_t read_cast_error(int32_t *out, bool clear) {

@@ -38,6 +38,9 @@ cudaError_t launch_cast_transpose_dynamic(const void *x, fp8ds_dtype x_dtype, in
                                           fp8ds_format fmt, float *scale, uint8_t *y, uint8_t *yt, float *amax,
                                           float *scale_inv, cudaStream_t stream);
 
+// yt[c, r] = y[r, c] for a uint8 tensor [rows, cols].
+cudaError_t launch_transpose_u8(const uint8_t *y, int64_t rows, int64_t cols, uint8_t *yt, cudaStream_t stream);
+
 cudaError_t launch_update_scales(int64_t num_tensors, int32_t hist_len, float *amax_history,
                                  float *scale, float *scale_inv, const uint8_t *formats,
                                  fp8ds_amax_algo algo, cudaStream_t stream);

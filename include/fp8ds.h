@@ -142,6 +142,19 @@ fp8ds_status fp8_cast_transpose_amax_dynamic(const void *x, fp8ds_dtype x_dtype,
                                              float *scale_inv, fp8ds_stream stream);
 
 /*
+ * fp8_transpose -- the FP8 transpose cache of a tensor that arrived already
+ * cast [TE820: transpose_2d(cache=True) fills a Float8Tensor's transpose;
+ * F8E312: a weight all-gathered in FP8 still needs its transpose for the
+ * backward]:  yt[c, r] = y[r, c], bytes copied unchanged.
+ *   y [rows, cols] uint8, yt [cols, rows] uint8 (must not overlap y).
+ * 16-byte aligned pointers with rows and cols multiples of 16 take the
+ * vectorised path; other shapes are still transposed exactly.
+ * Errors: FP8DS_ERR_INVALID_ARG for negative sizes, NULL or aliasing pointers.
+ */
+fp8ds_status fp8_transpose(const uint8_t *y, int64_t rows, int64_t cols, uint8_t *yt,
+                           fp8ds_stream stream);
+
+/*
  * fp8_update_scales -- the delayed-scaling recipe update of T FP8 meta tensors
  * in ONE launch [TE820 "FP8 scale update kernel"; TE761 DelayedScaling(
  * amax_history_len=16, amax_compute_algo="max"); F8E312 amax buffers of all

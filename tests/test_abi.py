@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
     for n in ("fp8_quantize", "fp8_cast_transpose_amax", "fp8_update_scales", "fp8_gemm",
               "fp8_gemm_ex", "fp8_gemm_workspace_size", "fp8_gemm_noalloc", "fp8_gemm_cast",
               "fp8_linear_fwd_ex", "fp8_linear_bwd_ex", "fp8_cast_transpose_amax_noop",
-              "fp8_cast_transpose_amax_dynamic",
+              "fp8_cast_transpose_amax_dynamic", "fp8_transpose",
               "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
               "fp8ds_version"):
         assert n in names
