@@ -28,6 +28,10 @@ ERR_TIMEOUT = 4
 
 _FMT_NAMES = {"e4m3": E4M3, "e5m2": E5M2, E4M3: E4M3, E5M2: E5M2}
 
+K_MAJOR = 0      # operand [m, k] / [n, k] row-major
+MN_MAJOR = 1     # operand [k, m] / [k, n] row-major
+_MAJOR = {"k": K_MAJOR, "mn": MN_MAJOR, K_MAJOR: K_MAJOR, MN_MAJOR: MN_MAJOR}
+
 
 class Fp8dsError(RuntimeError):
     def __init__(self, status, message):
@@ -75,13 +79,15 @@ _SIGS = {
                     ctypes.c_size_t, _P],
     "fp8_gemm_workspace_size": [ctypes.POINTER(ctypes.c_size_t)],
     "fp8_gemm_noalloc": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
-    "fp8_gemm_cast": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _I64, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
+    "fp8_gemm_cast": [_P, _INT, _INT, _P, _P, _INT, _INT, _P, _P, _INT, _I64, _I64, _I64, _INT, _P, _P, _P, _P, _P,
+                      _P],
     "fp8_linear_fwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _INT,
                        _I32, _P, _P, _P, _P],
     "fp8_linear_fwd_ex": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _INT,
                           _I32, _P, _P, _P, ctypes.POINTER(_Fp8Io), _P],
-    "fp8_linear_bwd_ex": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P,
+    "fp8_linear_bwd_ex": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P, _P,
                           _INT, _P, _P, _P, _P, ctypes.POINTER(_Fp8Io), _P],
+    "fp8_gemm_major": [_P, _INT, _INT, _P, _P, _INT, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
     "fp8_linear_bwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P,
                        _INT, _P, _P, _P, _P, _P],
     "fp8ds_device_status": [ctypes.POINTER(_I32), _I32],
@@ -201,10 +207,14 @@ def fp8_gemm_noalloc(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, d, bias=None,
 
 
 def fp8_gemm_cast(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, out_fmt, out_scale, d8, d8t=None,
-                  out_amax=None, out_scale_inv=None, bias=None, stream=None):
-    m, k = a.shape
-    n = b.shape[0]
-    _check(_lib.fp8_gemm_cast(_ptr(a), _fmt(a_fmt), _ptr(a_scale_inv), _ptr(b), _fmt(b_fmt),
+                  out_amax=None, out_scale_inv=None, bias=None, a_major="k", b_major="k", stream=None):
+    """GEMM with an FP8 output; a is [m, k] ("k") or [k, m] ("mn"), b is
+    [n, k] ("k") or [k, n] ("mn")."""
+    am, bm = _MAJOR[a_major], _MAJOR[b_major]
+    m = a.shape[1] if am == MN_MAJOR else a.shape[0]
+    k = a.shape[0] if am == MN_MAJOR else a.shape[1]
+    n = b.shape[1] if bm == MN_MAJOR else b.shape[0]
+    _check(_lib.fp8_gemm_cast(_ptr(a), _fmt(a_fmt), am, _ptr(a_scale_inv), _ptr(b), _fmt(b_fmt), bm,
                               _ptr(b_scale_inv), _ptr(bias), F32 if bias is None else _dtype(bias), m, n, k,
                               _fmt(out_fmt), _ptr(out_scale), _ptr(d8), _ptr(d8t), _ptr(out_amax),
                               _ptr(out_scale_inv), _stream(stream)))
@@ -245,7 +255,7 @@ class Fp8Meta:
 class Fp8Linear:
     """A linear layer's fp32 master weight, optional bias and FP8 weight cache."""
 
-    def __init__(self, w, bias, meta_in, meta_w, meta_grad, workspace=None, w_noop_flag=None):
+    def __init__(self, w, bias, meta_in, meta_w, meta_grad, workspace=None, w_noop_flag=None, transpose=True):
         """w_noop_flag: optional device int32 tensor; when given, the forward
         always enqueues the weight cast and the GPU skips it while the flag is
         non-zero (graph-capturable weight caching)."""
@@ -255,7 +265,8 @@ class Fp8Linear:
         self.workspace = workspace
         self.w_noop_flag = w_noop_flag
         self.w8 = torch.empty(out_f, in_f, dtype=torch.uint8, device=w.device)
-        self.w8t = torch.empty(in_f, out_f, dtype=torch.uint8, device=w.device)
+        # transpose=False: no cached weight transpose (the backward reads w8 MN-major)
+        self.w8t = torch.empty(in_f, out_f, dtype=torch.uint8, device=w.device) if transpose else None
         self.w_scale_inv = torch.ones(1, dtype=torch.float32, device=w.device)
         ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
         self._c = _Linear(_ptr(w), _ptr(bias), F32 if bias is None else _dtype(bias), in_f, out_f,
@@ -313,15 +324,30 @@ def fp8_linear_fwd_ex(lin, meta, x, y, is_first_microbatch, x8, x8t=None, x_scal
 
 
 def fp8_linear_bwd_ex(lin, meta, dy, x8t, x_scale_inv, dw, dy8, dy8t, dy_scale_inv, dx=None, in_cast=False,
-                      out_meta=None, out8=None, out8t=None, out_scale_inv=None, stream=None):
+                      out_meta=None, out8=None, out8t=None, out_scale_inv=None, x8=None, stream=None):
     """fp8_linear_bwd with FP8 hand-over: in_cast -> dy8/dy8t/dy_scale_inv
     already hold the cast gradient (dy may be None); out_meta -> the dgrad is
-    cast in the GEMM epilogue into out8/out8t/out_scale_inv."""
+    cast in the GEMM epilogue into out8/out8t/out_scale_inv.  Transposes are
+    optional: x8t None -> the wgrad reads x8; dy8t None -> it reads dy8; a
+    linear without w8t -> the dgrad reads w8 (all MN-major)."""
     io = _io(in_cast, out_meta, out8, out8t, out_scale_inv)
     _check(_lib.fp8_linear_bwd_ex(ctypes.byref(lin._c), ctypes.byref(meta._c), _ptr(dy),
-                                  BF16 if dy is None else _dtype(dy), dy8.shape[0], _ptr(x8t),
+                                  BF16 if dy is None else _dtype(dy), dy8.shape[0], _ptr(x8), _ptr(x8t),
                                   _ptr(x_scale_inv), _ptr(dx), BF16 if dx is None else _dtype(dx), _ptr(dw),
                                   _ptr(dy8), _ptr(dy8t), _ptr(dy_scale_inv), ctypes.byref(io), _stream(stream)))
+
+
+
+def fp8_gemm_major(a, a_fmt, a_major, a_scale_inv, b, b_fmt, b_major, b_scale_inv, d, bias=None, stream=None):
+    """D[m, n] = A(m, k) B(n, k) scaled; a is [m, k] ("k") or [k, m] ("mn"),
+    b is [n, k] ("k") or [k, n] ("mn")."""
+    am, bm = _MAJOR[a_major], _MAJOR[b_major]
+    m = a.shape[1] if am == MN_MAJOR else a.shape[0]
+    k = a.shape[0] if am == MN_MAJOR else a.shape[1]
+    n = b.shape[1] if bm == MN_MAJOR else b.shape[0]
+    _check(_lib.fp8_gemm_major(_ptr(a), _fmt(a_fmt), am, _ptr(a_scale_inv), _ptr(b), _fmt(b_fmt), bm,
+                               _ptr(b_scale_inv), _ptr(bias), F32 if bias is None else _dtype(bias), _ptr(d),
+                               _dtype(d), m, n, k, _stream(stream)))
 
 
 def fp8ds_device_status(clear=True):

@@ -107,9 +107,12 @@ static fp8ds_status check_cast(const char *fn, const void *x, int x_dtype, int64
     return FP8DS_OK;
 }
 
-static fp8ds_status check_gemm(const uint8_t *a, int fa, const float *sa, const uint8_t *b, int fb,
-                               const float *sb, const void *bias, int bias_dtype, const void *d, int d_dtype,
-                               int64_t m, int64_t n, int64_t k) {
+// a_mn / b_mn: the operand is stored MN-major ([k, m] / [k, n] row-major);
+// its row pitch is then m (n) bytes instead of k, which the tensor map needs
+// to be a multiple of 16.
+static fp8ds_status check_gemm_layout(const uint8_t *a, int fa, const float *sa, bool a_mn, const uint8_t *b, int fb,
+                                      const float *sb, bool b_mn, const void *bias, int bias_dtype, const void *d,
+                                      int d_dtype, int64_t m, int64_t n, int64_t k) {
     if (a == nullptr || b == nullptr || d == nullptr || sa == nullptr || sb == nullptr)
         return invalid("fp8_gemm: a, b, d and the scale_inv pointers must not be NULL");
     if (!valid_fmt(fa) || !valid_fmt(fb)) return invalid("fp8_gemm: unknown FP8 format");
@@ -117,7 +120,10 @@ static fp8ds_status check_gemm(const uint8_t *a, int fa, const float *sa, const 
         return invalid("fp8_gemm: unknown output or bias dtype");
     if (m <= 0 || n <= 0 || k <= 0) return invalid("fp8_gemm: m, n, k must be positive");
     if (m > 0x7FFFFFFF || n > 0x7FFFFFFF || k > 0x7FFFFFFF) return invalid("fp8_gemm: size exceeds 2^31-1");
-    if (k % 16 != 0) return invalid("fp8_gemm: k (%lld) must be a multiple of 16", (long long)k);
+    if ((!a_mn || !b_mn) && k % 16 != 0)
+        return invalid("fp8_gemm: k (%lld) must be a multiple of 16 for a K-major operand", (long long)k);
+    if (a_mn && m % 16 != 0) return invalid("fp8_gemm: m (%lld) must be a multiple of 16 for an MN-major a", (long long)m);
+    if (b_mn && n % 16 != 0) return invalid("fp8_gemm: n (%lld) must be a multiple of 16 for an MN-major b", (long long)n);
     if (d_dtype == FP8DS_BF16 && n % 8 != 0) return invalid("fp8_gemm: n must be a multiple of 8 for bf16 output");
     if (d_dtype == FP8DS_F32 && n % 4 != 0) return invalid("fp8_gemm: n must be a multiple of 4 for fp32 output");
     if (!aligned16(a) || !aligned16(b) || !aligned16(d))
@@ -136,6 +142,12 @@ static fp8ds_status check_cast_out(const char *fn, const uint8_t *d8, const uint
     if (!aligned16(d8) || (d8t != nullptr && !aligned16(d8t)))
         return invalid("%s: the FP8 outputs must be 16-byte aligned", fn);
     return FP8DS_OK;
+}
+
+static fp8ds_status check_gemm(const uint8_t *a, int fa, const float *sa, const uint8_t *b, int fb,
+                               const float *sb, const void *bias, int bias_dtype, const void *d, int d_dtype,
+                               int64_t m, int64_t n, int64_t k) {
+    return check_gemm_layout(a, fa, sa, false, b, fb, sb, false, bias, bias_dtype, d, d_dtype, m, n, k);
 }
 
 static fp8ds_status check_meta(const char *fn, const fp8ds_meta *meta, int32_t idx) {
@@ -263,19 +275,40 @@ fp8ds_status fp8_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float 
                                stream);
 }
 
-fp8ds_status fp8_gemm_cast(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
-                           fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
-                           int64_t m, int64_t n, int64_t k, fp8ds_format out_fmt, const float *out_scale,
-                           uint8_t *d8, uint8_t *d8t, float *out_amax, float *out_scale_inv, fp8ds_stream stream) {
+fp8ds_status fp8_gemm_major(const uint8_t *a, fp8ds_format a_fmt, fp8ds_major a_major, const float *a_scale_inv,
+                            const uint8_t *b, fp8ds_format b_fmt, fp8ds_major b_major, const float *b_scale_inv,
+                            const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype, int64_t m,
+                            int64_t n, int64_t k, fp8ds_stream stream) {
     clear_error();
-    fp8ds_status st =
-        check_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d8, FP8DS_BF16, m, n, k);
+    if ((a_major != FP8DS_K_MAJOR && a_major != FP8DS_MN_MAJOR) ||
+        (b_major != FP8DS_K_MAJOR && b_major != FP8DS_MN_MAJOR))
+        return invalid("fp8_gemm_major: unknown operand layout");
+    const bool a_mn = a_major == FP8DS_MN_MAJOR, b_mn = b_major == FP8DS_MN_MAJOR;
+    fp8ds_status st = check_gemm_layout(a, a_fmt, a_scale_inv, a_mn, b, b_fmt, b_scale_inv, b_mn, bias, bias_dtype,
+                                        d, d_dtype, m, n, k);
+    if (st != FP8DS_OK) return st;
+    return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k, nullptr,
+                       0, stream, nullptr, a_mn, b_mn);
+}
+
+fp8ds_status fp8_gemm_cast(const uint8_t *a, fp8ds_format a_fmt, fp8ds_major a_major, const float *a_scale_inv,
+                           const uint8_t *b, fp8ds_format b_fmt, fp8ds_major b_major, const float *b_scale_inv,
+                           const void *bias, fp8ds_dtype bias_dtype, int64_t m, int64_t n, int64_t k,
+                           fp8ds_format out_fmt, const float *out_scale, uint8_t *d8, uint8_t *d8t, float *out_amax,
+                           float *out_scale_inv, fp8ds_stream stream) {
+    clear_error();
+    if ((a_major != FP8DS_K_MAJOR && a_major != FP8DS_MN_MAJOR) ||
+        (b_major != FP8DS_K_MAJOR && b_major != FP8DS_MN_MAJOR))
+        return invalid("fp8_gemm_cast: unknown operand layout");
+    const bool a_mn = a_major == FP8DS_MN_MAJOR, b_mn = b_major == FP8DS_MN_MAJOR;
+    fp8ds_status st = check_gemm_layout(a, a_fmt, a_scale_inv, a_mn, b, b_fmt, b_scale_inv, b_mn, bias, bias_dtype,
+                                        d8, FP8DS_BF16, m, n, k);
     if (st != FP8DS_OK) return st;
     if (!valid_fmt(out_fmt)) return invalid("fp8_gemm_cast: unknown output FP8 format %d", out_fmt);
     if ((st = check_cast_out("fp8_gemm_cast", d8, d8t, out_scale, m, n)) != FP8DS_OK) return st;
     const GemmCastOut cast{out_fmt, out_scale, d8t, out_amax, out_scale_inv};
     return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d8, FP8DS_BF16, m, n, k,
-                       nullptr, 0, stream, &cast);
+                       nullptr, 0, stream, &cast, a_mn, b_mn);
 }
 
 // The linear forward and backward, with the options of the _ex forms (NULL:
@@ -286,8 +319,7 @@ static fp8ds_status linear_fwd(const char *fn, fp8ds_linear *lin, const fp8ds_me
                                fp8ds_dtype x_dtype, int64_t m, void *y, fp8ds_dtype y_dtype,
                                int32_t is_first_microbatch, uint8_t *x8, uint8_t *x8t, float *x_scale_inv,
                                const fp8ds_fp8_io *io, cudaStream_t s) {
-    if (lin == nullptr || lin->w == nullptr || lin->w8 == nullptr || lin->w8t == nullptr ||
-        lin->w_scale_inv == nullptr)
+    if (lin == nullptr || lin->w == nullptr || lin->w8 == nullptr || lin->w_scale_inv == nullptr)
         return invalid("%s: incomplete linear handle", fn);
     const bool in_cast = io != nullptr && io->in_cast != 0;
     const bool out_cast = io != nullptr && io->out_meta >= 0;
@@ -336,35 +368,42 @@ static fp8ds_status linear_fwd(const char *fn, fp8ds_linear *lin, const fp8ds_me
                        lin->bias_dtype, y, y_dtype, m, N, K, lin->workspace, lin->workspace_bytes, s);
 }
 
+// Transposes are optional: without w8t the dgrad reads w8 MN-major, without
+// dy8t the wgrad reads dy8 MN-major (and the gradient cast writes no
+// transpose), without x8t it reads x8 MN-major.
 static fp8ds_status linear_bwd(const char *fn, const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy,
-                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8t, const float *x_scale_inv,
-                               void *dx, fp8ds_dtype dx_dtype, float *dw, uint8_t *dy8, uint8_t *dy8t,
-                               float *dy_scale_inv, const fp8ds_fp8_io *io, cudaStream_t s) {
-    if (lin == nullptr || lin->w8t == nullptr || lin->w_scale_inv == nullptr)
+                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8, const uint8_t *x8t,
+                               const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype, float *dw, uint8_t *dy8,
+                               uint8_t *dy8t, float *dy_scale_inv, const fp8ds_fp8_io *io, cudaStream_t s) {
+    if (lin == nullptr || lin->w8 == nullptr || lin->w_scale_inv == nullptr)
         return invalid("%s: incomplete linear handle", fn);
     if (!lin->cache_valid) return invalid("%s: the weight cache is empty (run the forward first)", fn);
     const bool in_cast = io != nullptr && io->in_cast != 0;
     const bool out_cast = io != nullptr && io->out_meta >= 0;
-    if ((!in_cast && dy == nullptr) || x8t == nullptr || x_scale_inv == nullptr || dw == nullptr ||
-        dy8 == nullptr || dy8t == nullptr || dy_scale_inv == nullptr)
+    if ((!in_cast && dy == nullptr) || (x8t == nullptr && x8 == nullptr) || x_scale_inv == nullptr ||
+        dw == nullptr || dy8 == nullptr || dy_scale_inv == nullptr)
         return invalid("%s: NULL pointer argument", fn);
+    const bool w_mn = lin->w8t == nullptr, dy_mn = dy8t == nullptr, x_mn = x8t == nullptr;
+    const uint8_t *wb = w_mn ? lin->w8 : lin->w8t;         // dgrad B
+    const uint8_t *ga = dy_mn ? dy8 : dy8t;                // wgrad A
+    const uint8_t *gb = x_mn ? x8 : x8t;                   // wgrad B
     fp8ds_status st;
     if ((st = check_meta(fn, meta, lin->meta_grad)) != FP8DS_OK) return st;
     if (out_cast && (st = check_meta(fn, meta, io->out_meta)) != FP8DS_OK) return st;
     const int64_t K = lin->in_features, N = lin->out_features;
     if (!in_cast && (st = check_cast(fn, dy, dy_dtype, m, N, FP8DS_E5M2, meta->scale, dy8)) != FP8DS_OK) return st;
     if (out_cast) {
-        if ((st = check_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv, nullptr,
-                             FP8DS_F32, io->out8, FP8DS_BF16, m, K, N)) != FP8DS_OK)
+        if ((st = check_gemm_layout(dy8, FP8DS_E5M2, dy_scale_inv, false, wb, FP8DS_E4M3, lin->w_scale_inv, w_mn,
+                                    nullptr, FP8DS_F32, io->out8, FP8DS_BF16, m, K, N)) != FP8DS_OK)
             return st;
         if ((st = check_cast_out(fn, io->out8, io->out8t, meta->scale, m, K)) != FP8DS_OK) return st;
-    } else if (dx != nullptr && (st = check_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3,
-                                                 lin->w_scale_inv, nullptr, FP8DS_F32, dx, dx_dtype, m, K, N)) !=
-                                    FP8DS_OK) {
+    } else if (dx != nullptr &&
+               (st = check_gemm_layout(dy8, FP8DS_E5M2, dy_scale_inv, false, wb, FP8DS_E4M3, lin->w_scale_inv, w_mn,
+                                       nullptr, FP8DS_F32, dx, dx_dtype, m, K, N)) != FP8DS_OK) {
         return st;
     }
-    if ((st = check_gemm(dy8t, FP8DS_E5M2, dy_scale_inv, x8t, FP8DS_E4M3, x_scale_inv, nullptr, FP8DS_F32, dw,
-                         FP8DS_F32, N, K, m)) != FP8DS_OK)
+    if ((st = check_gemm_layout(ga, FP8DS_E5M2, dy_scale_inv, dy_mn, gb, FP8DS_E4M3, x_scale_inv, x_mn, nullptr,
+                                FP8DS_F32, dw, FP8DS_F32, N, K, m)) != FP8DS_OK)
         return st;
     const int32_t hg = lin->meta_grad;
     if (!in_cast) {
@@ -376,16 +415,16 @@ static fp8ds_status linear_bwd(const char *fn, const fp8ds_linear *lin, const fp
     if (out_cast) {
         const int32_t ho = io->out_meta;
         const GemmCastOut cast{FP8DS_E5M2, meta->scale + ho, io->out8t, meta->amax_history + ho, io->out_scale_inv};
-        st = launch_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv, nullptr, FP8DS_F32,
-                         io->out8, FP8DS_BF16, m, K, N, lin->workspace, lin->workspace_bytes, s, &cast);
+        st = launch_gemm(dy8, FP8DS_E5M2, dy_scale_inv, wb, FP8DS_E4M3, lin->w_scale_inv, nullptr, FP8DS_F32,
+                         io->out8, FP8DS_BF16, m, K, N, lin->workspace, lin->workspace_bytes, s, &cast, false, w_mn);
         if (st != FP8DS_OK) return st;
     } else if (dx != nullptr) {
-        st = launch_gemm(dy8, FP8DS_E5M2, dy_scale_inv, lin->w8t, FP8DS_E4M3, lin->w_scale_inv, nullptr, FP8DS_F32,
-                         dx, dx_dtype, m, K, N, lin->workspace, lin->workspace_bytes, s);
+        st = launch_gemm(dy8, FP8DS_E5M2, dy_scale_inv, wb, FP8DS_E4M3, lin->w_scale_inv, nullptr, FP8DS_F32, dx,
+                         dx_dtype, m, K, N, lin->workspace, lin->workspace_bytes, s, nullptr, false, w_mn);
         if (st != FP8DS_OK) return st;
     }
-    return launch_gemm(dy8t, FP8DS_E5M2, dy_scale_inv, x8t, FP8DS_E4M3, x_scale_inv, nullptr, FP8DS_F32, dw,
-                       FP8DS_F32, N, K, m, lin->workspace, lin->workspace_bytes, s);
+    return launch_gemm(ga, FP8DS_E5M2, dy_scale_inv, gb, FP8DS_E4M3, x_scale_inv, nullptr, FP8DS_F32, dw, FP8DS_F32, N,
+                       K, m, lin->workspace, lin->workspace_bytes, s, nullptr, dy_mn, x_mn);
 }
 
 fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const void *x, fp8ds_dtype x_dtype,
@@ -408,16 +447,16 @@ fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, con
                             int64_t m, const uint8_t *x8t, const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
                             float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv, fp8ds_stream stream) {
     clear_error();
-    return linear_bwd("fp8_linear_bwd", lin, meta, dy, dy_dtype, m, x8t, x_scale_inv, dx, dx_dtype, dw, dy8, dy8t,
-                      dy_scale_inv, nullptr, stream);
+    return linear_bwd("fp8_linear_bwd", lin, meta, dy, dy_dtype, m, nullptr, x8t, x_scale_inv, dx, dx_dtype, dw, dy8,
+                      dy8t, dy_scale_inv, nullptr, stream);
 }
 
 fp8ds_status fp8_linear_bwd_ex(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy,
-                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8t, const float *x_scale_inv,
-                               void *dx, fp8ds_dtype dx_dtype, float *dw, uint8_t *dy8, uint8_t *dy8t,
-                               float *dy_scale_inv, const fp8ds_fp8_io *io, fp8ds_stream stream) {
+                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8, const uint8_t *x8t,
+                               const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype, float *dw, uint8_t *dy8,
+                               uint8_t *dy8t, float *dy_scale_inv, const fp8ds_fp8_io *io, fp8ds_stream stream) {
     clear_error();
-    return linear_bwd("fp8_linear_bwd_ex", lin, meta, dy, dy_dtype, m, x8t, x_scale_inv, dx, dx_dtype, dw, dy8, dy8t,
+    return linear_bwd("fp8_linear_bwd_ex", lin, meta, dy, dy_dtype, m, x8, x8t, x_scale_inv, dx, dx_dtype, dw, dy8, dy8t,
                       dy_scale_inv, io, stream);
 }
 

@@ -60,12 +60,14 @@ struct GemmCastOut {
 // Returns FP8DS_OK or an error (message set) for tensor-map or launch failures.
 // workspace (may be NULL) enables the stream-K schedule when it holds at
 // least gemm_workspace_bytes().  With `cast`, d receives FP8 codes and
-// d_dtype is ignored.
+// d_dtype is ignored.  a_mn / b_mn: the operand is stored MN-major, a as
+// [k, m] and b as [k, n] row-major (otherwise a is [m, k] and b [n, k]).
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
                          const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
                          const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
                          int64_t m, int64_t n, int64_t k, void *workspace, size_t workspace_bytes,
-                         cudaStream_t stream, const GemmCastOut *cast = nullptr);
+                         cudaStream_t stream, const GemmCastOut *cast = nullptr, bool a_mn = false,
+                         bool b_mn = false);
 
 // Workspace bytes the stream-K schedule needs on the current device.
 size_t gemm_workspace_bytes();

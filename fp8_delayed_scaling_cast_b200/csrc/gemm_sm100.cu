@@ -279,6 +279,32 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
     return d;
 }
 
+// MN-major operand tile with the 128-byte swizzle (8-bit elements): each
+// K row holds 128 consecutive M (or N) elements, 8 K rows form one 1 KB
+// swizzle atom, atoms follow each other along K (SBO = 1 KB), and a second
+// group of 128 M (N) elements sits LBO bytes further (the one-CTA kernel's
+// 256-column B tile: two TMA boxes 16 KB apart).  The same fields as the
+// K-major descriptor otherwise (version 1, layout SWIZZLE_128B).
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr, uint32_t lbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    d |= static_cast<uint64_t>(2u) << 61;
+    return d;
+}
+
+// Descriptor of a 128 x BK operand tile and its advance (in 16-byte units)
+// per K step of UMMA_K elements: 32 bytes along the swizzled row (K-major)
+// or 32 rows of 128 bytes (MN-major).
+__device__ __forceinline__ uint64_t operand_desc(uint32_t smem_addr, bool mn_major, uint32_t lbo_bytes) {
+    return mn_major ? sw128_mnmajor_desc(smem_addr, lbo_bytes) : sw128_kmajor_desc(smem_addr);
+}
+__device__ __forceinline__ uint64_t operand_kstep(int k, bool mn_major) {
+    return static_cast<uint64_t>(mn_major ? (k * UMMA_K * 128) >> 4 : (k * UMMA_K) >> 4);
+}
+
 __device__ __forceinline__ void umma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -344,6 +370,7 @@ struct Params {
     int32_t M, N, K;
     int32_t tiles_m, tiles_n, num_kb;
     uint32_t idesc;
+    int32_t a_mn, b_mn;   // 1: the operand is stored MN-major ([K, M] / [K, N] row-major)
     // stream-K (pair kernel only): 0 = whole tiles per cluster
     int32_t stream_k;
     uint32_t epoch;       // non-zero per launch; partials are published with it
@@ -879,8 +906,19 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                         break;
                     }
                     mbar_arrive_expect_tx(&sm.full[stage], S1_A_STAGE + S1_B_STAGE);
-                    tma_load_2d(&tmap_a, &sm.full[stage], sm.a + stage * S1_A_STAGE, kb * BK, m_blk * S1_BM);
-                    tma_load_2d(&tmap_b, &sm.full[stage], sm.b + stage * S1_B_STAGE, kb * BK, n_blk * ACC_N);
+                    uint8_t *a_dst = sm.a + stage * S1_A_STAGE, *b_dst = sm.b + stage * S1_B_STAGE;
+                    if (p.a_mn)
+                        tma_load_2d(&tmap_a, &sm.full[stage], a_dst, m_blk * S1_BM, kb * BK);
+                    else
+                        tma_load_2d(&tmap_a, &sm.full[stage], a_dst, kb * BK, m_blk * S1_BM);
+                    if (p.b_mn) {
+                        // two 128-column boxes: the tile's column groups, 16 KB apart
+                        tma_load_2d(&tmap_b, &sm.full[stage], b_dst, n_blk * ACC_N, kb * BK);
+                        tma_load_2d(&tmap_b, &sm.full[stage], b_dst + S1_B_STAGE / 2, n_blk * ACC_N + ACC_N / 2,
+                                    kb * BK);
+                    } else {
+                        tma_load_2d(&tmap_b, &sm.full[stage], b_dst, kb * BK, n_blk * ACC_N);
+                    }
                     ++issued;
                     if (++stage == S1_STAGES) {
                         stage = 0;
@@ -921,13 +959,12 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t a_desc = sw128_kmajor_desc(smem_u32(sm.a + stage * S1_A_STAGE));
-                    const uint64_t b_desc = sw128_kmajor_desc(smem_u32(sm.b + stage * S1_B_STAGE));
+                    const uint64_t a_desc = operand_desc(smem_u32(sm.a + stage * S1_A_STAGE), p.a_mn, 0);
+                    const uint64_t b_desc = operand_desc(smem_u32(sm.b + stage * S1_B_STAGE), p.b_mn, S1_B_STAGE / 2);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
-                        // advance the start address by k * 32 bytes inside the swizzle row
-                        const uint64_t adv = static_cast<uint64_t>((k * UMMA_K) >> 4);
-                        umma_f8f6f4(d_tmem, a_desc + adv, b_desc + adv, p.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                        umma_f8f6f4(d_tmem, a_desc + operand_kstep(k, p.a_mn), b_desc + operand_kstep(k, p.b_mn),
+                                    p.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
                     }
                     umma_commit(&sm.empty[stage]);
                     if (++stage == S1_STAGES) {
@@ -1032,10 +1069,17 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     if (leader) mbar_arrive_expect_tx(&sm.full[stage], 2 * (A_STAGE + S2_B_STAGE));
                     const uint32_t full_leader = map_to_cta(smem_u32(&sm.full[stage]), 0u);
 #pragma unroll
-                    for (int h = 0; h < M_SUB; ++h)
-                        tma_load_2d_pair(&tmap_a, full_leader, sm.a + stage * A_STAGE + h * S2_BM * BK, kb * BK,
-                                         a_row + h * 2 * S2_BM);
-                    tma_load_2d_pair(&tmap_b, full_leader, sm.b + stage * S2_B_STAGE, kb * BK, b_row);
+                    for (int h = 0; h < M_SUB; ++h) {
+                        uint8_t *a_dst = sm.a + stage * A_STAGE + h * S2_BM * BK;
+                        if (p.a_mn)
+                            tma_load_2d_pair(&tmap_a, full_leader, a_dst, a_row + h * 2 * S2_BM, kb * BK);
+                        else
+                            tma_load_2d_pair(&tmap_a, full_leader, a_dst, kb * BK, a_row + h * 2 * S2_BM);
+                    }
+                    if (p.b_mn)
+                        tma_load_2d_pair(&tmap_b, full_leader, sm.b + stage * S2_B_STAGE, b_row, kb * BK);
+                    else
+                        tma_load_2d_pair(&tmap_b, full_leader, sm.b + stage * S2_B_STAGE, kb * BK, b_row);
                     ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -1074,16 +1118,16 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t b_desc = sw128_kmajor_desc(smem_u32(sm.b + stage * S2_B_STAGE));
+                    const uint64_t b_desc = operand_desc(smem_u32(sm.b + stage * S2_B_STAGE), p.b_mn, 0);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
-                        const uint64_t adv = static_cast<uint64_t>((k * UMMA_K) >> 4);
 #pragma unroll
                         for (int h = 0; h < M_SUB; ++h) {
                             const uint64_t a_desc =
-                                sw128_kmajor_desc(smem_u32(sm.a + stage * A_STAGE + h * S2_BM * BK));
-                            umma_f8f6f4_pair(tmem_base + static_cast<uint32_t>((acc + h) * ACC_N), a_desc + adv,
-                                             b_desc + adv, p.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+                                operand_desc(smem_u32(sm.a + stage * A_STAGE + h * S2_BM * BK), p.a_mn, 0);
+                            umma_f8f6f4_pair(tmem_base + static_cast<uint32_t>((acc + h) * ACC_N),
+                                             a_desc + operand_kstep(k, p.a_mn), b_desc + operand_kstep(k, p.b_mn),
+                                             p.idesc, (kb > kb0 || k > 0) ? 1u : 0u);
                         }
                     }
                     umma_commit_pair_to(&sm.empty[stage], 0x3);
@@ -1124,12 +1168,15 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint6
 
 // Instruction descriptor of tcgen05.mma.kind::f8f6f4 (dense, K-major A and B):
 // [4,6) D format (1 = fp32), [7,10) A format, [10,13) B format (0 = E4M3,
-// 1 = E5M2), [15] / [16] A / B major (0 = K), [17,23) N >> 3, [24,29) M >> 4.
-uint32_t make_idesc(fp8ds_format fa, fp8ds_format fb, int m, int n) {
+// 1 = E5M2), [15] / [16] A / B major (0 = K, 1 = MN), [17,23) N >> 3,
+// [24,29) M >> 4.
+uint32_t make_idesc(fp8ds_format fa, fp8ds_format fb, int m, int n, bool a_mn, bool b_mn) {
     uint32_t d = 0;
     d |= 1u << 4;
     d |= static_cast<uint32_t>(fa == FP8DS_E5M2 ? 1 : 0) << 7;
     d |= static_cast<uint32_t>(fb == FP8DS_E5M2 ? 1 : 0) << 10;
+    d |= static_cast<uint32_t>(a_mn ? 1 : 0) << 15;
+    d |= static_cast<uint32_t>(b_mn ? 1 : 0) << 16;
     d |= static_cast<uint32_t>(n >> 3) << 17;
     d |= static_cast<uint32_t>(m >> 4) << 24;
     return d;
@@ -1208,15 +1255,21 @@ size_t gemm_workspace_bytes() {
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
                          fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
                          void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, void *workspace,
-                         size_t workspace_bytes, cudaStream_t stream, const GemmCastOut *cast) {
+                         size_t workspace_bytes, cudaStream_t stream, const GemmCastOut *cast, bool a_mn,
+                         bool b_mn) {
     const int out = cast != nullptr ? OUT_FP8 : (d_dtype == FP8DS_BF16 ? OUT_BF16 : OUT_F32);
     const bool pair = m > S1_BM;
     // Long contractions amortise the non-overlapped epilogue of the 512-row
     // pair tile; short ones keep the double-buffered 256-row tile.
     const int m_sub = (pair && m > 2 * S2_BM && k >= FP8DS_MSUB2_MIN_K) ? 2 : 1;
     CUtensorMap ta, tb, td;
-    bool ok = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, k, m, k, BK, pair ? S2_BM : S1_BM) &&
-              encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, k, n, k, BK, pair ? S2_BN_HALF : ACC_N);
+    // K-major operands: [rows, k] boxes of BK x rows; MN-major: [k, rows]
+    // boxes of 128 columns x BK rows (the one-CTA B tile loads two of them)
+    const uint32_t a_rows = pair ? S2_BM : S1_BM, b_rows = pair ? S2_BN_HALF : ACC_N;
+    bool ok = (a_mn ? encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, m, k, m, 128, BK)
+                    : encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a, k, m, k, BK, a_rows)) &&
+              (b_mn ? encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, n, k, n, 128, BK)
+                    : encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, k, n, k, BK, b_rows));
     if (out == OUT_FP8) {
         // the FP8 epilogue stores with plain global stores; the map stays a
         // valid description of the codes (it is only prefetched)
@@ -1242,7 +1295,9 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.tiles_m = static_cast<int32_t>((m + tile_m - 1) / tile_m);
     p.tiles_n = static_cast<int32_t>((n + ACC_N - 1) / ACC_N);
     p.num_kb = static_cast<int32_t>((k + BK - 1) / BK);
-    p.idesc = make_idesc(a_fmt, b_fmt, pair ? 2 * S2_BM : S1_BM, ACC_N);
+    p.idesc = make_idesc(a_fmt, b_fmt, pair ? 2 * S2_BM : S1_BM, ACC_N, a_mn, b_mn);
+    p.a_mn = a_mn ? 1 : 0;
+    p.b_mn = b_mn ? 1 : 0;
     p.stream_k = 0;
     p.epoch = 0;
     p.flags = nullptr;

@@ -58,6 +58,15 @@ typedef enum { FP8DS_E4M3 = 0, FP8DS_E5M2 = 1 } fp8ds_format;
 typedef enum { FP8DS_F32 = 0, FP8DS_BF16 = 1 } fp8ds_dtype;
 
 /*
+ * Storage order of a GEMM operand.  K_MAJOR: a [m, k] / b [n, k] row-major
+ * (k contiguous, the "TN" layout of torch._scaled_mm(a, b.t())).  MN_MAJOR:
+ * a [k, m] / b [k, n] row-major -- the tensor as its producer wrote it,
+ * read transposed by the tensor core (sm_100's tcgen05 reads 8-bit operands
+ * in either order, so no FP8 transpose has to be materialised).
+ */
+typedef enum { FP8DS_K_MAJOR = 0, FP8DS_MN_MAJOR = 1 } fp8ds_major;
+
+/*
  * Amax used by the update [TE761 recipe: amax_compute_algo, "max" in the
  * repro]: MAX = the max over the history window; MOST_RECENT = the amax
  * recorded in the current step alone (the recipe parameter's other choice).
@@ -266,6 +275,27 @@ fp8ds_status fp8_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float 
                               int64_t m, int64_t n, int64_t k, fp8ds_stream stream);
 
 /*
+ * fp8_gemm_major -- fp8_gemm with either storage order per operand
+ * (fp8ds_major).  Same result as fp8_gemm on the transposed operands:
+ *   d[m,n] = (sum_k A(m,k) B(n,k)) * *a_scale_inv * *b_scale_inv (+ bias[n])
+ *   A(m,k) = a[m*k + k'] (K_MAJOR) or a[k*m + m'] (MN_MAJOR), likewise B.
+ * The backward of a linear needs no transposed copies with it: the wgrad
+ * dW = dY^T X reads dY8 [tokens, out] and X8 [tokens, in] MN-major, the
+ * dgrad dX = dY W reads W8 [out, in] MN-major (the pages' TE and
+ * float8_experimental designs cast transposes because Hopper's FP8 tensor
+ * cores read only K-major operands).
+ * Requirements: as fp8_gemm, except that k % 16 == 0 is needed only with a
+ * K-major operand; m % 16 == 0 for an MN-major a, n % 16 == 0 for an
+ * MN-major b.  Errors: as fp8_gemm; FP8DS_ERR_INVALID_ARG for an unknown
+ * layout.
+ */
+fp8ds_status fp8_gemm_major(const uint8_t *a, fp8ds_format a_fmt, fp8ds_major a_major,
+                            const float *a_scale_inv, const uint8_t *b, fp8ds_format b_fmt,
+                            fp8ds_major b_major, const float *b_scale_inv, const void *bias,
+                            fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype, int64_t m,
+                            int64_t n, int64_t k, fp8ds_stream stream);
+
+/*
  * fp8_gemm_cast -- the GEMM with an FP8 output for the next layer [PTFP8
  * torch._scaled_mm with out_dtype=float8_e4m3fn, returning the output and its
  * amax].  Reading used here: the FP8 output is the cast that the next layer
@@ -281,14 +311,17 @@ fp8ds_status fp8_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float 
  * out_scale_inv) without h ever reaching memory.  out_scale is normally the
  * next layer's delayed scale (meta.scale[t]) and out_amax its history slot 0
  * (amax_history[0, t]).
- *   a, b, bias, m, n, k, formats: as fp8_gemm.
+ *   a, b, bias, m, n, k, formats: as fp8_gemm; a_major / b_major as
+ *   fp8_gemm_major (the fused dgrad of a linear without a weight transpose
+ *   reads w8 MN-major).
  *   d8 [m, n] uint8, d8t [n, m] uint8 or NULL; out_scale [1] fp32.
  * Requirements: as fp8_gemm, plus n % 16 == 0, m % 16 == 0 when d8t is not
  * NULL, d8 / d8t 16-byte aligned.  Errors: as fp8_gemm.
  */
-fp8ds_status fp8_gemm_cast(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,
-                           const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
-                           const void *bias, fp8ds_dtype bias_dtype, int64_t m, int64_t n, int64_t k,
+fp8ds_status fp8_gemm_cast(const uint8_t *a, fp8ds_format a_fmt, fp8ds_major a_major,
+                           const float *a_scale_inv, const uint8_t *b, fp8ds_format b_fmt,
+                           fp8ds_major b_major, const float *b_scale_inv, const void *bias,
+                           fp8ds_dtype bias_dtype, int64_t m, int64_t n, int64_t k,
                            fp8ds_format out_fmt, const float *out_scale, uint8_t *d8, uint8_t *d8t,
                            float *out_amax, float *out_scale_inv, fp8ds_stream stream);
 
@@ -322,7 +355,8 @@ typedef struct {
     int64_t in_features;
     int64_t out_features;
     uint8_t *w8;               /* [out_features, in_features] cached FP8 weight */
-    uint8_t *w8t;              /* [in_features, out_features] cached FP8 transpose */
+    uint8_t *w8t;              /* [in_features, out_features] cached FP8 transpose, or NULL
+                                  (then the backward reads w8 MN-major) */
     float *w_scale_inv;        /* [1] private scale_inv of the cached weight */
     int32_t meta_in, meta_w, meta_grad;
     int32_t cache_valid;
@@ -410,9 +444,18 @@ fp8ds_status fp8_linear_fwd_ex(fp8ds_linear *lin, const fp8ds_meta *meta, const 
                                int32_t is_first_microbatch, uint8_t *x8, uint8_t *x8t,
                                float *x_scale_inv, const fp8ds_fp8_io *io, fp8ds_stream stream);
 
-/* fp8_linear_bwd with the options above (io may be NULL: same as fp8_linear_bwd). */
+/*
+ * fp8_linear_bwd with the options above (io may be NULL), and with every
+ * transposed copy optional (fp8_gemm_major reads the untransposed tensors):
+ *   x8t NULL  -> the wgrad reads x8 [m, in_features] (required then);
+ *   dy8t NULL -> the gradient cast writes no transpose and the wgrad reads
+ *                dy8 [m, out_features];
+ *   lin->w8t NULL (also accepted by the forward, which then writes no weight
+ *                transpose) -> the dgrad reads w8 [out_features, in_features].
+ * MN-major reads need in_features % 16 == 0 and out_features % 16 == 0.
+ */
 fp8ds_status fp8_linear_bwd_ex(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy,
-                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8t,
+                               fp8ds_dtype dy_dtype, int64_t m, const uint8_t *x8, const uint8_t *x8t,
                                const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
                                float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv,
                                const fp8ds_fp8_io *io, fp8ds_stream stream);

@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
     for n in ("fp8_quantize", "fp8_cast_transpose_amax", "fp8_update_scales", "fp8_gemm",
               "fp8_gemm_ex", "fp8_gemm_workspace_size", "fp8_gemm_noalloc", "fp8_gemm_cast",
               "fp8_linear_fwd_ex", "fp8_linear_bwd_ex", "fp8_cast_transpose_amax_noop",
-              "fp8_cast_transpose_amax_dynamic", "fp8_transpose",
+              "fp8_cast_transpose_amax_dynamic", "fp8_transpose", "fp8_gemm_major",
               "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
               "fp8ds_version"):
         assert n in names
@@ -127,8 +127,9 @@ def test_gemm_cast_argument_checks(lib):
     L = lib._lib
     s = P(0)
 
-    def call(m=128, n=256, k=128, fmt=0, scale=FAKE, d8=FAKE, d8t=None):
-        return L.fp8_gemm_cast(FAKE, 0, FAKE, FAKE, 0, FAKE, None, 0, m, n, k, fmt, scale, d8, d8t, None, None, s)
+    def call(m=128, n=256, k=128, fmt=0, scale=FAKE, d8=FAKE, d8t=None, am=0):
+        return L.fp8_gemm_cast(FAKE, 0, am, FAKE, FAKE, 0, 0, FAKE, None, 0, m, n, k, fmt, scale, d8, d8t, None, None,
+                               s)
 
     assert call(n=264) == lib.ERR_INVALID_ARG and "multiple of 16" in lib.fp8ds_last_error()
     assert call(m=120, d8t=FAKE) == lib.ERR_INVALID_ARG and "transposed" in lib.fp8ds_last_error()
@@ -137,6 +138,7 @@ def test_gemm_cast_argument_checks(lib):
     assert call(d8=None) == lib.ERR_INVALID_ARG
     assert call(d8t=FAKE_ODD) == lib.ERR_INVALID_ARG and "aligned" in lib.fp8ds_last_error()
     assert call(k=120) == lib.ERR_INVALID_ARG
+    assert call(am=3) == lib.ERR_INVALID_ARG and "layout" in lib.fp8ds_last_error()
 
 
 def test_linear_ex_argument_checks(lib):
@@ -161,8 +163,8 @@ def test_linear_ex_argument_checks(lib):
         "multiple of 16" in lib.fp8ds_last_error()
 
     def bwd(io, lin_, dy=FAKE, m=128):
-        return L.fp8_linear_bwd_ex(ctypes.byref(lin_), ctypes.byref(meta), dy, 1, m, FAKE, FAKE, FAKE, 1, FAKE,
-                                   FAKE, FAKE, FAKE, ctypes.byref(io), s)
+        return L.fp8_linear_bwd_ex(ctypes.byref(lin_), ctypes.byref(meta), dy, 1, m, None, FAKE, FAKE, FAKE, 1,
+                                   FAKE, FAKE, FAKE, FAKE, ctypes.byref(io), s)
 
     assert bwd(lib._Fp8Io(0, -1, None, None, None), lin) == lib.ERR_INVALID_ARG and \
         "cache" in lib.fp8ds_last_error()
@@ -174,3 +176,20 @@ def test_linear_ex_argument_checks(lib):
         "transposed" in lib.fp8ds_last_error()
     assert bwd(lib._Fp8Io(1, 11, FAKE, FAKE, FAKE), cached, dy=None) == lib.ERR_INVALID_ARG and \
         "out of range" in lib.fp8ds_last_error()
+
+
+def test_gemm_major_argument_checks(lib):
+    """Operand layouts: an MN-major a needs m % 16, an MN-major b needs n % 16,
+    k % 16 only with a K-major operand; unknown layouts are refused.  Every
+    call below fails a check (no launch)."""
+    L = lib._lib
+    s = P(0)
+
+    def call(am=0, bm=0, m=128, n=256, k=128):
+        return L.fp8_gemm_major(FAKE, 0, am, FAKE, FAKE, 0, bm, FAKE, None, 0, FAKE, 1, m, n, k, s)
+
+    assert call(am=2) == lib.ERR_INVALID_ARG and "layout" in lib.fp8ds_last_error()
+    assert call(am=1, m=120) == lib.ERR_INVALID_ARG and "MN-major a" in lib.fp8ds_last_error()
+    assert call(bm=1, n=264) == lib.ERR_INVALID_ARG and "MN-major b" in lib.fp8ds_last_error()
+    assert call(am=0, bm=1, k=120) == lib.ERR_INVALID_ARG and "K-major" in lib.fp8ds_last_error()
+    assert call(am=1, bm=1, k=120, n=12) == lib.ERR_INVALID_ARG   # k is free, but n % 16 is not met

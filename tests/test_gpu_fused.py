@@ -111,12 +111,13 @@ class _Mlp:
     """fc1 (hidden -> ffn) and fc2 (ffn -> hidden) with metas [X, W1, dH, H, W2, dY]
     and all device buffers of one training step."""
 
-    def __init__(self, fp8, tokens, hidden, ffn, workspace=None):
+    def __init__(self, fp8, tokens, hidden, ffn, workspace=None, transposes=True):
         w1, b1, w2, b2 = inputs.mlp_pair(seed=0, tokens=tokens, hidden=hidden, ratio=ffn // hidden)
         self.fp8 = fp8
         self.meta = fp8.Fp8Meta(["e4m3", "e4m3", "e5m2", "e4m3", "e4m3", "e5m2"], hist_len=16)
-        self.fc1 = fp8.Fp8Linear(w1.cuda(), b1.cuda(), 0, 1, 2, workspace=workspace)
-        self.fc2 = fp8.Fp8Linear(w2.cuda(), b2.cuda(), 3, 4, 5, workspace=workspace)
+        self.fc1 = fp8.Fp8Linear(w1.cuda(), b1.cuda(), 0, 1, 2, workspace=workspace, transpose=transposes)
+        self.fc2 = fp8.Fp8Linear(w2.cuda(), b2.cuda(), 3, 4, 5, workspace=workspace, transpose=transposes)
+        self.transposes = transposes
         M, Hd, F = tokens, hidden, ffn
         u = lambda *s: torch.zeros(*s, dtype=torch.uint8, device="cuda")   # noqa: E731
         f = lambda *s: torch.zeros(*s, dtype=torch.float32, device="cuda")  # noqa: E731
@@ -151,9 +152,22 @@ class _Mlp:
                               self.si[3:4], dx=self.dx, in_cast=True)
         m.update()
 
+    def step_no_transposes(self, x, dy):
+        """The fused step with no transposed copy anywhere: the GEMMs read
+        X8, H8, dY8, dH8 and the weights MN-major where the transpose was used."""
+        fp8, m = self.fp8, self.meta
+        fp8.fp8_linear_fwd_ex(self.fc1, m, x, None, True, self.x8, None, self.si[0:1], out_meta=3,
+                              out8=self.h8, out8t=None, out_scale_inv=self.si[1:2])
+        fp8.fp8_linear_fwd_ex(self.fc2, m, None, self.y, True, self.h8, None, self.si[1:2], in_cast=True)
+        fp8.fp8_linear_bwd_ex(self.fc2, m, dy, None, self.si[1:2], self.dw2, self.dy8, None, self.si[2:3],
+                              out_meta=2, out8=self.dh8, out8t=None, out_scale_inv=self.si[3:4], x8=self.h8)
+        fp8.fp8_linear_bwd_ex(self.fc1, m, None, None, self.si[0:1], self.dw1, self.dh8, None, self.si[3:4],
+                              dx=self.dx, in_cast=True, x8=self.x8)
+        m.update()
 
-def _compare(u, f, what):
-    for name in ("x8", "x8t", "h8", "h8t", "dy8", "dy8t", "dh8", "dh8t"):
+
+def _compare(u, f, what, names=("x8", "x8t", "h8", "h8t", "dy8", "dy8t", "dh8", "dh8t")):
+    for name in names:
         assert_bytes_equal(u8(getattr(f, name)), u8(getattr(u, name)), "%s: %s" % (what, name))
     for name in ("y", "dx"):
         assert_bytes_equal(host_bits(getattr(f, name)), host_bits(getattr(u, name)), "%s: %s" % (what, name))
@@ -182,3 +196,24 @@ def test_mlp_fp8_handover_equals_unfused(fp8, tokens, hidden, ffn, use_ws):
         torch.cuda.synchronize()
         assert fp8.fp8ds_device_status() == 0
         _compare(un, fu, "step %d" % step)
+
+
+@pytest.mark.parametrize("tokens,hidden,ffn", [(384, 256, 1024), (8192, 2048, 8192)])
+def test_mlp_without_transposes_equals_unfused(fp8, tokens, hidden, ffn):
+    """The B200 layout of the step: no FP8 transpose is ever written (casts
+    without yt, weight caches without w8t, FP8 epilogues without the
+    transposed output); the wgrads read X8/H8 and dY8/dH8 and the dgrads the
+    weights MN-major.  Every output, FP8 tensor and meta equals the unfused
+    step that casts and reads transposes, over three steps."""
+    un = _Mlp(fp8, tokens, hidden, ffn)
+    nt = _Mlp(fp8, tokens, hidden, ffn, transposes=False)
+    for step in range(3):
+        x, dy = inputs.mlp_step_inputs(step, tokens=tokens, hidden=hidden)
+        xd, dyd = x.cuda(), dy.cuda()
+        un.step_unfused(xd, dyd)
+        nt.step_no_transposes(xd, dyd)
+        torch.cuda.synchronize()
+        assert fp8.fp8ds_device_status() == 0
+        _compare(un, nt, "step %d" % step, names=("x8", "h8", "dy8", "dh8"))
+        assert_bytes_equal(u8(nt.fc1.w8), u8(un.fc1.w8), "step %d: w1 cache" % step)
+        assert_bytes_equal(u8(nt.fc2.w8), u8(un.fc2.w8), "step %d: w2 cache" % step)
