@@ -647,12 +647,21 @@ __device__ __forceinline__ void store_segment(uint8_t *dst, int64_t left, const 
 }
 
 __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint8_t *box, int half, uint8_t *d8,
-                                                  uint8_t *d8t, int64_t n_base, int32_t m_row0, float sab,
+                                                  uint8_t *d8t, const CUtensorMap *tmap_d, int64_t n_base,
+                                                  int32_t m_row0, float sab,
                                                   const float *bias_s, uint32_t empty_bar_cluster, bool arrive,
                                                   int mode, float *slot, int h, int q, float s_out, int fmt,
                                                   int32_t m_total, int32_t n_total, float &amax) {
     constexpr int CHUNKS = ACC_N / 32 / 2;
     const int32_t m = m_row0 + lane;
+    // Without the transpose the warp's 32 rows x 128 code bytes are one
+    // 128-byte-swizzled staging box and one TMA store; with it, the codes go
+    // out with plain stores beside the transposed ones.
+    const bool staged = d8t == nullptr;
+    if (staged && mode != 1) {
+        if (lane == 0) tma_store_wait_read<0>();
+        __syncwarp();
+    }
     const uint64_t sab2 = pack_f32x2(sab, sab);
     const uint64_t s2 = pack_f32x2(s_out, s_out);
     uint32_t r[32];
@@ -690,7 +699,13 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
         }
         // the registers of r are free: start the next chunk's TMEM load
         if (c + 1 < CHUNKS) tmem_ld32(t_row + col0 + 32, r);
-        if (mode != 1) {
+        if (mode != 1 && staged) {
+            // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
+            *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c) ^ (lane & 7)) * 16) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c + 1) ^ (lane & 7)) * 16) =
+                make_uint4(w[4], w[5], w[6], w[7]);
+        } else if (mode != 1) {
             const int64_t n0 = n_base + col0;
             if (m < m_total && n0 < n_total)
                 store_segment(d8 + static_cast<int64_t>(m) * n_total + n0, n_total - n0, w);
@@ -713,6 +728,14 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
             }
         }
         if (c + 1 < CHUNKS) tmem_ld_wait();
+    }
+    if (staged && mode != 1) {
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * CHUNKS * 32), m_row0);
+            tma_store_commit();
+        }
     }
 }
 
@@ -814,9 +837,9 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
                                    static_cast<uint32_t>((acc + h) * ACC_N);
             const int32_t m_row0 = (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32;
             if constexpr (OUT == OUT_FP8)
-                epilogue_tile_fp8(t_row, lane, box, half, p.out_d8, p.out_d8t, static_cast<int64_t>(n_blk) * ACC_N,
-                                  m_row0, sab, bias_s, empty_addr, h == m_sub - 1, mode, slot, h, q, s_out,
-                                  p.out_fmt, p.M, p.N, amax);
+                epilogue_tile_fp8(t_row, lane, box, half, p.out_d8, p.out_d8t, tmap_d,
+                                  static_cast<int64_t>(n_blk) * ACC_N, m_row0, sab, bias_s, empty_addr,
+                                  h == m_sub - 1, mode, slot, h, q, s_out, p.out_fmt, p.M, p.N, amax);
             else
                 epilogue_tile<OUT == OUT_BF16>(t_row, lane, box, half, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
                                                m_row0, sab, bias_s, empty_addr, h == m_sub - 1, mode, slot, h, q);
@@ -1271,9 +1294,9 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
               (b_mn ? encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, n, k, n, 128, BK)
                     : encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b, k, n, k, BK, b_rows));
     if (out == OUT_FP8) {
-        // the FP8 epilogue stores with plain global stores; the map stays a
-        // valid description of the codes (it is only prefetched)
-        ok = ok && encode_tmap_2d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT8, d, n, m, n, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+        // codes [m, n]: 128-byte x 32-row swizzled boxes (the store path
+        // without transpose; with it the epilogue uses plain stores)
+        ok = ok && encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_UINT8, d, n, m, n, 128, 32);
     } else {
         ok = ok && (out == OUT_BF16 ? encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, n, m, n * 2, 64, 32)
                                     : encode_2d(&td, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d, n, m, n * 4, 32, 32));

@@ -59,6 +59,10 @@ CASES = [
     (1024, 512, 4096, "e4m3", None, True, 0.0),      # 512-row pair tiles (long K)
     (1024, 512, 4096, "e5m2", "f32", False, 1e9),    # no transpose; a larger running amax is kept
     (2048, 8192, 2048, "e4m3", "f32", True, 0.0),    # the MLP's fc1 shape class
+    # without the transpose the codes leave through the staged TMA store
+    (128, 256, 128, "e4m3", "f32", False, 0.0),
+    (400, 528, 256, "e5m2", "bf16", False, 0.0),
+    (2048, 8192, 2048, "e4m3", "f32", False, 0.0),
 ]
 
 
