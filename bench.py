@@ -427,6 +427,27 @@ def time_cast_workload(fp8, device, reps=100):
     return res
 
 
+def time_update_576(fp8, device, reps=200):
+    """One fp8_update_scales launch over the 576 metas of the 32-block model
+    (32 blocks x 6 linears x input/weight/grad), history 16, launched back to
+    back (the history starts filled with amaxes; every launch reads and
+    rewrites all 16 slots of every meta).  Mean per launch."""
+    T = 32 * 6 * 3
+    meta = fp8.Fp8Meta(["e4m3", "e4m3", "e5m2"] * (T // 3), hist_len=16, device=device)
+    g = torch.Generator(device="cpu").manual_seed(11)
+    meta.amax_history.copy_(torch.rand(16, T, generator=g).to(device) * 10)
+    for _ in range(10):
+        meta.update()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        meta.update()
+    e1.record()
+    torch.cuda.synchronize()
+    return 1e3 * e0.elapsed_time(e1) / reps
+
+
 def time_headline_gemm(fp8, device, reps=50, warmup=10):
     """8192x2048x8192 and 8192x8192x2048 e4m3 GEMMs (bf16 out), timed alone:
     10 warm-up and 50 timed launches.  torch._scaled_mm (a library GEMM) is
@@ -840,6 +861,7 @@ def main():
     c2_us = statistics.mean([c2["e4m3"]["us_mean"], c2["e5m2"]["us_mean"]])
     c2_gbs = C2_BYTES / (c2_us * 1e-6) / 1e9
     heads = time_headline_gemm(fp8, device)
+    upd576_us = time_update_576(fp8, device)
 
     # end to end through the public API with host buffers
     e2e_ms, h2d, d2h = e2e_linear_api(fp8, step, device, max(10, args.steps // 2), 3)
@@ -909,6 +931,7 @@ def main():
             "dynamic_note": "amax pass + scale + cast (input read twice) vs the delayed cast's one read",
         },
         "update_scales_us": 1e3 * statistics.mean(upd_ms),
+        "update_scales_576_metas_us": upd576_us,
         "gemm_us": {k: 1e3 * statistics.mean(v) for k, v in gemm_by_key.items()},
         "cast_us": {k: 1e3 * statistics.mean(v) for k, v in cast_ms.items()},
         "kernels_sum_ms_per_step": kernel_ms,

@@ -370,7 +370,7 @@ typedef struct {
  *   1. cast x -> x8 (and x8t if not NULL) with meta.scale[meta_in], amax into
  *      amax_history[0, meta_in], private scale_inv into *x_scale_inv;
  *   2. if is_first_microbatch is -1 (None: always), 1 (True: refresh and keep),
- *      or 0 (False) with no valid cache: cast w -> w8 and w8t with
+ *      or 0 (False) with no valid cache: cast w -> w8 and w8t (if not NULL) with
  *      meta.scale[meta_w], amax into amax_history[0, meta_w], private
  *      scale_inv into *w_scale_inv; sets cache_valid.  With 0 and a valid
  *      cache the cached weight and its frozen scale_inv are reused;
@@ -382,7 +382,8 @@ typedef struct {
  * is_first_microbatch is then ignored for the weight.  Write 0 to the flag
  * for a microbatch that must refresh the cache, 1 for the others.
  *   x [m, in_features] (x_dtype); y [m, out_features] (y_dtype);
- *   x8 [m, in_features], x8t [in_features, m] or NULL (needed by the backward).
+ *   x8 [m, in_features], x8t [in_features, m] or NULL (fp8_linear_bwd reads
+ *   x8t; fp8_linear_bwd_ex reads x8 MN-major when x8t is NULL).
  * The delayed-scaling update is not part of the forward: call
  * fp8_update_scales once per step over the whole meta.
  * Errors: as the calls it makes; nothing is enqueued if the arguments fail.
@@ -401,6 +402,9 @@ fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const voi
  *   3. wgrad: dw[out, in] (fp32) = dy8t . (x8t)^T with *dy_scale_inv * *x_scale_inv.
  *   dy [m, out_features] (dy_dtype); x8t [in_features, m] and x_scale_inv from
  *   the forward; dy8 [m, out_features], dy8t [out_features, m] workspaces.
+ *   dy8t may be NULL (no gradient transpose is written; the wgrad reads dy8
+ *   MN-major), and a linear without w8t has its dgrad read w8 MN-major (see
+ *   fp8_gemm_major; out_features % 16 == 0 / in_features % 16 == 0 then).
  * Requires lin->cache_valid.  Errors: as the calls it makes.
  */
 fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy,

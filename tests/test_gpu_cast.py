@@ -267,3 +267,52 @@ def test_dynamic_scaling_all_zero_keeps_scale(fp8):
     torch.cuda.synchronize()
     assert am.item() == 0.0 and s.item() == 5.0 and si.item() == np.float32(0.2)
     assert bool((y == 0).all())
+
+
+def test_cast_transpose_beyond_2g_elements(fp8):
+    """A bf16 [65536, 32776] cast (2.15e9 elements: more than 2^31, so every
+    byte offset past 2 GB must be formed in 64 bits; 32776 columns leave a
+    ragged last column tile).  The input is drawn in seeded row chunks
+    (generator 4000 + chunk, N(0,1)) straight to the device.  Checked: the
+    amax over the whole tensor (oracle amax of every chunk), the scale_inv,
+    and the FP8 bytes of sampled rows of y and of yt (oracle casts of those
+    rows and columns)."""
+    R, C, CH = 65536, 32776, 4096
+    xd = torch.empty(R, C, dtype=torch.bfloat16, device="cuda")
+    am_ref = np.float32(0.0)
+    rows = np.array([0, 1, 4095, 4096, 32767, 32768, 65534, 65535], np.int64)
+    cols = np.array([0, 1, 63, 64, 16383, 16384, 32767, 32768, 32775], np.int64)
+    row_bits, col_bits = {}, np.empty((R, cols.size), np.uint16)
+    for c in range(R // CH):
+        xc = inputs.normal((CH, C), inputs.gen(4000 + c)).to(torch.bfloat16)
+        if c == R // CH - 1:
+            xc[CH - 1, C - 1] = 3072.0           # the largest entry (exact in bf16), last row and column
+        bits = host_bits(xc)
+        am_ref = o.amax(bits, am_ref)
+        for r in rows[(rows >= c * CH) & (rows < (c + 1) * CH)]:
+            row_bits[int(r)] = bits[r - c * CH].copy()
+        col_bits[c * CH:(c + 1) * CH] = bits[:, cols]
+        xd[c * CH:(c + 1) * CH].copy_(xc)
+        del xc, bits
+    s = np.float32(448.0) / np.float32(1000.0)
+    y = torch.empty(R, C, dtype=torch.uint8, device="cuda")
+    yt = torch.empty(C, R, dtype=torch.uint8, device="cuda")
+    sd = torch.tensor([s], device="cuda")
+    am = torch.zeros(1, device="cuda")
+    si = torch.zeros(1, device="cuda")
+    fp8.fp8_cast_transpose_amax(xd, "e4m3", sd, y, yt, am, si)
+    torch.cuda.synchronize()
+    assert fp8.fp8ds_device_status() == 0
+    assert_f32_bits_equal(am.cpu().numpy(), [am_ref], "amax")
+    assert am.item() == 3072.0
+    assert_f32_bits_equal(si.cpu().numpy(), [np.float32(1.0) / s], "scale_inv")
+    ridx = torch.from_numpy(rows).cuda()
+    got_rows = y.index_select(0, ridx).cpu().numpy()
+    for k, r in enumerate(rows):
+        ry, _, _, _ = o.cast_transpose_amax(row_bits[int(r)][None, :], o.E4M3, s, transpose=False)
+        assert_bytes_equal(got_rows[k], ry[0], "y row %d" % r)
+    got_cols = yt.index_select(0, torch.from_numpy(cols).cuda()).cpu().numpy()
+    ry, _, _, _ = o.cast_transpose_amax(np.ascontiguousarray(col_bits.T), o.E4M3, s, transpose=False)
+    assert_bytes_equal(got_cols, ry, "yt rows (x columns)")
+    del xd, y, yt
+    torch.cuda.empty_cache()
