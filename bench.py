@@ -292,6 +292,17 @@ class MlpStep:
             sync_amax(m)
         m.update()
 
+    def run_casts(self, i):
+        """The native step's four delayed-scaling casts alone (X, W1, W2 from
+        fp32, dY from bf16; y only, no transpose), on step i's inputs."""
+        fp8, m, fc1, fc2 = self.fp8, self.meta, self.fc1n, self.fc2n
+        x, dy = self.xs[i % len(self.xs)], self.dys[i % len(self.dys)]
+        amax = m.amax_history[0]
+        fp8.fp8_cast_transpose_amax(x, "e4m3", m.scale[0:1], self.x8, None, amax[0:1], self.si[0:1])
+        fp8.fp8_cast_transpose_amax(fc1.w, "e4m3", m.scale[1:2], fc1.w8, None, amax[1:2], fc1.w_scale_inv)
+        fp8.fp8_cast_transpose_amax(fc2.w, "e4m3", m.scale[4:5], fc2.w8, None, amax[4:5], fc2.w_scale_inv)
+        fp8.fp8_cast_transpose_amax(dy, "e5m2", m.scale[5:6], self.dy8, None, amax[5:6], self.si[2:3])
+
     def run_gemms(self):
         """The native step's six GEMM launches alone, in step order, on the
         step's own operands, outputs, layouts and epilogues, with nothing
@@ -659,16 +670,27 @@ def single_kernel(args):
             run = lambda: fp8.fp8_gemm_cast(a, "e4m3", sa, b, "e4m3", sa, "e4m3", so, d8, None, am, si)  # noqa: E731
         work, unit = 2.0 * M * N * K / 1e12, "TFLOP/s"
     else:
+        # the bf16 [8192, 2048] workload, or (--cast-in f32) the fp32 input
+        # of the same shape that the step's X and weight casts read; --no-yt
+        # writes y only, as the native step does
         base = inputs.spiky_bf16().to(dev)
+        if args.cast_in == "f32":
+            base = base.float()
         xs = [base] + [base.roll(i * 17, dims=1).contiguous() for i in range(1, 8)]
         y = torch.empty(C2_ROWS, C2_COLS, dtype=torch.uint8, device=dev)
-        yt = torch.empty(C2_COLS, C2_ROWS, dtype=torch.uint8, device=dev)
+        yt = None
+        if not args.no_yt and args.kernel != "quantize":
+            yt = torch.empty(C2_COLS, C2_ROWS, dtype=torch.uint8, device=dev)
         s = torch.ones(1, device=dev)
         am = torch.zeros(1, device=dev)
         si = torch.zeros(1, device=dev)
         it = iter(range(1 << 30))
-        run = lambda: fp8.fp8_cast_transpose_amax(xs[next(it) % 8], args.fmt, s, y, yt, am, si)  # noqa: E731
-        work, unit = C2_BYTES / 1e9, "GB/s"
+        if args.kernel == "quantize":                    # the flat (1-D) cast of the same bytes
+            run = lambda: fp8.fp8_quantize(xs[next(it) % 8], args.fmt, s, y, am, si)  # noqa: E731
+        else:
+            run = lambda: fp8.fp8_cast_transpose_amax(xs[next(it) % 8], args.fmt, s, y, yt, am, si)  # noqa: E731
+        work = C2_ROWS * C2_COLS * (base.element_size() + 1 + (0 if yt is None else 1)) / 1e9
+        unit = "GB/s"
     for _ in range(2):
         run()
     torch.cuda.synchronize()
@@ -679,7 +701,8 @@ def single_kernel(args):
     s1.record()
     torch.cuda.synchronize()
     us = 1e3 * s0.elapsed_time(s1) / args.reps
-    print(json.dumps({"kernel": args.kernel, "us": us, "rate": work / (us * 1e-6), "unit": unit,
+    print(json.dumps({"kernel": args.kernel, "shape": args.shape if args.kernel.startswith("gemm") else None,
+                      "cast_in": args.cast_in, "yt": not args.no_yt, "us": us, "rate": work / (us * 1e-6), "unit": unit,
                       "status": fp8.fp8ds_device_status()}))
 
 
@@ -694,11 +717,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=None,
                     help="tokens of the oracle's sample (default 128; 8 per step for --impl reference)")
-    ap.add_argument("--kernel", choices=["gemm", "gemmcast", "cast"], default=None,
+    ap.add_argument("--kernel", choices=["gemm", "gemmcast", "cast", "quantize"], default=None,
                     help="run one kernel alone (2 warm-up + --reps launches), for profilers")
     ap.add_argument("--shape", default="8192x2048x8192", help="MxNxK for --kernel gemm")
     ap.add_argument("--major", default="k,k", help="operand layouts a,b for --kernel gemm: k or mn each")
     ap.add_argument("--fmt", default="e4m3", help="FP8 format for --kernel cast")
+    ap.add_argument("--cast-in", default="bf16", choices=["bf16", "f32"], help="input dtype for --kernel cast")
+    ap.add_argument("--no-yt", action="store_true", help="--kernel cast writes y only (no transpose)")
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     if args.kernel:
@@ -830,6 +855,20 @@ def main():
     gemm_clock_info = gclocks.stop() if gclocks else None
     gemm_b2b_ms = g0.elapsed_time(g1) / (STEP_GEMMS * args.steps)
 
+    # the step's four casts back to back, K rounds over the rotating inputs
+    # (234 MB read per round, more than L2): the cast kernels' own rate in
+    # the step's shapes, free of the per-launch event brackets' host gaps
+    for i in range(2):
+        step.run_casts(i)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier_sync(world)
+    c0.record()
+    for i in range(args.steps):
+        step.run_casts(i)
+    c1.record()
+    barrier_sync(world)
+    cast_b2b_ms = max_over_ranks(c0.elapsed_time(c1) / args.steps, world, device)
+
     per = log.summary()
     gemm_ms = [t for _, t in per["gemm"]]
     gemm_by_key = {}
@@ -853,7 +892,8 @@ def main():
             gemm_peak, gemm_peak_kind = fp8_peak_sus, "sustained"
     cast_total_ms = sum(sum(v) for v in cast_ms.values()) / args.steps
     kernel_ms = (sum(gemm_ms) + sum(upd_ms)) / args.steps + cast_total_ms
-    cast_gbs_step = STEP_CAST_BYTES_FUSED / (cast_total_ms * 1e-3) / 1e9
+    cast_gbs_step = STEP_CAST_BYTES_FUSED / (cast_b2b_ms * 1e-3) / 1e9
+    cast_gbs_bracketed = STEP_CAST_BYTES_FUSED / (cast_total_ms * 1e-3) / 1e9
     value = world * STEP_FLOP / (ms * 1e-3) / 1e12
 
     # standalone: cast-transpose-amax workload and the headline GEMM shapes
@@ -927,6 +967,10 @@ def main():
             "bytes_per_launch": C2_BYTES, "achieved": c2_gbs, "peak": pk["hbm"], "unit": "GB/s",
             "frac": c2_gbs / pk["hbm"], "bound": "hbm",
             "in_step_gbs": cast_gbs_step, "in_step_frac": cast_gbs_step / pk["hbm"],
+            "in_step_us": 1e3 * cast_b2b_ms, "in_step_bytes": STEP_CAST_BYTES_FUSED,
+            "in_step_note": "the step's 4 casts (X, W1, W2 fp32; dY bf16; y only) back to back, K rounds, "
+                            "CUDA events around the loop",
+            "in_step_event_bracketed_gbs": cast_gbs_bracketed,
             "dynamic_scaling_e4m3_us": c2["dynamic_e4m3"]["us_mean"],
             "dynamic_note": "amax pass + scale + cast (input read twice) vs the delayed cast's one read",
         },

@@ -72,10 +72,12 @@ constexpr int EPI_BYTES = EPI_WARPS * EPI_BOX_BYTES + 256 * 4;  // + the tile's 
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int SMEM_ALIGN = 1024;
 constexpr int GROUP_M = 8;
-// Smallest K for which the pair kernel takes the 512-row tile (compile-time
-// setting; 4096 measured best on B200 for the MLP shapes).
+// Smallest K for which the pair kernel may take the 512-row tile (compile-
+// time setting).  On B200 the 512-row tile measured 3-4% faster than the
+// 256-row one at 8192 x 8192 x 2048 and at K = 8192, as long as its last
+// wave is no emptier (checked at launch).
 #ifndef FP8DS_MSUB2_MIN_K
-#define FP8DS_MSUB2_MIN_K 4096
+#define FP8DS_MSUB2_MIN_K 2048
 #endif
 // Output kinds of the epilogue.
 constexpr int OUT_F32 = 0;
@@ -94,8 +96,9 @@ constexpr int S1_SMEM = SMEM_ALIGN + S1_STAGES * (S1_A_STAGE + S1_B_STAGE) + EPI
 // 2-SM kernel: pair tile (M_SUB x 256) x 256.  Per CTA and stage: M_SUB
 // boxes of 128 rows of A and 128 rows of B.  M_SUB = 1: 6 stages of 32 KB,
 // two accumulators (double-buffered).  M_SUB = 2: 4 stages of 48 KB, the two
-// M halves fill all 512 TMEM columns (one accumulator set, not overlapped
-// with the epilogue) in exchange for 25% fewer loaded bytes per FLOP.
+// M halves fill all 512 TMEM columns (one accumulator set) in exchange for
+// 25% fewer loaded bytes per FLOP; the halves are released to the next tile
+// one at a time, so only the epilogue's first half is not overlapped.
 constexpr int S2_BM = 128;           // rows of A (and of D) per CTA and M half
 constexpr int S2_BN_HALF = 128;      // rows of B per CTA
 constexpr int S2_B_STAGE = S2_BN_HALF * BK;
@@ -787,7 +790,7 @@ template <int OUT>
 __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap *tmap_d, const Params &p,
                                               uint32_t tmem_base, int warp, int lane, int cluster, int clusters,
                                               int m_sub, int rows_per_sub, int row_offset, int acc_bufs,
-                                              uint32_t tempty_rank, int rank) {
+                                              uint32_t tempty_rank, int rank, bool split) {
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - EPI_WARP0) >> 2;  // which half of the accumulator columns
     uint8_t *box = sm.epi + (warp - EPI_WARP0) * EPI_BOX_BYTES;
@@ -831,18 +834,24 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
         stage_bias(bias_s, p, static_cast<int64_t>(n_blk) * ACC_N, epi_tid);
         epilogue_bar();
         tc_fence_after();
-        const uint32_t empty_addr = map_to_cta(smem_u32(&sm.tempty[acc]), tempty_rank);
+        // An accumulator is released whole (tempty[acc]) after its last row
+        // block, or with `split` (a single accumulator set of two M halves)
+        // half by half (tempty[h]), so that the next tile's half-0 MMAs
+        // start while half 1 is still being read.
+        const uint32_t empty_base = map_to_cta(smem_u32(&sm.tempty[acc]), tempty_rank);
         for (int h = 0; h < m_sub; ++h) {
+            const uint32_t empty_addr = empty_base + static_cast<uint32_t>(split ? h * sizeof(uint64_t) : 0);
+            const bool release = split || h == m_sub - 1;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>((acc + h) * ACC_N);
             const int32_t m_row0 = (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32;
             if constexpr (OUT == OUT_FP8)
                 epilogue_tile_fp8(t_row, lane, box, half, p.out_d8, p.out_d8t, tmap_d,
-                                  static_cast<int64_t>(n_blk) * ACC_N, m_row0, sab, bias_s, empty_addr,
-                                  h == m_sub - 1, mode, slot, h, q, s_out, p.out_fmt, p.M, p.N, amax);
+                                  static_cast<int64_t>(n_blk) * ACC_N, m_row0, sab, bias_s, empty_addr, release,
+                                  mode, slot, h, q, s_out, p.out_fmt, p.M, p.N, amax);
             else
                 epilogue_tile<OUT == OUT_BF16>(t_row, lane, box, half, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
-                                               m_row0, sab, bias_s, empty_addr, h == m_sub - 1, mode, slot, h, q);
+                                               m_row0, sab, bias_s, empty_addr, release, mode, slot, h, q);
         }
         if (mode == 1) {
             // Publish: every epilogue thread's partial stores precede the flag.
@@ -1003,7 +1012,8 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         __syncwarp();
     } else {
-        epilogue_loop<OUT>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u, 0);
+        epilogue_loop<OUT>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u, 0,
+                           false);
     }
 
     tc_fence_before();
@@ -1029,6 +1039,10 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     constexpr int STAGES = PC::STAGES;
     constexpr int A_STAGE = PC::A_STAGE;
     constexpr int ACC_BUFS = PC::ACC_BUFS;
+    // Half-by-half release of the 512-row tile's accumulator (FP8 output,
+    // whose longer epilogue it hides best; measured neutral-to-negative with
+    // bf16 and fp32 outputs).
+    constexpr bool SPLIT = M_SUB == 2 && OUT == OUT_FP8;
     extern __shared__ uint8_t smem_raw[];
     const Smem sm = carve<STAGES, A_STAGE, S2_B_STAGE>(smem_raw);
     const int warp = threadIdx.x >> 5;
@@ -1135,7 +1149,59 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     break;
                 }
                 tc_fence_after();
-                for (int kb = kb0; kb < kb1; ++kb) {
+                int kb = kb0;
+                if constexpr (SPLIT) {
+                    // The epilogue frees the two M halves one after the other
+                    // (tempty[0], then tempty[1]).  The first `pre` k-blocks
+                    // run their half-0 MMAs as soon as half 0 is free, holding
+                    // their stages; their half-1 MMAs follow once half 1 is
+                    // free, and only then are the stages released.  One stage
+                    // stays out of this so that the main loop resumes on a
+                    // loaded stage while the held ones refill.  Within each
+                    // half the accumulation order over (k-block, k) is
+                    // unchanged.
+                    const int pre = kb1 - kb0 < STAGES - 1 ? kb1 - kb0 : STAGES - 1;
+                    int st = stage;
+                    uint32_t ph = phase;
+                    for (int j = 0; j < pre && ok; ++j) {
+                        if (!mbar_wait(&sm.full[st], ph, sm.abort_flag, SITE_MMA_FULL)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t b_desc = operand_desc(smem_u32(sm.b + st * S2_B_STAGE), p.b_mn, 0);
+                        const uint64_t a_desc = operand_desc(smem_u32(sm.a + st * A_STAGE), p.a_mn, 0);
+#pragma unroll
+                        for (int k = 0; k < BK / UMMA_K; ++k)
+                            umma_f8f6f4_pair(tmem_base, a_desc + operand_kstep(k, p.a_mn),
+                                             b_desc + operand_kstep(k, p.b_mn), p.idesc, (j > 0 || k > 0) ? 1u : 0u);
+                        if (++st == STAGES) {
+                            st = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                    if (!ok || !mbar_wait(&sm.tempty[1], acc_phase ^ 1u, sm.abort_flag, SITE_MMA_TMEM_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int j = 0; j < pre; ++j) {
+                        const uint64_t b_desc = operand_desc(smem_u32(sm.b + stage * S2_B_STAGE), p.b_mn, 0);
+                        const uint64_t a_desc =
+                            operand_desc(smem_u32(sm.a + stage * A_STAGE + S2_BM * BK), p.a_mn, 0);
+#pragma unroll
+                        for (int k = 0; k < BK / UMMA_K; ++k)
+                            umma_f8f6f4_pair(tmem_base + static_cast<uint32_t>(ACC_N), a_desc + operand_kstep(k, p.a_mn),
+                                             b_desc + operand_kstep(k, p.b_mn), p.idesc, (j > 0 || k > 0) ? 1u : 0u);
+                        umma_commit_pair_to(&sm.empty[stage], 0x3);
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    kb = kb0 + pre;
+                }
+                for (; kb < kb1; ++kb) {
                     if (!mbar_wait(&sm.full[stage], phase, sm.abort_flag, SITE_MMA_FULL)) {
                         ok = false;
                         break;
@@ -1167,7 +1233,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         __syncwarp();
     } else {
         epilogue_loop<OUT>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, M_SUB, 2 * S2_BM,
-                           static_cast<int>(rank) * S2_BM, ACC_BUFS, 0u, static_cast<int>(rank));
+                           static_cast<int>(rank) * S2_BM, ACC_BUFS, 0u, static_cast<int>(rank), SPLIT);
     }
 
     tc_fence_before();
@@ -1282,9 +1348,21 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
                          bool b_mn) {
     const int out = cast != nullptr ? OUT_FP8 : (d_dtype == FP8DS_BF16 ? OUT_BF16 : OUT_F32);
     const bool pair = m > S1_BM;
-    // Long contractions amortise the non-overlapped epilogue of the 512-row
-    // pair tile; short ones keep the double-buffered 256-row tile.
-    const int m_sub = (pair && m > 2 * S2_BM && k >= FP8DS_MSUB2_MIN_K) ? 2 : 1;
+    // Long contractions amortise the partly exposed epilogue of the 512-row
+    // pair tile; short ones keep the double-buffered 256-row tile.  The
+    // 512-row tile is also declined when its tiles fill the last wave of
+    // pairs less well than the 256-row ones (e.g. 4096 x 8192: 256 tiles =
+    // 3.46 waves of 74 pairs against 512 = 6.92 waves).
+    int m_sub = 1;
+    if (pair && m > 2 * S2_BM && k >= FP8DS_MSUB2_MIN_K) {
+        static int cached_pairs[64] = {};
+        const int64_t cap = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached_pairs);
+        const int64_t tn = (n + ACC_N - 1) / ACC_N;
+        const int64_t t1 = ((m + 2 * S2_BM - 1) / (2 * S2_BM)) * tn, t2 = ((m + 4 * S2_BM - 1) / (4 * S2_BM)) * tn;
+        // wave fill tiles / (waves * cap), compared without division
+        const int64_t w1 = (t1 + cap - 1) / cap, w2 = (t2 + cap - 1) / cap;
+        if (cap <= 0 || t2 * w1 * 50 >= t1 * w2 * 49) m_sub = 2;      // fill(512) >= fill(256) - 2%
+    }
     CUtensorMap ta, tb, td;
     // K-major operands: [rows, k] boxes of BK x rows; MN-major: [k, rows]
     // boxes of 128 columns x BK rows (the one-CTA B tile loads two of them)

@@ -56,8 +56,11 @@ CASES = [
     (128, 256, 128, "e4m3", "f32", True, 0.0),       # one-CTA kernel (M <= 128)
     (400, 528, 256, "e4m3", "f32", True, 0.0),       # CTA pairs, 256-row tiles, ragged M and N
     (400, 528, 256, "e5m2", "bf16", True, 0.0),
-    (1024, 512, 4096, "e4m3", None, True, 0.0),      # 512-row pair tiles (long K)
+    (1024, 512, 4096, "e4m3", None, True, 0.0),      # long K, few tiles (256-row pair tiles)
     (1024, 512, 4096, "e5m2", "f32", False, 1e9),    # no transpose; a larger running amax is kept
+    # 512-row pair tiles (released to the next tile half by half), ragged in M, N and K
+    (1040, 4880, 4112, "e4m3", "f32", False, 0.0),
+    (1008, 4880, 2064, "e5m2", "bf16", True, 0.0),
     (2048, 8192, 2048, "e4m3", "f32", True, 0.0),    # the MLP's fc1 shape class
     # without the transpose the codes leave through the staged TMA store
     (128, 256, 128, "e4m3", "f32", False, 0.0),

@@ -83,13 +83,16 @@ def _compare(d, ref, rows, out_dtype, what, ops):
 
 
 # M <= 128 runs the 1-SM kernel, larger M the CTA-pair kernel: pair tile
-# 256 x 256, or 512 x 256 when M > 256 and K >= 4096.  Covered: ragged M
-# inside a pair and inside the 512-row tile, a second CTA with one row, B rows
-# of the second CTA entirely out of range (N <= 128), a partial last k-block,
-# more tiles than SM pairs.
+# 256 x 256, or 512 x 256 when M > 256, K >= 2048 and the 512-row tiles fill
+# the last wave of pairs as well (at least ~75 tiles of 256 rows).  Covered:
+# ragged M inside a pair and inside the 512-row tile (1040 = 2 x 512 + 16,
+# 1000), a second CTA with one row, B rows of the second CTA entirely out of
+# range (N <= 128), a partial last k-block, more tiles than SM pairs, long K
+# with few tiles (which keeps the 256-row tile).
 SHAPES = [(128, 256, 128), (128, 512, 256), (300, 520, 272), (1, 8, 16), (129, 264, 144),
           (256, 256, 1024), (4096, 8, 256), (1000, 136, 528), (4096, 2048, 256),
-          (2048, 8192, 1024), (600, 264, 4096), (1024, 512, 4112), (257, 136, 4096)]
+          (2048, 8192, 1024), (600, 264, 4096), (1024, 512, 4112), (257, 136, 4096),
+          (1040, 4880, 4112), (1000, 4880, 2064)]
 
 
 @pytest.mark.parametrize("shape", SHAPES)

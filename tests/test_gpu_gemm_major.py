@@ -51,11 +51,11 @@ def _run(fp8, a, fa, am, sa, b, fb, bm, sb, out_dtype):
 
 
 LAYOUTS = [("k", "mn"), ("mn", "k"), ("mn", "mn")]
-# (M, N, K): one-CTA kernel, pair 256-row tiles, 512-row tiles (K >= 4096),
-# ragged edges (a partial last k-block, M and N off the tile grid), more tiles
-# than SM pairs.
+# (M, N, K): one-CTA kernel, pair 256-row tiles, 512-row tiles (K >= 2048
+# with enough tiles), ragged edges (a partial last k-block, M and N off the
+# tile grid), more tiles than SM pairs.
 SHAPES = [(128, 256, 128), (64, 512, 256), (384, 512, 512), (400, 528, 272), (1024, 512, 4096),
-          (2048, 8192, 1024), (8192, 2048, 8192)]
+          (2048, 8192, 1024), (1040, 4880, 2064), (8192, 2048, 8192)]
 
 
 @pytest.mark.parametrize("layout", LAYOUTS)
