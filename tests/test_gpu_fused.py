@@ -186,11 +186,13 @@ def _compare(u, f, what, names=("x8", "x8t", "h8", "h8t", "dy8", "dy8t", "dh8", 
 
 
 @pytest.mark.parametrize("tokens,hidden,ffn,use_ws", [(384, 256, 1024, False), (1024, 512, 2048, True),
-                                                      (8192, 2048, 8192, False)])
+                                                      (7168, 2048, 2048, True), (8192, 2048, 8192, False)])
 def test_mlp_fp8_handover_equals_unfused(fp8, tokens, hidden, ffn, use_ws):
     """Three delayed-scaling steps of the MLP pair, fused and unfused side by
     side from the same inputs; with a workspace the stream-K schedule may run
-    (the same in both)."""
+    (the same in both).  At 7168 tokens every GEMM takes 112 tiles of 512 x
+    256 and runs stream-K; the FP8-output ones also release their
+    accumulator half by half."""
     ws_u = fp8.gemm_workspace() if use_ws else None
     ws_f = fp8.gemm_workspace() if use_ws else None
     un = _Mlp(fp8, tokens, hidden, ffn, ws_u)

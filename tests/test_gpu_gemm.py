@@ -180,8 +180,9 @@ def test_gemm_repeatable(fp8):
 # the stream-K schedule: every pair takes an equal share of the (tile,
 # k-block) work and tiles split between two pairs are combined through the
 # workspace.  (4096, 2048, 256): 128 tiles of 256x256; (4608, 2304, 4096):
-# 81 tiles of 512x256; both have more tiles than the 74 pairs of a B200 and
-# are not whole waves.
+# 162 tiles of 256x256 (its 81 tiles of 512x256 would fill the last wave
+# worse); (7168, 2048, 2048): 112 tiles of 512x256.  All have more tiles than
+# the 74 pairs of a B200 and are not whole waves.
 
 @pytest.fixture(scope="module")
 def ws(fp8):
@@ -192,7 +193,7 @@ def _flags_clear(ws):
     return int(ws[:4096].view(torch.int32).abs().sum().item()) == 0
 
 
-@pytest.mark.parametrize("shape", [(4096, 2048, 256), (4608, 2304, 4096)])
+@pytest.mark.parametrize("shape", [(4096, 2048, 256), (4608, 2304, 4096), (7168, 2048, 2048)])
 @pytest.mark.parametrize("fa,fb", [("e4m3", "e4m3"), ("e5m2", "e4m3")])
 def test_gemm_stream_k_integer_exact(fp8, ws, shape, fa, fb):
     """Integer operands: every partial sum, and the sum of two partials, is
