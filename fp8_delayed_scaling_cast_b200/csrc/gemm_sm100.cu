@@ -520,7 +520,15 @@ __device__ __forceinline__ void partial_io(int mode, uint32_t (&r)[32], float *s
 // of chunk c + 1 is issued as soon as chunk c has been converted, into the
 // same registers, so its latency overlaps chunk c's staging and store; the
 // loop is fully unrolled so that every load has its own registers.
-template <bool OUT_BF16>
+// Four bias values from the tile's shared-memory copy.  BIAS false: the bias
+// is absent and its (zero) copy is not read; the arithmetic is the same fma
+// with +0.
+template <bool BIAS>
+__device__ __forceinline__ float4 bias4(const float *bs) {
+    return BIAS ? *reinterpret_cast<const float4 *>(bs) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+}
+
+template <bool OUT_BF16, bool BIAS>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *box, int half,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                               float sab, const float *bias_s, uint32_t empty_bar_cluster,
@@ -557,11 +565,14 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             if (OUT_BF16) {
                 uint32_t packed[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float v0 = fmaf(__uint_as_float(r[2 * j]), sab, bs[2 * j]);
-                    const float v1 = fmaf(__uint_as_float(r[2 * j + 1]), sab, bs[2 * j + 1]);
-                    __nv_bfloat162 hv = __floats2bfloat162_rn(v0, v1);
-                    packed[j] = *reinterpret_cast<uint32_t *>(&hv);
+                for (int j = 0; j < 8; ++j) {
+                    const float4 b = bias4<BIAS>(bs + 4 * j);
+                    __nv_bfloat162 ha = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j]), sab, b.x),
+                                                              fmaf(__uint_as_float(r[4 * j + 1]), sab, b.y));
+                    __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j + 2]), sab, b.z),
+                                                              fmaf(__uint_as_float(r[4 * j + 3]), sab, b.w));
+                    packed[2 * j] = *reinterpret_cast<uint32_t *>(&ha);
+                    packed[2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
                 }
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -573,11 +584,12 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     const int pc = k ^ (lane & 7);
+                    const float4 b = bias4<BIAS>(bs + 4 * k);
                     *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
-                        make_uint4(__float_as_uint(fmaf(__uint_as_float(r[4 * k]), sab, bs[4 * k])),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 1]), sab, bs[4 * k + 1])),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 2]), sab, bs[4 * k + 2])),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 3]), sab, bs[4 * k + 3])));
+                        make_uint4(__float_as_uint(fmaf(__uint_as_float(r[4 * k]), sab, b.x)),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 1]), sab, b.y)),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 2]), sab, b.z)),
+                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 3]), sab, b.w)));
                 }
             }
         }
@@ -649,6 +661,7 @@ __device__ __forceinline__ void store_segment(uint8_t *dst, int64_t left, const 
     }
 }
 
+template <bool BIAS>
 __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint8_t *box, int half, uint8_t *d8,
                                                   uint8_t *d8t, const CUtensorMap *tmap_d, int64_t n_base,
                                                   int32_t m_row0, float sab,
@@ -684,7 +697,7 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
             const float *bs = bias_s + col0;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float4 b = *reinterpret_cast<const float4 *>(bs + 4 * j);
+                const float4 b = bias4<BIAS>(bs + 4 * j);
                 const uint64_t v01 = fma_f32x2(pack_f32x2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])),
                                                sab2, pack_f32x2(b.x, b.y));
                 const uint64_t v23 = fma_f32x2(
@@ -845,13 +858,24 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>((acc + h) * ACC_N);
             const int32_t m_row0 = (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32;
-            if constexpr (OUT == OUT_FP8)
-                epilogue_tile_fp8(t_row, lane, box, half, p.out_d8, p.out_d8t, tmap_d,
-                                  static_cast<int64_t>(n_blk) * ACC_N, m_row0, sab, bias_s, empty_addr, release,
-                                  mode, slot, h, q, s_out, p.out_fmt, p.M, p.N, amax);
-            else
-                epilogue_tile<OUT == OUT_BF16>(t_row, lane, box, half, tmap_d, static_cast<int64_t>(n_blk) * ACC_N,
-                                               m_row0, sab, bias_s, empty_addr, release, mode, slot, h, q);
+            const int64_t n_base = static_cast<int64_t>(n_blk) * ACC_N;
+            if constexpr (OUT == OUT_FP8) {
+                if (p.bias_kind != 0)
+                    epilogue_tile_fp8<true>(t_row, lane, box, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
+                                            bias_s, empty_addr, release, mode, slot, h, q, s_out, p.out_fmt, p.M, p.N,
+                                            amax);
+                else
+                    epilogue_tile_fp8<false>(t_row, lane, box, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
+                                             bias_s, empty_addr, release, mode, slot, h, q, s_out, p.out_fmt, p.M, p.N,
+                                             amax);
+            } else {
+                if (p.bias_kind != 0)
+                    epilogue_tile<OUT == OUT_BF16, true>(t_row, lane, box, half, tmap_d, n_base, m_row0, sab, bias_s,
+                                                         empty_addr, release, mode, slot, h, q);
+                else
+                    epilogue_tile<OUT == OUT_BF16, false>(t_row, lane, box, half, tmap_d, n_base, m_row0, sab, bias_s,
+                                                          empty_addr, release, mode, slot, h, q);
+            }
         }
         if (mode == 1) {
             // Publish: every epilogue thread's partial stores precede the flag.
@@ -1191,8 +1215,9 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                             operand_desc(smem_u32(sm.a + stage * A_STAGE + S2_BM * BK), p.a_mn, 0);
 #pragma unroll
                         for (int k = 0; k < BK / UMMA_K; ++k)
-                            umma_f8f6f4_pair(tmem_base + static_cast<uint32_t>(ACC_N), a_desc + operand_kstep(k, p.a_mn),
-                                             b_desc + operand_kstep(k, p.b_mn), p.idesc, (j > 0 || k > 0) ? 1u : 0u);
+                            umma_f8f6f4_pair(tmem_base + static_cast<uint32_t>(ACC_N),
+                                             a_desc + operand_kstep(k, p.a_mn), b_desc + operand_kstep(k, p.b_mn),
+                                             p.idesc, (j > 0 || k > 0) ? 1u : 0u);
                         umma_commit_pair_to(&sm.empty[stage], 0x3);
                         if (++stage == STAGES) {
                             stage = 0;
