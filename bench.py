@@ -400,9 +400,47 @@ def max_over_ranks(v, world, device):
 
 # ---------------------------------------------------------- measurements --
 
+def graph_time_us(run, reps):
+    """Mean device time per call of run(i), i = 0 .. reps-1, with the calls
+    captured once in a CUDA graph and the graph replayed between two CUDA
+    events on the launching stream.  Short kernels issued one by one from
+    Python wait on the host (about 10-17 us per call on these boxes); in the
+    graph they run back to back as they would behind a long kernel."""
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(reps):
+            run(i)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del graph
+    return 1e3 * e0.elapsed_time(e1) / reps
+
+
+def host_issue_time_us(run, reps):
+    """The same calls issued one by one from Python, CUDA events around the
+    loop: the host's per-call cost when it exceeds the kernel's."""
+    for i in range(3):
+        run(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(reps):
+        run(i)
+    e1.record()
+    torch.cuda.synchronize()
+    return 1e3 * e0.elapsed_time(e1) / reps
+
+
 def time_cast_workload(fp8, device, reps=100):
     """bf16 [8192, 2048] (0.1% spikes) -> e4m3 and e5m2 with transpose and amax,
-    over 8 rotating input buffers (268 MB > L2); per-launch CUDA-event times."""
+    over 8 rotating input buffers (268 MB > L2); per-launch device times of
+    graph-replayed launches, plus the host-issued loop for context."""
     base = inputs.spiky_bf16().to(device)
     xs = [base] + [base.roll(i * 17, dims=1).contiguous() for i in range(1, 8)]
     y = torch.empty(C2_ROWS, C2_COLS, dtype=torch.uint8, device=device)
@@ -412,51 +450,35 @@ def time_cast_workload(fp8, device, reps=100):
     si = torch.zeros(1, device=device)
     res = {}
     for fmt in ("e4m3", "e5m2"):
+        def cast(i, fmt=fmt):
+            fp8.fp8_cast_transpose_amax(xs[i % 8], fmt, s, y, yt, am, si)
         for i in range(5):
-            fp8.fp8_cast_transpose_amax(xs[i % 8], fmt, s, y, yt, am, si)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record()
-        for i in range(reps):
-            fp8.fp8_cast_transpose_amax(xs[i % 8], fmt, s, y, yt, am, si)
-        e1.record()
-        torch.cuda.synchronize()
-        res[fmt] = {"us_mean": 1e3 * e0.elapsed_time(e1) / reps}
+            cast(i)
+        res[fmt] = {"us_mean": graph_time_us(cast, reps), "us_host_issued": host_issue_time_us(cast, reps)}
     # dynamic scaling of the same tensors (amax pass, scale, cast: the input
     # is read twice) for comparison with the delayed cast above
     sd = torch.ones(1, device=device)
+
+    def dyn(i):
+        fp8.fp8_cast_transpose_amax_dynamic(xs[i % 8], "e4m3", sd, y, yt, am, si)
     for i in range(5):
-        fp8.fp8_cast_transpose_amax_dynamic(xs[i % 8], "e4m3", sd, y, yt, am, si)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    e0.record()
-    for i in range(reps):
-        fp8.fp8_cast_transpose_amax_dynamic(xs[i % 8], "e4m3", sd, y, yt, am, si)
-    e1.record()
-    torch.cuda.synchronize()
-    res["dynamic_e4m3"] = {"us_mean": 1e3 * e0.elapsed_time(e1) / reps}
+        dyn(i)
+    res["dynamic_e4m3"] = {"us_mean": graph_time_us(dyn, reps)}
     return res
 
 
 def time_update_576(fp8, device, reps=200):
     """One fp8_update_scales launch over the 576 metas of the 32-block model
     (32 blocks x 6 linears x input/weight/grad), history 16, launched back to
-    back (the history starts filled with amaxes; every launch reads and
-    rewrites all 16 slots of every meta).  Mean per launch."""
+    back from a CUDA graph (the history starts filled with amaxes; every
+    launch reads and rewrites all 16 slots of every meta).  Mean per launch."""
     T = 32 * 6 * 3
     meta = fp8.Fp8Meta(["e4m3", "e4m3", "e5m2"] * (T // 3), hist_len=16, device=device)
     g = torch.Generator(device="cpu").manual_seed(11)
     meta.amax_history.copy_(torch.rand(16, T, generator=g).to(device) * 10)
     for _ in range(10):
         meta.update()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(reps):
-        meta.update()
-    e1.record()
-    torch.cuda.synchronize()
-    return 1e3 * e0.elapsed_time(e1) / reps
+    return graph_time_us(lambda i: meta.update(), reps)
 
 
 def time_headline_gemm(fp8, device, reps=50, warmup=10):
@@ -856,18 +878,12 @@ def main():
     gemm_b2b_ms = g0.elapsed_time(g1) / (STEP_GEMMS * args.steps)
 
     # the step's four casts back to back, K rounds over the rotating inputs
-    # (234 MB read per round, more than L2): the cast kernels' own rate in
-    # the step's shapes, free of the per-launch event brackets' host gaps
+    # (234 MB read per round, more than L2), replayed from a CUDA graph: the
+    # cast kernels' own rate in the step's shapes, free of host issue gaps
     for i in range(2):
         step.run_casts(i)
-    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier_sync(world)
-    c0.record()
-    for i in range(args.steps):
-        step.run_casts(i)
-    c1.record()
-    barrier_sync(world)
-    cast_b2b_ms = max_over_ranks(c0.elapsed_time(c1) / args.steps, world, device)
+    cast_b2b_ms = max_over_ranks(graph_time_us(step.run_casts, args.steps) * 1e-3, world, device)
 
     per = log.summary()
     gemm_ms = [t for _, t in per["gemm"]]
@@ -969,7 +985,10 @@ def main():
             "in_step_gbs": cast_gbs_step, "in_step_frac": cast_gbs_step / pk["hbm"],
             "in_step_us": 1e3 * cast_b2b_ms, "in_step_bytes": STEP_CAST_BYTES_FUSED,
             "in_step_note": "the step's 4 casts (X, W1, W2 fp32; dY bf16; y only) back to back, K rounds, "
-                            "CUDA events around the loop",
+                            "replayed from a CUDA graph, CUDA events around the replay",
+            "us_host_issued": {"e4m3": c2["e4m3"]["us_host_issued"], "e5m2": c2["e5m2"]["us_host_issued"]},
+            "timing": "100 launches over the 8 inputs captured in a CUDA graph, replayed between CUDA events; "
+                      "us_host_issued: the same launches issued one by one from Python",
             "in_step_event_bracketed_gbs": cast_gbs_bracketed,
             "dynamic_scaling_e4m3_us": c2["dynamic_e4m3"]["us_mean"],
             "dynamic_note": "amax pass + scale + cast (input read twice) vs the delayed cast's one read",
