@@ -634,10 +634,14 @@ def committed_gemm_traffic(root):
     return float(fields["traffic_bytes_per_launch"]), "ncu capture of the step's 6 GEMM launches (%s)" % TRAFFIC_PROFILE
 
 
-def time_graph_step(step, steps):
+def time_graph_step(step, steps, device):
     """The fused step captured once in a CUDA graph and replayed `steps` times
     (no host work per step beyond the replay call).  The graph reads the
-    first input set; returns device ms per step and host us per replay."""
+    first input set.  Blocks of graph replays alternate with blocks of the
+    same step issued eagerly on the same input set, so that both see the
+    same clock (the power cap lowers it as the run goes on); the SM clock is
+    sampled over the section.  Returns device ms per step for both, and the
+    host us per replay."""
     saved = step.xs, step.dys
     step.xs, step.dys = saved[0][:1], saved[1][:1]
     torch.cuda.synchronize()
@@ -647,20 +651,39 @@ def time_graph_step(step, steps):
     for _ in range(3):
         graph.replay()
     torch.cuda.synchronize()
-    s = torch.cuda.Event(enable_timing=True)
-    e = torch.cuda.Event(enable_timing=True)
-    h0 = time.perf_counter()
-    s.record()
-    for _ in range(steps):
-        graph.replay()
-    e.record()
-    host_s = time.perf_counter() - h0
-    torch.cuda.synchronize()
-    ms = s.elapsed_time(e) / steps
+    clocks = ClockSampler(device)
+    clocks.start()
+    time.sleep(0.1)
+    clocks.mark_start()
+    graph_ms, eager_ms, host_s = [], [], 0.0
+    for _ in range(2):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(steps):
+            step.run_linear_api(0)
+        e.record()
+        torch.cuda.synchronize()
+        eager_ms.append(s.elapsed_time(e) / steps)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        h0 = time.perf_counter()
+        s.record()
+        for _ in range(steps):
+            graph.replay()
+        e.record()
+        host_s += time.perf_counter() - h0
+        torch.cuda.synchronize()
+        graph_ms.append(s.elapsed_time(e) / steps)
+    clocks.mark_end()
+    clock_info = clocks.stop()
     step.xs, step.dys = saved
     del graph
+    ms = statistics.mean(graph_ms)
     return {"ms_per_step": ms, "value": STEP_FLOP / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-            "host_us_per_step": 1e6 * host_s / steps}
+            "host_us_per_step": 1e6 * host_s / (2 * steps),
+            "eager_same_section_ms_per_step": statistics.mean(eager_ms),
+            "blocks_ms": {"eager": eager_ms, "graph": graph_ms}, "clocks": clock_info}
 
 
 def single_kernel(args):
@@ -844,7 +867,7 @@ def main():
 
     # the fused step replayed from a CUDA graph (one GPU: the amax sync of
     # several ranks is not captured)
-    graph_info = time_graph_step(step, args.steps) if world == 1 else None
+    graph_info = time_graph_step(step, args.steps, device) if world == 1 else None
 
     # per-kernel durations: the same launches, one C call per kernel, each
     # bracketed by CUDA events on the launching stream (K more steps)

@@ -29,6 +29,7 @@
 // +-max, and turns every NaN (either sign, any payload) into 0x7F; the GPU
 // tests pin that behaviour for every bf16 pattern and every fp32 pattern in
 // the formats' range.
+#include <atomic>
 #include <cuda_bf16.h>
 
 #include "fp8ds_internal.h"
@@ -548,20 +549,22 @@ cudaError_t ct_launch_tma(const void *x, int64_t rows, int64_t cols, const float
                         R::BOX_COLS, CT_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
         return ct_launch_elem<T, FMT, WRITE_T>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
     auto kernel = cast_transpose_tma_kernel<T, FMT, WRITE_T>;
-    static bool configured[64] = {};
-    static int per_sm[64] = {};
+    // per device: CTAs per SM once the kernel's shared-memory limit is set
+    // (0 = not yet; concurrent first calls may both set it, to the same value)
+    static std::atomic<int> per_sm[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
-    if (!configured[dev]) {
+    int n_sm = per_sm[dev].load(std::memory_order_relaxed);
+    if (n_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, R::SMEM);
         if (e != cudaSuccess) return e;
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, CT_THREADS, R::SMEM) != cudaSuccess || n < 1) n = 1;
-        per_sm[dev] = n;
-        configured[dev] = true;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n_sm, kernel, CT_THREADS, R::SMEM) != cudaSuccess ||
+            n_sm < 1)
+            n_sm = 1;
+        per_sm[dev].store(n_sm, std::memory_order_relaxed);
     }
-    const int64_t cap = static_cast<int64_t>(num_sms()) * per_sm[dev];
+    const int64_t cap = static_cast<int64_t>(num_sms()) * n_sm;
     const int grid = static_cast<int>(num_tiles < cap ? (num_tiles > 0 ? num_tiles : 1) : cap);
     return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), R::SMEM, stream, 1, tm, static_cast<int32_t>(rows),
                       static_cast<int32_t>(cols), scale, y, yt, amax, scale_inv, static_cast<int32_t>(tiles_c),

@@ -1296,23 +1296,26 @@ uint32_t make_idesc(fp8ds_format fa, fp8ds_format fb, int m, int n, bool a_mn, b
     return d;
 }
 
+// Per-device flags and counts below are computed once; concurrent first
+// calls may both compute them and store the same value.
 template <typename K>
-cudaError_t set_smem_once(K kernel, int bytes, bool (&done)[64]) {
+cudaError_t set_smem_once(K kernel, int bytes, std::atomic<bool> (&done)[64]) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev].store(true, std::memory_order_relaxed);
     return e;
 }
 
 // Number of CTA pairs of a 2-SM kernel that fit on the device at once.
 template <typename K>
-int max_pairs(K kernel, int smem_bytes, int (&cached)[64]) {
+int max_pairs(K kernel, int smem_bytes, std::atomic<int> (&cached)[64]) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms() / 2;
-    if (cached[dev] == 0) {
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
         cfg.blockDim = dim3(THREADS, 1, 1);
@@ -1324,18 +1327,17 @@ int max_pairs(K kernel, int smem_bytes, int (&cached)[64]) {
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) n = num_sms() / 2;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 template <int OUT, int M_SUB>
 cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
                        cudaStream_t stream) {
-    static bool done[64] = {};
-    static int cached_pairs[64] = {};
+    static std::atomic<bool> done[64];
+    static std::atomic<int> cached_pairs[64];
     auto kernel = fp8_gemm_2sm_kernel<OUT, M_SUB>;
     constexpr int smem = Pair<M_SUB>::SMEM;
     cudaError_t e = set_smem_once(kernel, smem, done);
@@ -1349,7 +1351,7 @@ cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
 template <int OUT>
 cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
                        cudaStream_t stream) {
-    static bool done[64] = {};
+    static std::atomic<bool> done[64];
     auto kernel = fp8_gemm_1sm_kernel<OUT>;
     cudaError_t e = set_smem_once(kernel, S1_SMEM, done);
     if (e != cudaSuccess) return e;
@@ -1361,7 +1363,7 @@ cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
 }  // namespace
 
 size_t gemm_workspace_bytes() {
-    static int cached[64] = {};
+    static std::atomic<int> cached[64];
     const int pairs = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached);
     return WS_FLAG_BYTES + static_cast<size_t>(pairs) * 2 * WS_SLOT_FLOATS * sizeof(float);
 }
@@ -1380,7 +1382,7 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     // 3.46 waves of 74 pairs against 512 = 6.92 waves).
     int m_sub = 1;
     if (pair && m > 2 * S2_BM && k >= FP8DS_MSUB2_MIN_K) {
-        static int cached_pairs[64] = {};
+        static std::atomic<int> cached_pairs[64];
         const int64_t cap = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached_pairs);
         const int64_t tn = (n + ACC_N - 1) / ACC_N;
         const int64_t t1 = ((m + 2 * S2_BM - 1) / (2 * S2_BM)) * tn, t2 = ((m + 4 * S2_BM - 1) / (4 * S2_BM)) * tn;
@@ -1437,7 +1439,7 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     if (pair && workspace != nullptr && workspace_bytes >= gemm_workspace_bytes()) {
         // Stream-K when whole tiles would leave a ragged last wave: at least
         // one tile per pair, fewer than 8 waves, not a whole number of waves.
-        static int cached[64] = {};
+        static std::atomic<int> cached[64];
         const int cap = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached);
         const int tiles = p.tiles_m * p.tiles_n;
         if (tiles >= cap && tiles % cap != 0 && tiles < 8 * cap && cap <= static_cast<int>(WS_FLAG_BYTES / 8)) {
