@@ -230,11 +230,12 @@ fp8ds_status fp8_gemm_workspace_size(size_t *bytes);
  * between two pairs is combined through the workspace: one pair stores its
  * fp32 partial accumulator there and publishes it, the other adds it before
  * the epilogue.  The result satisfies the same bounds as fp8_gemm (the two
- * partials are added in fp32).  On B200 under the 1 kW power cap the
- * whole-tile schedule of fp8_gemm measured faster for 8192 x 2048 x 8192
- * class shapes (idle SMs in the last wave let the busy ones clock higher);
- * the stream-K schedule is for cases where a profile shows the ragged last
- * wave dominating.
+ * partials are added in fp32).  On B200 the whole-tile schedule of fp8_gemm
+ * measured faster on the MLP shapes (8192 x 2048 x 8192: 95-97 against
+ * 114-117 us): the partial's store and reload cost about 15 us, one
+ * dependent load per 32 columns, and every extra tile segment adds an
+ * epilogue that the 512-row tile cannot overlap.  The stream-K schedule is
+ * for cases where a profile shows the ragged last wave dominating.
  *   workspace  16-byte aligned device memory of at least
  *              fp8_gemm_workspace_size() bytes, ZERO-FILLED before its first
  *              use; the library leaves its publication words at zero after
