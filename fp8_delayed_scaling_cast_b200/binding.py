@@ -71,6 +71,8 @@ _SIGS = {
     "fp8_quantize": [_P, _INT, _I64, _INT, _P, _P, _P, _P, _P],
     "fp8_cast_transpose_amax": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
     "fp8_cast_transpose_amax_noop": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P, _P],
+    "fp8_cast_transpose_amax_pair": [_P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P,
+                                     _INT, _INT, _P],
     "fp8_cast_transpose_amax_dynamic": [_P, _INT, _I64, _I64, _INT, _P, _P, _P, _P, _P, _P],
     "fp8_transpose": [_P, _I64, _I64, _P, _P],
     "fp8_update_scales": [_I64, _I32, _P, _P, _P, _P, _INT, _P],
@@ -168,6 +170,20 @@ def fp8_cast_transpose_amax_noop(x, fmt, scale, y, yt, amax, scale_inv, noop_fla
     _check(_lib.fp8_cast_transpose_amax_noop(_ptr(x), _dtype(x), rows, cols, _fmt(fmt), _ptr(scale), _ptr(y),
                                              _ptr(yt), _ptr(amax), _ptr(scale_inv), _ptr(noop_flag),
                                              _stream(stream)))
+
+
+def fp8_cast_transpose_amax_pair(xa, xb, fmt, scale_a, ya, scale_b, yb, yt_a=None, amax_a=None, scale_inv_a=None,
+                                 yt_b=None, amax_b=None, scale_inv_b=None, noop_b=None, stream=None):
+    """Two casts of one dtype and format (b optionally skipped by a device
+    flag), one launch where both suit it."""
+    if xa.dtype != xb.dtype:
+        raise TypeError("fp8_cast_transpose_amax_pair: both inputs must have one dtype")
+    ra, ca = xa.shape
+    rb, cb = xb.shape
+    _check(_lib.fp8_cast_transpose_amax_pair(_ptr(xa), ra, ca, _ptr(scale_a), _ptr(ya), _ptr(yt_a), _ptr(amax_a),
+                                             _ptr(scale_inv_a), _ptr(xb), rb, cb, _ptr(scale_b), _ptr(yb),
+                                             _ptr(yt_b), _ptr(amax_b), _ptr(scale_inv_b), _ptr(noop_b),
+                                             _dtype(xa), _fmt(fmt), _stream(stream)))
 
 
 def fp8_cast_transpose_amax_dynamic(x, fmt, scale, y, yt=None, amax=None, scale_inv=None, stream=None):

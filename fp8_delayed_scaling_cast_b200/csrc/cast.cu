@@ -321,15 +321,26 @@ struct RingLoad8<float, FMT> {
     }
 };
 
+// One tensor of a cast launch.  A launch casts one or two tensors of the same
+// input type and format (the linear forward's input and weight in one
+// launch); their tiles are numbered job 0 first, then job 1.  A job whose
+// noop flag holds non-zero at run time is skipped whole: no load, store,
+// amax or scale_inv of it happens.
+struct CastJob {
+    const float *scale;
+    uint8_t *y, *yt;
+    float *amax, *scale_inv;
+    const int32_t *noop;
+    int32_t rows, cols, tiles_c, num_tiles;
+};
+
 // Vectorised-path requirements (checked on the host): x 16-byte aligned
 // (TMA), cols % 8 == 0, rows % 16 == 0, y and yt 16-byte aligned.  Tiles
 // that reach past the tensor read zeros (TMA fill) and store element-wise.
 template <typename T, int FMT, bool WRITE_T>
 __global__ void __launch_bounds__(CT_THREADS, 3)
-cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t rows, int32_t cols,
-                          const float *__restrict__ scale_ptr, uint8_t *__restrict__ y, uint8_t *__restrict__ yt,
-                          float *__restrict__ amax, float *__restrict__ scale_inv, int32_t tiles_c,
-                          int32_t num_tiles, const int32_t *__restrict__ noop) {
+cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap0, const __grid_constant__ CUtensorMap tmap1,
+                          const CastJob job0, const CastJob job1) {
     using R = TmaRing<T>;
     constexpr int STAGES = R::STAGES;
     extern __shared__ uint8_t dsm[];
@@ -340,30 +351,46 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
     __shared__ uint32_t tsm[2][CT_COLS * CT_TSTRIDE];
     const int tid = threadIdx.x;
     const int cc = tid & 7, rg = tid >> 3;
-    float m = 0.0f;
+    float m0 = 0.0f, m1 = 0.0f;
 
     if (tid == 0) {
         for (int i = 0; i < STAGES; ++i) ptx::mbar_init(&full[i], 1);
         ptx::fence_barrier_init();
         ptx::fence_async_smem();
-        ptx::prefetch_tmap(&tmap_x);
+        ptx::prefetch_tmap(&tmap0);
+        if (job1.num_tiles > 0) ptx::prefetch_tmap(&tmap1);
     }
     ptx::pdl_wait();
     ptx::pdl_launch_dependents();
-    // device-side skip (whole grid), before any load is issued
-    if (noop != nullptr && __ldg(noop) != 0) return;
-    const float s = __ldg(scale_ptr);
-    if (tid == 0 && blockIdx.x == 0 && scale_inv != nullptr) *scale_inv = __frcp_rn(s);
+    // device-side skips (whole jobs), before any load is issued
+    const int32_t n0 = (job0.noop != nullptr && __ldg(job0.noop) != 0) ? 0 : job0.num_tiles;
+    const int32_t n1 = (job1.noop != nullptr && __ldg(job1.noop) != 0) ? 0 : job1.num_tiles;
+    const int32_t num_tiles = n0 + n1;
+    if (num_tiles == 0) return;
+    const float s0 = n0 > 0 ? __ldg(job0.scale) : 0.0f;
+    const float s1 = n1 > 0 ? __ldg(job1.scale) : 0.0f;
+    if (tid == 0 && blockIdx.x == 0) {
+        if (n0 > 0 && job0.scale_inv != nullptr) *job0.scale_inv = __frcp_rn(s0);
+        if (n1 > 0 && job1.scale_inv != nullptr) *job1.scale_inv = __frcp_rn(s1);
+    }
     __syncthreads();
+    // Tile t of the launch: job (t >= n0) and its tile index within the job.
+    auto which = [&](int t, int &j, int &lt) {
+        j = t >= n0 ? 1 : 0;
+        lt = j ? t - n0 : t;
+    };
     // Thread 0 keeps up to STAGES tiles of this CTA in flight.
     int issued = 0;
     auto issue = [&](int tile, int stage) {
-        const int32_t r0 = (tile / tiles_c) * CT_ROWS;
-        const int32_t c0 = (tile % tiles_c) * CT_COLS;
+        int j, lt;
+        which(tile, j, lt);
+        const CastJob &J = j ? job1 : job0;
+        const int32_t r0 = (lt / J.tiles_c) * CT_ROWS;
+        const int32_t c0 = (lt % J.tiles_c) * CT_COLS;
         ptx::mbar_arrive_expect_tx(&full[stage], R::STAGE_BYTES);
 #pragma unroll
         for (int b = 0; b < R::BOXES; ++b)
-            ptx::tma_load_2d(&tmap_x, &full[stage], ring + stage * R::STAGE_BYTES + b * R::BOX_BYTES,
+            ptx::tma_load_2d(j ? &tmap1 : &tmap0, &full[stage], ring + stage * R::STAGE_BYTES + b * R::BOX_BYTES,
                              c0 + b * R::BOX_COLS, r0);
         ++issued;
     };
@@ -376,8 +403,12 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
 
     // yt stores of a tile whose transposed words are in tsm[buf].
     auto store_yt = [&](int tile, int buf) {
-        const int32_t r0 = (tile / tiles_c) * CT_ROWS;
-        const int32_t c0 = (tile % tiles_c) * CT_COLS;
+        int j, lt;
+        which(tile, j, lt);
+        const CastJob &J = j ? job1 : job0;
+        const int32_t rows = J.rows, cols = J.cols;
+        const int32_t r0 = (lt / J.tiles_c) * CT_ROWS;
+        const int32_t c0 = (lt % J.tiles_c) * CT_COLS;
         const bool full_tile = (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
@@ -386,7 +417,7 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
             const uint32_t *tp = tsm[buf] + c * CT_TSTRIDE + 4 * q;
             const uint4 v = make_uint4(tp[0], tp[1], tp[2], tp[3]);
             const int32_t gc = c0 + c, gr = r0 + 16 * q;
-            uint8_t *dst = yt + static_cast<int64_t>(gc) * rows + gr;
+            uint8_t *dst = J.yt + static_cast<int64_t>(gc) * rows + gr;
             if (full_tile) {
                 *reinterpret_cast<uint4 *>(dst) = v;
             } else if (gc < cols) {
@@ -418,16 +449,22 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
             const int next = prev + STAGES * gridDim.x;  // the stage tile i-1 used
             if (next < num_tiles) issue(next, (it - 1) % STAGES);
         }
+        int j, lt;
+        which(tile, j, lt);
+        const CastJob &J = j ? job1 : job0;
+        const int32_t rows = J.rows, cols = J.cols;
+        const float s = j ? s1 : s0;
+        float &m = j ? m1 : m0;
         const uint8_t *st = ring + stage * R::STAGE_BYTES;
-        const int32_t r0 = (tile / tiles_c) * CT_ROWS;
-        const int32_t c0 = (tile % tiles_c) * CT_COLS;
+        const int32_t r0 = (lt / J.tiles_c) * CT_ROWS;
+        const int32_t c0 = (lt % J.tiles_c) * CT_COLS;
         const bool full_tile = (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
         uint2 w[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) w[i] = RingLoad8<T, FMT>::cast(st, 4 * rg + i, cc, s, m);
         {
             const int32_t gr0 = r0 + 4 * rg, gc0 = c0 + 8 * cc;
-            uint8_t *yp = y + static_cast<int64_t>(gr0) * cols + gc0;
+            uint8_t *yp = J.y + static_cast<int64_t>(gr0) * cols + gc0;
             if (full_tile) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) *reinterpret_cast<uint2 *>(yp + static_cast<int64_t>(i) * cols) = w[i];
@@ -466,10 +503,14 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap_x, int32_t ro
     // Loads issued but never consumed (only after a timeout) must land before
     // the CTA exits.
     if (tid == 0) {
-        for (int j = it; j < issued; ++j)
-            ptx::mbar_wait_for(&full[j % STAGES], static_cast<uint32_t>((j / STAGES) & 1), ptx::DRAIN_NS);
+        for (int jj = it; jj < issued; ++jj)
+            ptx::mbar_wait_for(&full[jj % STAGES], static_cast<uint32_t>((jj / STAGES) & 1), ptx::DRAIN_NS);
     }
-    block_amax_commit<CT_THREADS>(m, amax);
+    if (n0 > 0) block_amax_commit<CT_THREADS>(m0, job0.amax);
+    if (n1 > 0) {
+        __syncthreads();  // the first commit's reduction buffer is free again
+        block_amax_commit<CT_THREADS>(m1, job1.amax);
+    }
 }
 
 // ---------------------------------------------------------------- quantize --
@@ -536,18 +577,43 @@ cudaError_t ct_launch_elem(const void *x, int64_t rows, int64_t cols, const floa
                       scale, y, yt, amax, scale_inv, tiles_c, num_tiles, noop);
 }
 
-template <typename T, int FMT, bool WRITE_T>
-cudaError_t ct_launch_tma(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
-                          float *amax, float *scale_inv, const int32_t *noop, cudaStream_t stream) {
+// One tensor of a cast as the host sees it.
+struct HostCast {
+    const void *x;
+    int64_t rows, cols;
+    const float *scale;
+    uint8_t *y, *yt;
+    float *amax, *scale_inv;
+    const int32_t *noop;
+};
+
+// The TMA kernel's requirements (the element-wise kernel takes the rest).
+bool tma_eligible(const HostCast &c) {
+    return c.rows > 0 && c.cols > 0 && aligned16(c.x) && aligned16(c.y) && (c.yt == nullptr || aligned16(c.yt)) &&
+           (c.cols % 8 == 0) && (c.rows % 16 == 0) && c.rows < (int64_t(1) << 31) && c.cols < (int64_t(1) << 31);
+}
+
+// Tensor map and job of one tensor; false if the map cannot be encoded.
+template <typename T>
+bool make_job(const HostCast &c, CUtensorMap *tm, CastJob *job) {
     using R = TmaRing<T>;
-    const int64_t tiles_c = (cols + CT_COLS - 1) / CT_COLS;
-    const int64_t tiles_r = (rows + CT_ROWS - 1) / CT_ROWS;
-    const int64_t num_tiles = tiles_c * tiles_r;
-    CUtensorMap tm;
-    if (!encode_tmap_2d(&tm, sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, x,
-                        static_cast<uint64_t>(cols), static_cast<uint64_t>(rows), static_cast<uint64_t>(cols) * sizeof(T),
-                        R::BOX_COLS, CT_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
-        return ct_launch_elem<T, FMT, WRITE_T>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
+    if (!encode_tmap_2d(tm, sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c.x,
+                        static_cast<uint64_t>(c.cols), static_cast<uint64_t>(c.rows),
+                        static_cast<uint64_t>(c.cols) * sizeof(T), R::BOX_COLS, CT_ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+        return false;
+    const int64_t tiles_c = (c.cols + CT_COLS - 1) / CT_COLS;
+    const int64_t num_tiles = tiles_c * ((c.rows + CT_ROWS - 1) / CT_ROWS);
+    *job = CastJob{c.scale, c.y, c.yt, c.amax, c.scale_inv, c.noop, static_cast<int32_t>(c.rows),
+                   static_cast<int32_t>(c.cols), static_cast<int32_t>(tiles_c), static_cast<int32_t>(num_tiles)};
+    return true;
+}
+
+// One launch of the TMA kernel over job 0 and job 1 (job 1 may have no tiles).
+template <typename T, int FMT, bool WRITE_T>
+cudaError_t ct_launch_tma(const CUtensorMap &t0, const CastJob &j0, const CUtensorMap &t1, const CastJob &j1,
+                          cudaStream_t stream) {
+    using R = TmaRing<T>;
+    const int64_t num_tiles = static_cast<int64_t>(j0.num_tiles) + j1.num_tiles;
     auto kernel = cast_transpose_tma_kernel<T, FMT, WRITE_T>;
     // per device: CTAs per SM once the kernel's shared-memory limit is set
     // (0 = not yet; concurrent first calls may both set it, to the same value)
@@ -566,22 +632,37 @@ cudaError_t ct_launch_tma(const void *x, int64_t rows, int64_t cols, const float
     }
     const int64_t cap = static_cast<int64_t>(num_sms()) * n_sm;
     const int grid = static_cast<int>(num_tiles < cap ? (num_tiles > 0 ? num_tiles : 1) : cap);
-    return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), R::SMEM, stream, 1, tm, static_cast<int32_t>(rows),
-                      static_cast<int32_t>(cols), scale, y, yt, amax, scale_inv, static_cast<int32_t>(tiles_c),
-                      static_cast<int32_t>(num_tiles), noop);
+    return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), R::SMEM, stream, 1, t0, t1, j0, j1);
 }
 
 template <typename T, int FMT>
 cudaError_t ct_dispatch(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
                         float *amax, float *scale_inv, const int32_t *noop, cudaStream_t stream) {
-    const bool vec = rows > 0 && cols > 0 && aligned16(x) && aligned16(y) && (yt == nullptr || aligned16(yt)) &&
-                     (cols % 8 == 0) && (rows % 16 == 0) && rows < (int64_t(1) << 31) && cols < (int64_t(1) << 31);
-    if (yt != nullptr) {
-        return vec ? ct_launch_tma<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
-                   : ct_launch_elem<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
+    const HostCast c{x, rows, cols, scale, y, yt, amax, scale_inv, noop};
+    CUtensorMap tm;
+    CastJob job, none;
+    if (tma_eligible(c) && make_job<T>(c, &tm, &job)) {
+        none = job;
+        none.num_tiles = 0;
+        return yt != nullptr ? ct_launch_tma<T, FMT, true>(tm, job, tm, none, stream)
+                             : ct_launch_tma<T, FMT, false>(tm, job, tm, none, stream);
     }
-    return vec ? ct_launch_tma<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
-               : ct_launch_elem<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
+    return yt != nullptr ? ct_launch_elem<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
+                         : ct_launch_elem<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
+}
+
+// Two tensors of one input type and format in one launch, when both suit the
+// TMA kernel and both or neither write a transpose; false (nothing launched)
+// otherwise.
+template <typename T, int FMT>
+bool ct_dispatch_pair(const HostCast &a, const HostCast &b, cudaStream_t stream, cudaError_t *err) {
+    if ((a.yt == nullptr) != (b.yt == nullptr) || !tma_eligible(a) || !tma_eligible(b)) return false;
+    CUtensorMap t0, t1;
+    CastJob j0, j1;
+    if (!make_job<T>(a, &t0, &j0) || !make_job<T>(b, &t1, &j1)) return false;
+    *err = a.yt != nullptr ? ct_launch_tma<T, FMT, true>(t0, j0, t1, j1, stream)
+                           : ct_launch_tma<T, FMT, false>(t0, j0, t1, j1, stream);
+    return true;
 }
 
 template <typename T, int FMT>
@@ -770,6 +851,28 @@ cudaError_t launch_cast_transpose(const void *x, fp8ds_dtype x_dtype, int64_t ro
     return fmt == FP8DS_E4M3
                ? ct_dispatch<uint16_t, FP8DS_E4M3>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
                : ct_dispatch<uint16_t, FP8DS_E5M2>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
+}
+
+cudaError_t launch_cast_transpose_pair(const void *xa, int64_t rows_a, int64_t cols_a, const float *scale_a,
+                                       uint8_t *ya, uint8_t *yta, float *amax_a, float *scale_inv_a, const void *xb,
+                                       int64_t rows_b, int64_t cols_b, const float *scale_b, uint8_t *yb,
+                                       uint8_t *ytb, float *amax_b, float *scale_inv_b, const int32_t *noop_b,
+                                       fp8ds_dtype x_dtype, fp8ds_format fmt, cudaStream_t stream) {
+    const HostCast a{xa, rows_a, cols_a, scale_a, ya, yta, amax_a, scale_inv_a, nullptr};
+    const HostCast b{xb, rows_b, cols_b, scale_b, yb, ytb, amax_b, scale_inv_b, noop_b};
+    cudaError_t e = cudaSuccess;
+    bool one;
+    if (x_dtype == FP8DS_F32)
+        one = fmt == FP8DS_E4M3 ? ct_dispatch_pair<float, FP8DS_E4M3>(a, b, stream, &e)
+                                : ct_dispatch_pair<float, FP8DS_E5M2>(a, b, stream, &e);
+    else
+        one = fmt == FP8DS_E4M3 ? ct_dispatch_pair<uint16_t, FP8DS_E4M3>(a, b, stream, &e)
+                                : ct_dispatch_pair<uint16_t, FP8DS_E5M2>(a, b, stream, &e);
+    if (one) return e;
+    e = launch_cast_transpose(xa, x_dtype, rows_a, cols_a, fmt, scale_a, ya, yta, amax_a, scale_inv_a, stream);
+    if (e != cudaSuccess) return e;
+    return launch_cast_transpose(xb, x_dtype, rows_b, cols_b, fmt, scale_b, yb, ytb, amax_b, scale_inv_b, stream,
+                                 noop_b);
 }
 
 cudaError_t launch_quantize(const void *x, fp8ds_dtype x_dtype, int64_t n, fp8ds_format fmt,

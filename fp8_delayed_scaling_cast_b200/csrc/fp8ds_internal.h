@@ -31,6 +31,16 @@ cudaError_t launch_cast_transpose(const void *x, fp8ds_dtype x_dtype, int64_t ro
                                   float *amax, float *scale_inv, cudaStream_t stream,
                                   const int32_t *noop = nullptr);
 
+// Two casts of one input dtype and format (a: no noop flag; b: noop_b may be
+// NULL), in one launch when both suit the TMA kernel and both or neither
+// write a transpose, else as two launches.  Results as two calls of
+// launch_cast_transpose.
+cudaError_t launch_cast_transpose_pair(const void *xa, int64_t rows_a, int64_t cols_a, const float *scale_a,
+                                       uint8_t *ya, uint8_t *yta, float *amax_a, float *scale_inv_a, const void *xb,
+                                       int64_t rows_b, int64_t cols_b, const float *scale_b, uint8_t *yb,
+                                       uint8_t *ytb, float *amax_b, float *scale_inv_b, const int32_t *noop_b,
+                                       fp8ds_dtype x_dtype, fp8ds_format fmt, cudaStream_t stream);
+
 // Dynamic scaling: amax = max |x| (written, not accumulated), then
 // scale = fp8_max / amax (kept when that is not finite and positive),
 // scale_inv = 1 / scale, then the cast with that scale.

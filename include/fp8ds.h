@@ -131,6 +131,31 @@ fp8ds_status fp8_cast_transpose_amax_noop(const void *x, fp8ds_dtype x_dtype, in
                                           const int32_t *noop_flag, fp8ds_stream stream);
 
 /*
+ * fp8_cast_transpose_amax_pair -- two independent fp8_cast_transpose_amax
+ * calls of one input dtype and one FP8 format, issued as one kernel launch
+ * where possible [TE820 and TE761: per-call launches of small kernels are the
+ * CPU and launch overhead the pages set out to remove; a linear's forward
+ * casts its input and its weight back to back].  Tensor a is cast exactly as
+ * fp8_cast_transpose_amax(x_a, ..., scale_a, y_a, yt_a, amax_a, scale_inv_a),
+ * tensor b exactly as fp8_cast_transpose_amax_noop(x_b, ..., noop_b) (or the
+ * plain call when noop_b is NULL).  One launch when both tensors suit the TMA
+ * path (x and y 16-byte aligned, cols % 8 == 0, rows % 16 == 0) and both or
+ * neither have a transpose output; otherwise two launches, one per tensor.
+ * The results are the same bytes either way (amax is a max, so its order
+ * does not matter).  Tensors a and b must not overlap in memory, except that
+ * they may share scale, amax or scale_inv only if the caller wants their
+ * combined effect (amax is atomically maxed).
+ * Errors: as fp8_cast_transpose_amax, for either tensor.
+ */
+fp8ds_status fp8_cast_transpose_amax_pair(const void *x_a, int64_t rows_a, int64_t cols_a,
+                                          const float *scale_a, uint8_t *y_a, uint8_t *yt_a,
+                                          float *amax_a, float *scale_inv_a, const void *x_b,
+                                          int64_t rows_b, int64_t cols_b, const float *scale_b,
+                                          uint8_t *y_b, uint8_t *yt_b, float *amax_b,
+                                          float *scale_inv_b, const int32_t *noop_b,
+                                          fp8ds_dtype x_dtype, fp8ds_format fmt, fp8ds_stream stream);
+
+/*
  * fp8_cast_transpose_amax_dynamic -- dynamic scaling, for comparison with the
  * delayed recipe [F8E312: delayed vs dynamic scaling; "delayed scaling is
  * theoretically faster than dynamic scaling (less memory reads)" is the

@@ -32,6 +32,7 @@ def test_header_declares_the_boundary():
     for n in ("fp8_quantize", "fp8_cast_transpose_amax", "fp8_update_scales", "fp8_gemm",
               "fp8_gemm_ex", "fp8_gemm_workspace_size", "fp8_gemm_noalloc", "fp8_gemm_cast",
               "fp8_linear_fwd_ex", "fp8_linear_bwd_ex", "fp8_cast_transpose_amax_noop",
+              "fp8_cast_transpose_amax_pair",
               "fp8_cast_transpose_amax_dynamic", "fp8_transpose", "fp8_gemm_major",
               "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
               "fp8ds_version"):
@@ -91,6 +92,19 @@ def test_cast_and_update_argument_checks(lib):
     assert L.fp8_quantize(FAKE, 5, 16, 0, FAKE, FAKE, None, None, s) == lib.ERR_INVALID_ARG
     assert L.fp8_cast_transpose_amax(FAKE, 0, 4, -4, 0, FAKE, FAKE, None, None, None, s) == lib.ERR_INVALID_ARG
     assert L.fp8_cast_transpose_amax(FAKE, 0, 4, 4, 0, None, FAKE, None, None, None, s) == lib.ERR_INVALID_ARG
+    # the pair call checks both tensors before anything is launched
+    pair_ok = [FAKE, 16, 16, FAKE, FAKE, None, None, None, FAKE, 16, 16, FAKE, FAKE, None, None, None, None, 0, 0, s]
+
+    def pair(**kw):
+        a = list(pair_ok)
+        for i, v in kw.items():
+            a[int(i[1:])] = v
+        return L.fp8_cast_transpose_amax_pair(*a)
+    assert pair(a10=-16) == lib.ERR_INVALID_ARG and "(b)" in lib.fp8ds_last_error()
+    assert pair(a3=None) == lib.ERR_INVALID_ARG and "(a)" in lib.fp8ds_last_error()
+    assert pair(a12=None) == lib.ERR_INVALID_ARG and "(b)" in lib.fp8ds_last_error()
+    assert pair(a17=5) == lib.ERR_INVALID_ARG
+    assert pair(a18=4) == lib.ERR_INVALID_ARG
     assert L.fp8_update_scales(-1, 16, FAKE, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG
     assert L.fp8_update_scales(4, 0, FAKE, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG
     assert L.fp8_update_scales(4, 16, None, FAKE, FAKE, FAKE, 0, s) == lib.ERR_INVALID_ARG

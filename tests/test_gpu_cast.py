@@ -69,6 +69,68 @@ def test_cast_transpose_shapes(fp8, shape, dtype, fmt):
     _check_ct(fp8, x, fmt, 3.71875, amax0=0.25)
 
 
+def _gpu_pair(fp8, xa, xb, fmt, sa, sb, transpose, amax0=(0.0, 0.0), noop_b=None):
+    """fp8_cast_transpose_amax_pair on fresh outputs (y, yt filled 0xAA)."""
+    outs = []
+    for x, am0 in ((xa, amax0[0]), (xb, amax0[1])):
+        R, C = x.shape
+        outs.append([torch.full((R, C), 0xAA, dtype=torch.uint8, device="cuda"),
+                     torch.full((C, R), 0xAA, dtype=torch.uint8, device="cuda") if transpose else None,
+                     torch.tensor([am0], dtype=torch.float32, device="cuda"), torch.zeros(1, device="cuda")])
+    (ya, yta, ama, sia), (yb, ytb, amb, sib) = outs
+    fp8.fp8_cast_transpose_amax_pair(xa.cuda(), xb.cuda(), fmt, torch.tensor([sa], device="cuda"), ya,
+                                     torch.tensor([sb], device="cuda"), yb, yt_a=yta, amax_a=ama, scale_inv_a=sia,
+                                     yt_b=ytb, amax_b=amb, scale_inv_b=sib, noop_b=noop_b)
+    torch.cuda.synchronize()
+    assert fp8.fp8ds_device_status() == 0
+    return [[u8(t) if t is not None and t.dtype == torch.uint8 else (None if t is None else t.cpu().numpy())
+             for t in o_] for o_ in outs]
+
+
+def _check_against_oracle(got, x, fmt, scale, amax0, transpose, what):
+    y, yt, am, si = got
+    ry, ryt, ram, rsi = o.cast_transpose_amax(host_bits(x), FMT[fmt], scale, amax0, transpose)
+    assert_bytes_equal(y, ry, what + " y")
+    if transpose:
+        assert_bytes_equal(yt, ryt, what + " yt")
+    assert_f32_bits_equal(am, [ram], what + " amax")
+    assert_f32_bits_equal(si, [rsi], what + " scale_inv")
+
+
+# (shape a, shape b, dtype, format, transpose).  Both TMA-eligible: one launch
+# whose tiles run over a, then b (a linear's input and weight); b with ragged
+# tiles; b not TMA-eligible (cols % 8 != 0): two launches.
+PAIRS = [((256, 512), (1024, 256), torch.float32, "e4m3", False),
+         ((256, 512), (1024, 256), torch.float32, "e4m3", True),
+         ((512, 2048), (144, 136), torch.bfloat16, "e5m2", True),
+         ((128, 64), (128, 64), torch.float32, "e5m2", True),
+         ((256, 512), (100, 36), torch.float32, "e4m3", False)]
+
+
+@pytest.mark.parametrize("sa_shape,sb_shape,dtype,fmt,transpose", PAIRS)
+def test_cast_pair_matches_oracle(fp8, sa_shape, sb_shape, dtype, fmt, transpose):
+    xa = (inputs.normal(sa_shape, inputs.gen(11)) * 40).to(dtype)
+    xb = (inputs.normal(sb_shape, inputs.gen(12)) * 300).to(dtype)
+    ga, gb = _gpu_pair(fp8, xa, xb, fmt, 3.71875, 0.5, transpose, amax0=(0.25, 1e9))
+    _check_against_oracle(ga, xa, fmt, 3.71875, 0.25, transpose, "a")
+    _check_against_oracle(gb, xb, fmt, 0.5, 1e9, transpose, "b")
+
+
+def test_cast_pair_noop_skips_b(fp8):
+    """With b's device flag set nothing of b is written; a is cast as usual."""
+    xa = inputs.normal((256, 512), inputs.gen(13)) * 40
+    xb = inputs.normal((512, 256), inputs.gen(14)) * 40
+    for flag in (1, 0):
+        f = torch.tensor([flag], dtype=torch.int32, device="cuda")
+        ga, gb = _gpu_pair(fp8, xa, xb, "e4m3", 2.0, 4.0, True, amax0=(0.0, 7.5), noop_b=f)
+        _check_against_oracle(ga, xa, "e4m3", 2.0, 0.0, True, "a (flag %d)" % flag)
+        if flag:
+            assert (gb[0] == 0xAA).all() and (gb[1] == 0xAA).all()
+            assert gb[2][0] == np.float32(7.5) and gb[3][0] == 0.0
+        else:
+            _check_against_oracle(gb, xb, "e4m3", 4.0, 7.5, True, "b (flag 0)")
+
+
 @pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
 def test_cast_transpose_no_transpose_and_empty(fp8, fmt):
     x = inputs.normal((64, 96), inputs.gen(3))
