@@ -401,6 +401,9 @@ typedef struct {
  *      scale_inv into *w_scale_inv; sets cache_valid.  With 0 and a valid
  *      cache the cached weight and its frozen scale_inv are reused;
  *   3. y = fp8_gemm(x8, w8, *x_scale_inv, *w_scale_inv, bias).
+ * When x is fp32 and the weight is recast, steps 1 and 2 are one launch
+ * (fp8_cast_transpose_amax_pair) where the shapes allow; the bytes are the
+ * same as with two.
  * With lin->w_noop_flag set, step 2 is decided on the device instead [TE820:
  * a CUDA graph captured around the forward must not bake in the weight-cache
  * decision]: the weight cast is always enqueued and skips itself while
