@@ -23,7 +23,10 @@
 //   - amax is reduced with warp shuffles, then once per CTA, then one atomic
 //     max on the float's bit pattern (non-negative floats order like ints);
 //   - grids are sized to fill every SM with resident CTAs and loop over
-//     tiles (grid-stride), so the atomics are few.
+//     tiles (grid-stride), so the atomics are few;
+//   - one launch may cast two tensors of one dtype and format (a linear's
+//     input and weight): its tiles run over the first, then the second, so
+//     the launch's ramp and last-tile tail are paid once.
 // The cast itself is the hardware conversion cvt.rn.satfinite.{e4m3,e5m2}x2,
 // which rounds to nearest-even, saturates finite overflow and infinities to
 // +-max, and turns every NaN (either sign, any payload) into 0x7F; the GPU
@@ -284,7 +287,7 @@ cast_transpose_kernel(const T *__restrict__ x, int64_t rows, int64_t cols,
 // Shared-memory ring of input tiles (one 128 x 64 tile per stage).
 template <typename T>
 struct TmaRing {
-    static constexpr int STAGES = sizeof(T) == 2 ? 3 : 2;   // bf16: 3 CTAs per SM; fp32: 2
+    static constexpr int STAGES = sizeof(T) == 2 ? 3 : 2;   // stages of 16 KB (bf16) or 32 KB (fp32)
     static constexpr int BOX_COLS = 128 / sizeof(T);             // one 128-byte swizzle row per box row
     static constexpr int BOXES = CT_COLS / BOX_COLS;              // 1 (bf16) or 2 (fp32)
     static constexpr int BOX_BYTES = CT_ROWS * 128;               // 16 KB
