@@ -87,6 +87,19 @@ META_NAMES = ["fc1.in", "fc1.w", "fc1.grad", "fc2.in", "fc2.w", "fc2.grad"]
 META_FMTS = ["e4m3", "e4m3", "e5m2", "e4m3", "e4m3", "e5m2"]
 
 
+def step_config(world):
+    """The workload both arms name in their JSON line."""
+    return {
+        "workload": "MLP pair 2048->8192->2048 fwd+bwd at 8192 tokens (batch 8 x seq 1024), "
+                    "HYBRID delayed scaling, amax history 16, weights recast every step, "
+                    "H and dH handed over in FP8 from the GEMM epilogues, no FP8 transposes "
+                    "(MN-major operand reads)",
+        "tokens": TOKENS, "hidden": HIDDEN, "ffn": FFN, "gemms_per_step": STEP_GEMMS,
+        "parallelism": "dp%d" % world,
+        "l2": "inputs larger than L2: about 1.5 GB touched per step, X/dY rotate over 2 sets",
+    }
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -805,8 +818,7 @@ def main():
             "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "MLP pair 2048->8192->2048 fwd+bwd, HYBRID delayed scaling",
-                       "tokens": args.cpu_tokens},
+            "config": step_config(world),
             "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -981,15 +993,7 @@ def main():
         "vs_baseline": None,
         "dtype": "fp8(e4m3,e5m2)xfp8->f32",
         "data": "synthetic",
-        "config": {
-            "workload": "MLP pair 2048->8192->2048 fwd+bwd at 8192 tokens (batch 8 x seq 1024), "
-                        "HYBRID delayed scaling, amax history 16, weights recast every step, "
-                        "H and dH handed over in FP8 from the GEMM epilogues, no FP8 transposes "
-                        "(MN-major operand reads)",
-            "tokens": TOKENS, "hidden": HIDDEN, "ffn": FFN, "gemms_per_step": STEP_GEMMS,
-            "parallelism": "dp%d" % world,
-            "l2": "inputs larger than L2: about 1.5 GB touched per step, X/dY rotate over 2 sets",
-        },
+        "config": step_config(world),
         "roofline": {
             "kernel": "fp8_gemm_2sm_kernel (tcgen05 CTA pairs; bf16 / fp32 / FP8 out)",
             "bound": "tensor", "achieved": gemm_tflops, "peak": gemm_peak, "unit": "TFLOP/s",
