@@ -207,3 +207,21 @@ def test_gemm_major_argument_checks(lib):
     assert call(bm=1, n=264) == lib.ERR_INVALID_ARG and "MN-major b" in lib.fp8ds_last_error()
     assert call(am=0, bm=1, k=120) == lib.ERR_INVALID_ARG and "K-major" in lib.fp8ds_last_error()
     assert call(am=1, bm=1, k=120, n=12) == lib.ERR_INVALID_ARG   # k is free, but n % 16 is not met
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/fp8ds.h compiles as strict C99 and as C++ on its own (no CUDA
+    or torch headers), so any C caller can use the boundary."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "fp8ds.h"\nint main(void) { return fp8_gemm_workspace_size(0) == FP8DS_OK; }\n')
+    for lang, std in (("c", "-std=c99"), ("c++", "-std=c++17")):
+        r = subprocess.run([cc, "-x", lang, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-I" + inc, "-c",
+                            str(src), "-o", str(tmp_path / ("o_" + lang.replace("+", "p")))],
+                           capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
