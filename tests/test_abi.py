@@ -225,3 +225,37 @@ def test_header_is_plain_c(tmp_path):
                             str(src), "-o", str(tmp_path / ("o_" + lang.replace("+", "p")))],
                            capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+
+
+def test_c_program_links_and_calls_the_library(tmp_path, lib):
+    """A plain C program links libfp8ds.so and gets its version string and
+    an argument-check error (host-only paths: no device is touched)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    inc = os.path.join(ROOT, "include")
+    libdir = os.path.dirname(lib.LIB_PATH)
+    src = tmp_path / "client.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "fp8ds.h"
+int main(void) {
+    float scale = 1.0f;
+    unsigned char y[16];
+    float x[16] = {0};
+    fp8ds_status st = fp8_cast_transpose_amax(x, FP8DS_F32, 4, -4, FP8DS_E4M3, &scale, y, NULL, NULL, NULL, NULL);
+    printf("%s|%d|%s\n", fp8ds_version(), (int)st, fp8ds_last_error());
+    return st == FP8DS_ERR_INVALID_ARG && strlen(fp8ds_last_error()) > 0 ? 0 : 1;
+}
+''')
+    exe = tmp_path / "client"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I" + inc, str(src), "-o", str(exe), "-L" + libdir,
+                        "-l:libfp8ds.so", "-Wl,-rpath," + libdir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stdout + r.stderr
+    version, status, msg = r.stdout.strip().split("|")
+    assert "sm_100a" in version and int(status) == lib.ERR_INVALID_ARG and "negative" in msg
