@@ -67,8 +67,22 @@ constexpr int EPI_WARPS = 8;               // two per TMEM lane quarter
 constexpr int THREADS = 64 + 32 * EPI_WARPS; // producer warp, MMA warp, epilogue warps
 constexpr int EPI_WARP0 = 2;
 constexpr int TMEM_COLS = 512; // two accumulators
+// Epilogue shape (compile-time settings): TMEM columns per tcgen05.ld (32 or
+// 64) and staging boxes per epilogue warp (1, or 2 so that a box is filled
+// while the previous one's TMA store still reads shared memory; the second
+// box takes the shared memory of one ring stage).
+#ifndef FP8DS_EPI_LD
+#define FP8DS_EPI_LD 32
+#endif
+#ifndef FP8DS_EPI_BOXES
+#define FP8DS_EPI_BOXES 1
+#endif
+constexpr int EPI_LD = FP8DS_EPI_LD;
+constexpr int EPI_NBOX = FP8DS_EPI_BOXES;
+static_assert(EPI_LD == 32 || EPI_LD == 64, "TMEM load width must be 32 or 64 columns");
+static_assert(EPI_NBOX == 1 || EPI_NBOX == 2, "one or two staging boxes per epilogue warp");
 constexpr int EPI_BOX_BYTES = 32 * 128;  // staging box: 32 rows x 128 bytes
-constexpr int EPI_BYTES = EPI_WARPS * EPI_BOX_BYTES + 256 * 4;  // + the tile's bias (fp32 x 256)
+constexpr int EPI_BYTES = EPI_WARPS * EPI_NBOX * EPI_BOX_BYTES + 256 * 4;  // + the tile's bias (fp32 x 256)
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr int SMEM_ALIGN = 1024;
 constexpr int GROUP_M = 8;
@@ -88,7 +102,7 @@ constexpr unsigned long long DRAIN_NS = 200000000ull;     // 0.2 s
 
 // 1-SM kernel: tile 128 x 256, 4 stages of 16 KB (A) + 32 KB (B).
 constexpr int S1_BM = 128;
-constexpr int S1_STAGES = 4;
+constexpr int S1_STAGES = 4 - (EPI_NBOX - 1);
 constexpr int S1_A_STAGE = S1_BM * BK;
 constexpr int S1_B_STAGE = ACC_N * BK;
 constexpr int S1_SMEM = SMEM_ALIGN + S1_STAGES * (S1_A_STAGE + S1_B_STAGE) + EPI_BYTES + 256;
@@ -104,7 +118,7 @@ constexpr int S2_BN_HALF = 128;      // rows of B per CTA
 constexpr int S2_B_STAGE = S2_BN_HALF * BK;
 template <int M_SUB>
 struct Pair {
-    static constexpr int STAGES = M_SUB == 1 ? 6 : 4;
+    static constexpr int STAGES = (M_SUB == 1 ? 6 : 4) - (EPI_NBOX - 1);
     static constexpr int A_STAGE = M_SUB * S2_BM * BK;
     static constexpr int ACC_BUFS = M_SUB == 1 ? 2 : 1;
     static constexpr int SMEM = SMEM_ALIGN + STAGES * (A_STAGE + S2_B_STAGE) + EPI_BYTES + 256;
@@ -363,6 +377,28 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+}
+
+// tcgen05.ld of EPI_LD columns (32 lanes x 32 bits each) into r.
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld32(taddr, r); }
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[64]) { tmem_ld64(taddr, r); }
+
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 struct Params {
@@ -495,7 +531,7 @@ __device__ __forceinline__ float4 *partial_at(float *slot, int h, int q, int col
 }
 
 // Store (mode 1) or add (mode 2) the partial accumulator of 32 columns.
-__device__ __forceinline__ void partial_io(int mode, uint32_t (&r)[32], float *slot, int h, int q, int col0,
+__device__ __forceinline__ void partial_io(int mode, uint32_t *r, float *slot, int h, int q, int col0,
                                            int lane) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -529,77 +565,87 @@ __device__ __forceinline__ float4 bias4(const float *bs) {
 }
 
 template <bool OUT_BF16, bool BIAS>
-__device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *box, int half,
+__device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *boxes, int &nbox, int half,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                               float sab, const float *bias_s, uint32_t empty_bar_cluster,
                                               bool arrive, int mode, float *slot, int h, int q) {
-    constexpr int COLS_PER_BOX = OUT_BF16 ? 64 : 32;
-    constexpr int LOADS_PER_BOX = OUT_BF16 ? 2 : 1;
-    constexpr int CHUNKS = ACC_N / 32 / 2;
-    uint32_t r[32];
-    tmem_ld32(t_row + half * CHUNKS * 32, r);
+    constexpr int SUBS_PER_BOX = OUT_BF16 ? 2 : 1;  // 32-column sub-blocks per staging box
+    constexpr int CHUNKS = ACC_N / 2 / EPI_LD;      // TMEM loads per warp and row block
+    constexpr int SUBS = EPI_LD / 32;               // 32-column sub-blocks per load
+    uint32_t r[EPI_LD];
+    tmem_ld(t_row + half * (ACC_N / 2), r);
     tmem_ld_wait();
 #pragma unroll
     for (int c = 0; c < CHUNKS; ++c) {
-        const int col0 = (half * CHUNKS + c) * 32;
-        const int hh = c % LOADS_PER_BOX;
-        const int bx = col0 / COLS_PER_BOX;
         if (arrive && c == CHUNKS - 1) {
             // every TMEM load of this accumulator has completed
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
         }
-        if (mode != 0) partial_io(mode, r, slot, h, q, col0, lane);
-        if (mode != 1) {
-            if (hh == 0) {
-                // Staging buffer reuse: the previous store from it must have
-                // finished reading shared memory.
-                if (lane == 0) tma_store_wait_read<0>();
+#pragma unroll
+        for (int sb = 0; sb < SUBS; ++sb) {
+            uint32_t *rr = r + 32 * sb;
+            const int col0 = half * (ACC_N / 2) + (c * SUBS + sb) * 32;  // accumulator column
+            const int hh = (col0 / 32) % SUBS_PER_BOX;
+            const bool last_of_chunk = sb == SUBS - 1;
+            if (mode != 0) partial_io(mode, rr, slot, h, q, col0, lane);
+            if (mode != 1) {
+                uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
+                if (hh == 0) {
+                    // Staging buffer reuse: the store issued from this box
+                    // EPI_NBOX stores ago must have finished reading it.
+                    if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
+                    __syncwarp();
+                }
+                const float *bs = bias_s + col0;
+                // 32 columns -> 128 bytes (fp32) or 64 bytes (bf16) of row `lane`;
+                // 16-byte chunk k of the row goes to chunk k ^ (lane & 7) (the
+                // 128-byte swizzle the output tensor map expects).
+                if (OUT_BF16) {
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 b = bias4<BIAS>(bs + 4 * j);
+                        __nv_bfloat162 ha = __floats2bfloat162_rn(fmaf(__uint_as_float(rr[4 * j]), sab, b.x),
+                                                                  fmaf(__uint_as_float(rr[4 * j + 1]), sab, b.y));
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(rr[4 * j + 2]), sab, b.z),
+                                                                  fmaf(__uint_as_float(rr[4 * j + 3]), sab, b.w));
+                        packed[2 * j] = *reinterpret_cast<uint32_t *>(&ha);
+                        packed[2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int pc = (hh * 4 + k) ^ (lane & 7);
+                        *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
+                            make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int pc = k ^ (lane & 7);
+                        const float4 b = bias4<BIAS>(bs + 4 * k);
+                        *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
+                            make_uint4(__float_as_uint(fmaf(__uint_as_float(rr[4 * k]), sab, b.x)),
+                                       __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 1]), sab, b.y)),
+                                       __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 2]), sab, b.z)),
+                                       __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 3]), sab, b.w)));
+                    }
+                }
+            }
+            // the registers of r are free: start the next chunk's TMEM load
+            if (last_of_chunk && c + 1 < CHUNKS) tmem_ld(t_row + half * (ACC_N / 2) + (c + 1) * EPI_LD, r);
+            if (mode != 1 && hh == SUBS_PER_BOX - 1) {
+                uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
+                fence_async_smem();
                 __syncwarp();
-            }
-            const float *bs = bias_s + col0;
-            // 32 columns -> 128 bytes (fp32) or 64 bytes (bf16) of row `lane`;
-            // 16-byte chunk k of the row goes to chunk k ^ (lane & 7) (the
-            // 128-byte swizzle the output tensor map expects).
-            if (OUT_BF16) {
-                uint32_t packed[16];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 b = bias4<BIAS>(bs + 4 * j);
-                    __nv_bfloat162 ha = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j]), sab, b.x),
-                                                              fmaf(__uint_as_float(r[4 * j + 1]), sab, b.y));
-                    __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j + 2]), sab, b.z),
-                                                              fmaf(__uint_as_float(r[4 * j + 3]), sab, b.w));
-                    packed[2 * j] = *reinterpret_cast<uint32_t *>(&ha);
-                    packed[2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
+                if (lane == 0) {
+                    tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + (col0 / (32 * SUBS_PER_BOX)) *
+                                                                               (32 * SUBS_PER_BOX)),
+                                 m_row0);
+                    tma_store_commit();
                 }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int pc = (hh * 4 + k) ^ (lane & 7);
-                    *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
-                        make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int pc = k ^ (lane & 7);
-                    const float4 b = bias4<BIAS>(bs + 4 * k);
-                    *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
-                        make_uint4(__float_as_uint(fmaf(__uint_as_float(r[4 * k]), sab, b.x)),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 1]), sab, b.y)),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 2]), sab, b.z)),
-                                   __float_as_uint(fmaf(__uint_as_float(r[4 * k + 3]), sab, b.w)));
-                }
-            }
-        }
-        if (c + 1 < CHUNKS) tmem_ld32(t_row + col0 + 32, r);
-        if (mode != 1 && hh == LOADS_PER_BOX - 1) {
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + bx * COLS_PER_BOX), m_row0);
-                tma_store_commit();
+                ++nbox;
             }
         }
         if (c + 1 < CHUNKS) tmem_ld_wait();
@@ -662,85 +708,94 @@ __device__ __forceinline__ void store_segment(uint8_t *dst, int64_t left, const 
 }
 
 template <bool BIAS>
-__device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint8_t *box, int half, uint8_t *d8,
-                                                  uint8_t *d8t, const CUtensorMap *tmap_d, int64_t n_base,
-                                                  int32_t m_row0, float sab,
+__device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint8_t *boxes, int &nbox, int half,
+                                                  uint8_t *d8, uint8_t *d8t, const CUtensorMap *tmap_d,
+                                                  int64_t n_base, int32_t m_row0, float sab,
                                                   const float *bias_s, uint32_t empty_bar_cluster, bool arrive,
                                                   int mode, float *slot, int h, int q, float s_out, int fmt,
                                                   int32_t m_total, int32_t n_total, float &amax) {
-    constexpr int CHUNKS = ACC_N / 32 / 2;
+    constexpr int CHUNKS = ACC_N / 2 / EPI_LD;  // TMEM loads per warp and row block
+    constexpr int SUBS = EPI_LD / 32;           // 32-column sub-blocks per load
     const int32_t m = m_row0 + lane;
     // Without the transpose the warp's 32 rows x 128 code bytes are one
     // 128-byte-swizzled staging box and one TMA store; with it, the codes go
-    // out with plain stores beside the transposed ones.
+    // out with plain stores beside the transposed ones (in box 0's memory).
     const bool staged = d8t == nullptr;
+    uint8_t *box = staged ? boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES : boxes;
     if (staged && mode != 1) {
-        if (lane == 0) tma_store_wait_read<0>();
+        if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
         __syncwarp();
     }
     const uint64_t sab2 = pack_f32x2(sab, sab);
     const uint64_t s2 = pack_f32x2(s_out, s_out);
-    uint32_t r[32];
-    tmem_ld32(t_row + half * CHUNKS * 32, r);
+    uint32_t r[EPI_LD];
+    tmem_ld(t_row + half * (ACC_N / 2), r);
     tmem_ld_wait();
 #pragma unroll
     for (int c = 0; c < CHUNKS; ++c) {
-        const int col0 = (half * CHUNKS + c) * 32;
         if (arrive && c == CHUNKS - 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(empty_bar_cluster);
         }
-        if (mode != 0) partial_io(mode, r, slot, h, q, col0, lane);
-        uint32_t w[8];
-        if (mode != 1) {
-            const float *bs = bias_s + col0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 b = bias4<BIAS>(bs + 4 * j);
-                const uint64_t v01 = fma_f32x2(pack_f32x2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])),
-                                               sab2, pack_f32x2(b.x, b.y));
-                const uint64_t v23 = fma_f32x2(
-                    pack_f32x2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), sab2,
-                    pack_f32x2(b.z, b.w));
-                const __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
-                const __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
-                const float h0 = __low2float(ha), h1 = __high2float(ha);
-                const float h2 = __low2float(hb), h3 = __high2float(hb);
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
-                const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
-                const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
-                w[j] = cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) | (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
-            }
-        }
-        // the registers of r are free: start the next chunk's TMEM load
-        if (c + 1 < CHUNKS) tmem_ld32(t_row + col0 + 32, r);
-        if (mode != 1 && staged) {
-            // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
-            *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c) ^ (lane & 7)) * 16) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-            *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c + 1) ^ (lane & 7)) * 16) =
-                make_uint4(w[4], w[5], w[6], w[7]);
-        } else if (mode != 1) {
-            const int64_t n0 = n_base + col0;
-            if (m < m_total && n0 < n_total)
-                store_segment(d8 + static_cast<int64_t>(m) * n_total + n0, n_total - n0, w);
-            if (d8t != nullptr) {
-                uint8_t *tile = box + (c & 1) * FP8_TILE_BYTES;
-                *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE + 16) = make_uint4(w[4], w[5], w[6], w[7]);
-                __syncwarp();
-                uint32_t t[8];
+        for (int sb = 0; sb < SUBS; ++sb) {
+            uint32_t *rr = r + 32 * sb;
+            const int cs = c * SUBS + sb;              // sub-block within the warp's 128 columns
+            const int col0 = half * (ACC_N / 2) + cs * 32;
+            if (mode != 0) partial_io(mode, rr, slot, h, q, col0, lane);
+            uint32_t w[8];
+            if (mode != 1) {
+                const float *bs = bias_s + col0;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    t[i] = static_cast<uint32_t>(tile[(4 * i) * FP8_TSTRIDE + lane]) |
-                           (static_cast<uint32_t>(tile[(4 * i + 1) * FP8_TSTRIDE + lane]) << 8) |
-                           (static_cast<uint32_t>(tile[(4 * i + 2) * FP8_TSTRIDE + lane]) << 16) |
-                           (static_cast<uint32_t>(tile[(4 * i + 3) * FP8_TSTRIDE + lane]) << 24);
+                for (int j = 0; j < 8; ++j) {
+                    const float4 b = bias4<BIAS>(bs + 4 * j);
+                    const uint64_t v01 = fma_f32x2(
+                        pack_f32x2(__uint_as_float(rr[4 * j]), __uint_as_float(rr[4 * j + 1])), sab2,
+                        pack_f32x2(b.x, b.y));
+                    const uint64_t v23 = fma_f32x2(
+                        pack_f32x2(__uint_as_float(rr[4 * j + 2]), __uint_as_float(rr[4 * j + 3])), sab2,
+                        pack_f32x2(b.z, b.w));
+                    const __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
+                    const __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
+                    const float h0 = __low2float(ha), h1 = __high2float(ha);
+                    const float h2 = __low2float(hb), h3 = __high2float(hb);
+                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+                    const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
+                    const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
+                    w[j] = cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) |
+                           (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
                 }
-                const int64_t n = n0 + lane;
-                if (n < n_total && m_row0 < m_total)
-                    store_segment(d8t + n * m_total + m_row0, static_cast<int64_t>(m_total) - m_row0, t);
+            }
+            // the registers of r are free: start the next chunk's TMEM load
+            if (sb == SUBS - 1 && c + 1 < CHUNKS) tmem_ld(t_row + half * (ACC_N / 2) + (c + 1) * EPI_LD, r);
+            if (mode != 1 && staged) {
+                // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
+                *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * cs) ^ (lane & 7)) * 16) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * cs + 1) ^ (lane & 7)) * 16) =
+                    make_uint4(w[4], w[5], w[6], w[7]);
+            } else if (mode != 1) {
+                const int64_t n0 = n_base + col0;
+                if (m < m_total && n0 < n_total)
+                    store_segment(d8 + static_cast<int64_t>(m) * n_total + n0, n_total - n0, w);
+                if (d8t != nullptr) {
+                    uint8_t *tile = box + (cs & 1) * FP8_TILE_BYTES;
+                    *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4 *>(tile + lane * FP8_TSTRIDE + 16) = make_uint4(w[4], w[5], w[6], w[7]);
+                    __syncwarp();
+                    uint32_t t[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        t[i] = static_cast<uint32_t>(tile[(4 * i) * FP8_TSTRIDE + lane]) |
+                               (static_cast<uint32_t>(tile[(4 * i + 1) * FP8_TSTRIDE + lane]) << 8) |
+                               (static_cast<uint32_t>(tile[(4 * i + 2) * FP8_TSTRIDE + lane]) << 16) |
+                               (static_cast<uint32_t>(tile[(4 * i + 3) * FP8_TSTRIDE + lane]) << 24);
+                    }
+                    const int64_t n = n0 + lane;
+                    if (n < n_total && m_row0 < m_total)
+                        store_segment(d8t + n * m_total + m_row0, static_cast<int64_t>(m_total) - m_row0, t);
+                }
             }
         }
         if (c + 1 < CHUNKS) tmem_ld_wait();
@@ -749,9 +804,10 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
-            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * CHUNKS * 32), m_row0);
+            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)), m_row0);
             tma_store_commit();
         }
+        ++nbox;
     }
 }
 
@@ -806,8 +862,9 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
                                               uint32_t tempty_rank, int rank, bool split) {
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - EPI_WARP0) >> 2;  // which half of the accumulator columns
-    uint8_t *box = sm.epi + (warp - EPI_WARP0) * EPI_BOX_BYTES;
-    float *bias_s = reinterpret_cast<float *>(sm.epi + EPI_WARPS * EPI_BOX_BYTES);
+    uint8_t *boxes = sm.epi + (warp - EPI_WARP0) * EPI_NBOX * EPI_BOX_BYTES;
+    int nbox = 0;  // staging boxes this warp has filled (boxes alternate)
+    float *bias_s = reinterpret_cast<float *>(sm.epi + EPI_WARPS * EPI_NBOX * EPI_BOX_BYTES);
     const int epi_tid = (warp - EPI_WARP0) * 32 + lane;
     const float sab = __fmul_rn(__ldg(p.a_scale_inv), __ldg(p.b_scale_inv));
     const float s_out = OUT == OUT_FP8 ? __ldg(p.out_scale) : 0.0f;
@@ -861,19 +918,19 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             const int64_t n_base = static_cast<int64_t>(n_blk) * ACC_N;
             if constexpr (OUT == OUT_FP8) {
                 if (p.bias_kind != 0)
-                    epilogue_tile_fp8<true>(t_row, lane, box, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
+                    epilogue_tile_fp8<true>(t_row, lane, boxes, nbox, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
                                             bias_s, empty_addr, release, mode, slot, h, q, s_out, p.out_fmt, p.M, p.N,
                                             amax);
                 else
-                    epilogue_tile_fp8<false>(t_row, lane, box, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
+                    epilogue_tile_fp8<false>(t_row, lane, boxes, nbox, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
                                              bias_s, empty_addr, release, mode, slot, h, q, s_out, p.out_fmt, p.M, p.N,
                                              amax);
             } else {
                 if (p.bias_kind != 0)
-                    epilogue_tile<OUT == OUT_BF16, true>(t_row, lane, box, half, tmap_d, n_base, m_row0, sab, bias_s,
+                    epilogue_tile<OUT == OUT_BF16, true>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab, bias_s,
                                                          empty_addr, release, mode, slot, h, q);
                 else
-                    epilogue_tile<OUT == OUT_BF16, false>(t_row, lane, box, half, tmap_d, n_base, m_row0, sab, bias_s,
+                    epilogue_tile<OUT == OUT_BF16, false>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab, bias_s,
                                                           empty_addr, release, mode, slot, h, q);
             }
         }

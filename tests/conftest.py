@@ -27,3 +27,20 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Summary of the bf16 GEMM output checks: how far the GPU's bf16 results
+    sat from the fp64 reference, in bf16 ulps."""
+    try:
+        from tests.gpu_util import BF16_CHECKS
+    except Exception:  # pragma: no cover
+        return
+    if not BF16_CHECKS:
+        return
+    worst = max(BF16_CHECKS, key=lambda c: c[1])
+    least = min(BF16_CHECKS, key=lambda c: c[2])
+    n = sum(c[3] for c in BF16_CHECKS)
+    terminalreporter.write_line(
+        "bf16 GEMM checks: %d checks, %d elements; max %.3f ulp (%s); lowest share within 1 ulp %.6f (%s)"
+        % (len(BF16_CHECKS), n, worst[1], worst[0], least[2], least[0]))

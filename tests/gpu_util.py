@@ -83,10 +83,25 @@ def accumulation_allowance(absdot, K):
     return (np.ceil(K / 32.0) + 2) * 2.0 ** -24 * np.asarray(absdot, np.float64)
 
 
+# Largest share of a bf16 output's elements that may lie beyond the plain
+# 1-ulp bound (inside the accumulation allowance): the allowance exists for
+# the rare elements whose |D_ref| cancels far below sum_k |a_k b_k|; a
+# regression that pushes many elements into it fails here.
+BF16_BEYOND_ULP_MAX_SHARE = 1e-3
+BF16_BEYOND_ULP_MIN_COUNT = 2
+
+# (what, max ulp, share within 1 ulp, elements) of every bf16 check of the
+# session; tests/conftest.py prints the summary at the end of the run.
+BF16_CHECKS = []
+
+
 def check_gemm_bf16(got_bits, ref, what, absdot=None, K=None):
     """bf16 output: every element within 1 bf16 ulp (at |bf16_rne(D_ref)|) of
     the fp64 reference, widened by the fp32 accumulation bound where
-    cancellation makes |D_ref| small against sum_k |a_k b_k|."""
+    cancellation makes |D_ref| small against sum_k |a_k b_k|.  At most
+    BF16_BEYOND_ULP_MAX_SHARE of the elements (and never more than
+    BF16_BEYOND_ULP_MIN_COUNT on small outputs) may need the widening.
+    Returns (max ulp, share of elements within 1 ulp)."""
     got = o.bf16_bits_to_f32(got_bits).astype(np.float64)
     ulp = bf16_ulp(o.round_bf16(ref))
     tol = ulp if absdot is None else ulp + accumulation_allowance(absdot, K)
@@ -98,5 +113,11 @@ def check_gemm_bf16(got_bits, ref, what, absdot=None, K=None):
                              "%.2f x tol)" % (what, int(bad.sum()), np.unravel_index(i, ref.shape),
                                               got.flat[i], ref.flat[i], (diff / ulp).flat[i],
                                               (diff / tol).flat[i]))
-    within = float((diff <= ulp).mean())
-    return float((diff / ulp).max()), within
+    beyond = int((diff > ulp).sum())
+    max_ulp = float((diff / ulp).max()) if diff.size else 0.0
+    within = 1.0 - beyond / diff.size if diff.size else 1.0
+    BF16_CHECKS.append((what, max_ulp, within, int(diff.size)))
+    limit = max(BF16_BEYOND_ULP_MIN_COUNT, int(BF16_BEYOND_ULP_MAX_SHARE * diff.size))
+    assert beyond <= limit, "%s: %d of %d elements beyond 1 bf16 ulp (inside the accumulation allowance), " \
+        "more than %d; max %.2f ulp" % (what, beyond, diff.size, limit, max_ulp)
+    return max_ulp, within

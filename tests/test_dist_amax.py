@@ -17,6 +17,7 @@ import torch.multiprocessing as mp
 
 import oracle as o
 from fp8_delayed_scaling_cast_b200 import inputs
+from fp8_delayed_scaling_cast_b200.dist import sync_amax
 
 WORLD = 2
 STEPS = 20
@@ -43,6 +44,15 @@ def _batch(step):
 W = inputs.normal((16, 32), inputs.gen(9), 0.02).numpy()
 
 
+class _HistView:
+    """What sync_amax reads from a meta: the [H, T] history as a torch tensor
+    (here a view of the oracle's numpy history, sharing its memory)."""
+
+    def __init__(self, hist):
+        assert hist.flags["C_CONTIGUOUS"]
+        self.amax_history = torch.from_numpy(hist)
+
+
 def _rank_main(rank, port, out):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -59,9 +69,9 @@ def _rank_main(rank, port, out):
         meta.record(0, am_x)
         meta.record(1, am_w)
         meta.record(2, am_g)
-        row = torch.from_numpy(meta.hist[0].copy())
-        dist.all_reduce(row, op=dist.ReduceOp.MAX)
-        meta.hist[0] = row.numpy()
+        # the product's exchange, on a torch view that shares the oracle's
+        # history memory (row 0 is reduced in place)
+        sync_amax(_HistView(meta.hist))
         meta.update()
     out[rank] = (meta.hist.copy(), meta.scale.copy(), meta.scale_inv.copy())
     dist.destroy_process_group()
