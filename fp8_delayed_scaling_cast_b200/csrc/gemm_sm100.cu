@@ -377,7 +377,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+__device__ __forceinline__ __attribute__((unused)) void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -395,9 +395,15 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
         : "r"(taddr));
 }
 
-// tcgen05.ld of EPI_LD columns (32 lanes x 32 bits each) into r.
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[32]) { tmem_ld32(taddr, r); }
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[64]) { tmem_ld64(taddr, r); }
+// tcgen05.ld of N = 32 or 64 columns (32 lanes x 32 bits each) into r.
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N == 32 || N == 64, "TMEM load width");
+    if constexpr (N == 32)
+        tmem_ld32(taddr, r);
+    else
+        tmem_ld64(taddr, r);
+}
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -1425,28 +1431,56 @@ size_t gemm_workspace_bytes() {
     return WS_FLAG_BYTES + static_cast<size_t>(pairs) * 2 * WS_SLOT_FLOATS * sizeof(float);
 }
 
+namespace {
+
+// Tile schedule of a GEMM on the current device: kernel (one CTA or a CTA
+// pair), pair-tile rows, tile count, and whether a workspace turns it into
+// the stream-K schedule.
+struct GemmPlan {
+    bool pair;
+    int m_sub;
+    int64_t tiles;
+    bool stream_k;   // with a large enough workspace
+};
+
+GemmPlan plan_gemm(int64_t m, int64_t n, int64_t k) {
+    static std::atomic<int> cached_pairs[64];
+    GemmPlan g;
+    g.pair = m > S1_BM;
+    // Long contractions amortise the partly exposed epilogue of the 512-row
+    // pair tile; short ones keep the double-buffered 256-row tile.  The
+    // 512-row tile is also declined when its tiles fill the last wave of
+    // pairs less well than the 256-row ones (e.g. 4096 x 8192: 256 tiles =
+    // 3.46 waves of 74 pairs against 512 = 6.92 waves).
+    g.m_sub = 1;
+    const int64_t cap = g.pair ? max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached_pairs) : 0;
+    const int64_t tn = (n + ACC_N - 1) / ACC_N;
+    if (g.pair && m > 2 * S2_BM && k >= FP8DS_MSUB2_MIN_K) {
+        const int64_t t1 = ((m + 2 * S2_BM - 1) / (2 * S2_BM)) * tn, t2 = ((m + 4 * S2_BM - 1) / (4 * S2_BM)) * tn;
+        // wave fill tiles / (waves * cap), compared without division
+        const int64_t w1 = (t1 + cap - 1) / cap, w2 = (t2 + cap - 1) / cap;
+        if (cap <= 0 || t2 * w1 * 50 >= t1 * w2 * 49) g.m_sub = 2;      // fill(512) >= fill(256) - 2%
+    }
+    const int64_t tile_m = g.pair ? g.m_sub * 2 * S2_BM : S1_BM;
+    g.tiles = ((m + tile_m - 1) / tile_m) * tn;
+    // Stream-K when whole tiles would leave a ragged last wave: at least one
+    // tile per pair, fewer than 8 waves, not a whole number of waves.
+    g.stream_k = g.pair && cap > 0 && g.tiles >= cap && g.tiles % cap != 0 && g.tiles < 8 * cap &&
+                 cap <= static_cast<int64_t>(WS_FLAG_BYTES / 8);
+    return g;
+}
+
+}  // namespace
+
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
                          fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
                          void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, void *workspace,
                          size_t workspace_bytes, cudaStream_t stream, const GemmCastOut *cast, bool a_mn,
                          bool b_mn) {
     const int out = cast != nullptr ? OUT_FP8 : (d_dtype == FP8DS_BF16 ? OUT_BF16 : OUT_F32);
-    const bool pair = m > S1_BM;
-    // Long contractions amortise the partly exposed epilogue of the 512-row
-    // pair tile; short ones keep the double-buffered 256-row tile.  The
-    // 512-row tile is also declined when its tiles fill the last wave of
-    // pairs less well than the 256-row ones (e.g. 4096 x 8192: 256 tiles =
-    // 3.46 waves of 74 pairs against 512 = 6.92 waves).
-    int m_sub = 1;
-    if (pair && m > 2 * S2_BM && k >= FP8DS_MSUB2_MIN_K) {
-        static std::atomic<int> cached_pairs[64];
-        const int64_t cap = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached_pairs);
-        const int64_t tn = (n + ACC_N - 1) / ACC_N;
-        const int64_t t1 = ((m + 2 * S2_BM - 1) / (2 * S2_BM)) * tn, t2 = ((m + 4 * S2_BM - 1) / (4 * S2_BM)) * tn;
-        // wave fill tiles / (waves * cap), compared without division
-        const int64_t w1 = (t1 + cap - 1) / cap, w2 = (t2 + cap - 1) / cap;
-        if (cap <= 0 || t2 * w1 * 50 >= t1 * w2 * 49) m_sub = 2;      // fill(512) >= fill(256) - 2%
-    }
+    const GemmPlan plan = plan_gemm(m, n, k);
+    const bool pair = plan.pair;
+    const int m_sub = plan.m_sub;
     CUtensorMap ta, tb, td;
     // K-major operands: [rows, k] boxes of BK x rows; MN-major: [k, rows]
     // boxes of 128 columns x BK rows (the one-CTA B tile loads two of them)
@@ -1493,21 +1527,14 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.out_fmt = cast != nullptr ? static_cast<int32_t>(cast->fmt) : 0;
     p.out_d8 = cast != nullptr ? static_cast<uint8_t *>(d) : nullptr;
     p.out_d8t = cast != nullptr ? cast->d8t : nullptr;
-    if (pair && workspace != nullptr && workspace_bytes >= gemm_workspace_bytes()) {
-        // Stream-K when whole tiles would leave a ragged last wave: at least
-        // one tile per pair, fewer than 8 waves, not a whole number of waves.
-        static std::atomic<int> cached[64];
-        const int cap = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached);
-        const int tiles = p.tiles_m * p.tiles_n;
-        if (tiles >= cap && tiles % cap != 0 && tiles < 8 * cap && cap <= static_cast<int>(WS_FLAG_BYTES / 8)) {
-            static std::atomic<uint32_t> launches{0};
-            uint32_t e = ++launches;
-            if (e == 0) e = ++launches;
-            p.stream_k = 1;
-            p.epoch = e;
-            p.flags = static_cast<int32_t *>(workspace);
-            p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + WS_FLAG_BYTES);
-        }
+    if (plan.stream_k && workspace != nullptr && workspace_bytes >= gemm_workspace_bytes()) {
+        static std::atomic<uint32_t> launches{0};
+        uint32_t e = ++launches;
+        if (e == 0) e = ++launches;
+        p.stream_k = 1;
+        p.epoch = e;
+        p.flags = static_cast<int32_t *>(workspace);
+        p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + WS_FLAG_BYTES);
     }
     cudaError_t e;
     if (pair && m_sub == 2) {
@@ -1577,8 +1604,16 @@ fp8ds_status launch_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const flo
                   need, NOALLOC_SCRATCH_BYTES);
         return FP8DS_ERR_INVALID_ARG;
     }
-    // The array keeps whatever the previous call left: the publication words
-    // must start at zero.
+    // Whole tiles (no ragged last wave, or the one-CTA kernel) need no
+    // scratch: the same launch as fp8_gemm, nothing else enqueued.
+    if (!plan_gemm(m, n, k).stream_k)
+        return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k,
+                           nullptr, 0, stream);
+    // The array keeps whatever the previous call left.  Each stream-K launch
+    // publishes its partials under a fresh non-zero epoch and its consumers
+    // clear the words they read, so stale words cannot match; the words are
+    // still cleared here so that a launch that ended early (a bounded wait
+    // gave up) leaves nothing behind for the next one.
     e = cudaMemsetAsync(ws, 0, WS_FLAG_BYTES, stream);
     if (e != cudaSuccess) {
         set_error("fp8_gemm_noalloc: clearing the scratch failed: %s", cudaGetErrorString(e));

@@ -284,12 +284,16 @@ fp8ds_status fp8_gemm_ex(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
  * engine at start-up, or C code that only receives tensor pointers and owns
  * no allocator -- yet want the same GEMM.
  *   Arguments, layouts and results as fp8_gemm.  Calls no allocator (no
- *   cudaMalloc/cudaFree, no library routine that allocates); it only enqueues
- *   a 4 KiB memset of the scratch's publication words and the GEMM on
- *   `stream`.
+ *   cudaMalloc/cudaFree, no library routine that allocates).  When the
+ *   shape's tiles leave a ragged last wave of CTA pairs (the stream-K case)
+ *   it enqueues a 4 KiB memset of the scratch's publication words and the
+ *   GEMM on `stream`; otherwise only the GEMM, exactly as fp8_gemm.
  *   The first call on a device looks up the scratch's device address (a
  *   runtime query, done once per device with that device current); make that
- *   first call before any stream capture on the device.
+ *   first call before any stream capture on the device.  The address, like
+ *   the library's other per-device settings (kernel attributes, occupancy
+ *   figures), is kept for the life of the process: after cudaDeviceReset on
+ *   a device, do not call the library on that device again.
  *   All calls share the one scratch: calls that may overlap on the GPU (other
  *   streams, other threads) race and must be ordered by the caller.
  * Errors: as fp8_gemm; FP8DS_ERR_INVALID_ARG if the device needs more
