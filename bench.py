@@ -14,20 +14,23 @@ is laid out for B200:
   either order.
 The results are identical to the unfused, transpose-based calls.
 
-Per step: 4 casts with amax (X, W1, W2, dY) in 3 launches (fc1's forward
-casts X and W1 in one), 6 FP8 GEMMs (fwd, dgrad, wgrad of both linears;
-1.649 TFLOP), 1 update launch.  The unfused step (every linear casts its own
-input and gradient with transposes, 6 casts in 5 launches) is
-timed beside it and reported as "unfused_step".  Under torchrun every rank runs its
+Per step: 4 casts with amax (X, W1, W2, dY) in 2 launches (the weight-cache
+refresh of both linears with X as an extra cast, then dY in the backward),
+6 FP8 GEMMs (fwd, dgrad, wgrad of both linears; 1.649 TFLOP), 1 update
+launch.  The unfused step (every linear casts its own input and gradient with
+transposes, 6 casts in 5 launches) is timed beside it and reported as
+"unfused_step".  Under torchrun every rank runs its
 own batch (data parallel, weak scaling) and the ranks max-reduce the current
 amaxes over NCCL before the update (the amax sync of delayed scaling).
 
-Printed (rank 0, one JSON line): whole-job GEMM TFLOP/s of the step, the
+Printed (rank 0, one compact JSON line): whole-job GEMM TFLOP/s of the step,
+the cast-transpose-amax workload bf16 [8192, 2048] -> e4m3/e5m2 in GB/s, the
 roofline of the dominant kernel (the GEMM) from CUDA events over the timed
-region, the cast-transpose-amax workload bf16 [8192, 2048] -> e4m3/e5m2 in
-GB/s, the end-to-end figure through the public linear API with pinned host
-inputs, the oracle's CPU baseline on a bounded sample, and the SM clocks
-sampled during the timed region.
+region, the end-to-end figure through the public linear API with pinned host
+inputs, the TEBlock forward over four microbatches and the 32-block forward
+(576 metas), the oracle's CPU baseline on a bounded sample, and the SM clocks
+sampled during the timed region.  --detail PATH also writes the per-kernel
+breakdown and the notes on how each figure was taken.
 """
 import argparse
 import json
@@ -276,6 +279,20 @@ class MlpStep:
         self.dw1 = e(FFN, HIDDEN, dt=f32)
         self.dw2 = e(HIDDEN, FFN, dt=f32)
         self.si = e(4, dt=f32)  # private scale_invs of x8, h8, dy8, dh8
+        # the native step casts X, W1 and W2 in one launch: the weight-cache
+        # refresh of both linears with X as an extra cast (job arrays built once)
+        self.group = fp8.LinearGroup([self.fc1n, self.fc2n])
+        self._xjobs = {}
+
+    def xjob(self, x):
+        """The X cast of the native step as a job array (built once per input
+        buffer)."""
+        key = x.data_ptr()
+        if key not in self._xjobs:
+            amax = self.meta.amax_history[0]
+            self._xjobs[key] = (x, self.fp8.cast_jobs([self.fp8.cast_job(x, "e4m3", self.meta.scale[0:1], self.x8,
+                                                                         None, amax[0:1], self.si[0:1])]))
+        return self._xjobs[key][1]
 
     def run_linear_api(self, i, sync_amax=None, fused=True):
         """The step through the public linear API (what a user calls).  fused:
@@ -285,9 +302,10 @@ class MlpStep:
         x, dy = self.xs[i % len(self.xs)], self.dys[i % len(self.dys)]
         if fused:
             fc1, fc2 = self.fc1n, self.fc2n
-            fp8.fp8_linear_fwd_ex(fc1, m, x, None, True, self.x8, None, self.si[0:1], out_meta=3,
-                                  out8=self.h8, out_scale_inv=self.si[1:2])
-            fp8.fp8_linear_fwd_ex(fc2, m, None, self.y, True, self.h8, None, self.si[1:2], in_cast=True)
+            fp8.fp8_linear_refresh_weights(self.group, m, self.xjob(x))
+            fp8.fp8_linear_fwd_ex(fc1, m, None, None, False, self.x8, None, self.si[0:1], in_cast=True,
+                                  out_meta=3, out8=self.h8, out_scale_inv=self.si[1:2])
+            fp8.fp8_linear_fwd_ex(fc2, m, None, self.y, False, self.h8, None, self.si[1:2], in_cast=True)
             fp8.fp8_linear_bwd_ex(fc2, m, dy, None, self.si[1:2], self.dw2, self.dy8, None, self.si[2:3],
                                   out_meta=2, out8=self.dh8, out_scale_inv=self.si[3:4], x8=self.h8)
             fp8.fp8_linear_bwd_ex(fc1, m, None, None, self.si[0:1], self.dw1, self.dh8, None, self.si[3:4],
@@ -307,16 +325,13 @@ class MlpStep:
         m.update()
 
     def run_casts(self, i):
-        """The native step's delayed-scaling casts alone (X and W1 from fp32 in
-        one launch, as fc1's forward issues them; W2 from fp32; dY from bf16;
-        y only, no transpose), on step i's inputs."""
-        fp8, m, fc1, fc2 = self.fp8, self.meta, self.fc1n, self.fc2n
+        """The native step's delayed-scaling casts alone (X, W1 and W2 from
+        fp32 in one launch, as the step issues them; dY from bf16; y only, no
+        transpose), on step i's inputs."""
+        fp8, m, fc2 = self.fp8, self.meta, self.fc2n
         x, dy = self.xs[i % len(self.xs)], self.dys[i % len(self.dys)]
         amax = m.amax_history[0]
-        fp8.fp8_cast_transpose_amax_pair(x, fc1.w, "e4m3", m.scale[0:1], self.x8, m.scale[1:2], fc1.w8,
-                                         amax_a=amax[0:1], scale_inv_a=self.si[0:1], amax_b=amax[1:2],
-                                         scale_inv_b=fc1.w_scale_inv)
-        fp8.fp8_cast_transpose_amax(fc2.w, "e4m3", m.scale[4:5], fc2.w8, None, amax[4:5], fc2.w_scale_inv)
+        fp8.fp8_linear_refresh_weights(self.group, m, self.xjob(x))
         fp8.fp8_cast_transpose_amax(dy, "e5m2", m.scale[5:6], self.dy8, None, amax[5:6], self.si[2:3])
 
     def run_gemms(self):
@@ -349,15 +364,11 @@ class MlpStep:
 
         fc1, fc2 = self.fc1n, self.fc2n
         amax = m.amax_history[0]
-        # fc1's forward casts its input and its weight in one launch
-        timed("cast", "x+w1", lambda: fp8.fp8_cast_transpose_amax_pair(
-            x, fc1.w, "e4m3", m.scale[0:1], self.x8, m.scale[1:2], fc1.w8, amax_a=amax[0:1], scale_inv_a=self.si[0:1],
-            amax_b=amax[1:2], scale_inv_b=fc1.w_scale_inv))
+        # X, W1 and W2 in one launch
+        timed("cast", "x+w1+w2", lambda: fp8.fp8_linear_refresh_weights(self.group, m, self.xjob(x)))
         timed("gemm", "fc1.fwd", lambda: fp8.fp8_gemm_cast(
             self.x8, "e4m3", self.si[0:1], fc1.w8, "e4m3", fc1.w_scale_inv, "e4m3", m.scale[3:4], self.h8, None,
             amax[3:4], self.si[1:2], bias=fc1.bias))
-        timed("cast", "w2", lambda: fp8.fp8_cast_transpose_amax(fc2.w, "e4m3", m.scale[4:5], fc2.w8, None,
-                                                                 amax[4:5], fc2.w_scale_inv))
         timed("gemm", "fc2.fwd", lambda: fp8.fp8_gemm(self.h8, "e4m3", self.si[1:2], fc2.w8, "e4m3",
                                                        fc2.w_scale_inv, self.y, bias=fc2.bias))
         timed("cast", "dy", lambda: fp8.fp8_cast_transpose_amax(dy, "e5m2", m.scale[5:6], self.dy8, None, amax[5:6],
@@ -376,8 +387,141 @@ class MlpStep:
         timed("update", "update", m.update)
 
 
-# fused step: 3 cast launches (X with W1, W2, dY), 6 GEMMs, 1 update
-LAUNCHES_PER_STEP = 3 + 6 + 1
+class TeblockForward:
+    """Forward of `blocks` TEBlocks (six linears each: 2048 -> 12288 (+bias),
+    6144, 2048, 4096, 8192 (+bias), and 8192 -> 2048 (+bias)) at 8192 tokens,
+    fp32 master weights ~ N(0, 0.02) and input X ~ U[0,1) fp32 drawn on the
+    device from a seeded generator, bf16 outputs, HYBRID e4m3, history 16.
+    The path per block, through the public API:
+      - one fp8_cast_transpose_amax_multi launch casts X for the five K = 2048
+        linears, each with its own meta (the pages' te.Linear casts its own
+        input);
+      - the six GEMMs (fp8_linear_fwd_ex with in_cast); fc1 hands H to fc2 in
+        FP8 from its epilogue (no bf16 H, no separate H cast);
+    plus, per step, the weight-cache refresh of every linear in one launch
+    (fp8_linear_refresh_weights) when the weights are recast, and one
+    fp8_update_scales over all 18 * blocks metas.  Native B200 layout: no FP8
+    transposes (the backward would read X8, H8 and the weights MN-major)."""
+
+    def __init__(self, fp8, device, blocks, seed=0):
+        self.fp8 = fp8
+        L = 6 * blocks
+        self.blocks = blocks
+        self.meta = fp8.Fp8Meta(["e4m3", "e4m3", "e5m2"] * L, hist_len=16, device=device)
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        self.lins = []
+        for i in range(L):
+            out_f, in_f, has_bias = inputs.TEBLOCK_LINEARS[i % 6]
+            w = torch.randn(out_f, in_f, generator=g, device=device) * 0.02
+            bias = torch.randn(out_f, generator=g, device=device) * 0.02 if has_bias else None
+            self.lins.append(fp8.Fp8Linear(w, bias, 3 * i, 3 * i + 1, 3 * i + 2, transpose=False))
+        self.group = fp8.LinearGroup(self.lins)
+        self.x = torch.rand(TOKENS, HIDDEN, generator=g, device=device)
+        u8, bf = torch.uint8, torch.bfloat16
+        self.x8 = [torch.empty(TOKENS, HIDDEN, dtype=u8, device=device) for _ in range(5)]
+        self.h8 = torch.empty(TOKENS, FFN, dtype=u8, device=device)
+        self.ys = [torch.empty(TOKENS, out_f, dtype=bf, device=device) for out_f, _, _ in inputs.TEBLOCK_LINEARS]
+        self.si = torch.zeros(6, dtype=torch.float32, device=device)   # private scale_invs of the inputs
+        amax = self.meta.amax_history[0]
+        self.xjobs = []
+        for b in range(blocks):
+            jobs = []
+            for j in range(5):
+                t = 3 * (6 * b + j)
+                jobs.append(fp8.cast_job(self.x, "e4m3", self.meta.scale[t:t + 1], self.x8[j], None,
+                                         amax[t:t + 1], self.si[j:j + 1]))
+            self.xjobs.append(fp8.cast_jobs(jobs))
+        self.flop = blocks * sum(2.0 * TOKENS * o * i for o, i, _ in inputs.TEBLOCK_LINEARS)
+
+    def launches(self, refresh):
+        return (1 if refresh else 0) + self.blocks * (1 + 6) + 1
+
+    def run(self, refresh):
+        fp8, m = self.fp8, self.meta
+        if refresh:
+            fp8.fp8_linear_refresh_weights(self.group, m)
+        for b in range(self.blocks):
+            fp8.fp8_cast_transpose_amax_multi(self.xjobs[b])
+            lins = self.lins[6 * b:6 * b + 6]
+            for j in range(4):
+                fp8.fp8_linear_fwd_ex(lins[j], m, None, self.ys[j], False, self.x8[j], None, self.si[j:j + 1],
+                                      in_cast=True)
+            fp8.fp8_linear_fwd_ex(lins[4], m, None, None, False, self.x8[4], None, self.si[4:5], in_cast=True,
+                                  out_meta=lins[5]._c.meta_in, out8=self.h8, out_scale_inv=self.si[5:6])
+            fp8.fp8_linear_fwd_ex(lins[5], m, None, self.ys[5], False, self.h8, None, self.si[5:6], in_cast=True)
+        m.update()
+
+
+def time_teblock_microbatches(fp8, device, rounds):
+    """The TEBlock forward over 4 microbatches (is_first_microbatch True, then
+    False x3: the weight caches are refreshed at microbatch 0 and reused), the
+    update after each microbatch; CUDA events around every microbatch, over
+    `rounds` rounds after one warm-up round."""
+    tb = TeblockForward(fp8, device, blocks=1)
+    for mb in range(4):
+        tb.run(mb == 0)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(rounds)]
+    for r in range(rounds):
+        ev[r][0].record()
+        for mb in range(4):
+            tb.run(mb == 0)
+            ev[r][mb + 1].record()
+    torch.cuda.synchronize()
+    per_mb = [[ev[r][mb].elapsed_time(ev[r][mb + 1]) for r in range(rounds)] for mb in range(4)]
+    refresh_ms = statistics.mean(per_mb[0])
+    reuse_ms = statistics.mean(per_mb[1] + per_mb[2] + per_mb[3])
+    out = {"refresh_mb_ms": refresh_ms, "reuse_mb_ms": reuse_ms,
+           "reuse_tflops": tb.flop / (reuse_ms * 1e-3) / 1e12, "refresh_tflops": tb.flop / (refresh_ms * 1e-3) / 1e12,
+           "launches_refresh_mb": tb.launches(True), "launches_reuse_mb": tb.launches(False)}
+    del tb
+    torch.cuda.empty_cache()
+    return out
+
+
+def time_toy_model(fp8, device, steps):
+    """The 32-block forward (192 linears, 576 metas, weights recast every
+    step): device ms per step issued eagerly, the host time to issue one
+    step, and the same step captured once in a CUDA graph and replayed."""
+    toy = TeblockForward(fp8, device, blocks=32)
+    for _ in range(2):
+        toy.run(True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    h0 = time.perf_counter()
+    for _ in range(steps):
+        toy.run(True)
+    host_s = time.perf_counter() - h0
+    e1.record()
+    torch.cuda.synchronize()
+    eager_ms = e0.elapsed_time(e1) / steps
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        toy.run(True)
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    h0 = time.perf_counter()
+    for _ in range(steps):
+        graph.replay()
+    ghost_s = time.perf_counter() - h0
+    e1.record()
+    torch.cuda.synchronize()
+    graph_ms = e0.elapsed_time(e1) / steps
+    status = fp8.fp8ds_device_status()
+    out = {"ms_per_step": eager_ms, "tflops": toy.flop / (eager_ms * 1e-3) / 1e12,
+           "host_us_per_step": 1e6 * host_s / steps, "graph_ms_per_step": graph_ms,
+           "graph_host_us_per_step": 1e6 * ghost_s / steps, "launches_per_step": toy.launches(True),
+           "device_status": status}
+    del graph, toy
+    torch.cuda.empty_cache()
+    return out
+
+
+# native step: 2 cast launches (X with W1 and W2, dY), 6 GEMMs, 1 update
+LAUNCHES_PER_STEP = 2 + 6 + 1
 # unfused step: X with W1, H, W2, dY, dH casts, 6 GEMMs, 1 update
 LAUNCHES_PER_STEP_UNFUSED = 5 + 6 + 1
 
@@ -709,7 +853,24 @@ def single_kernel(args):
     ones (used under ncu with -s 2)."""
     from fp8_delayed_scaling_cast_b200 import binding as fp8
     dev = torch.device("cuda", 0)
-    if args.kernel in ("gemm", "gemmcast"):
+    if args.kernel == "castmulti":
+        # the step's X, W1 and W2 casts (fp32 [8192, 2048], [8192, 2048],
+        # [2048, 8192] -> e4m3, y only) in one fp8_cast_transpose_amax_multi
+        # launch; 201 MB read per launch, more than L2
+        g = torch.Generator(device=dev)
+        g.manual_seed(5)
+        srcs = [torch.rand(TOKENS, HIDDEN, generator=g, device=dev),
+                torch.randn(FFN, HIDDEN, generator=g, device=dev) * 0.02,
+                torch.randn(HIDDEN, FFN, generator=g, device=dev) * 0.02]
+        outs = [torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in srcs]
+        sc = torch.ones(3, device=dev)
+        am = torch.zeros(3, device=dev)
+        si = torch.zeros(3, device=dev)
+        jobs = fp8.cast_jobs([fp8.cast_job(t, "e4m3", sc[i:i + 1], o, None, am[i:i + 1], si[i:i + 1])
+                              for i, (t, o) in enumerate(zip(srcs, outs))])
+        run = lambda: fp8.fp8_cast_transpose_amax_multi(jobs)  # noqa: E731
+        work, unit = sum(t.numel() * 5 for t in srcs) / 1e9, "GB/s"
+    elif args.kernel in ("gemm", "gemmcast"):
         M, N, K = (int(v) for v in args.shape.split("x"))
         g = torch.Generator(device="cpu").manual_seed(3)
         a = torch.randint(0, 0x7F, (M, K), generator=g, dtype=torch.uint8).to(dev)
@@ -780,7 +941,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=None,
                     help="tokens of the oracle's sample (default 128; 8 per step for --impl reference)")
-    ap.add_argument("--kernel", choices=["gemm", "gemmcast", "cast", "quantize"], default=None,
+    ap.add_argument("--kernel", choices=["gemm", "gemmcast", "cast", "castmulti", "quantize"], default=None,
                     help="run one kernel alone (2 warm-up + --reps launches), for profilers")
     ap.add_argument("--shape", default="8192x2048x8192", help="MxNxK for --kernel gemm")
     ap.add_argument("--major", default="k,k", help="operand layouts a,b for --kernel gemm: k or mn each")
@@ -788,6 +949,8 @@ def main():
     ap.add_argument("--cast-in", default="bf16", choices=["bf16", "f32"], help="input dtype for --kernel cast")
     ap.add_argument("--no-yt", action="store_true", help="--kernel cast writes y only (no transpose)")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--detail", default=None, help="also write the per-kernel breakdown and notes (JSON) here")
+    ap.add_argument("--no-models", action="store_true", help="skip the TEBlock and 32-block forward timings")
     args = ap.parse_args()
     if args.kernel:
         return single_kernel(args)
@@ -964,6 +1127,16 @@ def main():
     e2e_ms = max_over_ranks(e2e_ms, world, device)
     status = status or fp8.fp8ds_device_status()
 
+    # the TEBlock forward (4 microbatches, cache refreshed at the first) and
+    # the 32-block forward (576 metas): rank 0's GPU only, after the step
+    teblock = toy = None
+    if world == 1 and not args.no_models:
+        del step
+        torch.cuda.empty_cache()
+        teblock = time_teblock_microbatches(fp8, device, rounds=max(3, min(args.steps, 10)))
+        toy = time_toy_model(fp8, device, steps=max(3, min(args.steps, 10)))
+        status = status or toy["device_status"]
+
     if world > 1:
         barrier_sync(world)
         torch.distributed.destroy_process_group()
@@ -980,6 +1153,7 @@ def main():
                "sample": "oracle step (6 casts, 6 fp64 GEMMs, update) at %d of %d tokens, full "
                          "weights; %.1f s" % (args.cpu_tokens, TOKENS, dt)}
 
+    r3 = lambda v: None if v is None else round(v, 3)  # noqa: E731
     line = {
         "metric": METRIC,
         "value": value,
@@ -994,62 +1168,69 @@ def main():
         "dtype": "fp8(e4m3,e5m2)xfp8->f32",
         "data": "synthetic",
         "config": step_config(world),
-        "roofline": {
-            "kernel": "fp8_gemm_2sm_kernel (tcgen05 CTA pairs; bf16 / fp32 / FP8 out)",
-            "bound": "tensor", "achieved": gemm_tflops, "peak": gemm_peak, "unit": "TFLOP/s",
-            "frac": gemm_tflops / gemm_peak, "traffic": traffic, "traffic_unit": "bytes per launch",
-            "traffic_note": traffic_note, "algorithmic_bytes_per_launch": GEMM_ALG_BYTES,
-            "peak_kind": gemm_peak_kind,
-            "peak_note": "fp8 dense = 2 x measured bf16 (%s): burst %.1f, sustained %.1f TFLOP/s (frac %.3f / %.3f); "
-                         "sustained is used when the SM clock over the GEMM loop sat >10%% below max" % (
-                             pk["src"], fp8_peak, fp8_peak_sus, gemm_tflops / fp8_peak, gemm_tflops / fp8_peak_sus),
-            "clocks": gemm_clock_info,
-            "flop_per_launch": GEMM_FLOP, "launch_us": 1e3 * gemm_avg_b2b,
-            "timing": "the step's 6 GEMM launches (same operands, outputs, epilogues) back to back for K rounds, "
-                      "CUDA events around the loop on the launching stream; mean per launch",
-            "launch_us_event_bracketed": 1e3 * gemm_avg,
-        },
         "cast_transpose_amax": {
-            "workload": "bf16 [8192, 2048] (0.1%% spikes x1000) -> FP8 + transpose + amax, 8 rotating inputs",
-            "e4m3_us": c2["e4m3"]["us_mean"], "e5m2_us": c2["e5m2"]["us_mean"],
-            "bytes_per_launch": C2_BYTES, "achieved": c2_gbs, "peak": pk["hbm"], "unit": "GB/s",
-            "frac": c2_gbs / pk["hbm"], "bound": "hbm",
-            "in_step_gbs": cast_gbs_step, "in_step_frac": cast_gbs_step / pk["hbm"],
-            "in_step_us": 1e3 * cast_b2b_ms, "in_step_bytes": STEP_CAST_BYTES_FUSED,
-            "in_step_note": "the step's cast launches (X with W1 in one, W2: fp32; dY bf16; y only) back to back, "
-                            "K rounds, "
-                            "replayed from a CUDA graph, CUDA events around the replay",
-            "us_host_issued": {"e4m3": c2["e4m3"]["us_host_issued"], "e5m2": c2["e5m2"]["us_host_issued"]},
-            "timing": "100 launches over the 8 inputs captured in a CUDA graph, replayed between CUDA events; "
-                      "us_host_issued: the same launches issued one by one from Python",
-            "in_step_event_bracketed_gbs": cast_gbs_bracketed,
-            "dynamic_scaling_e4m3_us": c2["dynamic_e4m3"]["us_mean"],
-            "dynamic_note": "amax pass + scale + cast (input read twice) vs the delayed cast's one read",
+            "bf16_8192x2048_e4m3_us": r3(c2["e4m3"]["us_mean"]), "e5m2_us": r3(c2["e5m2"]["us_mean"]),
+            "gbs": r3(c2_gbs), "peak_gbs": pk["hbm"], "frac": r3(c2_gbs / pk["hbm"]),
+            "in_step_us": r3(1e3 * cast_b2b_ms), "in_step_gbs": r3(cast_gbs_step),
+            "in_step_frac": r3(cast_gbs_step / pk["hbm"]), "dynamic_e4m3_us": r3(c2["dynamic_e4m3"]["us_mean"]),
         },
-        "update_scales_us": 1e3 * statistics.mean(upd_ms),
-        "update_scales_576_metas_us": upd576_us,
-        "gemm_us": {k: 1e3 * statistics.mean(v) for k, v in gemm_by_key.items()},
-        "cast_us": {k: 1e3 * statistics.mean(v) for k, v in cast_ms.items()},
-        "kernels_sum_ms_per_step": kernel_ms,
-        "gemm_alone": heads,
-        "step_roofline_frac": ((STEP_FLOP / (fp8_peak * 1e12)) + (STEP_CAST_BYTES_FUSED / (pk["hbm"] * 1e9))) /
-                              (ms * 1e-3),
-        "host_us_per_step": host_us,
-        "graph_step": graph_info,
-        "unfused_step": {"ms_per_step": ms_unfused, "value": world * STEP_FLOP / (ms_unfused * 1e-3) / 1e12,
-                         "unit": "TFLOP/s", "gpu_launches_per_step": LAUNCHES_PER_STEP_UNFUSED,
-                         "api": "fp8_linear_fwd/bwd: every linear casts its own input and gradient, with "
-                                "transposes, K-major operands only"},
-        "e2e": {"value": world * STEP_FLOP / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "fp8_linear_fwd_ex/bwd_ex + fp8_update_scales, pinned host X/dY, double-buffered copies"},
+        "roofline": {
+            "bound": "tensor", "achieved": r3(gemm_tflops), "peak": gemm_peak, "unit": "TFLOP/s",
+            "frac": r3(gemm_tflops / gemm_peak), "traffic": traffic,
+            "kernel": "fp8_gemm_2sm_kernel", "launch_us": r3(1e3 * gemm_avg_b2b), "peak_kind": gemm_peak_kind,
+            "peak_src": pk["src"], "frac_burst": r3(gemm_tflops / fp8_peak),
+        },
+        "e2e": {"value": r3(world * STEP_FLOP / (e2e_ms * 1e-3) / 1e12), "unit": "TFLOP/s",
+                "ms_per_step": r3(e2e_ms), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "gpu_launches_per_step": LAUNCHES_PER_STEP,
-        "launch_mode": "programmatic dependent launch (griddepcontrol) on every kernel",
+        "gemm_alone": {k: {"us": r3(v["us_mean"]), "tflops": r3(v["tflops"]),
+                           "torch_scaled_mm_us": r3(v["context_torch_scaled_mm"].get("us_mean"))}
+                       for k, v in heads.items()},
+        "teblock_fwd_4mb": None if teblock is None else {k: r3(v) for k, v in teblock.items()},
+        "toy32_fwd": None if toy is None else {k: r3(v) for k, v in toy.items() if k != "device_status"},
+        "graph_step": None if graph_info is None else {"ms_per_step": r3(graph_info["ms_per_step"]),
+                                                      "host_us_per_step": r3(graph_info["host_us_per_step"])},
+        "host_us_per_step": r3(host_us),
+        "unfused_step_ms": r3(ms_unfused),
+        "update_576_metas_us": r3(upd576_us),
+        "step_roofline_frac": r3(((STEP_FLOP / (fp8_peak * 1e12)) + (STEP_CAST_BYTES_FUSED / (pk["hbm"] * 1e9))) /
+                                 (ms * 1e-3)),
         "device_status": status,
         "clocks": clock_info,
         "cpu_baseline": cpu,
     }
+    if args.detail:
+        detail = {
+            "gemm_event_bracketed_us": {k: 1e3 * statistics.mean(v) for k, v in gemm_by_key.items()},
+            "cast_event_bracketed_us": {k: 1e3 * statistics.mean(v) for k, v in cast_ms.items()},
+            "update_event_bracketed_us": 1e3 * statistics.mean(upd_ms),
+            "kernels_event_bracketed_sum_ms_per_step": kernel_ms,
+            "event_bracketed_note": "each launch bracketed by CUDA events: the events break the PDL overlap and "
+                                    "add host gaps, so these run 5-20% above the back-to-back figures and their "
+                                    "sum exceeds ms_per_step",
+            "roofline_timing": "the step's 6 GEMM launches (same operands, outputs, epilogues) back to back for K "
+                               "rounds, CUDA events around the loop on the launching stream; mean per launch",
+            "roofline_traffic_note": traffic_note, "gemm_algorithmic_bytes_per_launch": GEMM_ALG_BYTES,
+            "gemm_clocks": gemm_clock_info,
+            "peak_note": "fp8 dense = 2 x measured bf16 (%s): burst %.1f, sustained %.1f TFLOP/s; sustained is "
+                         "used when the SM clock over the GEMM loop sat >10%% below max" % (
+                             pk["src"], fp8_peak, fp8_peak_sus),
+            "cast_workload": c2,
+            "cast_in_step_event_bracketed_gbs": cast_gbs_bracketed,
+            "cast_timing": "100 launches over 8 rotating inputs captured in a CUDA graph, replayed between CUDA "
+                           "events; us_host_issued: the same launches issued one by one from Python; in_step: the "
+                           "step's 2 cast launches (X+W1+W2 fp32 in one, dY bf16; y only) back to back, K rounds, "
+                           "replayed from a CUDA graph",
+            "graph_step": graph_info,
+            "gemm_alone": heads,
+            "teblock_fwd_4mb": teblock,
+            "toy32_fwd": toy,
+            "e2e_api": "fp8_linear_refresh_weights + fp8_linear_fwd_ex/bwd_ex + fp8_update_scales, pinned host "
+                       "X/dY, double-buffered copies",
+        }
+        with open(args.detail, "w") as f:
+            json.dump(detail, f, indent=1)
     print(json.dumps(line))
 
 

@@ -63,6 +63,11 @@ class _Linear(ctypes.Structure):
                 ("workspace", _P), ("workspace_bytes", ctypes.c_size_t), ("w_noop_flag", _P)]
 
 
+class _CastJob(ctypes.Structure):
+    _fields_ = [("x", _P), ("x_dtype", _INT), ("rows", _I64), ("cols", _I64), ("fmt", _INT), ("scale", _P),
+                ("y", _P), ("yt", _P), ("amax", _P), ("scale_inv", _P), ("noop_flag", _P)]
+
+
 class _Fp8Io(ctypes.Structure):
     _fields_ = [("in_cast", _I32), ("out_meta", _I32), ("out8", _P), ("out8t", _P), ("out_scale_inv", _P)]
 
@@ -93,6 +98,10 @@ _SIGS = {
     "fp8_linear_bwd": [ctypes.POINTER(_Linear), ctypes.POINTER(_Meta), _P, _INT, _I64, _P, _P, _P,
                        _INT, _P, _P, _P, _P, _P],
     "fp8ds_device_status": [ctypes.POINTER(_I32), _I32],
+    "fp8_cast_transpose_amax_multi": [ctypes.POINTER(_CastJob), _I32, _P],
+    "fp8ds_test_stream_k_withhold": [_I32, ctypes.c_uint64],
+    "fp8_linear_refresh_weights": [ctypes.POINTER(ctypes.POINTER(_Linear)), _I32, ctypes.POINTER(_Meta),
+                                   ctypes.POINTER(_CastJob), _I32, _P],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -184,6 +193,33 @@ def fp8_cast_transpose_amax_pair(xa, xb, fmt, scale_a, ya, scale_b, yb, yt_a=Non
                                              _ptr(scale_inv_a), _ptr(xb), rb, cb, _ptr(scale_b), _ptr(yb),
                                              _ptr(yt_b), _ptr(amax_b), _ptr(scale_inv_b), _ptr(noop_b),
                                              _dtype(xa), _fmt(fmt), _stream(stream)))
+
+
+def cast_job(x, fmt, scale, y, yt=None, amax=None, scale_inv=None, noop_flag=None):
+    """One job record of fp8_cast_transpose_amax_multi / the extra casts of
+    fp8_linear_refresh_weights: the arguments of fp8_cast_transpose_amax_noop
+    (x 2-D; a 1-D x is cast as one row)."""
+    rows, cols = (x.shape[0], x.shape[1]) if x.dim() == 2 else (1, x.numel())
+    return _CastJob(_ptr(x), _dtype(x), rows, cols, _fmt(fmt), _ptr(scale), _ptr(y), _ptr(yt), _ptr(amax),
+                    _ptr(scale_inv), _ptr(noop_flag))
+
+
+def _job_array(jobs):
+    if isinstance(jobs, ctypes.Array):
+        return jobs
+    return (_CastJob * len(jobs))(*jobs) if len(jobs) else None
+
+
+def cast_jobs(jobs):
+    """A reusable job array (list of cast_job records -> ctypes array), so that
+    repeated calls skip the marshalling."""
+    return (_CastJob * len(jobs))(*jobs)
+
+
+def fp8_cast_transpose_amax_multi(jobs, stream=None):
+    """Many casts in one launch; jobs: cast_job records or a cast_jobs array."""
+    arr = _job_array(jobs)
+    _check(_lib.fp8_cast_transpose_amax_multi(arr, 0 if arr is None else len(arr), _stream(stream)))
 
 
 def fp8_cast_transpose_amax_dynamic(x, fmt, scale, y, yt=None, amax=None, scale_inv=None, stream=None):
@@ -311,6 +347,28 @@ class Fp8Linear:
 
     def invalidate_cache(self):
         self._c.cache_valid = 0
+
+
+class LinearGroup:
+    """Handles of several Fp8Linear layers as the C array that
+    fp8_linear_refresh_weights takes (built once, reused every step)."""
+
+    def __init__(self, lins):
+        self.lins = list(lins)
+        self._arr = (ctypes.POINTER(_Linear) * len(self.lins))(*[ctypes.pointer(l._c) for l in self.lins])
+
+    def __len__(self):
+        return len(self.lins)
+
+
+def fp8_linear_refresh_weights(lins, meta, extra=(), stream=None):
+    """Recast the FP8 weight caches of all `lins` (an LinearGroup or a list of
+    Fp8Linear) and the `extra` casts (cast_job records or a cast_jobs array)
+    in one launch; the forwards that follow pass is_first_microbatch=False."""
+    group = lins if isinstance(lins, LinearGroup) else LinearGroup(lins)
+    ex = _job_array(extra)
+    _check(_lib.fp8_linear_refresh_weights(group._arr, len(group), ctypes.byref(meta._c), ex,
+                                           0 if ex is None else len(ex), _stream(stream)))
 
 
 def fp8_linear_fwd(lin, meta, x, y, is_first_microbatch, x8, x8t=None, x_scale_inv=None,

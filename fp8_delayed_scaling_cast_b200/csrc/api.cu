@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "fp8ds_internal.h"
 
@@ -212,6 +213,29 @@ fp8ds_status fp8_cast_transpose_amax_pair(const void *x_a, int64_t rows_a, int64
                                                   rows_b, cols_b, scale_b, y_b, yt_b, amax_b, scale_inv_b, noop_b,
                                                   x_dtype, fmt, stream),
                        "fp8_cast_transpose_amax_pair");
+}
+
+// Checks of one job of a multi-tensor cast (the message names the job).
+static fp8ds_status check_cast_job(const char *fn, const fp8ds_cast_job &j, int32_t i) {
+    char what[96];
+    snprintf(what, sizeof what, "%s (job %d)", fn, static_cast<int>(i));
+    fp8ds_status st = check_cast(what, j.x, j.x_dtype, j.rows, j.cols, j.fmt, j.scale, j.y);
+    if (st != FP8DS_OK) return st;
+    if (j.yt != nullptr && (j.rows >= (int64_t(1) << 31) || j.cols >= (int64_t(1) << 31)))
+        return invalid("%s: rows and cols must be below 2^31 with a transpose", what);
+    return FP8DS_OK;
+}
+
+fp8ds_status fp8_cast_transpose_amax_multi(const fp8ds_cast_job *jobs, int32_t num_jobs, fp8ds_stream stream) {
+    clear_error();
+    if (num_jobs < 0) return invalid("fp8_cast_transpose_amax_multi: num_jobs < 0");
+    if (num_jobs > 0 && jobs == nullptr) return invalid("fp8_cast_transpose_amax_multi: jobs must not be NULL");
+    for (int32_t i = 0; i < num_jobs; ++i) {
+        fp8ds_status st = check_cast_job("fp8_cast_transpose_amax_multi", jobs[i], i);
+        if (st != FP8DS_OK) return st;
+    }
+    if (num_jobs == 0) return FP8DS_OK;
+    return cuda_status(launch_cast_multi(jobs, num_jobs, stream), "fp8_cast_transpose_amax_multi");
 }
 
 fp8ds_status fp8_cast_transpose_amax_dynamic(const void *x, fp8ds_dtype x_dtype, int64_t rows, int64_t cols,
@@ -474,6 +498,48 @@ fp8ds_status fp8_linear_fwd_ex(fp8ds_linear *lin, const fp8ds_meta *meta, const 
                       x_scale_inv, io, stream);
 }
 
+fp8ds_status fp8_linear_refresh_weights(fp8ds_linear *const *lins, int32_t num_lins, const fp8ds_meta *meta,
+                                        const fp8ds_cast_job *extra, int32_t num_extra, fp8ds_stream stream) {
+    clear_error();
+    const char *fn = "fp8_linear_refresh_weights";
+    if (num_lins < 0 || num_extra < 0) return invalid("%s: negative count", fn);
+    if ((num_lins > 0 && lins == nullptr) || (num_extra > 0 && extra == nullptr))
+        return invalid("%s: NULL array", fn);
+    std::vector<fp8ds_cast_job> jobs;
+    jobs.reserve(static_cast<size_t>(num_lins) + static_cast<size_t>(num_extra));
+    for (int32_t i = 0; i < num_lins; ++i) {
+        const fp8ds_linear *lin = lins[i];
+        if (lin == nullptr || lin->w == nullptr || lin->w8 == nullptr || lin->w_scale_inv == nullptr)
+            return invalid("%s: incomplete linear handle %d", fn, static_cast<int>(i));
+        fp8ds_status st = check_meta(fn, meta, lin->meta_w);
+        if (st != FP8DS_OK) return st;
+        fp8ds_cast_job j;
+        j.x = lin->w;
+        j.x_dtype = FP8DS_F32;
+        j.rows = lin->out_features;
+        j.cols = lin->in_features;
+        j.fmt = FP8DS_E4M3;
+        j.scale = meta->scale + lin->meta_w;
+        j.y = lin->w8;
+        j.yt = lin->w8t;
+        j.amax = meta->amax_history + lin->meta_w;
+        j.scale_inv = lin->w_scale_inv;
+        j.noop_flag = lin->w_noop_flag;
+        if ((st = check_cast_job(fn, j, i)) != FP8DS_OK) return st;
+        jobs.push_back(j);
+    }
+    for (int32_t i = 0; i < num_extra; ++i) {
+        fp8ds_status st = check_cast_job(fn, extra[i], num_lins + i);
+        if (st != FP8DS_OK) return st;
+        jobs.push_back(extra[i]);
+    }
+    if (jobs.empty()) return FP8DS_OK;
+    fp8ds_status st = cuda_status(launch_cast_multi(jobs.data(), static_cast<int32_t>(jobs.size()), stream), fn);
+    if (st != FP8DS_OK) return st;
+    for (int32_t i = 0; i < num_lins; ++i) lins[i]->cache_valid = 1;
+    return FP8DS_OK;
+}
+
 fp8ds_status fp8_linear_bwd(const fp8ds_linear *lin, const fp8ds_meta *meta, const void *dy, fp8ds_dtype dy_dtype,
                             int64_t m, const uint8_t *x8t, const float *x_scale_inv, void *dx, fp8ds_dtype dx_dtype,
                             float *dw, uint8_t *dy8, uint8_t *dy8t, float *dy_scale_inv, fp8ds_stream stream) {
@@ -497,6 +563,12 @@ fp8ds_status fp8ds_device_status(int32_t *code_out, int32_t clear) {
     clear_error();
     if (code_out == nullptr) return invalid("fp8ds_device_status: code_out must not be NULL");
     return cuda_status(read_device_error(code_out, clear != 0), "fp8ds_device_status");
+}
+
+fp8ds_status fp8ds_test_stream_k_withhold(int32_t withhold, uint64_t wait_ns) {
+    clear_error();
+    set_stream_k_withhold(withhold != 0 ? 1 : 0, static_cast<unsigned long long>(wait_ns));
+    return FP8DS_OK;
 }
 
 const char *fp8ds_version(void) { return "fp8ds 0.1.0 (sm_100a)"; }

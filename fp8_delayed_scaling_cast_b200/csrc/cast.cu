@@ -553,6 +553,229 @@ quantize_kernel(const T *__restrict__ x, int64_t n, const float *__restrict__ sc
     block_amax_commit<Q_THREADS>(m, amax);
 }
 
+// ------------------------------------------------ many tensors, one launch --
+
+// Up to MC_MAX_JOBS tensors of any input dtype, FP8 format and shape, with or
+// without transpose, cast in one launch ("[PyTorch] Refactor FP8 workspaces
+// in linear modules": the weight workspaces of every linear refreshed
+// together; "CPU Overhead of te.Linear FP8 Layers": per-tensor launches are
+// the overhead to remove).  The job list travels by value in the kernel
+// parameters, so a captured CUDA graph replays it unchanged.
+//
+// Work units ("tiles") are numbered job after job.  A job without transpose
+// is a flat array cut into tiles of 16 KB of input: each of the 256 threads
+// issues four coalesced 16-byte loads (a warp reads 512 contiguous bytes per
+// load), then casts and stores their codes.  A job with transpose uses the
+// 128 x 64 tiles and the shared-memory transpose of cast_transpose_kernel.
+// CTA c of G takes the contiguous tile range [c*T/G, (c+1)*T/G), so it meets
+// each job in one stretch: its amax is reduced across the CTA and max-ed into
+// the job's amax once per stretch.
+constexpr int MC_THREADS = 256;
+constexpr int MC_LOADS = 4;                                  // 16-byte loads per thread and flat tile
+constexpr int MC_FLAT_BYTES = MC_THREADS * MC_LOADS * 16;    // input bytes per flat tile
+constexpr int MC_MAX_JOBS = 256;
+
+enum : uint32_t {
+    MC_BF16 = 1u,    // input bf16 (else fp32)
+    MC_E5M2 = 2u,    // output e5m2 (else e4m3)
+    MC_T = 4u,       // writes the transpose (2-D tiles)
+    MC_VEC = 8u,     // 16-byte vector path allowed (alignment and shape)
+};
+
+struct MultiJob {
+    const void *x;
+    uint8_t *y, *yt;
+    const float *scale;
+    float *amax, *scale_inv;
+    const int32_t *noop;
+    int64_t n;            // elements (rows * cols)
+    int32_t rows, cols;   // 2-D shape (transpose jobs)
+    uint32_t tile0;       // first tile of this job in the launch
+    uint32_t tiles_c;     // column tiles (transpose jobs)
+    uint32_t kind;        // MC_* bits
+};
+
+struct MultiParams {
+    MultiJob jobs[MC_MAX_JOBS];
+    int32_t num_jobs;
+    uint32_t total_tiles;
+};
+
+// Flat tile `lt` of a job without transpose.
+template <typename T, int FMT>
+__device__ __forceinline__ void mc_flat_tile(const MultiJob &J, uint32_t lt, float s, float &m) {
+    constexpr int PER16 = 16 / static_cast<int>(sizeof(T));           // elements per 16-byte load
+    constexpr int64_t TILE = MC_FLAT_BYTES / static_cast<int>(sizeof(T));
+    const int64_t base = static_cast<int64_t>(lt) * TILE;
+    const T *x = static_cast<const T *>(J.x);
+    const int tid = threadIdx.x;
+    if ((J.kind & MC_VEC) && base + TILE <= J.n) {
+        uint4 v[MC_LOADS];
+#pragma unroll
+        for (int k = 0; k < MC_LOADS; ++k)
+            v[k] = __ldg(reinterpret_cast<const uint4 *>(x + base) + k * MC_THREADS + tid);
+#pragma unroll
+        for (int k = 0; k < MC_LOADS; ++k) {
+            const int64_t e = base + static_cast<int64_t>(k * MC_THREADS + tid) * PER16;
+            if constexpr (sizeof(T) == 4) {
+                *reinterpret_cast<uint32_t *>(J.y + e) =
+                    cast4<FMT>(__uint_as_float(v[k].x), __uint_as_float(v[k].y), __uint_as_float(v[k].z),
+                               __uint_as_float(v[k].w), s, m);
+            } else {
+                *reinterpret_cast<uint2 *>(J.y + e) = Load8<uint16_t, FMT>::cast(v[k], s, m);
+            }
+        }
+    } else {
+        const int64_t end = base + TILE < J.n ? base + TILE : J.n;
+        for (int64_t i = base + tid; i < end; i += MC_THREADS) {
+            const float v = InElem<T>::load(x + i);
+            m = fmaxf(m, fabsf(v));
+            J.y[i] = static_cast<uint8_t>(cvt1<FMT>(__fmul_rn(v, s)));
+        }
+    }
+}
+
+// 128 x 64 tile `lt` of a job with transpose (the algorithm of
+// cast_transpose_kernel: 16-byte loads for interior tiles of aligned tensors,
+// element-wise otherwise; tsm is the CTA's padded transpose tile).  Every
+// thread of the CTA calls it (it contains block barriers).
+template <typename T, int FMT>
+__device__ __forceinline__ void mc_transpose_tile(const MultiJob &J, uint32_t lt, float s, float &m,
+                                                  uint32_t *tsm) {
+    const int tid = threadIdx.x;
+    const int64_t rows = J.rows, cols = J.cols;
+    const int64_t r0 = static_cast<int64_t>(lt / J.tiles_c) * CT_ROWS;
+    const int64_t c0 = static_cast<int64_t>(lt % J.tiles_c) * CT_COLS;
+    const T *x = static_cast<const T *>(J.x);
+    if ((J.kind & MC_VEC) && r0 + CT_ROWS <= rows && c0 + CT_COLS <= cols) {
+        const int cc = tid & 7, rg = tid >> 3;
+        using Raw = decltype(Load8<T, FMT>::raw(x));
+        Raw buf[4];
+        const T *xp = x + (r0 + 4 * rg) * cols + c0 + 8 * cc;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) buf[i] = Load8<T, FMT>::raw(xp + i * cols);
+        uint2 w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = Load8<T, FMT>::cast(buf[i], s, m);
+        uint8_t *yp = J.y + (r0 + 4 * rg) * cols + c0 + 8 * cc;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint2 *>(yp + i * cols) = w[i];
+        // 4 rows x 8 bytes -> 8 column words of 4 rows each
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t a0 = h ? w[0].y : w[0].x, a1 = h ? w[1].y : w[1].x;
+            const uint32_t a2 = h ? w[2].y : w[2].x, a3 = h ? w[3].y : w[3].x;
+            const uint32_t p01l = __byte_perm(a0, a1, 0x5140);
+            const uint32_t p01h = __byte_perm(a0, a1, 0x7362);
+            const uint32_t p23l = __byte_perm(a2, a3, 0x5140);
+            const uint32_t p23h = __byte_perm(a2, a3, 0x7362);
+            uint32_t *tw = tsm + (8 * cc + 4 * h) * CT_TSTRIDE + rg;
+            tw[0 * CT_TSTRIDE] = __byte_perm(p01l, p23l, 0x5410);
+            tw[1 * CT_TSTRIDE] = __byte_perm(p01l, p23l, 0x7632);
+            tw[2 * CT_TSTRIDE] = __byte_perm(p01h, p23h, 0x5410);
+            tw[3 * CT_TSTRIDE] = __byte_perm(p01h, p23h, 0x7632);
+        }
+        __syncthreads();
+        // 64 columns x 8 chunks of 16 rows; 2 chunks per thread
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int idx = tid + MC_THREADS * k;
+            const int c = idx >> 3, q = idx & 7;
+            const uint32_t *tp = tsm + c * CT_TSTRIDE + 4 * q;
+            *reinterpret_cast<uint4 *>(J.yt + (c0 + c) * rows + r0 + 16 * q) = make_uint4(tp[0], tp[1], tp[2], tp[3]);
+        }
+        __syncthreads();
+    } else {
+        uint8_t *tsm8 = reinterpret_cast<uint8_t *>(tsm);
+        for (int i = 0; i < (CT_ROWS * CT_COLS) / MC_THREADS; ++i) {
+            const int e = tid + MC_THREADS * i;
+            const int r = e / CT_COLS, c = e % CT_COLS;
+            const int64_t gr = r0 + r, gc = c0 + c;
+            uint32_t code = 0;
+            if (gr < rows && gc < cols) {
+                const float v = InElem<T>::load(x + gr * cols + gc);
+                m = fmaxf(m, fabsf(v));
+                code = cvt1<FMT>(__fmul_rn(v, s));
+                J.y[gr * cols + gc] = static_cast<uint8_t>(code);
+            }
+            tsm8[c * (CT_TSTRIDE * 4) + r] = static_cast<uint8_t>(code);
+        }
+        __syncthreads();
+        for (int i = 0; i < (CT_ROWS * CT_COLS) / MC_THREADS; ++i) {
+            const int e = tid + MC_THREADS * i;
+            const int c = e / CT_ROWS, r = e % CT_ROWS;
+            const int64_t gr = r0 + r, gc = c0 + c;
+            if (gr < rows && gc < cols) J.yt[gc * rows + gr] = tsm8[c * (CT_TSTRIDE * 4) + r];
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(MC_THREADS)
+cast_multi_kernel(const __grid_constant__ MultiParams p) {
+    __shared__ uint32_t tsm[CT_COLS * CT_TSTRIDE];
+    ptx::pdl_wait();
+    ptx::pdl_launch_dependents();
+    const int tid = threadIdx.x;
+    // Jobs with no elements own no tile: their scale_inv is written here.
+    if (blockIdx.x == 0 && tid == 0) {
+        for (int j = 0; j < p.num_jobs; ++j) {
+            const MultiJob &J = p.jobs[j];
+            if (J.n == 0 && J.scale_inv != nullptr && !(J.noop != nullptr && __ldg(J.noop) != 0))
+                *J.scale_inv = __frcp_rn(__ldg(J.scale));
+        }
+    }
+    const uint64_t T = p.total_tiles;
+    const uint32_t t_begin = static_cast<uint32_t>(T * blockIdx.x / gridDim.x);
+    const uint32_t t_end = static_cast<uint32_t>(T * (blockIdx.x + 1) / gridDim.x);
+    if (t_begin >= t_end) return;
+    // the last job whose first tile is at or before t_begin (jobs[0].tile0 = 0)
+    int lo = 0, hi = p.num_jobs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.jobs[mid].tile0 <= t_begin)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    int j = lo;
+    float m = 0.0f, s = 0.0f;
+    int cur = -1;
+    bool skip = true;
+    for (uint32_t t = t_begin; t < t_end; ++t) {
+        while (j + 1 < p.num_jobs && p.jobs[j + 1].tile0 <= t) ++j;
+        if (j != cur) {
+            // the CTA leaves job `cur`: one reduction and one atomic for its stretch
+            if (cur >= 0 && !skip) {
+                block_amax_commit<MC_THREADS>(m, p.jobs[cur].amax);
+                __syncthreads();   // the reduction buffer is free again
+            }
+            m = 0.0f;
+            cur = j;
+            const MultiJob &J = p.jobs[j];
+            skip = J.noop != nullptr && __ldg(J.noop) != 0;
+            if (!skip) {
+                s = __ldg(J.scale);
+                if (t == J.tile0 && tid == 0 && J.scale_inv != nullptr) *J.scale_inv = __frcp_rn(s);
+            }
+        }
+        if (skip) continue;
+        const MultiJob &J = p.jobs[j];
+        const uint32_t lt = t - J.tile0;
+        switch (J.kind & (MC_BF16 | MC_E5M2 | MC_T)) {
+            case 0: mc_flat_tile<float, FP8DS_E4M3>(J, lt, s, m); break;
+            case MC_E5M2: mc_flat_tile<float, FP8DS_E5M2>(J, lt, s, m); break;
+            case MC_BF16: mc_flat_tile<uint16_t, FP8DS_E4M3>(J, lt, s, m); break;
+            case MC_BF16 | MC_E5M2: mc_flat_tile<uint16_t, FP8DS_E5M2>(J, lt, s, m); break;
+            case MC_T: mc_transpose_tile<float, FP8DS_E4M3>(J, lt, s, m, tsm); break;
+            case MC_T | MC_E5M2: mc_transpose_tile<float, FP8DS_E5M2>(J, lt, s, m, tsm); break;
+            case MC_T | MC_BF16: mc_transpose_tile<uint16_t, FP8DS_E4M3>(J, lt, s, m, tsm); break;
+            default: mc_transpose_tile<uint16_t, FP8DS_E5M2>(J, lt, s, m, tsm); break;
+        }
+    }
+    if (cur >= 0 && !skip) block_amax_commit<MC_THREADS>(m, p.jobs[cur].amax);
+}
+
 // -------------------------------------------------------------- launchers --
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -834,6 +1057,71 @@ cudaError_t launch_transpose_u8(const uint8_t *y, int64_t rows, int64_t cols, ui
     auto kernel = transpose_u8_kernel<false>;
     return launch_pdl(kernel, dim3(grid_for(kernel, TR_THREADS, num_tiles)), dim3(TR_THREADS), 0, stream, 1, y, rows,
                       cols, yt, tiles_c, num_tiles);
+}
+
+cudaError_t launch_cast_multi(const fp8ds_cast_job *jobs, int32_t num_jobs, cudaStream_t stream) {
+    static std::atomic<int> per_sm[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    int n_sm = per_sm[dev].load(std::memory_order_relaxed);
+    if (n_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n_sm, cast_multi_kernel, MC_THREADS, 0) != cudaSuccess ||
+            n_sm < 1)
+            n_sm = 1;
+        per_sm[dev].store(n_sm, std::memory_order_relaxed);
+    }
+    const int64_t cap = static_cast<int64_t>(num_sms()) * n_sm;
+    int32_t done = 0;
+    while (done < num_jobs) {
+        MultiParams P;
+        uint64_t tiles = 0;
+        int32_t cnt = 0;
+        while (done + cnt < num_jobs && cnt < MC_MAX_JOBS) {
+            const fp8ds_cast_job &c = jobs[done + cnt];
+            const bool bf16 = c.x_dtype == FP8DS_BF16;
+            const bool tr = c.yt != nullptr;
+            const int64_t n = c.rows * c.cols;
+            uint64_t jt = 0, tiles_c = 0;
+            bool vec;
+            if (tr) {
+                tiles_c = static_cast<uint64_t>((c.cols + CT_COLS - 1) / CT_COLS);
+                jt = tiles_c * static_cast<uint64_t>((c.rows + CT_ROWS - 1) / CT_ROWS);
+                vec = aligned16(c.x) && aligned16(c.y) && aligned16(c.yt) && c.cols % 8 == 0 && c.rows % 16 == 0;
+            } else {
+                const int64_t per_tile = MC_FLAT_BYTES / (bf16 ? 2 : 4);
+                jt = static_cast<uint64_t>((n + per_tile - 1) / per_tile);
+                vec = aligned16(c.x) && aligned16(c.y);
+            }
+            if (tiles + jt > 0xFFFFFFFFull) break;   // next launch
+            MultiJob &J = P.jobs[cnt];
+            J.x = c.x;
+            J.y = c.y;
+            J.yt = c.yt;
+            J.scale = c.scale;
+            J.amax = c.amax;
+            J.scale_inv = c.scale_inv;
+            J.noop = c.noop_flag;
+            J.n = n;
+            J.rows = static_cast<int32_t>(tr ? c.rows : 0);
+            J.cols = static_cast<int32_t>(tr ? c.cols : 0);
+            J.tile0 = static_cast<uint32_t>(tiles);
+            J.tiles_c = static_cast<uint32_t>(tiles_c);
+            J.kind = (bf16 ? MC_BF16 : 0u) | (c.fmt == FP8DS_E5M2 ? MC_E5M2 : 0u) | (tr ? MC_T : 0u) |
+                     (vec ? MC_VEC : 0u);
+            tiles += jt;
+            ++cnt;
+        }
+        if (cnt == 0) return cudaErrorInvalidValue;   // one job alone exceeds 2^32 tiles
+        P.num_jobs = cnt;
+        P.total_tiles = static_cast<uint32_t>(tiles);
+        const int64_t g = static_cast<int64_t>(tiles) < cap ? static_cast<int64_t>(tiles) : cap;
+        cudaError_t e = launch_pdl(cast_multi_kernel, dim3(static_cast<unsigned>(g < 1 ? 1 : g)), dim3(MC_THREADS), 0,
+                                   stream, 1, P);
+        if (e != cudaSuccess) return e;
+        done += cnt;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t read_cast_error(int32_t *out, bool clear) {

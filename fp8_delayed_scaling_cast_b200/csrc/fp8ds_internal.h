@@ -48,6 +48,10 @@ cudaError_t launch_cast_transpose_dynamic(const void *x, fp8ds_dtype x_dtype, in
                                           fp8ds_format fmt, float *scale, uint8_t *y, uint8_t *yt, float *amax,
                                           float *scale_inv, cudaStream_t stream);
 
+// Up to 256 casts per launch (more: consecutive launches); jobs validated by
+// the caller (a transpose job needs rows, cols < 2^31).
+cudaError_t launch_cast_multi(const fp8ds_cast_job *jobs, int32_t num_jobs, cudaStream_t stream);
+
 // yt[c, r] = y[r, c] for a uint8 tensor [rows, cols].
 cudaError_t launch_transpose_u8(const uint8_t *y, int64_t rows, int64_t cols, uint8_t *yt, cudaStream_t stream);
 
@@ -87,6 +91,9 @@ fp8ds_status launch_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const flo
                                  const uint8_t *b, fp8ds_format b_fmt, const float *b_scale_inv,
                                  const void *bias, fp8ds_dtype bias_dtype, void *d, fp8ds_dtype d_dtype,
                                  int64_t m, int64_t n, int64_t k, cudaStream_t stream);
+
+// Error-path test setting of the stream-K GEMM (fp8ds_test_stream_k_withhold).
+void set_stream_k_withhold(int withhold, unsigned long long wait_ns);
 
 // Device error words written by kernels whose bounded waits give up (one per
 // translation unit); read_device_error returns the first non-zero one.

@@ -77,6 +77,12 @@ constexpr int TMEM_COLS = 512; // two accumulators
 #ifndef FP8DS_EPI_BOXES
 #define FP8DS_EPI_BOXES 1
 #endif
+// FP8DS_EPI_DIRECT: the epilogue stores D from registers with 32-byte
+// global stores (no shared-memory staging, no TMA store).
+#ifndef FP8DS_EPI_DIRECT
+#define FP8DS_EPI_DIRECT 0
+#endif
+constexpr bool EPI_DIRECT = FP8DS_EPI_DIRECT != 0;
 constexpr int EPI_LD = FP8DS_EPI_LD;
 constexpr int EPI_NBOX = FP8DS_EPI_BOXES;
 static_assert(EPI_LD == 32 || EPI_LD == 64, "TMEM load width must be 32 or 64 columns");
@@ -426,6 +432,12 @@ struct Params {
     float *out_amax;       // NULL or atomic-max target
     float *out_scale_inv;  // NULL or fl32(1 / out_scale)
     uint8_t *out_d8;       // [M, N] codes
+    // limit of the wait for another pair's partial sum, and (tests of the
+    // error path only) whether split tiles withhold their publication
+    unsigned long long partial_wait_ns;
+    int32_t withhold_partials;
+    void *out;             // D (fp32 / bf16 output) for the direct-store epilogue
+    int32_t out_v8;        // D and its row pitch are 32-byte aligned (32-byte stores)
     uint8_t *out_d8t;      // [N, M] codes or NULL
     int32_t out_fmt;
 };
@@ -570,11 +582,39 @@ __device__ __forceinline__ float4 bias4(const float *bs) {
     return BIAS ? *reinterpret_cast<const float4 *>(bs) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
+__device__ __forceinline__ void st_global_v8(void *p, const uint32_t *w) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
+// 32 columns of row m of D (bf16: 16 words, fp32: 32 words) from registers,
+// clipped at N (a multiple of 8 (bf16) or 4 (fp32): 16-byte granules are
+// wholly inside or outside).
+template <bool OUT_BF16>
+__device__ __forceinline__ void store_row_direct(void *out, int32_t m, int64_t n0, int32_t m_total, int32_t n_total,
+                                                 bool v8, const uint32_t *w) {
+    constexpr int WORDS = OUT_BF16 ? 16 : 32;
+    constexpr int COLS_PER_16B = OUT_BF16 ? 8 : 4;
+    if (m >= m_total || n0 >= n_total) return;
+    uint8_t *dst = static_cast<uint8_t *>(out) + (static_cast<int64_t>(m) * n_total + n0) * (OUT_BF16 ? 2 : 4);
+    if (v8 && n0 + 32 <= n_total) {
+#pragma unroll
+        for (int g = 0; g < WORDS / 8; ++g) st_global_v8(dst + 32 * g, w + 8 * g);
+    } else {
+#pragma unroll
+        for (int g = 0; g < WORDS / 4; ++g)
+            if (n0 + g * COLS_PER_16B < n_total)
+                *reinterpret_cast<uint4 *>(dst + 16 * g) = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+    }
+}
+
 template <bool OUT_BF16, bool BIAS>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *boxes, int &nbox, int half,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                               float sab, const float *bias_s, uint32_t empty_bar_cluster,
-                                              bool arrive, int mode, float *slot, int h, int q) {
+                                              bool arrive, int mode, float *slot, int h, int q, void *out,
+                                              int32_t m_total, int32_t n_total, bool v8) {
     constexpr int SUBS_PER_BOX = OUT_BF16 ? 2 : 1;  // 32-column sub-blocks per staging box
     constexpr int CHUNKS = ACC_N / 2 / EPI_LD;      // TMEM loads per warp and row block
     constexpr int SUBS = EPI_LD / 32;               // 32-column sub-blocks per load
@@ -596,7 +636,34 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             const int hh = (col0 / 32) % SUBS_PER_BOX;
             const bool last_of_chunk = sb == SUBS - 1;
             if (mode != 0) partial_io(mode, rr, slot, h, q, col0, lane);
-            if (mode != 1) {
+            if (EPI_DIRECT && mode != 1) {
+                const float *bs = bias_s + col0;
+                if (OUT_BF16) {
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float4 b = bias4<BIAS>(bs + 4 * j);
+                        __nv_bfloat162 ha = __floats2bfloat162_rn(fmaf(__uint_as_float(rr[4 * j]), sab, b.x),
+                                                                  fmaf(__uint_as_float(rr[4 * j + 1]), sab, b.y));
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(rr[4 * j + 2]), sab, b.z),
+                                                                  fmaf(__uint_as_float(rr[4 * j + 3]), sab, b.w));
+                        packed[2 * j] = *reinterpret_cast<uint32_t *>(&ha);
+                        packed[2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
+                    }
+                    store_row_direct<true>(out, m_row0 + lane, n_base + col0, m_total, n_total, v8, packed);
+                } else {
+                    uint32_t v[32];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const float4 b = bias4<BIAS>(bs + 4 * k);
+                        v[4 * k] = __float_as_uint(fmaf(__uint_as_float(rr[4 * k]), sab, b.x));
+                        v[4 * k + 1] = __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 1]), sab, b.y));
+                        v[4 * k + 2] = __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 2]), sab, b.z));
+                        v[4 * k + 3] = __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 3]), sab, b.w));
+                    }
+                    store_row_direct<false>(out, m_row0 + lane, n_base + col0, m_total, n_total, v8, v);
+                }
+            } else if (mode != 1) {
                 uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
                 if (hh == 0) {
                     // Staging buffer reuse: the store issued from this box
@@ -641,7 +708,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             }
             // the registers of r are free: start the next chunk's TMEM load
             if (last_of_chunk && c + 1 < CHUNKS) tmem_ld(t_row + half * (ACC_N / 2) + (c + 1) * EPI_LD, r);
-            if (mode != 1 && hh == SUBS_PER_BOX - 1) {
+            if (!EPI_DIRECT && mode != 1 && hh == SUBS_PER_BOX - 1) {
                 uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
                 fence_async_smem();
                 __syncwarp();
@@ -726,7 +793,7 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
     // Without the transpose the warp's 32 rows x 128 code bytes are one
     // 128-byte-swizzled staging box and one TMA store; with it, the codes go
     // out with plain stores beside the transposed ones (in box 0's memory).
-    const bool staged = d8t == nullptr;
+    const bool staged = !EPI_DIRECT && d8t == nullptr;
     uint8_t *box = staged ? boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES : boxes;
     if (staged && mode != 1) {
         if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
@@ -896,7 +963,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             // The other cluster wrote this partial at the start of its range.
             const uint64_t t0 = globaltimer();
             while (ld_acquire(flag) != static_cast<int32_t>(p.epoch)) {
-                if (*sm.abort_flag || globaltimer() - t0 > TIMEOUT_NS) {
+                if (*sm.abort_flag || globaltimer() - t0 > p.partial_wait_ns) {
                     *sm.abort_flag = 1;
                     record_error(SITE_EPI_PARTIAL);
                     ok = false;
@@ -934,10 +1001,12 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             } else {
                 if (p.bias_kind != 0)
                     epilogue_tile<OUT == OUT_BF16, true>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab, bias_s,
-                                                         empty_addr, release, mode, slot, h, q);
+                                                         empty_addr, release, mode, slot, h, q, p.out, p.M, p.N,
+                                                         p.out_v8 != 0);
                 else
-                    epilogue_tile<OUT == OUT_BF16, false>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab, bias_s,
-                                                          empty_addr, release, mode, slot, h, q);
+                    epilogue_tile<OUT == OUT_BF16, false>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab,
+                                                          bias_s, empty_addr, release, mode, slot, h, q, p.out, p.M,
+                                                          p.N, p.out_v8 != 0);
             }
         }
         if (mode == 1) {
@@ -945,7 +1014,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             epilogue_bar();
             if (epi_tid == 0) {
                 __threadfence();
-                st_release(flag, static_cast<int32_t>(p.epoch));
+                if (!p.withhold_partials) st_release(flag, static_cast<int32_t>(p.epoch));
             }
         } else if (mode == 2) {
             epilogue_bar();
@@ -1433,6 +1502,10 @@ size_t gemm_workspace_bytes() {
 
 namespace {
 
+// Error-path test setting (fp8ds_test_stream_k_withhold).
+std::atomic<int> g_test_withhold{0};
+std::atomic<unsigned long long> g_test_wait_ns{0};
+
 // Tile schedule of a GEMM on the current device: kernel (one CTA or a CTA
 // pair), pair-tile rows, tile count, and whether a workspace turns it into
 // the stream-K schedule.
@@ -1527,6 +1600,15 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.out_fmt = cast != nullptr ? static_cast<int32_t>(cast->fmt) : 0;
     p.out_d8 = cast != nullptr ? static_cast<uint8_t *>(d) : nullptr;
     p.out_d8t = cast != nullptr ? cast->d8t : nullptr;
+    p.partial_wait_ns = TIMEOUT_NS;
+    p.withhold_partials = 0;
+    if (g_test_withhold.load(std::memory_order_relaxed) != 0) {
+        p.withhold_partials = 1;
+        const unsigned long long w = g_test_wait_ns.load(std::memory_order_relaxed);
+        if (w != 0) p.partial_wait_ns = w;
+    }
+    p.out = d;
+    p.out_v8 = (reinterpret_cast<uintptr_t>(d) % 32 == 0) && (n * (out == OUT_F32 ? 4 : 2)) % 32 == 0;
     if (plan.stream_k && workspace != nullptr && workspace_bytes >= gemm_workspace_bytes()) {
         static std::atomic<uint32_t> launches{0};
         uint32_t e = ++launches;
@@ -1621,6 +1703,11 @@ fp8ds_status launch_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const flo
     }
     return launch_gemm(a, a_fmt, a_scale_inv, b, b_fmt, b_scale_inv, bias, bias_dtype, d, d_dtype, m, n, k, ws,
                        NOALLOC_SCRATCH_BYTES, stream);
+}
+
+void set_stream_k_withhold(int withhold, unsigned long long wait_ns) {
+    g_test_wait_ns.store(wait_ns, std::memory_order_relaxed);
+    g_test_withhold.store(withhold, std::memory_order_relaxed);
 }
 
 cudaError_t read_gemm_error(int32_t *out, bool clear) {

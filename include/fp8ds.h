@@ -156,6 +156,47 @@ fp8ds_status fp8_cast_transpose_amax_pair(const void *x_a, int64_t rows_a, int64
                                           fp8ds_dtype x_dtype, fp8ds_format fmt, fp8ds_stream stream);
 
 /*
+ * One tensor of fp8_cast_transpose_amax_multi: the arguments of
+ * fp8_cast_transpose_amax_noop gathered in a struct (host memory; the
+ * pointers inside are device pointers).
+ */
+typedef struct {
+    const void *x;             /* [rows, cols] row-major input (x_dtype) */
+    fp8ds_dtype x_dtype;
+    int64_t rows;
+    int64_t cols;
+    fp8ds_format fmt;
+    const float *scale;        /* [1] fp32, read on the device */
+    uint8_t *y;                /* [rows, cols] FP8 codes */
+    uint8_t *yt;               /* [cols, rows] FP8 transpose, or NULL */
+    float *amax;               /* [1] atomic-max target, or NULL */
+    float *scale_inv;          /* [1] private scale_inv, or NULL */
+    const int32_t *noop_flag;  /* device int32 or NULL: non-zero at run time skips this tensor */
+} fp8ds_cast_job;
+
+/*
+ * fp8_cast_transpose_amax_multi -- many independent casts in one kernel
+ * launch [TE820: the FP8 weight workspaces of all linears refreshed together
+ * ("fewer kernel launches"); TE761: the CPU time of launching per-tensor
+ * kernels is the overhead to remove].  Job i gives exactly the bytes of
+ * fp8_cast_transpose_amax_noop(jobs[i].x, ..., jobs[i].noop_flag) (the plain
+ * call when noop_flag is NULL): y, yt, the amax max-ed into *amax and
+ * *scale_inv.  Jobs may mix input dtypes, formats, shapes and transpose or
+ * none; a job with no elements only writes its scale_inv.
+ *   jobs      host array of num_jobs job records (read during the call only;
+ *             the job list is copied into the launch, so a captured CUDA graph
+ *             replays it).
+ * Up to 256 jobs go into one launch; a longer list is split into consecutive
+ * launches of up to 256.  Outputs of different jobs must not overlap (amax /
+ * scale_inv targets may be shared only if their combined effect is wanted).
+ * Errors: FP8DS_ERR_INVALID_ARG for num_jobs < 0, a NULL jobs array, any job
+ * that fp8_cast_transpose_amax would reject, or a job with a transpose whose
+ * rows or cols reach 2^31; nothing is enqueued then.
+ */
+fp8ds_status fp8_cast_transpose_amax_multi(const fp8ds_cast_job *jobs, int32_t num_jobs,
+                                           fp8ds_stream stream);
+
+/*
  * fp8_cast_transpose_amax_dynamic -- dynamic scaling, for comparison with the
  * delayed recipe [F8E312: delayed vs dynamic scaling; "delayed scaling is
  * theoretically faster than dynamic scaling (less memory reads)" is the
@@ -427,6 +468,27 @@ fp8ds_status fp8_linear_fwd(fp8ds_linear *lin, const fp8ds_meta *meta, const voi
                             float *x_scale_inv, fp8ds_stream stream);
 
 /*
+ * fp8_linear_refresh_weights -- refresh the FP8 weight caches of many linears
+ * in one launch [TE820: one weight workspace per linear, refreshed when
+ * is_first_microbatch is True or None; TE761: per-linear launch overhead].
+ * For every lins[i]: cast w -> w8 (and w8t if not NULL) in e4m3 with
+ * meta.scale[meta_w], amax into amax_history[0, meta_w], private scale_inv
+ * into *w_scale_inv (honouring w_noop_flag), exactly as fp8_linear_fwd's
+ * weight cast, then set cache_valid = 1.  The forwards that follow pass
+ * is_first_microbatch = 0 to use the refreshed caches.  `extra` (may be NULL
+ * with num_extra = 0) lists further casts of the same launch, e.g. a layer's
+ * input (then forwarded with fp8ds_fp8_io.in_cast).  All casts go through
+ * fp8_cast_transpose_amax_multi (one launch for up to 256 casts).
+ *   lins      host array of num_lins handle pointers.
+ * Errors: FP8DS_ERR_INVALID_ARG for an incomplete handle, a meta index out of
+ * range, or an invalid extra job; nothing is enqueued then and no cache_valid
+ * flag changes.
+ */
+fp8ds_status fp8_linear_refresh_weights(fp8ds_linear *const *lins, int32_t num_lins,
+                                        const fp8ds_meta *meta, const fp8ds_cast_job *extra,
+                                        int32_t num_extra, fp8ds_stream stream);
+
+/*
  * fp8_linear_bwd -- FP8 backward of one linear [TE761 HYBRID: e5m2 gradients]:
  *   1. cast dy -> e5m2 dy8 and dy8t with meta.scale[meta_grad], amax into
  *      amax_history[0, meta_grad], private scale_inv into *dy_scale_inv;
@@ -508,6 +570,24 @@ const char *fp8ds_last_error(void);
  * read fails.
  */
 fp8ds_status fp8ds_device_status(int32_t *code_out, int32_t clear);
+
+/*
+ * fp8ds_test_stream_k_withhold -- test setting for the error path of the
+ * stream-K GEMM; it has no counterpart on the pages and changes nothing the
+ * method computes.  With withhold != 0, every stream-K launch issued after
+ * the call (fp8_gemm_ex, fp8_gemm_noalloc and the linear calls with a
+ * workspace) runs with the CTA pairs that compute the later k-blocks of a
+ * split tile NOT publishing their partial sums: the pairs that own those
+ * tiles wait for a publication that never comes, give up after wait_ns
+ * nanoseconds (0: the default limit of 2 s), record FP8DS_ERR_TIMEOUT with
+ * site code 5 (the partial-sum wait) in the device error word
+ * (fp8ds_device_status: (5 << 8) | FP8DS_ERR_TIMEOUT), leave their split
+ * tiles unwritten and exit; the launch ends and the context stays usable.
+ * withhold = 0 (and wait_ns = 0) restores normal operation.  A process-wide
+ * host setting read when a GEMM is enqueued; a graph captured meanwhile
+ * keeps it.  Always returns FP8DS_OK.
+ */
+fp8ds_status fp8ds_test_stream_k_withhold(int32_t withhold, uint64_t wait_ns);
 
 /* Library version string. */
 const char *fp8ds_version(void);

@@ -35,7 +35,7 @@ def test_header_declares_the_boundary():
               "fp8_cast_transpose_amax_pair",
               "fp8_cast_transpose_amax_dynamic", "fp8_transpose", "fp8_gemm_major",
               "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
-              "fp8ds_version"):
+              "fp8ds_version", "fp8_cast_transpose_amax_multi", "fp8_linear_refresh_weights"):
         assert n in names
 
 
@@ -259,3 +259,46 @@ int main(void) {
     assert r.returncode == 0, r.stdout + r.stderr
     version, status, msg = r.stdout.strip().split("|")
     assert "sm_100a" in version and int(status) == lib.ERR_INVALID_ARG and "negative" in msg
+
+
+def test_multi_cast_and_refresh_argument_checks(lib):
+    """The multi-tensor cast and the weight-cache refresh check every job (and
+    every handle) before anything is launched, and name the bad job."""
+    L = lib._lib
+    s = P(0)
+    good = lib._CastJob(FAKE, 0, 64, 32, 0, FAKE, FAKE, None, None, None, None)
+    jobs = (lib._CastJob * 3)(good, good, good)
+    jobs[2].scale = None
+    assert L.fp8_cast_transpose_amax_multi(jobs, 3, s) == lib.ERR_INVALID_ARG
+    assert "job 2" in lib.fp8ds_last_error()
+    jobs[2].scale = FAKE
+    jobs[1].rows = -1
+    assert L.fp8_cast_transpose_amax_multi(jobs, 3, s) == lib.ERR_INVALID_ARG
+    assert "job 1" in lib.fp8ds_last_error()
+    jobs[1].rows = 64
+    jobs[0].fmt = 7
+    assert L.fp8_cast_transpose_amax_multi(jobs, 3, s) == lib.ERR_INVALID_ARG
+    jobs[0].fmt = 0
+    jobs[0].yt = FAKE
+    jobs[0].rows = 1 << 31
+    assert L.fp8_cast_transpose_amax_multi(jobs, 3, s) == lib.ERR_INVALID_ARG and "2^31" in lib.fp8ds_last_error()
+    assert L.fp8_cast_transpose_amax_multi(None, 2, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_cast_transpose_amax_multi(jobs, -1, s) == lib.ERR_INVALID_ARG
+    assert L.fp8_cast_transpose_amax_multi(None, 0, s) == lib.OK          # nothing to do
+    # refresh: an incomplete handle or a bad meta index rejects the whole call
+    # and leaves every cache flag as it was
+    meta = lib._Meta(FAKE, FAKE, FAKE, FAKE, 6, 16)
+    la = lib._Linear(FAKE, None, 0, 256, 512, FAKE, None, FAKE, 0, 1, 2, 0, None, 0)
+    lb = lib._Linear(FAKE, None, 0, 512, 256, None, None, FAKE, 3, 4, 5, 0, None, 0)
+    arr = (ctypes.POINTER(lib._Linear) * 2)(ctypes.pointer(la), ctypes.pointer(lb))
+    assert L.fp8_linear_refresh_weights(arr, 2, ctypes.byref(meta), None, 0, s) == lib.ERR_INVALID_ARG
+    assert "handle 1" in lib.fp8ds_last_error() and la.cache_valid == 0
+    lb.w8 = FAKE
+    lb.meta_w = 6
+    assert L.fp8_linear_refresh_weights(arr, 2, ctypes.byref(meta), None, 0, s) == lib.ERR_INVALID_ARG
+    assert "out of range" in lib.fp8ds_last_error() and la.cache_valid == 0
+    lb.meta_w = 4
+    bad_extra = (lib._CastJob * 1)(lib._CastJob(None, 0, 64, 32, 0, FAKE, FAKE, None, None, None, None))
+    assert L.fp8_linear_refresh_weights(arr, 2, ctypes.byref(meta), bad_extra, 1, s) == lib.ERR_INVALID_ARG
+    assert "job 2" in lib.fp8ds_last_error() and la.cache_valid == 0 and lb.cache_valid == 0
+    assert L.fp8_linear_refresh_weights(None, 1, ctypes.byref(meta), None, 0, s) == lib.ERR_INVALID_ARG

@@ -36,4 +36,4 @@ def test_step_accounting():
     assert bench.STEP_GEMMS == 6
     assert abs(bench.STEP_FLOP - 6 * 2.0 * 8192 * 8192 * 2048) < 1
     assert bench.STEP_CAST_BYTES_FUSED == 3 * 8192 * 2048 * 5 + 8192 * 2048 * 3
-    assert bench.LAUNCHES_PER_STEP == 10 and bench.LAUNCHES_PER_STEP_UNFUSED == 12
+    assert bench.LAUNCHES_PER_STEP == 9 and bench.LAUNCHES_PER_STEP_UNFUSED == 12

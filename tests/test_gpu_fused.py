@@ -173,6 +173,25 @@ class _Mlp:
         m.update()
 
 
+    def step_one_cast_launch(self, x, dy):
+        """The step without transposes whose X, W1 and W2 casts are one launch
+        (fp8_linear_refresh_weights with X as an extra job); the forwards then
+        reuse the refreshed caches and take X8 as already cast."""
+        fp8, m = self.fp8, self.meta
+        if not hasattr(self, "group"):
+            self.group = fp8.LinearGroup([self.fc1, self.fc2])
+        xjob = fp8.cast_job(x, "e4m3", m.scale[0:1], self.x8, None, m.amax_history[0, 0:1], self.si[0:1])
+        fp8.fp8_linear_refresh_weights(self.group, m, [xjob])
+        fp8.fp8_linear_fwd_ex(self.fc1, m, None, None, False, self.x8, None, self.si[0:1], in_cast=True,
+                              out_meta=3, out8=self.h8, out8t=None, out_scale_inv=self.si[1:2])
+        fp8.fp8_linear_fwd_ex(self.fc2, m, None, self.y, False, self.h8, None, self.si[1:2], in_cast=True)
+        fp8.fp8_linear_bwd_ex(self.fc2, m, dy, None, self.si[1:2], self.dw2, self.dy8, None, self.si[2:3],
+                              out_meta=2, out8=self.dh8, out8t=None, out_scale_inv=self.si[3:4], x8=self.h8)
+        fp8.fp8_linear_bwd_ex(self.fc1, m, None, None, self.si[0:1], self.dw1, self.dh8, None, self.si[3:4],
+                              dx=self.dx, in_cast=True, x8=self.x8)
+        m.update()
+
+
 def _compare(u, f, what, names=("x8", "x8t", "h8", "h8t", "dy8", "dy8t", "dh8", "dh8t")):
     for name in names:
         assert_bytes_equal(u8(getattr(f, name)), u8(getattr(u, name)), "%s: %s" % (what, name))
@@ -226,3 +245,22 @@ def test_mlp_without_transposes_equals_unfused(fp8, tokens, hidden, ffn):
         _compare(un, nt, "step %d" % step, names=("x8", "h8", "dy8", "dh8"))
         assert_bytes_equal(u8(nt.fc1.w8), u8(un.fc1.w8), "step %d: w1 cache" % step)
         assert_bytes_equal(u8(nt.fc2.w8), u8(un.fc2.w8), "step %d: w2 cache" % step)
+
+
+@pytest.mark.parametrize("tokens,hidden,ffn", [(384, 256, 1024), (8192, 2048, 8192)])
+def test_mlp_one_cast_launch_equals_unfused(fp8, tokens, hidden, ffn):
+    """The benchmarked step: X, W1 and W2 cast in one launch (the weight-cache
+    refresh of both linears with X as an extra job), no transposes.  Same
+    bytes, outputs and metas as the unfused step over three steps."""
+    un = _Mlp(fp8, tokens, hidden, ffn)
+    one = _Mlp(fp8, tokens, hidden, ffn, transposes=False)
+    for step in range(3):
+        x, dy = inputs.mlp_step_inputs(step, tokens=tokens, hidden=hidden)
+        xd, dyd = x.cuda(), dy.cuda()
+        un.step_unfused(xd, dyd)
+        one.step_one_cast_launch(xd, dyd)
+        torch.cuda.synchronize()
+        assert fp8.fp8ds_device_status() == 0
+        _compare(un, one, "step %d" % step, names=("x8", "h8", "dy8", "dh8"))
+        assert_bytes_equal(u8(one.fc1.w8), u8(un.fc1.w8), "step %d: w1 cache" % step)
+        assert_bytes_equal(u8(one.fc2.w8), u8(un.fc2.w8), "step %d: w2 cache" % step)

@@ -241,3 +241,46 @@ def test_gemm_stream_k_repeatable(fp8, ws):
     torch.cuda.synchronize()
     assert torch.equal(outs[0].view(torch.int32), outs[1].view(torch.int32))
     assert torch.equal(outs[0].view(torch.int32), outs[2].view(torch.int32))
+
+
+# ------------------------------------------------------------ error path --
+
+def test_stream_k_partial_wait_gives_up_and_reports(fp8, ws):
+    """The bounded wait for another pair's partial sum, made to run out: with
+    the test setting the pairs that compute the later k-blocks of every split
+    tile withhold their publication, so the owners of those tiles wait 5 ms,
+    give up, record a timeout at the partial-sum site in the device error word
+    and exit (no fault, no hang).  The context stays usable: the workspace's
+    publication words are clear and the next normal call is exact."""
+    M, N, K = 4096, 2048, 256                       # 128 tiles of 256 x 256
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    tiles = (M // 256) * (N // 256)
+    if not (pairs <= tiles < 8 * pairs and tiles % pairs != 0):
+        pytest.skip("%d tiles on %d CTA pairs: no split tiles" % (tiles, pairs))
+    a, av = _integer_codes((M, K), "e4m3", 25)
+    b, bv = _integer_codes((N, K), "e4m3", 26)
+    ad, bd = dev(a), dev(b)
+    sa, sb = torch.tensor([0.5], device="cuda"), torch.tensor([4.0], device="cuda")
+    assert fp8.fp8ds_device_status() == 0
+    d = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    assert fp8._lib.fp8ds_test_stream_k_withhold(1, 5_000_000) == fp8.OK
+    try:
+        fp8.fp8_gemm_ex(ad, "e4m3", sa, bd, "e4m3", sb, d, workspace=ws)
+        torch.cuda.synchronize()
+    finally:
+        assert fp8._lib.fp8ds_test_stream_k_withhold(0, 0) == fp8.OK
+    code = fp8.fp8ds_device_status()                 # read and cleared
+    assert code == (5 << 8) | fp8.ERR_TIMEOUT, hex(code)
+    assert fp8.fp8ds_device_status() == 0
+    assert _flags_clear(ws)
+    ref = (torch.from_numpy(av).double() @ torch.from_numpy(bv).double().T) * 2.0
+    # tiles computed whole (not split) are exact even in the aborted launch
+    got = d.cpu().double()
+    assert int((got == ref).sum()) > M * N // 4
+    # the next launch, without the setting, is exact everywhere
+    d.fill_(float("nan"))
+    fp8.fp8_gemm_ex(ad, "e4m3", sa, bd, "e4m3", sb, d, workspace=ws)
+    torch.cuda.synchronize()
+    assert fp8.fp8ds_device_status() == 0
+    assert torch.equal(d.cpu().double(), ref)
+    assert _flags_clear(ws)
