@@ -483,20 +483,29 @@ def time_teblock_microbatches(fp8, device, rounds):
 def time_toy_model(fp8, device, steps):
     """The 32-block forward (192 linears, 576 metas, weights recast every
     step): device ms per step issued eagerly, the host time to issue one
-    step, and the same step captured once in a CUDA graph and replayed."""
+    step into an idle queue (median of 3), and the same step captured once in
+    a CUDA graph and replayed (device ms and host us per replay)."""
     toy = TeblockForward(fp8, device, blocks=32)
     for _ in range(2):
         toy.run(True)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    h0 = time.perf_counter()
     for _ in range(steps):
         toy.run(True)
-    host_s = time.perf_counter() - h0
     e1.record()
     torch.cuda.synchronize()
     eager_ms = e0.elapsed_time(e1) / steps
+    # host time to issue one step into an idle queue (back to back, the
+    # launch queue fills and the host waits on the GPU)
+    host = []
+    for _ in range(3):
+        torch.cuda.synchronize()
+        h0 = time.perf_counter()
+        toy.run(True)
+        host.append(time.perf_counter() - h0)
+    torch.cuda.synchronize()
+    host_s = statistics.median(host) * steps
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         toy.run(True)

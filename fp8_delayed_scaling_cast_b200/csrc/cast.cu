@@ -324,11 +324,12 @@ struct RingLoad8<float, FMT> {
     }
 };
 
-// One tensor of a cast launch.  A launch casts one or two tensors of the same
-// input type and format (the linear forward's input and weight in one
-// launch); their tiles are numbered job 0 first, then job 1.  A job whose
-// noop flag holds non-zero at run time is skipped whole: no load, store,
-// amax or scale_inv of it happens.
+// One tensor of a cast launch.  A launch casts up to TMA_MAX_JOBS tensors of
+// one input type and format, all with or all without transpose (a linear
+// forward's input and weight; the MLP step's X, W1 and W2); their tiles are
+// numbered job after job.  A job whose noop flag holds non-zero at run time
+// is skipped whole: no load, store, amax or scale_inv of it happens.
+constexpr int TMA_MAX_JOBS = 8;
 struct CastJob {
     const float *scale;
     uint8_t *y, *yt;
@@ -336,14 +337,18 @@ struct CastJob {
     const int32_t *noop;
     int32_t rows, cols, tiles_c, num_tiles;
 };
+struct TmaJobs {
+    CUtensorMap maps[TMA_MAX_JOBS];
+    CastJob jobs[TMA_MAX_JOBS];
+    int32_t num_jobs;
+};
 
 // Vectorised-path requirements (checked on the host): x 16-byte aligned
 // (TMA), cols % 8 == 0, rows % 16 == 0, y and yt 16-byte aligned.  Tiles
 // that reach past the tensor read zeros (TMA fill) and store element-wise.
 template <typename T, int FMT, bool WRITE_T>
 __global__ void __launch_bounds__(CT_THREADS, 3)
-cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap0, const __grid_constant__ CUtensorMap tmap1,
-                          const CastJob job0, const CastJob job1) {
+cast_transpose_tma_kernel(const __grid_constant__ TmaJobs P) {
     using R = TmaRing<T>;
     constexpr int STAGES = R::STAGES;
     extern __shared__ uint8_t dsm[];
@@ -352,48 +357,52 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap0, const __gri
     // Transposed words of two consecutive tiles: tile i writes buffer i & 1
     // while the yt stores of tile i-1 read the other one.
     __shared__ uint32_t tsm[2][CT_COLS * CT_TSTRIDE];
+    // First tile of each job in the launch (a skipped job owns no tile).
+    __shared__ int32_t first_tile[TMA_MAX_JOBS + 1];
     const int tid = threadIdx.x;
     const int cc = tid & 7, rg = tid >> 3;
-    float m0 = 0.0f, m1 = 0.0f;
+    const int nj = P.num_jobs;
 
     if (tid == 0) {
         for (int i = 0; i < STAGES; ++i) ptx::mbar_init(&full[i], 1);
         ptx::fence_barrier_init();
         ptx::fence_async_smem();
-        ptx::prefetch_tmap(&tmap0);
-        if (job1.num_tiles > 0) ptx::prefetch_tmap(&tmap1);
     }
+    if (tid < nj) ptx::prefetch_tmap(&P.maps[tid]);
     ptx::pdl_wait();
     ptx::pdl_launch_dependents();
     // device-side skips (whole jobs), before any load is issued
-    const int32_t n0 = (job0.noop != nullptr && __ldg(job0.noop) != 0) ? 0 : job0.num_tiles;
-    const int32_t n1 = (job1.noop != nullptr && __ldg(job1.noop) != 0) ? 0 : job1.num_tiles;
-    const int32_t num_tiles = n0 + n1;
-    if (num_tiles == 0) return;
-    const float s0 = n0 > 0 ? __ldg(job0.scale) : 0.0f;
-    const float s1 = n1 > 0 ? __ldg(job1.scale) : 0.0f;
-    if (tid == 0 && blockIdx.x == 0) {
-        if (n0 > 0 && job0.scale_inv != nullptr) *job0.scale_inv = __frcp_rn(s0);
-        if (n1 > 0 && job1.scale_inv != nullptr) *job1.scale_inv = __frcp_rn(s1);
+    if (tid == 0) {
+        int32_t acc = 0;
+        for (int j = 0; j < nj; ++j) {
+            first_tile[j] = acc;
+            const CastJob &J = P.jobs[j];
+            if (J.noop != nullptr && __ldg(J.noop) != 0) continue;
+            acc += J.num_tiles;
+            if (blockIdx.x == 0 && J.scale_inv != nullptr) *J.scale_inv = __frcp_rn(__ldg(J.scale));
+        }
+        first_tile[nj] = acc;
     }
     __syncthreads();
-    // Tile t of the launch: job (t >= n0) and its tile index within the job.
-    auto which = [&](int t, int &j, int &lt) {
-        j = t >= n0 ? 1 : 0;
-        lt = j ? t - n0 : t;
+    const int32_t num_tiles = first_tile[nj];
+    if (num_tiles == 0) return;
+    // Job of tile t, advancing a cursor (tiles are visited in increasing order).
+    auto job_at = [&](int t, int &cur) {
+        while (t >= first_tile[cur + 1]) ++cur;
+        return cur;
     };
     // Thread 0 keeps up to STAGES tiles of this CTA in flight.
-    int issued = 0;
+    int issued = 0, pj = 0;
     auto issue = [&](int tile, int stage) {
-        int j, lt;
-        which(tile, j, lt);
-        const CastJob &J = j ? job1 : job0;
+        const int j = job_at(tile, pj);
+        const CastJob &J = P.jobs[j];
+        const int32_t lt = tile - first_tile[j];
         const int32_t r0 = (lt / J.tiles_c) * CT_ROWS;
         const int32_t c0 = (lt % J.tiles_c) * CT_COLS;
         ptx::mbar_arrive_expect_tx(&full[stage], R::STAGE_BYTES);
 #pragma unroll
         for (int b = 0; b < R::BOXES; ++b)
-            ptx::tma_load_2d(j ? &tmap1 : &tmap0, &full[stage], ring + stage * R::STAGE_BYTES + b * R::BOX_BYTES,
+            ptx::tma_load_2d(&P.maps[j], &full[stage], ring + stage * R::STAGE_BYTES + b * R::BOX_BYTES,
                              c0 + b * R::BOX_COLS, r0);
         ++issued;
     };
@@ -404,12 +413,11 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap0, const __gri
         }
     }
 
-    // yt stores of a tile whose transposed words are in tsm[buf].
-    auto store_yt = [&](int tile, int buf) {
-        int j, lt;
-        which(tile, j, lt);
-        const CastJob &J = j ? job1 : job0;
+    // yt stores of tile `tile` (job j) whose transposed words are in tsm[buf].
+    auto store_yt = [&](int tile, int j, int buf) {
+        const CastJob &J = P.jobs[j];
         const int32_t rows = J.rows, cols = J.cols;
+        const int32_t lt = tile - first_tile[j];
         const int32_t r0 = (lt / J.tiles_c) * CT_ROWS;
         const int32_t c0 = (lt % J.tiles_c) * CT_COLS;
         const bool full_tile = (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
@@ -435,9 +443,15 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap0, const __gri
     // One block barrier per tile.  Iteration i: wait for tile i; barrier
     // (all threads are past tile i-1: its stage can be refilled and its
     // transposed words are complete); refill; cast tile i into y and
-    // tsm[i & 1]; write yt of tile i-1 from tsm[(i-1) & 1].
+    // tsm[i & 1]; write yt of tile i-1 from tsm[(i-1) & 1].  The CTA's tiles
+    // go job after job: when the job changes, the amax of the previous one
+    // is reduced across the CTA and max-ed into its target.
     int it = 0;
-    int prev = -1;
+    int prev = -1, prev_j = -1;
+    int cj = 0;
+    // the scale of this CTA's first job is read while its first tiles load
+    int mj = blockIdx.x < num_tiles ? job_at(blockIdx.x, cj) : 0;
+    float m = 0.0f, s = __ldg(P.jobs[mj].scale);
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
         const int stage = it % STAGES;
         const uint32_t phase = static_cast<uint32_t>((it / STAGES) & 1);
@@ -452,13 +466,17 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap0, const __gri
             const int next = prev + STAGES * gridDim.x;  // the stage tile i-1 used
             if (next < num_tiles) issue(next, (it - 1) % STAGES);
         }
-        int j, lt;
-        which(tile, j, lt);
-        const CastJob &J = j ? job1 : job0;
+        const int j = job_at(tile, cj);
+        if (j != mj) {
+            block_amax_commit<CT_THREADS>(m, P.jobs[mj].amax);
+            m = 0.0f;
+            mj = j;
+            s = __ldg(P.jobs[j].scale);
+        }
+        const CastJob &J = P.jobs[j];
         const int32_t rows = J.rows, cols = J.cols;
-        const float s = j ? s1 : s0;
-        float &m = j ? m1 : m0;
         const uint8_t *st = ring + stage * R::STAGE_BYTES;
+        const int32_t lt = tile - first_tile[j];
         const int32_t r0 = (lt / J.tiles_c) * CT_ROWS;
         const int32_t c0 = (lt % J.tiles_c) * CT_COLS;
         const bool full_tile = (r0 + CT_ROWS <= rows) && (c0 + CT_COLS <= cols);
@@ -496,24 +514,21 @@ cast_transpose_tma_kernel(const __grid_constant__ CUtensorMap tmap0, const __gri
                 tw[2 * CT_TSTRIDE] = __byte_perm(p01h, p23h, 0x5410);
                 tw[3 * CT_TSTRIDE] = __byte_perm(p01h, p23h, 0x7632);
             }
-            if (prev >= 0) store_yt(prev, (it - 1) & 1);
+            if (prev >= 0) store_yt(prev, prev_j, (it - 1) & 1);
         }
         prev = tile;
+        prev_j = j;
     }
     // The last tile's transposed words: one more barrier, then its yt.
     __syncthreads();
-    if (WRITE_T && prev >= 0) store_yt(prev, (it - 1) & 1);
+    if (WRITE_T && prev >= 0) store_yt(prev, prev_j, (it - 1) & 1);
     // Loads issued but never consumed (only after a timeout) must land before
     // the CTA exits.
     if (tid == 0) {
         for (int jj = it; jj < issued; ++jj)
             ptx::mbar_wait_for(&full[jj % STAGES], static_cast<uint32_t>((jj / STAGES) & 1), ptx::DRAIN_NS);
     }
-    if (n0 > 0) block_amax_commit<CT_THREADS>(m0, job0.amax);
-    if (n1 > 0) {
-        __syncthreads();  // the first commit's reduction buffer is free again
-        block_amax_commit<CT_THREADS>(m1, job1.amax);
-    }
+    block_amax_commit<CT_THREADS>(m, P.jobs[mj].amax);
 }
 
 // ---------------------------------------------------------------- quantize --
@@ -834,12 +849,12 @@ bool make_job(const HostCast &c, CUtensorMap *tm, CastJob *job) {
     return true;
 }
 
-// One launch of the TMA kernel over job 0 and job 1 (job 1 may have no tiles).
+// One launch of the TMA kernel over P.num_jobs jobs.
 template <typename T, int FMT, bool WRITE_T>
-cudaError_t ct_launch_tma(const CUtensorMap &t0, const CastJob &j0, const CUtensorMap &t1, const CastJob &j1,
-                          cudaStream_t stream) {
+cudaError_t ct_launch_tma(const TmaJobs &P, cudaStream_t stream) {
     using R = TmaRing<T>;
-    const int64_t num_tiles = static_cast<int64_t>(j0.num_tiles) + j1.num_tiles;
+    int64_t num_tiles = 0;
+    for (int j = 0; j < P.num_jobs; ++j) num_tiles += P.jobs[j].num_tiles;
     auto kernel = cast_transpose_tma_kernel<T, FMT, WRITE_T>;
     // per device: CTAs per SM once the kernel's shared-memory limit is set
     // (0 = not yet; concurrent first calls may both set it, to the same value)
@@ -858,37 +873,41 @@ cudaError_t ct_launch_tma(const CUtensorMap &t0, const CastJob &j0, const CUtens
     }
     const int64_t cap = static_cast<int64_t>(num_sms()) * n_sm;
     const int grid = static_cast<int>(num_tiles < cap ? (num_tiles > 0 ? num_tiles : 1) : cap);
-    return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), R::SMEM, stream, 1, t0, t1, j0, j1);
+    return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), R::SMEM, stream, 1, P);
 }
 
 template <typename T, int FMT>
 cudaError_t ct_dispatch(const void *x, int64_t rows, int64_t cols, const float *scale, uint8_t *y, uint8_t *yt,
                         float *amax, float *scale_inv, const int32_t *noop, cudaStream_t stream) {
     const HostCast c{x, rows, cols, scale, y, yt, amax, scale_inv, noop};
-    CUtensorMap tm;
-    CastJob job, none;
-    if (tma_eligible(c) && make_job<T>(c, &tm, &job)) {
-        none = job;
-        none.num_tiles = 0;
-        return yt != nullptr ? ct_launch_tma<T, FMT, true>(tm, job, tm, none, stream)
-                             : ct_launch_tma<T, FMT, false>(tm, job, tm, none, stream);
-    }
+    TmaJobs P;
+    P.num_jobs = 1;
+    if (tma_eligible(c) && make_job<T>(c, &P.maps[0], &P.jobs[0]))
+        return yt != nullptr ? ct_launch_tma<T, FMT, true>(P, stream) : ct_launch_tma<T, FMT, false>(P, stream);
     return yt != nullptr ? ct_launch_elem<T, FMT, true>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream)
                          : ct_launch_elem<T, FMT, false>(x, rows, cols, scale, y, yt, amax, scale_inv, noop, stream);
 }
 
-// Two tensors of one input type and format in one launch, when both suit the
-// TMA kernel and both or neither write a transpose; false (nothing launched)
-// otherwise.
+// Up to TMA_MAX_JOBS tensors of one input type and format in one launch of
+// the TMA kernel, when every one suits it and all or none write a transpose;
+// false (nothing launched) otherwise.
+template <typename T, int FMT>
+bool ct_dispatch_jobs(const HostCast *c, int n, cudaStream_t stream, cudaError_t *err) {
+    if (n < 1 || n > TMA_MAX_JOBS) return false;
+    TmaJobs P;
+    P.num_jobs = n;
+    for (int j = 0; j < n; ++j) {
+        if ((c[j].yt == nullptr) != (c[0].yt == nullptr) || !tma_eligible(c[j])) return false;
+        if (!make_job<T>(c[j], &P.maps[j], &P.jobs[j])) return false;
+    }
+    *err = c[0].yt != nullptr ? ct_launch_tma<T, FMT, true>(P, stream) : ct_launch_tma<T, FMT, false>(P, stream);
+    return true;
+}
+
 template <typename T, int FMT>
 bool ct_dispatch_pair(const HostCast &a, const HostCast &b, cudaStream_t stream, cudaError_t *err) {
-    if ((a.yt == nullptr) != (b.yt == nullptr) || !tma_eligible(a) || !tma_eligible(b)) return false;
-    CUtensorMap t0, t1;
-    CastJob j0, j1;
-    if (!make_job<T>(a, &t0, &j0) || !make_job<T>(b, &t1, &j1)) return false;
-    *err = a.yt != nullptr ? ct_launch_tma<T, FMT, true>(t0, j0, t1, j1, stream)
-                           : ct_launch_tma<T, FMT, false>(t0, j0, t1, j1, stream);
-    return true;
+    const HostCast c[2] = {a, b};
+    return ct_dispatch_jobs<T, FMT>(c, 2, stream, err);
 }
 
 template <typename T, int FMT>
@@ -1059,7 +1078,26 @@ cudaError_t launch_transpose_u8(const uint8_t *y, int64_t rows, int64_t cols, ui
                       cols, yt, tiles_c, num_tiles);
 }
 
+// The TMA kernel's path for a short job list of one input type and format
+// whose tensors all suit it; false (nothing launched) otherwise.
+static bool cast_multi_tma(const fp8ds_cast_job *jobs, int32_t n, cudaStream_t stream, cudaError_t *err) {
+    if (n < 1 || n > TMA_MAX_JOBS) return false;
+    HostCast c[TMA_MAX_JOBS];
+    for (int32_t j = 0; j < n; ++j) {
+        if (jobs[j].x_dtype != jobs[0].x_dtype || jobs[j].fmt != jobs[0].fmt) return false;
+        c[j] = HostCast{jobs[j].x, jobs[j].rows, jobs[j].cols, jobs[j].scale, jobs[j].y, jobs[j].yt, jobs[j].amax,
+                        jobs[j].scale_inv, jobs[j].noop_flag};
+    }
+    if (jobs[0].x_dtype == FP8DS_F32)
+        return jobs[0].fmt == FP8DS_E4M3 ? ct_dispatch_jobs<float, FP8DS_E4M3>(c, n, stream, err)
+                                         : ct_dispatch_jobs<float, FP8DS_E5M2>(c, n, stream, err);
+    return jobs[0].fmt == FP8DS_E4M3 ? ct_dispatch_jobs<uint16_t, FP8DS_E4M3>(c, n, stream, err)
+                                     : ct_dispatch_jobs<uint16_t, FP8DS_E5M2>(c, n, stream, err);
+}
+
 cudaError_t launch_cast_multi(const fp8ds_cast_job *jobs, int32_t num_jobs, cudaStream_t stream) {
+    cudaError_t err = cudaSuccess;
+    if (cast_multi_tma(jobs, num_jobs, stream, &err)) return err;
     static std::atomic<int> per_sm[64];
     int dev = 0;
     cudaGetDevice(&dev);

@@ -83,6 +83,17 @@ constexpr int TMEM_COLS = 512; // two accumulators
 #define FP8DS_EPI_DIRECT 0
 #endif
 constexpr bool EPI_DIRECT = FP8DS_EPI_DIRECT != 0;
+// FP8DS_EPI_EARLY: whole-tile bf16 and FP8 epilogues read the accumulator
+// into registers and release TMEM before they stage and store D.
+#ifndef FP8DS_EPI_EARLY
+#define FP8DS_EPI_EARLY 1
+#endif
+constexpr bool EPI_EARLY = FP8DS_EPI_EARLY != 0 && !EPI_DIRECT;
+// FP8DS_SPLIT_BF16: the 512-row tile with bf16 output also releases its two
+// M halves one at a time (always done for FP8 output).
+#ifndef FP8DS_SPLIT_BF16
+#define FP8DS_SPLIT_BF16 0
+#endif
 constexpr int EPI_LD = FP8DS_EPI_LD;
 constexpr int EPI_NBOX = FP8DS_EPI_BOXES;
 static_assert(EPI_LD == 32 || EPI_LD == 64, "TMEM load width must be 32 or 64 columns");
@@ -884,6 +895,142 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
     }
 }
 
+// Whole-tile epilogues that release TMEM before they store (mode 0, staged
+// output).  Reading the accumulator out of TMEM is fast (8 warps drain
+// 256 bytes per SM cycle); converting, staging and storing D are the slow
+// part.  So each half of the accumulator is read and converted into
+// registers first and handed back to the MMA warp as soon as its last TMEM
+// load has completed; the staging and the TMA stores follow while the next
+// tile's MMAs already run.
+//
+// FP8 output: the codes of both halves fit in registers (32 words per half
+// and lane), so the whole accumulator is released before anything is stored.
+template <bool BIAS, int MSUB>
+__device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uint8_t *boxes, int &nbox, int half,
+                                                  const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row_h0,
+                                                  int32_t rows_per_sub, float sab, const float *bias_s,
+                                                  uint32_t empty_base, bool split, float s_out, int fmt,
+                                                  float &amax) {
+    constexpr int CH = ACC_N / 2 / 32;  // chunks of 32 columns per warp and half
+    const uint64_t sab2 = pack_f32x2(sab, sab);
+    const uint64_t s2 = pack_f32x2(s_out, s_out);
+    uint32_t codes[MSUB][CH * 8];
+    uint32_t r[32];
+#pragma unroll
+    for (int h = 0; h < MSUB; ++h) {
+        const uint32_t t_h = t_row0 + static_cast<uint32_t>(h * ACC_N + half * (ACC_N / 2));
+        tmem_ld32(t_h, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            if (c == CH - 1 && (split || h == MSUB - 1)) {
+                // every TMEM load of this half (or of the accumulator) is done
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(empty_base + static_cast<uint32_t>(split ? h * sizeof(uint64_t) : 0));
+            }
+            const float *bs = bias_s + half * (ACC_N / 2) + c * 32;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 b = bias4<BIAS>(bs + 4 * j);
+                const uint64_t v01 = fma_f32x2(pack_f32x2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])),
+                                               sab2, pack_f32x2(b.x, b.y));
+                const uint64_t v23 = fma_f32x2(
+                    pack_f32x2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), sab2,
+                    pack_f32x2(b.z, b.w));
+                const __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
+                const __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
+                const float h0 = __low2float(ha), h1 = __high2float(ha);
+                const float h2 = __low2float(hb), h3 = __high2float(hb);
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+                const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
+                const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
+                codes[h][8 * c + j] =
+                    cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) | (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
+            }
+            if (c + 1 < CH) {
+                tmem_ld32(t_h + static_cast<uint32_t>((c + 1) * 32), r);
+                tmem_ld_wait();
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < MSUB; ++h) {
+        uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
+        if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
+        __syncwarp();
+        // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
+#pragma unroll
+        for (int k = 0; k < 2 * CH; ++k)
+            *reinterpret_cast<uint4 *>(box + lane * 128 + (k ^ (lane & 7)) * 16) =
+                make_uint4(codes[h][4 * k], codes[h][4 * k + 1], codes[h][4 * k + 2], codes[h][4 * k + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)), m_row_h0 + h * rows_per_sub);
+            tma_store_commit();
+        }
+        ++nbox;
+    }
+}
+
+// bf16 output: the 128 columns of one half take 64 words per lane, so each
+// half is read, converted and released, then stored (two staging boxes of
+// 64 columns) before the next half is read.
+template <bool BIAS>
+__device__ __forceinline__ void epilogue_bf16_regs(uint32_t t_h, int lane, uint8_t *boxes, int &nbox, int half,
+                                                   const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
+                                                   float sab, const float *bias_s, uint32_t empty_addr,
+                                                   bool release) {
+    constexpr int CH = ACC_N / 2 / 32;
+    uint32_t packed[CH * 16];
+    uint32_t r[32];
+    tmem_ld32(t_h + static_cast<uint32_t>(half * (ACC_N / 2)), r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        if (release && c == CH - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(empty_addr);
+        }
+        const float *bs = bias_s + half * (ACC_N / 2) + c * 32;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 b = bias4<BIAS>(bs + 4 * j);
+            __nv_bfloat162 ha = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j]), sab, b.x),
+                                                      fmaf(__uint_as_float(r[4 * j + 1]), sab, b.y));
+            __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j + 2]), sab, b.z),
+                                                      fmaf(__uint_as_float(r[4 * j + 3]), sab, b.w));
+            packed[16 * c + 2 * j] = *reinterpret_cast<uint32_t *>(&ha);
+            packed[16 * c + 2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
+        }
+        if (c + 1 < CH) {
+            tmem_ld32(t_h + static_cast<uint32_t>(half * (ACC_N / 2) + (c + 1) * 32), r);
+            tmem_ld_wait();
+        }
+    }
+    // two boxes of 64 columns (128 bytes per row)
+#pragma unroll
+    for (int bx = 0; bx < 2; ++bx) {
+        uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
+        if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            *reinterpret_cast<uint4 *>(box + lane * 128 + (k ^ (lane & 7)) * 16) =
+                make_uint4(packed[32 * bx + 4 * k], packed[32 * bx + 4 * k + 1], packed[32 * bx + 4 * k + 2],
+                           packed[32 * bx + 4 * k + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2) + bx * 64), m_row0);
+            tma_store_commit();
+        }
+        ++nbox;
+    }
+}
+
 // Shared-memory carve-up common to both kernels.
 struct Smem {
     uint8_t *a, *b, *epi;
@@ -982,7 +1129,49 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
         // half by half (tempty[h]), so that the next tile's half-0 MMAs
         // start while half 1 is still being read.
         const uint32_t empty_base = map_to_cta(smem_u32(&sm.tempty[acc]), tempty_rank);
-        for (int h = 0; h < m_sub; ++h) {
+        const int64_t n_tile = static_cast<int64_t>(n_blk) * ACC_N;
+        const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * ACC_N);
+        const int32_t m_row_h0 = (m_blk * m_sub) * rows_per_sub + row_offset + q * 32;
+        bool done = false;
+        if constexpr (EPI_EARLY && OUT == OUT_FP8) {
+            if (mode == 0 && p.out_d8t == nullptr) {
+                if (m_sub == 2) {
+                    if (p.bias_kind != 0)
+                        epilogue_fp8_regs<true, 2>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
+                                                   rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt, amax);
+                    else
+                        epilogue_fp8_regs<false, 2>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
+                                                    rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt,
+                                                    amax);
+                } else {
+                    if (p.bias_kind != 0)
+                        epilogue_fp8_regs<true, 1>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
+                                                   rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt, amax);
+                    else
+                        epilogue_fp8_regs<false, 1>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
+                                                    rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt,
+                                                    amax);
+                }
+                done = true;
+            }
+        }
+        if constexpr (EPI_EARLY && OUT == OUT_BF16) {
+            if (mode == 0) {
+                for (int h = 0; h < m_sub; ++h) {
+                    const uint32_t empty_addr = empty_base + static_cast<uint32_t>(split ? h * sizeof(uint64_t) : 0);
+                    const bool release = split || h == m_sub - 1;
+                    const uint32_t t_h = t_acc + static_cast<uint32_t>(h * ACC_N);
+                    if (p.bias_kind != 0)
+                        epilogue_bf16_regs<true>(t_h, lane, boxes, nbox, half, tmap_d, n_tile,
+                                                 m_row_h0 + h * rows_per_sub, sab, bias_s, empty_addr, release);
+                    else
+                        epilogue_bf16_regs<false>(t_h, lane, boxes, nbox, half, tmap_d, n_tile,
+                                                  m_row_h0 + h * rows_per_sub, sab, bias_s, empty_addr, release);
+                }
+                done = true;
+            }
+        }
+        for (int h = 0; h < m_sub && !done; ++h) {
             const uint32_t empty_addr = empty_base + static_cast<uint32_t>(split ? h * sizeof(uint64_t) : 0);
             const bool release = split || h == m_sub - 1;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -1198,7 +1387,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     // Half-by-half release of the 512-row tile's accumulator (FP8 output,
     // whose longer epilogue it hides best; measured neutral-to-negative with
     // bf16 and fp32 outputs).
-    constexpr bool SPLIT = M_SUB == 2 && OUT == OUT_FP8;
+    constexpr bool SPLIT = M_SUB == 2 && (OUT == OUT_FP8 || (OUT == OUT_BF16 && FP8DS_SPLIT_BF16 != 0));
     extern __shared__ uint8_t smem_raw[];
     const Smem sm = carve<STAGES, A_STAGE, S2_B_STAGE>(smem_raw);
     const int warp = threadIdx.x >> 5;

@@ -117,6 +117,23 @@ def test_multi_cast_equals_single_calls(fp8):
         assert torch.equal(ja.si.view(torch.int32), jb.si.view(torch.int32)), i
 
 
+@pytest.mark.parametrize("dtype,fmt,transpose", [("f32", "e4m3", False), ("bf16", "e5m2", True)])
+def test_multi_cast_same_kind_jobs(fp8, dtype, fmt, transpose):
+    """Up to eight tensors of one input dtype and format, all with or all
+    without transpose, that suit the TMA path go through the TMA kernel in one
+    launch (the MLP step's X, W1, W2; a TEBlock's five inputs): every job
+    exact, a flagged job skipped, ragged edge tiles included."""
+    specs = [(512, 2048, 1.0, None), (1024, 512, 64.0, 0), (256, 1024, 0.5, 1), (208, 136, 2.0, None),
+             (2048, 256, 448.0 / 900.0, None), (16, 8, 4.0, None), (640, 64, 1.0, None), (128, 4096, 0.25, None)]
+    jobs = [_Job(fp8, r, c, dtype, fmt, transpose, seed=300 + i, scale=sc, noop=n)
+            for i, (r, c, sc, n) in enumerate(specs)]
+    fp8.fp8_cast_transpose_amax_multi([j.rec for j in jobs])
+    torch.cuda.synchronize()
+    assert fp8.fp8ds_device_status() == 0
+    for i, j in enumerate(jobs):
+        j.check("job %d" % i)
+
+
 def test_multi_cast_more_jobs_than_one_launch(fp8):
     """300 small tensors, more than the 256 of one launch (so two launches),
     mixed dtypes, formats and transposes: every cast exact."""

@@ -232,6 +232,7 @@ def test_mlp_pair_twenty_steps(fp8):
 TOY_BLOCKS = 32
 TOY_STEPS = 16
 TOY_CHECK_BLOCKS = (0, TOY_BLOCKS - 1)    # H amax checked against the oracle every step
+TOY_ALL_BLOCK_STEPS = (0, 7, TOY_STEPS - 1)   # ... and of all 32 blocks on these steps
 TOY_FULL_CHECKS = ((0, 0), (TOY_STEPS - 1, TOY_BLOCKS - 1))   # (step, block): casts in full, GEMM rows
 
 
@@ -245,7 +246,8 @@ def test_toy_model_576_metas(fp8):
     H amaxes of blocks 0 and 31 (oracle amax of the GPU's H), and all 576 metas
     after the update -- the oracle update runs on the oracle's amaxes, taking
     the other 30 blocks' H amaxes as recorded by the GPU (those H are GEMM
-    outputs).  The grad metas are never recorded: their scale stays 1.0.  Block
+    outputs) except on steps 0, 7 and 15, where the H amax of every block is
+    the oracle's amax of that block's H.  The grad metas are never recorded: their scale stays 1.0.  Block
     0 at the first step and block 31 at the last: every cast in full and the
     GEMM outputs on sampled rows."""
     M = inputs.TOKENS
@@ -278,7 +280,7 @@ def test_toy_model_576_metas(fp8):
                 i = blk * per_block + j
                 src = outs[fc1] if j == fc2 else xd
                 fp8.fp8_linear_fwd(lins[i], meta, src, outs[j], None, saved[j].x8, saved[j].x8t, saved[j].si)
-            if blk not in TOY_CHECK_BLOCKS:
+            if blk not in TOY_CHECK_BLOCKS and step not in TOY_ALL_BLOCK_STEPS:
                 continue
             torch.cuda.synchronize()
             h_bits = host_bits(outs[fc1])
