@@ -346,7 +346,9 @@ struct TmaJobs {
 // Vectorised-path requirements (checked on the host): x 16-byte aligned
 // (TMA), cols % 8 == 0, rows % 16 == 0, y and yt 16-byte aligned.  Tiles
 // that reach past the tensor read zeros (TMA fill) and store element-wise.
-template <typename T, int FMT, bool WRITE_T>
+// MULTI false: a launch of one tensor (job 0 only; every job index is the
+// constant 0, so the job's fields are read straight from the parameters).
+template <typename T, int FMT, bool WRITE_T, bool MULTI>
 __global__ void __launch_bounds__(CT_THREADS, 3)
 cast_transpose_tma_kernel(const __grid_constant__ TmaJobs P) {
     using R = TmaRing<T>;
@@ -361,7 +363,7 @@ cast_transpose_tma_kernel(const __grid_constant__ TmaJobs P) {
     __shared__ int32_t first_tile[TMA_MAX_JOBS + 1];
     const int tid = threadIdx.x;
     const int cc = tid & 7, rg = tid >> 3;
-    const int nj = P.num_jobs;
+    const int nj = MULTI ? P.num_jobs : 1;
 
     if (tid == 0) {
         for (int i = 0; i < STAGES; ++i) ptx::mbar_init(&full[i], 1);
@@ -388,8 +390,12 @@ cast_transpose_tma_kernel(const __grid_constant__ TmaJobs P) {
     if (num_tiles == 0) return;
     // Job of tile t, advancing a cursor (tiles are visited in increasing order).
     auto job_at = [&](int t, int &cur) {
-        while (t >= first_tile[cur + 1]) ++cur;
-        return cur;
+        if constexpr (MULTI) {
+            while (t >= first_tile[cur + 1]) ++cur;
+            return cur;
+        } else {
+            return 0;
+        }
     };
     // Thread 0 keeps up to STAGES tiles of this CTA in flight.
     int issued = 0, pj = 0;
@@ -850,12 +856,12 @@ bool make_job(const HostCast &c, CUtensorMap *tm, CastJob *job) {
 }
 
 // One launch of the TMA kernel over P.num_jobs jobs.
-template <typename T, int FMT, bool WRITE_T>
-cudaError_t ct_launch_tma(const TmaJobs &P, cudaStream_t stream) {
+template <typename T, int FMT, bool WRITE_T, bool MULTI>
+cudaError_t ct_launch_tma_k(const TmaJobs &P, cudaStream_t stream) {
     using R = TmaRing<T>;
     int64_t num_tiles = 0;
     for (int j = 0; j < P.num_jobs; ++j) num_tiles += P.jobs[j].num_tiles;
-    auto kernel = cast_transpose_tma_kernel<T, FMT, WRITE_T>;
+    auto kernel = cast_transpose_tma_kernel<T, FMT, WRITE_T, MULTI>;
     // per device: CTAs per SM once the kernel's shared-memory limit is set
     // (0 = not yet; concurrent first calls may both set it, to the same value)
     static std::atomic<int> per_sm[64];
@@ -874,6 +880,12 @@ cudaError_t ct_launch_tma(const TmaJobs &P, cudaStream_t stream) {
     const int64_t cap = static_cast<int64_t>(num_sms()) * n_sm;
     const int grid = static_cast<int>(num_tiles < cap ? (num_tiles > 0 ? num_tiles : 1) : cap);
     return launch_pdl(kernel, dim3(grid), dim3(CT_THREADS), R::SMEM, stream, 1, P);
+}
+
+template <typename T, int FMT, bool WRITE_T>
+cudaError_t ct_launch_tma(const TmaJobs &P, cudaStream_t stream) {
+    return P.num_jobs == 1 ? ct_launch_tma_k<T, FMT, WRITE_T, false>(P, stream)
+                           : ct_launch_tma_k<T, FMT, WRITE_T, true>(P, stream);
 }
 
 template <typename T, int FMT>

@@ -241,33 +241,76 @@ __device__ __noinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// L2 policy of the TMA traffic (FP8DS_L2_HINTS, compile-time setting):
+// operand loads marked evict_last and output stores evict_first, so that the
+// outputs streaming through L2 do not push out operand blocks that other CTA
+// pairs read again.
+#ifndef FP8DS_L2_HINTS
+#define FP8DS_L2_HINTS 0
+#endif
+#if FP8DS_L2_HINTS
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+#endif
+
 // TMA tile load into this CTA's shared memory, completion on a barrier of
 // this CTA.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,
                                             int32_t x, int32_t y) {
+#if FP8DS_L2_HINTS
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(l2_policy_evict_last())
+        : "memory");
+#else
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
+#endif
 }
 
 // TMA tile load into this CTA's shared memory whose completion is signalled
 // on a barrier of the pair's first CTA (bar_cluster_addr, shared::cluster).
 __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_cluster_addr, void *dst,
                                                  int32_t x, int32_t y) {
+#if FP8DS_L2_HINTS
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y), "l"(l2_policy_evict_last())
+        : "memory");
+#else
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y)
         : "memory");
+#endif
 }
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x,
                                              int32_t y) {
+#if FP8DS_L2_HINTS
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+                     map),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "l"(l2_policy_evict_first())
+                 : "memory");
+#else
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
                  "r"(smem_u32(src)), "r"(x), "r"(y)
                  : "memory");
+#endif
 }
 
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -903,8 +946,10 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
 // load has completed; the staging and the TMA stores follow while the next
 // tile's MMAs already run.
 //
-// FP8 output: the codes of both halves fit in registers (32 words per half
-// and lane), so the whole accumulator is released before anything is stored.
+// FP8 output: the codes of the first half go straight into the warp's
+// staging box (shared memory, not yet stored) and those of the last half
+// stay in registers (32 words per lane), so the whole accumulator is released
+// before anything is stored.
 template <bool BIAS, int MSUB>
 __device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uint8_t *boxes, int &nbox, int half,
                                                   const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row_h0,
@@ -914,8 +959,14 @@ __device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uin
     constexpr int CH = ACC_N / 2 / 32;  // chunks of 32 columns per warp and half
     const uint64_t sab2 = pack_f32x2(sab, sab);
     const uint64_t s2 = pack_f32x2(s_out, s_out);
-    uint32_t codes[MSUB][CH * 8];
+    uint32_t codes[CH * 8];
     uint32_t r[32];
+    uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
+    if (MSUB > 1) {
+        // the store last issued from this box must have finished reading it
+        if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
+        __syncwarp();
+    }
 #pragma unroll
     for (int h = 0; h < MSUB; ++h) {
         const uint32_t t_h = t_row0 + static_cast<uint32_t>(h * ACC_N + half * (ACC_N / 2));
@@ -930,6 +981,7 @@ __device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uin
                 if (lane == 0) mbar_arrive_cluster(empty_base + static_cast<uint32_t>(split ? h * sizeof(uint64_t) : 0));
             }
             const float *bs = bias_s + half * (ACC_N / 2) + c * 32;
+            uint32_t w[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float4 b = bias4<BIAS>(bs + 4 * j);
@@ -945,46 +997,66 @@ __device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uin
                 amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
                 const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
                 const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
-                codes[h][8 * c + j] =
-                    cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) | (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
+                w[j] = cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) | (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
             }
-            if (c + 1 < CH) {
-                tmem_ld32(t_h + static_cast<uint32_t>((c + 1) * 32), r);
-                tmem_ld_wait();
+            if (c + 1 < CH) tmem_ld32(t_h + static_cast<uint32_t>((c + 1) * 32), r);
+            if (h < MSUB - 1) {
+                // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
+                *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c) ^ (lane & 7)) * 16) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c + 1) ^ (lane & 7)) * 16) =
+                    make_uint4(w[4], w[5], w[6], w[7]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) codes[8 * c + j] = w[j];
             }
+            if (c + 1 < CH) tmem_ld_wait();
         }
     }
-#pragma unroll
-    for (int h = 0; h < MSUB; ++h) {
-        uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
-        if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
-        __syncwarp();
-        // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
-#pragma unroll
-        for (int k = 0; k < 2 * CH; ++k)
-            *reinterpret_cast<uint4 *>(box + lane * 128 + (k ^ (lane & 7)) * 16) =
-                make_uint4(codes[h][4 * k], codes[h][4 * k + 1], codes[h][4 * k + 2], codes[h][4 * k + 3]);
+    if (MSUB > 1) {
+        // the first half, staged while the accumulator was read
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
-            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)), m_row_h0 + h * rows_per_sub);
+            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)), m_row_h0);
             tma_store_commit();
         }
         ++nbox;
+        box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
     }
+    // the last half, from registers
+    if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 2 * CH; ++k)
+        *reinterpret_cast<uint4 *>(box + lane * 128 + (k ^ (lane & 7)) * 16) =
+            make_uint4(codes[4 * k], codes[4 * k + 1], codes[4 * k + 2], codes[4 * k + 3]);
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)),
+                     m_row_h0 + (MSUB - 1) * rows_per_sub);
+        tma_store_commit();
+    }
+    ++nbox;
 }
 
-// bf16 output: the 128 columns of one half take 64 words per lane, so each
-// half is read, converted and released, then stored (two staging boxes of
-// 64 columns) before the next half is read.
+// bf16 output: a half is 128 columns, two staging boxes of 64 columns.  The
+// first box is staged in shared memory while the half is read, the second
+// box's 32 words per lane stay in registers; the half is released (or, at
+// the last half, the accumulator) before the boxes are stored.  Halves are
+// read one after the other.
 template <bool BIAS>
 __device__ __forceinline__ void epilogue_bf16_regs(uint32_t t_h, int lane, uint8_t *boxes, int &nbox, int half,
                                                    const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                                    float sab, const float *bias_s, uint32_t empty_addr,
                                                    bool release) {
-    constexpr int CH = ACC_N / 2 / 32;
-    uint32_t packed[CH * 16];
+    constexpr int CH = ACC_N / 2 / 32;   // 4 chunks of 32 columns; 2 per box
+    uint32_t packed[16 * (CH / 2)];      // the second box
     uint32_t r[32];
+    uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
+    if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
+    __syncwarp();
     tmem_ld32(t_h + static_cast<uint32_t>(half * (ACC_N / 2)), r);
     tmem_ld_wait();
 #pragma unroll
@@ -995,6 +1067,7 @@ __device__ __forceinline__ void epilogue_bf16_regs(uint32_t t_h, int lane, uint8
             if (lane == 0) mbar_arrive_cluster(empty_addr);
         }
         const float *bs = bias_s + half * (ACC_N / 2) + c * 32;
+        uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float4 b = bias4<BIAS>(bs + 4 * j);
@@ -1002,33 +1075,45 @@ __device__ __forceinline__ void epilogue_bf16_regs(uint32_t t_h, int lane, uint8
                                                       fmaf(__uint_as_float(r[4 * j + 1]), sab, b.y));
             __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j + 2]), sab, b.z),
                                                       fmaf(__uint_as_float(r[4 * j + 3]), sab, b.w));
-            packed[16 * c + 2 * j] = *reinterpret_cast<uint32_t *>(&ha);
-            packed[16 * c + 2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
+            w[2 * j] = *reinterpret_cast<uint32_t *>(&ha);
+            w[2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
         }
-        if (c + 1 < CH) {
-            tmem_ld32(t_h + static_cast<uint32_t>(half * (ACC_N / 2) + (c + 1) * 32), r);
-            tmem_ld_wait();
-        }
-    }
-    // two boxes of 64 columns (128 bytes per row)
+        if (c + 1 < CH) tmem_ld32(t_h + static_cast<uint32_t>(half * (ACC_N / 2) + (c + 1) * 32), r);
+        if (c < CH / 2) {
+            // 32 columns = 64 bytes of the box row: 16-byte chunks (c % 2) * 4 + k,
+            // swizzled with lane & 7
 #pragma unroll
-    for (int bx = 0; bx < 2; ++bx) {
-        uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
-        if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
-        __syncwarp();
+            for (int k = 0; k < 4; ++k)
+                *reinterpret_cast<uint4 *>(box + lane * 128 + (((c % 2) * 4 + k) ^ (lane & 7)) * 16) =
+                    make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        } else {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4 *>(box + lane * 128 + (k ^ (lane & 7)) * 16) =
-                make_uint4(packed[32 * bx + 4 * k], packed[32 * bx + 4 * k + 1], packed[32 * bx + 4 * k + 2],
-                           packed[32 * bx + 4 * k + 3]);
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2) + bx * 64), m_row0);
-            tma_store_commit();
+            for (int j = 0; j < 16; ++j) packed[16 * (c - CH / 2) + j] = w[j];
         }
-        ++nbox;
+        if (c + 1 < CH) tmem_ld_wait();
     }
+    // first box (staged during the read), then the second from registers
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)), m_row0);
+        tma_store_commit();
+    }
+    ++nbox;
+    box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
+    if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<uint4 *>(box + lane * 128 + (k ^ (lane & 7)) * 16) =
+            make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+    fence_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2) + 64), m_row0);
+        tma_store_commit();
+    }
+    ++nbox;
 }
 
 // Shared-memory carve-up common to both kernels.
