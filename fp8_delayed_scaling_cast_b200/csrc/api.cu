@@ -6,8 +6,6 @@
 
 #include <atomic>
 #include <mutex>
-#include <set>
-#include <utility>
 #include <vector>
 
 #include "fp8ds_internal.h"
@@ -42,24 +40,6 @@ int num_sms() {
         cached[dev].store(n, std::memory_order_relaxed);
     }
     return n;
-}
-
-#ifndef FP8DS_CARVEOUT_MAX
-#define FP8DS_CARVEOUT_MAX 1
-#endif
-
-void ensure_carveout(const void *kernel) {
-#if FP8DS_CARVEOUT_MAX
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return;
-    static std::mutex mu;
-    static std::set<std::pair<const void *, int>> done;
-    std::lock_guard<std::mutex> g(mu);
-    if (done.insert({kernel, dev}).second)
-        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-#else
-    (void)kernel;
-#endif
 }
 
 namespace {

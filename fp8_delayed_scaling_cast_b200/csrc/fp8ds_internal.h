@@ -106,13 +106,6 @@ cudaError_t read_cast_error(int32_t *out, bool clear);
 bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
-// Every kernel of the library asks for the largest shared-memory carveout
-// (set once per kernel and device), so that consecutive launches of
-// different kernels -- casts, GEMMs, the update -- leave an SM's L1 /
-// shared-memory split unchanged between them (FP8DS_CARVEOUT_MAX, compile-
-// time setting).
-void ensure_carveout(const void *kernel);
-
 // Launches a kernel with programmatic stream serialization (the kernel may
 // start before the previous one in the stream completes; it synchronises
 // itself with griddepcontrol.wait) and, if cluster_x > 1, thread-block
@@ -120,7 +113,6 @@ void ensure_carveout(const void *kernel);
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                        unsigned cluster_x, Args &&...args) {
-    ensure_carveout(reinterpret_cast<const void *>(kernel));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;

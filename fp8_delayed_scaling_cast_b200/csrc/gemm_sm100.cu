@@ -241,10 +241,11 @@ __device__ __noinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     }
 }
 
-// L2 policy of the TMA traffic (FP8DS_L2_HINTS, compile-time setting):
-// operand loads marked evict_last and output stores evict_first, so that the
-// outputs streaming through L2 do not push out operand blocks that other CTA
-// pairs read again.
+// L2 policy of the TMA traffic (FP8DS_L2_HINTS, compile-time setting): 1 =
+// operand loads marked evict_last; 2 = also output stores evict_first, so
+// that the outputs streaming through L2 do not push out operand blocks that
+// other CTA pairs read again (but then a GEMM whose output feeds the next
+// one finds it in DRAM).
 #ifndef FP8DS_L2_HINTS
 #define FP8DS_L2_HINTS 0
 #endif
@@ -254,7 +255,7 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+__device__ __forceinline__ __attribute__((unused)) uint64_t l2_policy_evict_first() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
@@ -301,7 +302,7 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x,
                                              int32_t y) {
-#if FP8DS_L2_HINTS
+#if FP8DS_L2_HINTS >= 2
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
                      map),
                  "r"(smem_u32(src)), "r"(x), "r"(y), "l"(l2_policy_evict_first())
