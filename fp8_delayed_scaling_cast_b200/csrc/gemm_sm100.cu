@@ -241,77 +241,33 @@ __device__ __noinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     }
 }
 
-// L2 policy of the TMA traffic (FP8DS_L2_HINTS, compile-time setting): 1 =
-// operand loads marked evict_last; 2 = also output stores evict_first, so
-// that the outputs streaming through L2 do not push out operand blocks that
-// other CTA pairs read again (but then a GEMM whose output feeds the next
-// one finds it in DRAM).
-#ifndef FP8DS_L2_HINTS
-#define FP8DS_L2_HINTS 0
-#endif
-#if FP8DS_L2_HINTS
-__device__ __forceinline__ uint64_t l2_policy_evict_last() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-__device__ __forceinline__ __attribute__((unused)) uint64_t l2_policy_evict_first() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-#endif
-
 // TMA tile load into this CTA's shared memory, completion on a barrier of
 // this CTA.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,
                                             int32_t x, int32_t y) {
-#if FP8DS_L2_HINTS
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(l2_policy_evict_last())
-        : "memory");
-#else
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
         : "memory");
-#endif
 }
 
 // TMA tile load into this CTA's shared memory whose completion is signalled
 // on a barrier of the pair's first CTA (bar_cluster_addr, shared::cluster).
 __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_t bar_cluster_addr, void *dst,
                                                  int32_t x, int32_t y) {
-#if FP8DS_L2_HINTS
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y), "l"(l2_policy_evict_last())
-        : "memory");
-#else
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y)
         : "memory");
-#endif
 }
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t x,
                                              int32_t y) {
-#if FP8DS_L2_HINTS >= 2
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
-                     map),
-                 "r"(smem_u32(src)), "r"(x), "r"(y), "l"(l2_policy_evict_first())
-                 : "memory");
-#else
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
                  "r"(smem_u32(src)), "r"(x), "r"(y)
                  : "memory");
-#endif
 }
 
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -558,25 +514,31 @@ __device__ __forceinline__ bool epilogue_any(bool v) {
     return r != 0;
 }
 
-// Stage bias[n_base .. n_base+255] (0 when absent or past N) as fp32 in
-// shared memory; called by all epilogue threads between epilogue_any() and
-// epilogue_bar().
-__device__ __forceinline__ void stage_bias(float *bias_s, const Params &p, int64_t n_base, int epi_tid) {
+// The tile's bias, bias[n_base .. n_base+255] (0 when absent or past N), as
+// fp32: load_bias reads this thread's values from global memory (issued
+// before the epilogue waits for the accumulator, so the load overlaps the
+// wait), stage_bias stores them in shared memory once every epilogue warp is
+// done with the previous tile's copy.
+constexpr int BIAS_PER_THREAD = ACC_N / EPI_THREADS;
+__device__ __forceinline__ void load_bias(float (&v)[BIAS_PER_THREAD], const Params &p, int64_t n_base,
+                                          int epi_tid) {
 #pragma unroll
-    for (int i = 0; i < ACC_N / EPI_THREADS; ++i) {
-        const int c = epi_tid + i * EPI_THREADS;
-        const int64_t n = n_base + c;
-        float v = 0.0f;
+    for (int i = 0; i < BIAS_PER_THREAD; ++i) {
+        const int64_t n = n_base + epi_tid + i * EPI_THREADS;
+        v[i] = 0.0f;
         if (p.bias_kind != 0 && n < p.N) {
             if (p.bias_kind == 1) {
-                v = __ldg(static_cast<const float *>(p.bias) + n);
+                v[i] = __ldg(static_cast<const float *>(p.bias) + n);
             } else {
                 const uint16_t b = __ldg(static_cast<const uint16_t *>(p.bias) + n);
-                v = __uint_as_float(static_cast<uint32_t>(b) << 16);
+                v[i] = __uint_as_float(static_cast<uint32_t>(b) << 16);
             }
         }
-        bias_s[c] = v;
     }
+}
+__device__ __forceinline__ void stage_bias(float *bias_s, const float (&v)[BIAS_PER_THREAD], int epi_tid) {
+#pragma unroll
+    for (int i = 0; i < BIAS_PER_THREAD; ++i) bias_s[epi_tid + i * EPI_THREADS] = v[i];
 }
 
 // Tile order: groups of GROUP_M row-tiles; inside a group the row index runs
@@ -1184,6 +1146,8 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
         const uint32_t acc_phase = static_cast<uint32_t>(acc_bufs == 2 ? (local >> 1) : local) & 1u;
         ++local;
         const int mode = kb0 > 0 ? 1 : (kb1 < p.num_kb ? 2 : 0);
+        float bias_v[BIAS_PER_THREAD];
+        load_bias(bias_v, p, static_cast<int64_t>(n_blk) * ACC_N, epi_tid);
         bool ok = mbar_wait(&sm.tfull[acc], acc_phase, sm.abort_flag, SITE_EPI_TMEM_FULL);
         float *slot = nullptr;
         int32_t *flag = nullptr;
@@ -1207,7 +1171,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
         // All epilogue warps meet here every tile: they leave together if any
         // wait gave up, and none of them still reads the previous tile's bias.
         if (epilogue_any(!ok)) break;
-        stage_bias(bias_s, p, static_cast<int64_t>(n_blk) * ACC_N, epi_tid);
+        stage_bias(bias_s, bias_v, epi_tid);
         epilogue_bar();
         tc_fence_after();
         // An accumulator is released whole (tempty[acc]) after its last row
