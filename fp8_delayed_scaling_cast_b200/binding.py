@@ -85,6 +85,7 @@ _SIGS = {
     "fp8_gemm_ex": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P,
                     ctypes.c_size_t, _P],
     "fp8_gemm_workspace_size": [ctypes.POINTER(ctypes.c_size_t)],
+    "fp8_gemm_plan": [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)],
     "fp8_gemm_noalloc": [_P, _INT, _P, _P, _INT, _P, _P, _INT, _P, _INT, _I64, _I64, _I64, _P],
     "fp8_gemm_cast": [_P, _INT, _INT, _P, _P, _INT, _INT, _P, _P, _INT, _I64, _I64, _I64, _INT, _P, _P, _P, _P, _P,
                       _P],
@@ -284,6 +285,15 @@ def fp8_gemm_workspace_size():
     n = ctypes.c_size_t(0)
     _check(_lib.fp8_gemm_workspace_size(ctypes.byref(n)))
     return n.value
+
+
+def fp8_gemm_plan(m, n, k):
+    """The GEMM's tile schedule on the current device: dict with pair,
+    m_sub, tiles, stream_k (taken with a workspace) and resident pairs."""
+    info = (ctypes.c_int64 * 5)()
+    _check(_lib.fp8_gemm_plan(m, n, k, info))
+    return {"pair": bool(info[0]), "m_sub": int(info[1]), "tiles": int(info[2]), "stream_k": bool(info[3]),
+            "resident": int(info[4])}
 
 
 def gemm_workspace(device="cuda"):

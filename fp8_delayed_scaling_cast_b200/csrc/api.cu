@@ -294,6 +294,14 @@ fp8ds_status fp8_gemm_workspace_size(size_t *bytes) {
     return FP8DS_OK;
 }
 
+fp8ds_status fp8_gemm_plan(int64_t m, int64_t n, int64_t k, int64_t *info) {
+    clear_error();
+    if (info == nullptr) return invalid("fp8_gemm_plan: info must not be NULL");
+    if (m <= 0 || n <= 0 || k <= 0) return invalid("fp8_gemm_plan: m, n, k must be positive");
+    gemm_plan_info(m, n, k, info);
+    return FP8DS_OK;
+}
+
 fp8ds_status fp8_gemm_ex(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
                          fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
                          void *d, fp8ds_dtype d_dtype, int64_t m, int64_t n, int64_t k, void *workspace,

@@ -85,6 +85,8 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
 
 // Workspace bytes the stream-K schedule needs on the current device.
 size_t gemm_workspace_bytes();
+// The tile schedule of an m x n x k GEMM on the current device (fp8_gemm_plan).
+void gemm_plan_info(int64_t m, int64_t n, int64_t k, int64_t info[5]);
 
 // launch_gemm with the library's static device scratch as the workspace.
 fp8ds_status launch_gemm_noalloc(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv,

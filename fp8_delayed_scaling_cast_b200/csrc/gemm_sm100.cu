@@ -431,10 +431,12 @@ struct Params {
     int bias_kind;  // 0 none, 1 fp32, 2 bf16
     int32_t M, N, K;
     int32_t tiles_m, tiles_n, num_kb;
+    int32_t group_m;      // row tiles per raster group (tile_coords)
     uint32_t idesc;
     int32_t a_mn, b_mn;   // 1: the operand is stored MN-major ([K, M] / [K, N] row-major)
     // stream-K (pair kernel only): 0 = whole tiles per cluster
     int32_t stream_k;
+    int32_t sk_pairs;     // clusters the workspace has partial slots for
     uint32_t epoch;       // non-zero per launch; partials are published with it
     int32_t *flags;       // [clusters][2] publication words
     float *partials;      // [clusters][2 CTAs][2 row blocks][128 x 256] fp32
@@ -458,40 +460,41 @@ struct Params {
 constexpr size_t WS_FLAG_BYTES = 4096;  // room for 1024 clusters
 constexpr size_t WS_SLOT_FLOATS = 2 * 2 * 128 * 256;
 
-// Work assignment of a cluster (or CTA).  Stream-K: cluster c of C owns the
-// units [c*U/C, (c+1)*U/C) of the U = tiles * num_kb (tile, k-block) units in
-// tile order, as segments (tile, kb0, kb1); requires tiles >= C so that a
-// tile is split between at most two clusters.  Otherwise whole tiles c,
-// c + C, ...
+// Work assignment of a cluster (or CTA).  Whole tiles c, c + C, ... (C
+// clusters).  With stream-K, only the tiles of the whole waves go that way
+// (the first floor(T / C) * C of the T tiles); the U = R * num_kb (tile,
+// k-block) units of the R remaining tiles are shared out afterwards, cluster
+// c taking the units [c*U/C, (c+1)*U/C) in tile order as segments (tile,
+// kb0, kb1).  A split tile's segments belong to consecutive clusters, the
+// one with kb0 = 0 (the last segment of its cluster's range) storing D.
 struct Sched {
     int64_t u, u1;
-    int t, stride, num_tiles, num_kb;
-    bool sk;
+    int t, stride, dp_tiles, num_kb;
     __device__ __forceinline__ Sched(const Params &p, int c, int C) {
-        num_tiles = p.tiles_m * p.tiles_n;
+        const int num_tiles = p.tiles_m * p.tiles_n;
         num_kb = p.num_kb;
-        sk = p.stream_k != 0;
-        const int64_t U = static_cast<int64_t>(num_tiles) * num_kb;
-        u = U * c / C;
-        u1 = U * (c + 1) / C;
+        dp_tiles = p.stream_k != 0 ? (num_tiles / C) * C : num_tiles;
+        const int64_t base = static_cast<int64_t>(dp_tiles) * num_kb;
+        const int64_t U = static_cast<int64_t>(num_tiles - dp_tiles) * num_kb;
+        u = base + U * c / C;
+        u1 = base + U * (c + 1) / C;
         t = c;
         stride = C;
     }
     __device__ __forceinline__ bool next(int &tile, int &kb0, int &kb1) {
-        if (sk) {
-            if (u >= u1) return false;
-            tile = static_cast<int>(u / num_kb);
-            kb0 = static_cast<int>(u % num_kb);
-            const int64_t left = u1 - u;
-            kb1 = left < num_kb - kb0 ? kb0 + static_cast<int>(left) : num_kb;
-            u += kb1 - kb0;
+        if (t < dp_tiles) {
+            tile = t;
+            kb0 = 0;
+            kb1 = num_kb;
+            t += stride;
             return true;
         }
-        if (t >= num_tiles) return false;
-        tile = t;
-        kb0 = 0;
-        kb1 = num_kb;
-        t += stride;
+        if (u >= u1) return false;
+        tile = static_cast<int>(u / num_kb);
+        kb0 = static_cast<int>(u % num_kb);
+        const int64_t left = u1 - u;
+        kb1 = left < num_kb - kb0 ? kb0 + static_cast<int>(left) : num_kb;
+        u += kb1 - kb0;
         return true;
     }
 };
@@ -541,12 +544,14 @@ __device__ __forceinline__ void stage_bias(float *bias_s, const float (&v)[BIAS_
     for (int i = 0; i < BIAS_PER_THREAD; ++i) bias_s[epi_tid + i * EPI_THREADS] = v[i];
 }
 
-// Tile order: groups of GROUP_M row-tiles; inside a group the row index runs
-// fastest, so CTAs that run together share B columns and a band of A rows.
-__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int &m_blk, int &n_blk) {
-    const int group_size = GROUP_M * tiles_n;
-    const int first_m = (tile / group_size) * GROUP_M;
-    const int rows = min(tiles_m - first_m, GROUP_M);
+// Tile order: groups of `group` row-tiles; inside a group the row index runs
+// fastest, so CTAs that run together share B columns and a band of A rows
+// (group 1: whole rows of tiles, the column index running fastest).
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int group, int &m_blk,
+                                            int &n_blk) {
+    const int group_size = group * tiles_n;
+    const int first_m = (tile / group_size) * group;
+    const int rows = min(tiles_m - first_m, group);
     const int in_group = tile % group_size;
     m_blk = first_m + in_group % rows;
     n_blk = in_group / rows;
@@ -565,32 +570,56 @@ __device__ __forceinline__ float4 *partial_at(float *slot, int h, int q, int col
     return reinterpret_cast<float4 *>(slot) + ((h * 4 + q) * 64 + col / 4) * 32 + lane;
 }
 
-// Store (mode 1) or add (mode 2) the partial accumulator of 32 columns.
-__device__ __forceinline__ void partial_io(int mode, uint32_t *r, float *slot, int h, int q, int col0,
-                                           int lane) {
+// Add the partial of the next cluster (mode bit 2, from `in`), then store
+// the sum as this segment's partial (mode bit 1, to `out`), for 32 columns.
+constexpr int PART_OUT = 1;
+constexpr int PART_IN = 2;
+__device__ __forceinline__ void partial_io(int mode, uint32_t *r, const float *in, float *out, int h, int q,
+                                           int col0, int lane) {
+    if (mode & PART_IN) {
+        float4 v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float4 *ptr = partial_at(slot, h, q, col0 + 4 * i, lane);
-        if (mode == 1) {
-            *ptr = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-        } else {
-            const float4 v = __ldcg(ptr);
-            r[4 * i] = __float_as_uint(__uint_as_float(r[4 * i]) + v.x);
-            r[4 * i + 1] = __float_as_uint(__uint_as_float(r[4 * i + 1]) + v.y);
-            r[4 * i + 2] = __float_as_uint(__uint_as_float(r[4 * i + 2]) + v.z);
-            r[4 * i + 3] = __float_as_uint(__uint_as_float(r[4 * i + 3]) + v.w);
+        for (int i = 0; i < 8; ++i) v[i] = __ldcg(partial_at(const_cast<float *>(in), h, q, col0 + 4 * i, lane));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            r[4 * i] = __float_as_uint(__uint_as_float(r[4 * i]) + v[i].x);
+            r[4 * i + 1] = __float_as_uint(__uint_as_float(r[4 * i + 1]) + v[i].y);
+            r[4 * i + 2] = __float_as_uint(__uint_as_float(r[4 * i + 2]) + v[i].z);
+            r[4 * i + 3] = __float_as_uint(__uint_as_float(r[4 * i + 3]) + v[i].w);
         }
+    }
+    if (mode & PART_OUT) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            *partial_at(out, h, q, col0 + 4 * i, lane) =
+                make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]), __uint_as_float(r[4 * i + 2]),
+                            __uint_as_float(r[4 * i + 3]));
     }
 }
 
-// mode 0: convert and store D; mode 1: store the raw partial (no D); mode 2:
-// add the partial of the other cluster, then convert and store D.
-// The warp reads its 128 columns as four 32-column TMEM loads (which keeps
-// the live registers within the 168 that 10 warps per SM allow).  The load
-// of chunk c + 1 is issued as soon as chunk c has been converted, into the
-// same registers, so its latency overlaps chunk c's staging and store; the
-// loop is fully unrolled so that every load has its own registers.
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic; each lane rounds exactly as
+// the scalar fmaf / __fmul_rn).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
+}
+__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// D = acc * sab + bias for two adjacent columns (the raw TMEM words r0, r1).
+__device__ __forceinline__ uint64_t scale_bias2(uint32_t r0, uint32_t r1, uint64_t sab2, float b0, float b1) {
+    return fma_f32x2(pack_f32x2(__uint_as_float(r0), __uint_as_float(r1)), sab2, pack_f32x2(b0, b1));
+}
+
 // Four bias values from the tile's shared-memory copy.  BIAS false: the bias
 // is absent and its (zero) copy is not read; the arithmetic is the same fma
 // with +0.
@@ -626,15 +655,27 @@ __device__ __forceinline__ void store_row_direct(void *out, int32_t m, int64_t n
     }
 }
 
+// Stream-K modes (bits): 1 = the segment does not end the tile's k-range at
+// its start (kb0 > 0), so it stores its raw partial sum for the tile's owner
+// instead of D; 2 = the tile's k-range goes on after the segment (kb1 <
+// num_kb), so it first adds the partial of the cluster that holds the rest.
+// Mode 0 converts and stores D.
+// The warp reads its 128 columns as four 32-column TMEM loads (which keeps
+// the live registers within the 168 that 10 warps per SM allow).  The load
+// of chunk c + 1 is issued as soon as chunk c has been converted, into the
+// same registers, so its latency overlaps chunk c's staging and store; the
+// loop is fully unrolled so that every load has its own registers.
 template <bool OUT_BF16, bool BIAS>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *boxes, int &nbox, int half,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                               float sab, const float *bias_s, uint32_t empty_bar_cluster,
-                                              bool arrive, int mode, float *slot, int h, int q, void *out,
+                                              bool arrive, int mode, const float *p_in, float *p_out, int h, int q,
+                                              void *out,
                                               int32_t m_total, int32_t n_total, bool v8) {
     constexpr int SUBS_PER_BOX = OUT_BF16 ? 2 : 1;  // 32-column sub-blocks per staging box
     constexpr int CHUNKS = ACC_N / 2 / EPI_LD;      // TMEM loads per warp and row block
     constexpr int SUBS = EPI_LD / 32;               // 32-column sub-blocks per load
+    const uint64_t sab2 = pack_f32x2(sab, sab);
     uint32_t r[EPI_LD];
     tmem_ld(t_row + half * (ACC_N / 2), r);
     tmem_ld_wait();
@@ -652,8 +693,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             const int col0 = half * (ACC_N / 2) + (c * SUBS + sb) * 32;  // accumulator column
             const int hh = (col0 / 32) % SUBS_PER_BOX;
             const bool last_of_chunk = sb == SUBS - 1;
-            if (mode != 0) partial_io(mode, rr, slot, h, q, col0, lane);
-            if (EPI_DIRECT && mode != 1) {
+            if (mode != 0) partial_io(mode, rr, p_in, p_out, h, q, col0, lane);
+            if (EPI_DIRECT && !(mode & PART_OUT)) {
                 const float *bs = bias_s + col0;
                 if (OUT_BF16) {
                     uint32_t packed[16];
@@ -680,7 +721,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
                     }
                     store_row_direct<false>(out, m_row0 + lane, n_base + col0, m_total, n_total, v8, v);
                 }
-            } else if (mode != 1) {
+            } else if (!(mode & PART_OUT)) {
                 uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
                 if (hh == 0) {
                     // Staging buffer reuse: the store issued from this box
@@ -697,10 +738,10 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const float4 b = bias4<BIAS>(bs + 4 * j);
-                        __nv_bfloat162 ha = __floats2bfloat162_rn(fmaf(__uint_as_float(rr[4 * j]), sab, b.x),
-                                                                  fmaf(__uint_as_float(rr[4 * j + 1]), sab, b.y));
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(rr[4 * j + 2]), sab, b.z),
-                                                                  fmaf(__uint_as_float(rr[4 * j + 3]), sab, b.w));
+                        const uint64_t v01 = scale_bias2(rr[4 * j], rr[4 * j + 1], sab2, b.x, b.y);
+                        const uint64_t v23 = scale_bias2(rr[4 * j + 2], rr[4 * j + 3], sab2, b.z, b.w);
+                        __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
+                        __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
                         packed[2 * j] = *reinterpret_cast<uint32_t *>(&ha);
                         packed[2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
                     }
@@ -715,17 +756,17 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
                     for (int k = 0; k < 8; ++k) {
                         const int pc = k ^ (lane & 7);
                         const float4 b = bias4<BIAS>(bs + 4 * k);
+                        const uint64_t v01 = scale_bias2(rr[4 * k], rr[4 * k + 1], sab2, b.x, b.y);
+                        const uint64_t v23 = scale_bias2(rr[4 * k + 2], rr[4 * k + 3], sab2, b.z, b.w);
                         *reinterpret_cast<uint4 *>(box + lane * 128 + pc * 16) =
-                            make_uint4(__float_as_uint(fmaf(__uint_as_float(rr[4 * k]), sab, b.x)),
-                                       __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 1]), sab, b.y)),
-                                       __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 2]), sab, b.z)),
-                                       __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 3]), sab, b.w)));
+                            make_uint4(static_cast<uint32_t>(v01), static_cast<uint32_t>(v01 >> 32),
+                                       static_cast<uint32_t>(v23), static_cast<uint32_t>(v23 >> 32));
                     }
                 }
             }
             // the registers of r are free: start the next chunk's TMEM load
             if (last_of_chunk && c + 1 < CHUNKS) tmem_ld(t_row + half * (ACC_N / 2) + (c + 1) * EPI_LD, r);
-            if (!EPI_DIRECT && mode != 1 && hh == SUBS_PER_BOX - 1) {
+            if (!EPI_DIRECT && !(mode & PART_OUT) && hh == SUBS_PER_BOX - 1) {
                 uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
                 fence_async_smem();
                 __syncwarp();
@@ -740,24 +781,6 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
         }
         if (c + 1 < CHUNKS) tmem_ld_wait();
     }
-}
-
-// Packed pairs of fp32 (sm_100 f32x2 arithmetic; each lane rounds exactly as
-// the scalar fmaf / __fmul_rn).
-__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
-    return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
-}
-__device__ __forceinline__ float lo_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
-__device__ __forceinline__ float hi_f32(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
-__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
 }
 
 // Two FP8 codes (saturating, round to nearest even) packed in 16 bits:
@@ -802,7 +825,8 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
                                                   uint8_t *d8, uint8_t *d8t, const CUtensorMap *tmap_d,
                                                   int64_t n_base, int32_t m_row0, float sab,
                                                   const float *bias_s, uint32_t empty_bar_cluster, bool arrive,
-                                                  int mode, float *slot, int h, int q, float s_out, int fmt,
+                                                  int mode, const float *p_in, float *p_out, int h, int q,
+                                                  float s_out, int fmt,
                                                   int32_t m_total, int32_t n_total, float &amax) {
     constexpr int CHUNKS = ACC_N / 2 / EPI_LD;  // TMEM loads per warp and row block
     constexpr int SUBS = EPI_LD / 32;           // 32-column sub-blocks per load
@@ -812,7 +836,7 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
     // out with plain stores beside the transposed ones (in box 0's memory).
     const bool staged = !EPI_DIRECT && d8t == nullptr;
     uint8_t *box = staged ? boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES : boxes;
-    if (staged && mode != 1) {
+    if (staged && !(mode & PART_OUT)) {
         if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
         __syncwarp();
     }
@@ -833,9 +857,9 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
             uint32_t *rr = r + 32 * sb;
             const int cs = c * SUBS + sb;              // sub-block within the warp's 128 columns
             const int col0 = half * (ACC_N / 2) + cs * 32;
-            if (mode != 0) partial_io(mode, rr, slot, h, q, col0, lane);
+            if (mode != 0) partial_io(mode, rr, p_in, p_out, h, q, col0, lane);
             uint32_t w[8];
-            if (mode != 1) {
+            if (!(mode & PART_OUT)) {
                 const float *bs = bias_s + col0;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -859,13 +883,13 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
             }
             // the registers of r are free: start the next chunk's TMEM load
             if (sb == SUBS - 1 && c + 1 < CHUNKS) tmem_ld(t_row + half * (ACC_N / 2) + (c + 1) * EPI_LD, r);
-            if (mode != 1 && staged) {
+            if (!(mode & PART_OUT) && staged) {
                 // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
                 *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * cs) ^ (lane & 7)) * 16) =
                     make_uint4(w[0], w[1], w[2], w[3]);
                 *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * cs + 1) ^ (lane & 7)) * 16) =
                     make_uint4(w[4], w[5], w[6], w[7]);
-            } else if (mode != 1) {
+            } else if (!(mode & PART_OUT)) {
                 const int64_t n0 = n_base + col0;
                 if (m < m_total && n0 < n_total)
                     store_segment(d8 + static_cast<int64_t>(m) * n_total + n0, n_total - n0, w);
@@ -890,7 +914,7 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
         }
         if (c + 1 < CHUNKS) tmem_ld_wait();
     }
-    if (staged && mode != 1) {
+    if (staged && !(mode & PART_OUT)) {
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -948,11 +972,8 @@ __device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uin
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const float4 b = bias4<BIAS>(bs + 4 * j);
-                const uint64_t v01 = fma_f32x2(pack_f32x2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])),
-                                               sab2, pack_f32x2(b.x, b.y));
-                const uint64_t v23 = fma_f32x2(
-                    pack_f32x2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), sab2,
-                    pack_f32x2(b.z, b.w));
+                const uint64_t v01 = scale_bias2(r[4 * j], r[4 * j + 1], sab2, b.x, b.y);
+                const uint64_t v23 = scale_bias2(r[4 * j + 2], r[4 * j + 3], sab2, b.z, b.w);
                 const __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
                 const __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
                 const float h0 = __low2float(ha), h1 = __high2float(ha);
@@ -1016,6 +1037,7 @@ __device__ __forceinline__ void epilogue_bf16_regs(uint32_t t_h, int lane, uint8
                                                    bool release) {
     constexpr int CH = ACC_N / 2 / 32;   // 4 chunks of 32 columns; 2 per box
     uint32_t packed[16 * (CH / 2)];      // the second box
+    const uint64_t sab2 = pack_f32x2(sab, sab);
     uint32_t r[32];
     uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
     if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
@@ -1034,10 +1056,10 @@ __device__ __forceinline__ void epilogue_bf16_regs(uint32_t t_h, int lane, uint8
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float4 b = bias4<BIAS>(bs + 4 * j);
-            __nv_bfloat162 ha = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j]), sab, b.x),
-                                                      fmaf(__uint_as_float(r[4 * j + 1]), sab, b.y));
-            __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(r[4 * j + 2]), sab, b.z),
-                                                      fmaf(__uint_as_float(r[4 * j + 3]), sab, b.w));
+            const uint64_t v01 = scale_bias2(r[4 * j], r[4 * j + 1], sab2, b.x, b.y);
+            const uint64_t v23 = scale_bias2(r[4 * j + 2], r[4 * j + 3], sab2, b.z, b.w);
+            __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
+            __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
             w[2 * j] = *reinterpret_cast<uint32_t *>(&ha);
             w[2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
         }
@@ -1141,25 +1163,34 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
     int local = 0, tile, kb0, kb1;
     while (sched.next(tile, kb0, kb1)) {
         int m_blk, n_blk;
-        tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
+        tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, m_blk, n_blk);
         const int acc = acc_bufs == 2 ? (local & 1) : 0;
         const uint32_t acc_phase = static_cast<uint32_t>(acc_bufs == 2 ? (local >> 1) : local) & 1u;
         ++local;
-        const int mode = kb0 > 0 ? 1 : (kb1 < p.num_kb ? 2 : 0);
+        const int seg = (kb0 > 0 ? PART_OUT : 0) | (kb1 < p.num_kb ? PART_IN : 0);
+        const int mode = seg;
         float bias_v[BIAS_PER_THREAD];
         load_bias(bias_v, p, static_cast<int64_t>(n_blk) * ACC_N, epi_tid);
         bool ok = mbar_wait(&sm.tfull[acc], acc_phase, sm.abort_flag, SITE_EPI_TMEM_FULL);
-        float *slot = nullptr;
-        int32_t *flag = nullptr;
-        if (mode != 0) {
-            const int s = mode == 1 ? cluster : cluster + 1;
-            slot = p.partials + (static_cast<size_t>(s) * 2 + rank) * WS_SLOT_FLOATS;
-            flag = p.flags + s * 2 + rank;
+        // A cluster's partial slot and publication word (per CTA of the pair):
+        // this segment's own (PART_OUT) and the next cluster's (PART_IN).
+        float *p_out = nullptr;
+        const float *p_in = nullptr;
+        int32_t *out_flag = nullptr, *in_flag = nullptr;
+        if (seg & PART_OUT) {
+            p_out = p.partials + (static_cast<size_t>(cluster) * 2 + rank) * WS_SLOT_FLOATS;
+            out_flag = p.flags + cluster * 2 + rank;
         }
-        if (mode == 2 && ok && epi_tid == 0) {
-            // The other cluster wrote this partial at the start of its range.
+        if (seg & PART_IN) {
+            p_in = p.partials + (static_cast<size_t>(cluster + 1) * 2 + rank) * WS_SLOT_FLOATS;
+            in_flag = p.flags + (cluster + 1) * 2 + rank;
+        }
+        if ((seg & PART_IN) && ok && epi_tid == 0) {
+            // The rest of this tile's k-range is the first segment of the next
+            // cluster's range (which, if it does not reach the tile's end
+            // either, has added the partial of the cluster after it).
             const uint64_t t0 = globaltimer();
-            while (ld_acquire(flag) != static_cast<int32_t>(p.epoch)) {
+            while (ld_acquire(in_flag) != static_cast<int32_t>(p.epoch)) {
                 if (*sm.abort_flag || globaltimer() - t0 > p.partial_wait_ns) {
                     *sm.abort_flag = 1;
                     record_error(SITE_EPI_PARTIAL);
@@ -1231,33 +1262,37 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             if constexpr (OUT == OUT_FP8) {
                 if (p.bias_kind != 0)
                     epilogue_tile_fp8<true>(t_row, lane, boxes, nbox, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
-                                            bias_s, empty_addr, release, mode, slot, h, q, s_out, p.out_fmt, p.M, p.N,
+                                            bias_s, empty_addr, release, mode, p_in, p_out, h, q, s_out, p.out_fmt, p.M,
+                                            p.N,
                                             amax);
                 else
                     epilogue_tile_fp8<false>(t_row, lane, boxes, nbox, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
-                                             bias_s, empty_addr, release, mode, slot, h, q, s_out, p.out_fmt, p.M, p.N,
+                                             bias_s, empty_addr, release, mode, p_in, p_out, h, q, s_out, p.out_fmt, p.M,
+                                            p.N,
                                              amax);
             } else {
                 if (p.bias_kind != 0)
                     epilogue_tile<OUT == OUT_BF16, true>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab, bias_s,
-                                                         empty_addr, release, mode, slot, h, q, p.out, p.M, p.N,
+                                                         empty_addr, release, mode, p_in, p_out, h, q, p.out, p.M, p.N,
                                                          p.out_v8 != 0);
                 else
                     epilogue_tile<OUT == OUT_BF16, false>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab,
-                                                          bias_s, empty_addr, release, mode, slot, h, q, p.out, p.M,
+                                                          bias_s, empty_addr, release, mode, p_in, p_out, h, q, p.out, p.M,
                                                           p.N, p.out_v8 != 0);
             }
         }
-        if (mode == 1) {
-            // Publish: every epilogue thread's partial stores precede the flag.
+        if (seg != 0) {
+            // Every epilogue thread is done with the partials: the next
+            // cluster's slot is consumed (free for the next launch), and this
+            // segment's own partial stores precede its publication.
             epilogue_bar();
             if (epi_tid == 0) {
-                __threadfence();
-                if (!p.withhold_partials) st_release(flag, static_cast<int32_t>(p.epoch));
+                if (seg & PART_IN) *in_flag = 0;
+                if (seg & PART_OUT) {
+                    __threadfence();
+                    if (!p.withhold_partials) st_release(out_flag, static_cast<int32_t>(p.epoch));
+                }
             }
-        } else if (mode == 2) {
-            epilogue_bar();
-            if (epi_tid == 0) *flag = 0;  // consumed; the slot is free for the next launch
         }
     }
     if constexpr (OUT == OUT_FP8) {
@@ -1326,7 +1361,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             int tile, kb0, kb1;
             while (ok && sched.next(tile, kb0, kb1)) {
                 int m_blk, n_blk;
-                tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
+                tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, m_blk, n_blk);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&sm.empty[stage], phase ^ 1u, sm.abort_flag, SITE_PRODUCER_EMPTY)) {
                         ok = false;
@@ -1488,7 +1523,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             int tile, kb0, kb1;
             while (ok && sched.next(tile, kb0, kb1)) {
                 int m_blk, n_blk;
-                tile_coords(tile, p.tiles_m, p.tiles_n, m_blk, n_blk);
+                tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, m_blk, n_blk);
                 const int32_t a_row = m_blk * M_SUB * 2 * S2_BM + static_cast<int32_t>(rank) * S2_BM;
                 const int32_t b_row = n_blk * ACC_N + static_cast<int32_t>(rank) * S2_BN_HALF;
                 for (int kb = kb0; kb < kb1; ++kb) {
@@ -1715,7 +1750,9 @@ cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
     const int cap = max_pairs(kernel, smem, cached_pairs);
-    const int pairs = tiles < cap ? tiles : cap;
+    // a stream-K launch shares its remaining tiles' k-blocks among all pairs
+    // (as many as the workspace has partial slots for)
+    const int pairs = p.stream_k != 0 ? (cap < p.sk_pairs ? cap : p.sk_pairs) : (tiles < cap ? tiles : cap);
     return launch_pdl(kernel, dim3(2 * pairs), dim3(THREADS), smem, stream, 2, ta, tb, td, p);
 }
 
@@ -1752,6 +1789,7 @@ struct GemmPlan {
     bool pair;
     int m_sub;
     int64_t tiles;
+    int group_m;     // raster group (tile_coords)
     bool stream_k;   // with a large enough workspace
 };
 
@@ -1774,15 +1812,36 @@ GemmPlan plan_gemm(int64_t m, int64_t n, int64_t k) {
         if (cap <= 0 || t2 * w1 * 50 >= t1 * w2 * 49) g.m_sub = 2;      // fill(512) >= fill(256) - 2%
     }
     const int64_t tile_m = g.pair ? g.m_sub * 2 * S2_BM : S1_BM;
-    g.tiles = ((m + tile_m - 1) / tile_m) * tn;
-    // Stream-K when whole tiles would leave a ragged last wave: at least one
-    // tile per pair, fewer than 8 waves, not a whole number of waves.
-    g.stream_k = g.pair && cap > 0 && g.tiles >= cap && g.tiles % cap != 0 && g.tiles < 8 * cap &&
-                 cap <= static_cast<int64_t>(WS_FLAG_BYTES / 8);
+    const int64_t tm = (m + tile_m - 1) / tile_m;
+    g.tiles = tm * tn;
+    // Raster: row groups of GROUP_M tiles keep a band of A and the B columns
+    // in L2 over many waves.  A pair launch of at most two waves with more
+    // row tiles than column tiles takes whole rows of tiles instead, so that
+    // each A row block (the larger operand) is streamed by one wave only and
+    // the second wave re-reads only the smaller B.
+    g.group_m = (g.pair && cap > 0 && g.tiles <= 2 * cap && tm > tn) ? 1 : GROUP_M;
+    // Stream-K (given a workspace) when whole tiles would leave a ragged
+    // last wave worth balancing: R = tiles mod pairs with pairs / 3 <= R <=
+    // 7/8 pairs (a split tile then spans at most four clusters, and at
+    // least an eighth of a tile's time is saved), fewer than 8 waves, at
+    // least 8 k-blocks per tile, and a publication word for every cluster.
+    const int64_t rem = cap > 0 ? g.tiles % cap : 0;
+    g.stream_k = g.pair && cap > 0 && 3 * rem >= cap && 8 * rem <= 7 * cap && g.tiles < 8 * cap &&
+                 (k + BK - 1) / BK >= 8 && cap <= static_cast<int64_t>(WS_FLAG_BYTES / 8);
     return g;
 }
 
 }  // namespace
+
+void gemm_plan_info(int64_t m, int64_t n, int64_t k, int64_t info[5]) {
+    static std::atomic<int> cached_pairs[64];
+    const GemmPlan g = plan_gemm(m, n, k);
+    info[0] = g.pair ? 1 : 0;
+    info[1] = g.pair ? g.m_sub : 0;
+    info[2] = g.tiles;
+    info[3] = g.stream_k ? 1 : 0;
+    info[4] = g.pair ? max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached_pairs) : num_sms();
+}
 
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
                          fp8ds_format b_fmt, const float *b_scale_inv, const void *bias, fp8ds_dtype bias_dtype,
@@ -1826,10 +1885,12 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.tiles_m = static_cast<int32_t>((m + tile_m - 1) / tile_m);
     p.tiles_n = static_cast<int32_t>((n + ACC_N - 1) / ACC_N);
     p.num_kb = static_cast<int32_t>((k + BK - 1) / BK);
+    p.group_m = plan.group_m;
     p.idesc = make_idesc(a_fmt, b_fmt, pair ? 2 * S2_BM : S1_BM, ACC_N, a_mn, b_mn);
     p.a_mn = a_mn ? 1 : 0;
     p.b_mn = b_mn ? 1 : 0;
     p.stream_k = 0;
+    p.sk_pairs = 0;
     p.epoch = 0;
     p.flags = nullptr;
     p.partials = nullptr;
@@ -1853,6 +1914,8 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
         uint32_t e = ++launches;
         if (e == 0) e = ++launches;
         p.stream_k = 1;
+        const size_t slots = (workspace_bytes - WS_FLAG_BYTES) / (2 * WS_SLOT_FLOATS * sizeof(float));
+        p.sk_pairs = static_cast<int32_t>(slots < WS_FLAG_BYTES / 8 ? slots : WS_FLAG_BYTES / 8);
         p.epoch = e;
         p.flags = static_cast<int32_t *>(workspace);
         p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + WS_FLAG_BYTES);

@@ -290,18 +290,38 @@ fp8ds_status fp8_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale
 fp8ds_status fp8_gemm_workspace_size(size_t *bytes);
 
 /*
+ * fp8_gemm_plan -- the tile schedule that fp8_gemm, fp8_gemm_ex,
+ * fp8_gemm_cast and the linear calls take for an m x n x k product on the
+ * current device; it has no counterpart on the pages (it tells a caller
+ * whether a workspace would change anything).  Host only; no device work.
+ *   info [5] int64, written:
+ *     info[0]  1: CTA-pair tiles (m > 128); 0: one-CTA tiles of 128 x 256
+ *     info[1]  pair tiles of 256 (1) or 512 (2) rows x 256 columns; 0 for
+ *              one-CTA tiles
+ *     info[2]  number of tiles
+ *     info[3]  1 if a workspace (fp8_gemm_ex, fp8_gemm_noalloc) turns the
+ *              launch into the stream-K schedule, else 0
+ *     info[4]  CTA pairs (one-CTA tiles: CTAs) resident at once
+ * Errors: FP8DS_ERR_INVALID_ARG for a NULL info or m, n, k not positive.
+ */
+fp8ds_status fp8_gemm_plan(int64_t m, int64_t n, int64_t k, int64_t *info);
+
+/*
  * fp8_gemm_ex -- fp8_gemm with a caller-owned device workspace.  When the
- * tile count would leave a ragged last wave of CTA pairs, every pair then
- * takes an equal share of the (tile, k-block) work ("stream-K"); a tile split
- * between two pairs is combined through the workspace: one pair stores its
- * fp32 partial accumulator there and publishes it, the other adds it before
- * the epilogue.  The result satisfies the same bounds as fp8_gemm (the two
- * partials are added in fp32).  On B200 the whole-tile schedule of fp8_gemm
- * measured faster on the MLP shapes (8192 x 2048 x 8192: 95-97 against
- * 114-117 us): the partial's store and reload cost about 15 us, one
- * dependent load per 32 columns, and every extra tile segment adds an
- * epilogue that the 512-row tile cannot overlap.  The stream-K schedule is
- * for cases where a profile shows the ragged last wave dominating.
+ * tiles would leave a ragged last wave of CTA pairs (fp8_gemm_plan, info[3]),
+ * the whole waves still run as whole tiles and the k-blocks of the remaining
+ * tiles are shared out equally among all pairs ("stream-K"); a tile split
+ * between consecutive pairs is combined through the workspace in a fixed
+ * order: each pair that holds a later part stores its fp32 partial
+ * accumulator there (after adding the part after it, if any) and publishes
+ * it, and the pair that holds the tile's first k-blocks adds it and writes D.
+ * The result satisfies the same bounds as fp8_gemm (the partials are added
+ * in fp32) and is the same bits on every run.  On B200 the whole-tile
+ * schedule of fp8_gemm still measured faster on the MLP shapes (8192 x 2048
+ * x 8192: 99-100 us against 91-93 us): the schedule alone would save about
+ * 3 us, and storing and reloading the partials costs about 9.  The stream-K
+ * schedule is for cases where a profile shows the ragged last wave
+ * dominating.
  *   workspace  16-byte aligned device memory of at least
  *              fp8_gemm_workspace_size() bytes, ZERO-FILLED before its first
  *              use; the library leaves its publication words at zero after

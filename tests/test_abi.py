@@ -35,7 +35,8 @@ def test_header_declares_the_boundary():
               "fp8_cast_transpose_amax_pair",
               "fp8_cast_transpose_amax_dynamic", "fp8_transpose", "fp8_gemm_major",
               "fp8_linear_fwd", "fp8_linear_bwd", "fp8ds_last_error", "fp8ds_device_status",
-              "fp8ds_version", "fp8_cast_transpose_amax_multi", "fp8_linear_refresh_weights"):
+              "fp8ds_version", "fp8_cast_transpose_amax_multi", "fp8_linear_refresh_weights",
+              "fp8_gemm_plan"):
         assert n in names
 
 
@@ -81,6 +82,10 @@ def test_gemm_argument_checks(lib):
         lib.ERR_INVALID_ARG
     assert L.fp8_gemm_ex(FAKE, 0, FAKE, FAKE, 0, FAKE, None, 0, FAKE, 1, 128, 256, 128, FAKE_ODD, 64, s) == \
         lib.ERR_INVALID_ARG and "workspace" in lib.fp8ds_last_error()
+    # the schedule query checks its arguments before it asks the device
+    info = (ctypes.c_int64 * 5)()
+    assert L.fp8_gemm_plan(128, 256, 128, None) == lib.ERR_INVALID_ARG
+    assert L.fp8_gemm_plan(0, 256, 128, info) == lib.ERR_INVALID_ARG and "positive" in lib.fp8ds_last_error()
 
 
 def test_cast_and_update_argument_checks(lib):

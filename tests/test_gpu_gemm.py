@@ -176,13 +176,18 @@ def test_gemm_repeatable(fp8):
 
 
 # ------------------------------------------------------------------ stream-K --
-# With a workspace, shapes whose pair tiles would leave a ragged last wave run
-# the stream-K schedule: every pair takes an equal share of the (tile,
-# k-block) work and tiles split between two pairs are combined through the
-# workspace.  (4096, 2048, 256): 128 tiles of 256x256; (4608, 2304, 4096):
-# 162 tiles of 256x256 (its 81 tiles of 512x256 would fill the last wave
-# worse); (7168, 2048, 2048): 112 tiles of 512x256.  All have more tiles than
-# the 74 pairs of a B200 and are not whole waves.
+# With a workspace, shapes whose pair tiles leave a ragged last wave run the
+# stream-K schedule: the whole waves of tiles as before, then every pair takes
+# an equal share of the remaining tiles' (tile, k-block) units; a tile split
+# between two to four consecutive pairs is combined through the workspace in
+# a fixed order.  On the 74 pairs of a B200:
+#   (4096, 2048, 1024)  128 tiles of 256x256: 74 whole, 54 shared (up to
+#                       three pairs per tile)
+#   (4000, 2000, 1024)  the same with ragged M and N edges
+#   (7168, 2048, 2048)  112 tiles of 512x256: 74 whole, 38 shared
+#   (2048, 2048, 4096)  64 tiles of 256x256, all shared by the 74 pairs
+#   (8192, 2048, 8192), (2048, 8192, 8192)  the MLP's 128 tiles of 512x256
+SK_SHAPES = [(4096, 2048, 1024), (4000, 2000, 1024), (7168, 2048, 2048), (2048, 2048, 4096)]
 
 @pytest.fixture(scope="module")
 def ws(fp8):
@@ -193,12 +198,22 @@ def _flags_clear(ws):
     return int(ws[:4096].view(torch.int32).abs().sum().item()) == 0
 
 
-@pytest.mark.parametrize("shape", [(4096, 2048, 256), (4608, 2304, 4096), (7168, 2048, 2048)])
+def _require_stream_k(fp8, M, N, K):
+    """The shape must take the stream-K schedule; on a device with another
+    number of resident CTA pairs than a B200's 74 it may not (skip then)."""
+    plan = fp8.fp8_gemm_plan(M, N, K)
+    if not plan["stream_k"]:
+        assert plan["resident"] != 74, plan
+        pytest.skip("%d tiles on %d CTA pairs: no split tiles" % (plan["tiles"], plan["resident"]))
+
+
+@pytest.mark.parametrize("shape", SK_SHAPES)
 @pytest.mark.parametrize("fa,fb", [("e4m3", "e4m3"), ("e5m2", "e4m3")])
 def test_gemm_stream_k_integer_exact(fp8, ws, shape, fa, fb):
-    """Integer operands: every partial sum, and the sum of two partials, is
+    """Integer operands: every partial sum, and every sum of partials, is
     exact in fp32, so the split tiles must reproduce the exact product."""
     M, N, K = shape
+    _require_stream_k(fp8, M, N, K)
     a, av = _integer_codes((M, K), fa, 15)
     b, bv = _integer_codes((N, K), fb, 16)
     d = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
@@ -213,10 +228,11 @@ def test_gemm_stream_k_integer_exact(fp8, ws, shape, fa, fb):
     assert _flags_clear(ws)
 
 
-@pytest.mark.parametrize("shape", [(8192, 2048, 8192), (2048, 8192, 8192), (4096, 2048, 256)])
+@pytest.mark.parametrize("shape", [(8192, 2048, 8192), (2048, 8192, 8192), (4000, 2000, 1024)])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_gemm_stream_k_realistic(fp8, ws, shape, out_dtype):
     M, N, K = shape
+    _require_stream_k(fp8, M, N, K)
     a, b, sa, sb = _realistic_operands(M, N, K, "e4m3", "e4m3", seed=21)
     rows = _rows_for(M, N, K)
     ref = o.gemm(a, o.E4M3, b, o.E4M3, sa, sb, rows=rows)
@@ -231,7 +247,8 @@ def test_gemm_stream_k_realistic(fp8, ws, shape, out_dtype):
 
 def test_gemm_stream_k_repeatable(fp8, ws):
     """The split tiles are combined in a fixed order: same bits every run."""
-    a, b, sa, sb = _realistic_operands(4096, 2048, 256, "e4m3", "e4m3", seed=22)
+    _require_stream_k(fp8, 4096, 2048, 1024)
+    a, b, sa, sb = _realistic_operands(4096, 2048, 1024, "e4m3", "e4m3", seed=22)
     outs = []
     for _ in range(3):
         d = torch.empty(4096, 2048, dtype=torch.float32, device="cuda")
@@ -252,11 +269,8 @@ def test_stream_k_partial_wait_gives_up_and_reports(fp8, ws):
     give up, record a timeout at the partial-sum site in the device error word
     and exit (no fault, no hang).  The context stays usable: the workspace's
     publication words are clear and the next normal call is exact."""
-    M, N, K = 4096, 2048, 256                       # 128 tiles of 256 x 256
-    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
-    tiles = (M // 256) * (N // 256)
-    if not (pairs <= tiles < 8 * pairs and tiles % pairs != 0):
-        pytest.skip("%d tiles on %d CTA pairs: no split tiles" % (tiles, pairs))
+    M, N, K = 4096, 2048, 1024                      # 128 tiles of 256 x 256
+    _require_stream_k(fp8, M, N, K)
     a, av = _integer_codes((M, K), "e4m3", 25)
     b, bv = _integer_codes((N, K), "e4m3", 26)
     ad, bd = dev(a), dev(b)

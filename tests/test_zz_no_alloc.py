@@ -8,9 +8,9 @@ so that a run stopping at the first failure has run every other test; it
 passes alone in a fresh process as well.
 
 The shapes below leave a ragged last wave of CTA pairs on a B200, so the
-scratch is really used (a short and a long contraction; both run 256-row
-pair tiles, since their 512-row tiles would fill the last wave worse); the
-test checks that precondition against the device's SM count before it runs.  The
+scratch is really used (256-row and 512-row pair tiles); the test asks the
+library's own schedule (fp8_gemm_plan) whether the shape takes the split
+tiles on this device before it runs.  The
 output of two consecutive calls is compared with fp8_gemm (the existing entry
 point) within the tolerances of the other GEMM tests; the two calls also show
 that a call starts from whatever the previous one left in the shared scratch.
@@ -57,31 +57,19 @@ def _call_noalloc(fp8, a, sa, b, sb, d):
     assert st == fp8.OK, fp8.fp8ds_last_error()
 
 
-def _pair_tiles(M, N, K, pairs):
-    """Pair tiles of the launch: 256 x 256, or 512 x 256 from K = 2048 when
-    those fill the last wave of pairs at least as well (within 2 %)."""
-    tn = -(-N // 256)
-    t1 = -(-M // 256) * tn
-    t2 = -(-M // 512) * tn
-    if M > 256 and K >= 2048:
-        w1, w2 = -(-t1 // pairs), -(-t2 // pairs)
-        if t2 * w1 * 50 >= t1 * w2 * 49:
-            return t2
-    return t1
-
-
-@pytest.mark.parametrize("shape", [(4096, 2048, 256), (4608, 2304, 4096)])
+@pytest.mark.parametrize("shape", [(4096, 2048, 1024), (7168, 2048, 2048)])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_noalloc_matches_fp8_gemm_twice(fp8, shape, out_dtype):
     M, N, K = shape
     # The split-tile schedule (and with it the static scratch) is taken only
-    # when whole tiles leave a ragged last wave: at least one tile per CTA
-    # pair, fewer than 8 waves, not a whole number of waves.
-    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
-    tiles = _pair_tiles(M, N, K, pairs)
-    if not (pairs <= tiles < 8 * pairs and tiles % pairs != 0):
-        pytest.skip("%d pair tiles on %d CTA pairs: no ragged last wave, the scratch would not be used"
-                    % (tiles, pairs))
+    # when whole tiles leave a ragged last wave worth balancing; the library's
+    # own plan says whether this shape does on this device (on the 74 CTA
+    # pairs of a B200 both shapes do: 128 and 112 tiles).
+    plan = fp8.fp8_gemm_plan(M, N, K)
+    if not plan["stream_k"]:
+        assert plan["resident"] != 74, plan
+        pytest.skip("%d tiles on %d CTA pairs: no split tiles, the scratch would not be used"
+                    % (plan["tiles"], plan["resident"]))
     a, b, sa, sb = _operands(M, N, K, seed=31)
     ad, bd = dev(a), dev(b)
     sad = torch.tensor([sa], device="cuda")
