@@ -372,7 +372,6 @@ cast_transpose_tma_kernel(const __grid_constant__ TmaJobs P) {
     }
     if (tid < nj) ptx::prefetch_tmap(&P.maps[tid]);
     ptx::pdl_wait();
-    ptx::pdl_launch_dependents();
     // device-side skips (whole jobs), before any load is issued
     if (tid == 0) {
         int32_t acc = 0;
@@ -458,9 +457,19 @@ cast_transpose_tma_kernel(const __grid_constant__ TmaJobs P) {
     // the scale of this CTA's first job is read while its first tiles load
     int mj = blockIdx.x < num_tiles ? job_at(blockIdx.x, cj) : 0;
     float m = 0.0f, s = __ldg(P.jobs[mj].scale);
+    // The next kernel may launch (PDL) once every CTA has issued its last
+    // loads, not at the start: a dependent cast grid launched early measured
+    // 13 us slower behind this one (X + W1 + W2 then dY: 63 against 50 us),
+    // and waiting for the very end cost the GEMM that follows a cast in the
+    // step its prologue overlap; this point measured best for the step.
+    bool triggered = false;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
         const int stage = it % STAGES;
         const uint32_t phase = static_cast<uint32_t>((it / STAGES) & 1);
+        if (!triggered && static_cast<int64_t>(tile) + static_cast<int64_t>(STAGES) * gridDim.x >= num_tiles) {
+            ptx::pdl_launch_dependents();
+            triggered = true;
+        }
         const bool ok = ptx::mbar_wait_for(&full[stage], phase, ptx::TIMEOUT_NS);
         // Every thread leaves together if the tile never arrived.
         if (__syncthreads_or(!ok)) {
@@ -736,7 +745,6 @@ __global__ void __launch_bounds__(MC_THREADS)
 cast_multi_kernel(const __grid_constant__ MultiParams p) {
     __shared__ uint32_t tsm[CT_COLS * CT_TSTRIDE];
     ptx::pdl_wait();
-    ptx::pdl_launch_dependents();
     const int tid = threadIdx.x;
     // Jobs with no elements own no tile: their scale_inv is written here.
     if (blockIdx.x == 0 && tid == 0) {
@@ -764,6 +772,9 @@ cast_multi_kernel(const __grid_constant__ MultiParams p) {
     int cur = -1;
     bool skip = true;
     for (uint32_t t = t_begin; t < t_end; ++t) {
+        // dependents may launch once this CTA is into its last two tiles (as
+        // in the TMA kernel, not at the start)
+        if (t + 2 >= t_end && (t == t_begin || t + 2 == t_end)) ptx::pdl_launch_dependents();
         while (j + 1 < p.num_jobs && p.jobs[j + 1].tile0 <= t) ++j;
         if (j != cur) {
             // the CTA leaves job `cur`: one reduction and one atomic for its stretch
