@@ -175,6 +175,29 @@ def test_gemm_repeatable(fp8):
     assert torch.equal(d1.view(torch.int32), d2.view(torch.int32))
 
 
+def test_gemm_plan_reports_the_schedule(fp8):
+    """fp8_gemm_plan on this device: one-CTA tiles up to M = 128, the 512-row
+    pair tile for the MLP's K >= 2048 shapes, tile counts, and stream-K only
+    where whole tiles leave a ragged last wave worth balancing."""
+    small = fp8.fp8_gemm_plan(128, 256, 128)
+    assert not small["pair"] and small["m_sub"] == 0 and small["tiles"] == 1 and not small["stream_k"]
+    assert small["resident"] == torch.cuda.get_device_properties(0).multi_processor_count
+    fwd = fp8.fp8_gemm_plan(8192, 8192, 2048)
+    assert fwd["pair"] and fwd["m_sub"] == 2 and fwd["tiles"] == 16 * 32
+    pairs = fwd["resident"]
+    assert 0 < pairs <= torch.cuda.get_device_properties(0).multi_processor_count // 2
+    # 512 tiles: whole waves but the last, which is nearly full -> no stream-K
+    assert fwd["stream_k"] == (3 * (512 % pairs) >= pairs and 8 * (512 % pairs) <= 7 * pairs)
+    k8 = fp8.fp8_gemm_plan(8192, 2048, 8192)
+    assert k8["pair"] and k8["m_sub"] == 2 and k8["tiles"] == 16 * 8
+    short = fp8.fp8_gemm_plan(4096, 2048, 256)   # 128 tiles of 256 rows, but only 2 k-blocks
+    assert short["pair"] and short["m_sub"] == 1 and short["tiles"] == 16 * 8 and not short["stream_k"]
+    if pairs == 74:                               # a B200
+        assert not fwd["stream_k"] and k8["stream_k"]
+    with pytest.raises(fp8.Fp8dsError):
+        fp8.fp8_gemm_plan(0, 256, 128)
+
+
 # ------------------------------------------------------------------ stream-K --
 # With a workspace, shapes whose pair tiles leave a ragged last wave run the
 # stream-K schedule: the whole waves of tiles as before, then every pair takes
