@@ -933,96 +933,113 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
 // load has completed; the staging and the TMA stores follow while the next
 // tile's MMAs already run.
 //
-// FP8 output: the codes of the first half go straight into the warp's
-// staging box (shared memory, not yet stored) and those of the last half
-// stay in registers (32 words per lane), so the whole accumulator is released
-// before anything is stored.
+// FP8 output: only the bf16 rounding of D (acc * sa*sb + bias, two columns
+// per instruction) happens while a row block's accumulator is read; its 64
+// packed bf16 pairs per lane stay in registers and the row block is released
+// to the MMA warp right after its last TMEM load.  The delayed-scale
+// multiply, the FP8 conversion and the amax (as many conversion instructions
+// again, the slow part of this epilogue) are done later: for the first row
+// block of the 512-row tile chunk by chunk while the second block is read
+// (each chunk's packed words are converted, then replaced by the second
+// block's), otherwise after the release, while the next tile's MMAs run.
+// The codes go to the warp's staging box and out by TMA.
+template <bool BIAS>
+__device__ __forceinline__ void fp8_read_chunk(uint32_t (&pk)[64], int c, const uint32_t (&r)[32], uint64_t sab2,
+                                               const float *bs) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float4 b = bias4<BIAS>(bs + 4 * j);
+        const uint64_t v01 = scale_bias2(r[4 * j], r[4 * j + 1], sab2, b.x, b.y);
+        const uint64_t v23 = scale_bias2(r[4 * j + 2], r[4 * j + 3], sab2, b.z, b.w);
+        __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
+        __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
+        pk[16 * c + 2 * j] = *reinterpret_cast<uint32_t *>(&ha);
+        pk[16 * c + 2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
+    }
+}
+// Codes of chunk c (32 columns) from its packed bf16 pairs into the box row.
+__device__ __forceinline__ void fp8_convert_chunk(const uint32_t (&pk)[64], int c, uint8_t *box, int lane,
+                                                  uint64_t s2, int fmt, float &amax) {
+    uint32_t w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t ua = pk[16 * c + 2 * j], ub = pk[16 * c + 2 * j + 1];
+        const float h0 = __uint_as_float(ua << 16), h1 = __uint_as_float(ua & 0xFFFF0000u);
+        const float h2 = __uint_as_float(ub << 16), h3 = __uint_as_float(ub & 0xFFFF0000u);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+        const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
+        const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
+        w[j] = cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) | (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
+    }
+    // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
+    *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c) ^ (lane & 7)) * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c + 1) ^ (lane & 7)) * 16) =
+        make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 template <bool BIAS, int MSUB>
 __device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uint8_t *boxes, int &nbox, int half,
                                                   const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row_h0,
                                                   int32_t rows_per_sub, float sab, const float *bias_s,
                                                   uint32_t empty_base, bool split, float s_out, int fmt,
                                                   float &amax) {
-    constexpr int CH = ACC_N / 2 / 32;  // chunks of 32 columns per warp and half
+    constexpr int CH = ACC_N / 2 / 32;  // chunks of 32 columns per warp and row block
     const uint64_t sab2 = pack_f32x2(sab, sab);
     const uint64_t s2 = pack_f32x2(s_out, s_out);
-    uint32_t codes[CH * 8];
+    const float *bs = bias_s + half * (ACC_N / 2);
+    uint32_t pk[CH * 16];               // bf16(D) of a row block, two columns per word
     uint32_t r[32];
+    auto release = [&](int h) {
+        // every TMEM load of this row block (or of the accumulator) is done
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(empty_base + static_cast<uint32_t>(split ? h * sizeof(uint64_t) : 0));
+    };
+    auto store_box = [&](uint8_t *box, int h) {
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)), m_row_h0 + h * rows_per_sub);
+            tma_store_commit();
+        }
+        ++nbox;
+    };
+    // row block 0
+    const uint32_t t_h0 = t_row0 + static_cast<uint32_t>(half * (ACC_N / 2));
+    tmem_ld32(t_h0, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        fp8_read_chunk<BIAS>(pk, c, r, sab2, bs + c * 32);
+        if (c + 1 < CH) {
+            tmem_ld32(t_h0 + static_cast<uint32_t>((c + 1) * 32), r);
+            tmem_ld_wait();
+        }
+    }
+    if (split || MSUB == 1) release(0);
+    // the box's last store (the previous tile's) must have finished reading it
     uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
+    if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
+    __syncwarp();
     if (MSUB > 1) {
-        // the store last issued from this box must have finished reading it
+        // row block 1 is read while block 0 is converted, chunk by chunk
+        const uint32_t t_h1 = t_h0 + static_cast<uint32_t>(ACC_N);
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            tmem_ld32(t_h1 + static_cast<uint32_t>(c * 32), r);
+            fp8_convert_chunk(pk, c, box, lane, s2, fmt, amax);
+            tmem_ld_wait();
+            fp8_read_chunk<BIAS>(pk, c, r, sab2, bs + c * 32);
+        }
+        release(1);
+        store_box(box, 0);
+        box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
         if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
         __syncwarp();
     }
 #pragma unroll
-    for (int h = 0; h < MSUB; ++h) {
-        const uint32_t t_h = t_row0 + static_cast<uint32_t>(h * ACC_N + half * (ACC_N / 2));
-        tmem_ld32(t_h, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            if (c == CH - 1 && (split || h == MSUB - 1)) {
-                // every TMEM load of this half (or of the accumulator) is done
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(empty_base + static_cast<uint32_t>(split ? h * sizeof(uint64_t) : 0));
-            }
-            const float *bs = bias_s + half * (ACC_N / 2) + c * 32;
-            uint32_t w[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 b = bias4<BIAS>(bs + 4 * j);
-                const uint64_t v01 = scale_bias2(r[4 * j], r[4 * j + 1], sab2, b.x, b.y);
-                const uint64_t v23 = scale_bias2(r[4 * j + 2], r[4 * j + 3], sab2, b.z, b.w);
-                const __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
-                const __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
-                const float h0 = __low2float(ha), h1 = __high2float(ha);
-                const float h2 = __low2float(hb), h3 = __high2float(hb);
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
-                const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
-                const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
-                w[j] = cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) | (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
-            }
-            if (c + 1 < CH) tmem_ld32(t_h + static_cast<uint32_t>((c + 1) * 32), r);
-            if (h < MSUB - 1) {
-                // 16-byte chunk k of row `lane` goes to chunk k ^ (lane & 7)
-                *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c) ^ (lane & 7)) * 16) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4 *>(box + lane * 128 + ((2 * c + 1) ^ (lane & 7)) * 16) =
-                    make_uint4(w[4], w[5], w[6], w[7]);
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) codes[8 * c + j] = w[j];
-            }
-            if (c + 1 < CH) tmem_ld_wait();
-        }
-    }
-    if (MSUB > 1) {
-        // the first half, staged while the accumulator was read
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-            tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)), m_row_h0);
-            tma_store_commit();
-        }
-        ++nbox;
-        box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
-    }
-    // the last half, from registers
-    if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
-    __syncwarp();
-#pragma unroll
-    for (int k = 0; k < 2 * CH; ++k)
-        *reinterpret_cast<uint4 *>(box + lane * 128 + (k ^ (lane & 7)) * 16) =
-            make_uint4(codes[4 * k], codes[4 * k + 1], codes[4 * k + 2], codes[4 * k + 3]);
-    fence_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-        tma_store_2d(tmap_d, box, static_cast<int32_t>(n_base + half * (ACC_N / 2)),
-                     m_row_h0 + (MSUB - 1) * rows_per_sub);
-        tma_store_commit();
-    }
-    ++nbox;
+    for (int c = 0; c < CH; ++c) fp8_convert_chunk(pk, c, box, lane, s2, fmt, amax);
+    store_box(box, MSUB - 1);
 }
 
 // bf16 output: a half is 128 columns, two staging boxes of 64 columns.  The
