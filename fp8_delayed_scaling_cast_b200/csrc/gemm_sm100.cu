@@ -874,7 +874,8 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
                     const __nv_bfloat162 hb = __floats2bfloat162_rn(lo_f32(v23), hi_f32(v23));
                     const float h0 = __low2float(ha), h1 = __high2float(ha);
                     const float h2 = __low2float(hb), h3 = __high2float(hb);
-                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+                    if (m < m_total)  // rows past M (tile padding) count for no amax
+                        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
                     const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
                     const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
                     w[j] = cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) |
@@ -958,15 +959,17 @@ __device__ __forceinline__ void fp8_read_chunk(uint32_t (&pk)[64], int c, const 
     }
 }
 // Codes of chunk c (32 columns) from its packed bf16 pairs into the box row.
+// cmax: running max of |bf16(D)| over the row block's chunks (merged into the
+// amax by the caller only for rows below M).
 __device__ __forceinline__ void fp8_convert_chunk(const uint32_t (&pk)[64], int c, uint8_t *box, int lane,
-                                                  uint64_t s2, int fmt, float &amax) {
+                                                  uint64_t s2, int fmt, float &cmax) {
     uint32_t w[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const uint32_t ua = pk[16 * c + 2 * j], ub = pk[16 * c + 2 * j + 1];
         const float h0 = __uint_as_float(ua << 16), h1 = __uint_as_float(ua & 0xFFFF0000u);
         const float h2 = __uint_as_float(ub << 16), h3 = __uint_as_float(ub & 0xFFFF0000u);
-        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
+        cmax = fmaxf(cmax, fmaxf(fmaxf(fabsf(h0), fabsf(h1)), fmaxf(fabsf(h2), fabsf(h3))));
         const uint64_t p01 = mul_f32x2(pack_f32x2(h0, h1), s2);
         const uint64_t p23 = mul_f32x2(pack_f32x2(h2, h3), s2);
         w[j] = cvt_fp8x2(lo_f32(p01), hi_f32(p01), fmt) | (cvt_fp8x2(lo_f32(p23), hi_f32(p23), fmt) << 16);
@@ -982,11 +985,14 @@ __device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uin
                                                   const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row_h0,
                                                   int32_t rows_per_sub, float sab, const float *bias_s,
                                                   uint32_t empty_base, bool split, float s_out, int fmt,
-                                                  float &amax) {
+                                                  int32_t m_total, float &amax) {
     constexpr int CH = ACC_N / 2 / 32;  // chunks of 32 columns per warp and row block
     const uint64_t sab2 = pack_f32x2(sab, sab);
     const uint64_t s2 = pack_f32x2(s_out, s_out);
     const float *bs = bias_s + half * (ACC_N / 2);
+    // Rows past M (the last tile's padding: A read as zeros, so D is the bias
+    // alone there) are stored by no one and count for no amax.
+    float cmax = 0.0f;
     uint32_t pk[CH * 16];               // bf16(D) of a row block, two columns per word
     uint32_t r[32];
     auto release = [&](int h) {
@@ -1027,18 +1033,21 @@ __device__ __forceinline__ void epilogue_fp8_regs(uint32_t t_row0, int lane, uin
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
             tmem_ld32(t_h1 + static_cast<uint32_t>(c * 32), r);
-            fp8_convert_chunk(pk, c, box, lane, s2, fmt, amax);
+            fp8_convert_chunk(pk, c, box, lane, s2, fmt, cmax);
             tmem_ld_wait();
             fp8_read_chunk<BIAS>(pk, c, r, sab2, bs + c * 32);
         }
         release(1);
+        if (m_row_h0 + lane < m_total) amax = fmaxf(amax, cmax);
+        cmax = 0.0f;
         store_box(box, 0);
         box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
         if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
         __syncwarp();
     }
 #pragma unroll
-    for (int c = 0; c < CH; ++c) fp8_convert_chunk(pk, c, box, lane, s2, fmt, amax);
+    for (int c = 0; c < CH; ++c) fp8_convert_chunk(pk, c, box, lane, s2, fmt, cmax);
+    if (m_row_h0 + (MSUB - 1) * rows_per_sub + lane < m_total) amax = fmaxf(amax, cmax);
     store_box(box, MSUB - 1);
 }
 
@@ -1236,19 +1245,19 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
                 if (m_sub == 2) {
                     if (p.bias_kind != 0)
                         epilogue_fp8_regs<true, 2>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
-                                                   rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt, amax);
+                                                   rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt, p.M, amax);
                     else
                         epilogue_fp8_regs<false, 2>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
                                                     rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt,
-                                                    amax);
+                                                    p.M, amax);
                 } else {
                     if (p.bias_kind != 0)
                         epilogue_fp8_regs<true, 1>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
-                                                   rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt, amax);
+                                                   rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt, p.M, amax);
                     else
                         epilogue_fp8_regs<false, 1>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
                                                     rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt,
-                                                    amax);
+                                                    p.M, amax);
                 }
                 done = true;
             }

@@ -114,6 +114,38 @@ def test_gemm_cast_matches_cast_of_bf16_output(fp8, M, N, K, out_fmt, bias_kind,
     assert np.any((y & 0x7F) == (0x7E if fmt == o.E4M3 else 0x7B))
 
 
+@pytest.mark.parametrize("M,N,K,transpose", [
+    (100, 256, 32, False),     # one-CTA tile of 128 rows: rows 100-127 are padding
+    (300, 528, 32, False),     # 256-row pair tiles: rows 300-511 of the last tile
+    (304, 528, 32, True),      # the same through the transpose epilogue (M % 16 == 0)
+    (1040, 512, 2048, False),  # 512-row pair tiles: rows 1040-1535 of the last tile
+])
+def test_gemm_cast_amax_covers_output_rows_only(fp8, M, N, K, transpose):
+    """The amax is that of D's M rows.  The last tile's rows past M hold
+    acc = 0 (their A rows read as zeros), so there D would be the bias alone;
+    here the bias is -(K - 0.5) and every real row has acc = K, so the real
+    outputs are all 0.5 while the padding rows would give |D| = K - 0.5."""
+    one = 0x38                                    # e4m3 code of 1.0
+    a = np.full((M, K), one, dtype=np.uint8)
+    b = np.full((N, K), one, dtype=np.uint8)
+    assert o.decode(a[:1, :1], o.E4M3)[0, 0] == 1.0
+    bias = torch.full((N,), -(K - 0.5), dtype=torch.float32, device="cuda")
+    s1 = torch.ones(1, device="cuda")
+    d8 = torch.full((M, N), 0xAA, dtype=torch.uint8, device="cuda")
+    d8t = torch.full((N, M), 0xAA, dtype=torch.uint8, device="cuda") if transpose else None
+    am = torch.zeros(1, device="cuda")
+    si = torch.zeros(1, device="cuda")
+    fp8.fp8_gemm_cast(dev(a), "e4m3", s1, dev(b), "e4m3", s1, "e4m3", s1, d8, d8t, am, si, bias=bias)
+    torch.cuda.synchronize()
+    assert fp8.fp8ds_device_status() == 0
+    y, yt, oam, _ = o.cast_transpose_amax(np.full((M, N), 0.5, dtype=np.float32), o.E4M3, np.float32(1.0))
+    assert oam == 0.5
+    assert_bytes_equal(u8(d8), y, "codes")
+    if transpose:
+        assert_bytes_equal(u8(d8t), yt, "transposed codes")
+    assert_f32_bits_equal(am.cpu().numpy(), [oam], "amax")
+
+
 class _Mlp:
     """fc1 (hidden -> ffn) and fc2 (ffn -> hidden) with metas [X, W1, dH, H, W2, dY]
     and all device buffers of one training step."""
