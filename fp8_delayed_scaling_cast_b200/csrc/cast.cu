@@ -457,16 +457,16 @@ cast_transpose_tma_kernel(const __grid_constant__ TmaJobs P) {
     // the scale of this CTA's first job is read while its first tiles load
     int mj = blockIdx.x < num_tiles ? job_at(blockIdx.x, cj) : 0;
     float m = 0.0f, s = __ldg(P.jobs[mj].scale);
-    // The next kernel may launch (PDL) once every CTA has issued its last
-    // loads, not at the start: a dependent cast grid launched early measured
+    // The next kernel may launch (PDL) once every CTA has started its last
+    // tile, not at the start: a dependent cast grid launched early measured
     // 13 us slower behind this one (X + W1 + W2 then dY: 63 against 50 us),
     // and waiting for the very end cost the GEMM that follows a cast in the
-    // step its prologue overlap; this point measured best for the step.
+    // step its prologue overlap; this point measured best for both.
     bool triggered = false;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
         const int stage = it % STAGES;
         const uint32_t phase = static_cast<uint32_t>((it / STAGES) & 1);
-        if (!triggered && static_cast<int64_t>(tile) + static_cast<int64_t>(STAGES) * gridDim.x >= num_tiles) {
+        if (!triggered && static_cast<int64_t>(tile) + gridDim.x >= num_tiles) {
             ptx::pdl_launch_dependents();
             triggered = true;
         }
@@ -772,9 +772,9 @@ cast_multi_kernel(const __grid_constant__ MultiParams p) {
     int cur = -1;
     bool skip = true;
     for (uint32_t t = t_begin; t < t_end; ++t) {
-        // dependents may launch once this CTA is into its last two tiles (as
+        // dependents may launch once this CTA has started its last tile (as
         // in the TMA kernel, not at the start)
-        if (t + 2 >= t_end && (t == t_begin || t + 2 == t_end)) ptx::pdl_launch_dependents();
+        if (t + 1 == t_end) ptx::pdl_launch_dependents();
         while (j + 1 < p.num_jobs && p.jobs[j + 1].tile0 <= t) ++j;
         if (j != cur) {
             // the CTA leaves job `cur`: one reduction and one atomic for its stretch
