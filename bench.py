@@ -1199,6 +1199,8 @@ def main():
         "teblock_fwd_4mb": None if teblock is None else {k: r3(v) for k, v in teblock.items()},
         "toy32_fwd": None if toy is None else {k: r3(v) for k, v in toy.items() if k != "device_status"},
         "graph_step": None if graph_info is None else {"ms_per_step": r3(graph_info["ms_per_step"]),
+                                                      "eager_ms_same_section": r3(
+                                                          graph_info["eager_same_section_ms_per_step"]),
                                                       "host_us_per_step": r3(graph_info["host_us_per_step"])},
         "host_us_per_step": r3(host_us),
         "unfused_step_ms": r3(ms_unfused),
