@@ -944,12 +944,36 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
 // (each chunk's packed words are converted, then replaced by the second
 // block's), otherwise after the release, while the next tile's MMAs run.
 // The codes go to the warp's staging box and out by TMA.
+// The 32 bias values of a chunk from shared memory in one asm block: the
+// eight broadcast loads are issued back to back, so their latency is paid
+// once per chunk, not once per four columns.
+__device__ __forceinline__ void load_bias32(const float *bs, float (&b)[32]) {
+    asm volatile(
+        "ld.shared.v4.f32 {%0,%1,%2,%3}, [%32];\n\t"
+        "ld.shared.v4.f32 {%4,%5,%6,%7}, [%32+16];\n\t"
+        "ld.shared.v4.f32 {%8,%9,%10,%11}, [%32+32];\n\t"
+        "ld.shared.v4.f32 {%12,%13,%14,%15}, [%32+48];\n\t"
+        "ld.shared.v4.f32 {%16,%17,%18,%19}, [%32+64];\n\t"
+        "ld.shared.v4.f32 {%20,%21,%22,%23}, [%32+80];\n\t"
+        "ld.shared.v4.f32 {%24,%25,%26,%27}, [%32+96];\n\t"
+        "ld.shared.v4.f32 {%28,%29,%30,%31}, [%32+112];"
+        : "=f"(b[0]), "=f"(b[1]), "=f"(b[2]), "=f"(b[3]), "=f"(b[4]), "=f"(b[5]), "=f"(b[6]), "=f"(b[7]),
+          "=f"(b[8]), "=f"(b[9]), "=f"(b[10]), "=f"(b[11]), "=f"(b[12]), "=f"(b[13]), "=f"(b[14]), "=f"(b[15]),
+          "=f"(b[16]), "=f"(b[17]), "=f"(b[18]), "=f"(b[19]), "=f"(b[20]), "=f"(b[21]), "=f"(b[22]), "=f"(b[23]),
+          "=f"(b[24]), "=f"(b[25]), "=f"(b[26]), "=f"(b[27]), "=f"(b[28]), "=f"(b[29]), "=f"(b[30]), "=f"(b[31])
+        : "r"(smem_u32(bs))
+        : "memory");
+}
+
 template <bool BIAS>
 __device__ __forceinline__ void fp8_read_chunk(uint32_t (&pk)[64], int c, const uint32_t (&r)[32], uint64_t sab2,
                                                const float *bs) {
+    float bv[32];
+    if constexpr (BIAS) load_bias32(bs, bv);
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const float4 b = bias4<BIAS>(bs + 4 * j);
+        const float4 b = BIAS ? make_float4(bv[4 * j], bv[4 * j + 1], bv[4 * j + 2], bv[4 * j + 3])
+                              : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         const uint64_t v01 = scale_bias2(r[4 * j], r[4 * j + 1], sab2, b.x, b.y);
         const uint64_t v23 = scale_bias2(r[4 * j + 2], r[4 * j + 3], sab2, b.z, b.w);
         __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
@@ -1171,7 +1195,10 @@ __device__ __forceinline__ void st_release(int32_t *p, int32_t v) {
 // Stream-K segments: a tail (kb0 > 0, the first segment of this cluster)
 // publishes its partial in slot `cluster`; a head (kb0 == 0, kb1 < num_kb,
 // the last segment) adds the partial of slot cluster + 1 before storing D.
-template <int OUT>
+// BIAS: the launch has a bias (a kernel template parameter, so that each
+// kernel holds one epilogue variant and a kernel without a bias does not
+// stage one).
+template <int OUT, bool BIAS>
 __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap *tmap_d, const Params &p,
                                               uint32_t tmem_base, int warp, int lane, int cluster, int clusters,
                                               int m_sub, int rows_per_sub, int row_offset, int acc_bufs,
@@ -1196,7 +1223,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
         const int seg = (kb0 > 0 ? PART_OUT : 0) | (kb1 < p.num_kb ? PART_IN : 0);
         const int mode = seg;
         float bias_v[BIAS_PER_THREAD];
-        load_bias(bias_v, p, static_cast<int64_t>(n_blk) * ACC_N, epi_tid);
+        if constexpr (BIAS) load_bias(bias_v, p, static_cast<int64_t>(n_blk) * ACC_N, epi_tid);
         bool ok = mbar_wait(&sm.tfull[acc], acc_phase, sm.abort_flag, SITE_EPI_TMEM_FULL);
         // A cluster's partial slot and publication word (per CTA of the pair):
         // this segment's own (PART_OUT) and the next cluster's (PART_IN).
@@ -1226,10 +1253,13 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             }
         }
         // All epilogue warps meet here every tile: they leave together if any
-        // wait gave up, and none of them still reads the previous tile's bias.
+        // wait gave up, and none of them still reads the previous tile's bias
+        // (which is then staged and made visible to all of them).
         if (epilogue_any(!ok)) break;
-        stage_bias(bias_s, bias_v, epi_tid);
-        epilogue_bar();
+        if constexpr (BIAS) {
+            stage_bias(bias_s, bias_v, epi_tid);
+            epilogue_bar();
+        }
         tc_fence_after();
         // An accumulator is released whole (tempty[acc]) after its last row
         // block, or with `split` (a single accumulator set of two M halves)
@@ -1243,7 +1273,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
         if constexpr (EPI_EARLY && OUT == OUT_FP8) {
             if (mode == 0 && p.out_d8t == nullptr) {
                 if (m_sub == 2) {
-                    if (p.bias_kind != 0)
+                    if constexpr (BIAS)
                         epilogue_fp8_regs<true, 2>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
                                                    rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt, p.M, amax);
                     else
@@ -1251,7 +1281,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
                                                     rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt,
                                                     p.M, amax);
                 } else {
-                    if (p.bias_kind != 0)
+                    if constexpr (BIAS)
                         epilogue_fp8_regs<true, 1>(t_acc, lane, boxes, nbox, half, tmap_d, n_tile, m_row_h0,
                                                    rows_per_sub, sab, bias_s, empty_base, split, s_out, p.out_fmt, p.M, amax);
                     else
@@ -1268,7 +1298,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
                     const uint32_t empty_addr = empty_base + static_cast<uint32_t>(split ? h * sizeof(uint64_t) : 0);
                     const bool release = split || h == m_sub - 1;
                     const uint32_t t_h = t_acc + static_cast<uint32_t>(h * ACC_N);
-                    if (p.bias_kind != 0)
+                    if constexpr (BIAS)
                         epilogue_bf16_regs<true>(t_h, lane, boxes, nbox, half, tmap_d, n_tile,
                                                  m_row_h0 + h * rows_per_sub, sab, bias_s, empty_addr, release);
                     else
@@ -1286,7 +1316,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             const int32_t m_row0 = (m_blk * m_sub + h) * rows_per_sub + row_offset + q * 32;
             const int64_t n_base = static_cast<int64_t>(n_blk) * ACC_N;
             if constexpr (OUT == OUT_FP8) {
-                if (p.bias_kind != 0)
+                if constexpr (BIAS)
                     epilogue_tile_fp8<true>(t_row, lane, boxes, nbox, half, p.out_d8, p.out_d8t, tmap_d, n_base, m_row0, sab,
                                             bias_s, empty_addr, release, mode, p_in, p_out, h, q, s_out, p.out_fmt, p.M,
                                             p.N,
@@ -1297,7 +1327,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
                                             p.N,
                                              amax);
             } else {
-                if (p.bias_kind != 0)
+                if constexpr (BIAS)
                     epilogue_tile<OUT == OUT_BF16, true>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab, bias_s,
                                                          empty_addr, release, mode, p_in, p_out, h, q, p.out, p.M, p.N,
                                                          p.out_v8 != 0);
@@ -1336,7 +1366,7 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
 
 // ------------------------------------------------------------ 1-SM kernel --
 
-template <int OUT>
+template <int OUT, bool BIAS>
 __global__ void __launch_bounds__(THREADS, 1)
 fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d, const Params p) {
@@ -1468,7 +1498,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         __syncwarp();
     } else {
-        epilogue_loop<OUT>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u, 0,
+        epilogue_loop<OUT, BIAS>(sm, &tmap_d, p, tmem_base, warp, lane, blockIdx.x, gridDim.x, 1, S1_BM, 0, 2, 0u, 0,
                            false);
     }
 
@@ -1487,7 +1517,7 @@ fp8_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
 // tiles c, c + clusters, ...; a pair tile has M_SUB row blocks of 256 rows
 // and 256 columns.  CTA rank r of the pair owns rows r*128..r*128+127 of each
 // row block and loads rows r*128.. of the tile's 256 B rows.
-template <int OUT, int M_SUB>
+template <int OUT, int M_SUB, bool BIAS>
 __global__ void __launch_bounds__(THREADS, 1)
 fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const __grid_constant__ CUtensorMap tmap_d, const Params p) {
@@ -1689,7 +1719,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
         __syncwarp();
     } else {
-        epilogue_loop<OUT>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, M_SUB, 2 * S2_BM,
+        epilogue_loop<OUT, BIAS>(sm, &tmap_d, p, tmem_base, warp, lane, cluster_id, num_clusters, M_SUB, 2 * S2_BM,
                            static_cast<int>(rank) * S2_BM, ACC_BUFS, 0u, static_cast<int>(rank), SPLIT);
     }
 
@@ -1765,12 +1795,12 @@ int max_pairs(K kernel, int smem_bytes, std::atomic<int> (&cached)[64]) {
     return n;
 }
 
-template <int OUT, int M_SUB>
+template <int OUT, int M_SUB, bool BIAS>
 cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
                        cudaStream_t stream) {
     static std::atomic<bool> done[64];
     static std::atomic<int> cached_pairs[64];
-    auto kernel = fp8_gemm_2sm_kernel<OUT, M_SUB>;
+    auto kernel = fp8_gemm_2sm_kernel<OUT, M_SUB, BIAS>;
     constexpr int smem = Pair<M_SUB>::SMEM;
     cudaError_t e = set_smem_once(kernel, smem, done);
     if (e != cudaSuccess) return e;
@@ -1782,11 +1812,11 @@ cudaError_t launch_2sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
     return launch_pdl(kernel, dim3(2 * pairs), dim3(THREADS), smem, stream, 2, ta, tb, td, p);
 }
 
-template <int OUT>
+template <int OUT, bool BIAS>
 cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUtensorMap &td, const Params &p,
                        cudaStream_t stream) {
     static std::atomic<bool> done[64];
-    auto kernel = fp8_gemm_1sm_kernel<OUT>;
+    auto kernel = fp8_gemm_1sm_kernel<OUT, BIAS>;
     cudaError_t e = set_smem_once(kernel, S1_SMEM, done);
     if (e != cudaSuccess) return e;
     const int tiles = p.tiles_m * p.tiles_n;
@@ -1794,11 +1824,28 @@ cudaError_t launch_1sm(const CUtensorMap &ta, const CUtensorMap &tb, const CUten
     return launch_pdl(kernel, dim3(grid), dim3(THREADS), S1_SMEM, stream, 1, ta, tb, td, p);
 }
 
+// The kernel instantiation for an output kind, tile mode and bias presence.
+template <bool BIAS>
+cudaError_t launch_any(int out, bool pair, int m_sub, const CUtensorMap &ta, const CUtensorMap &tb,
+                       const CUtensorMap &td, const Params &p, cudaStream_t stream) {
+    if (pair && m_sub == 2)
+        return out == OUT_FP8    ? launch_2sm<OUT_FP8, 2, BIAS>(ta, tb, td, p, stream)
+               : out == OUT_BF16 ? launch_2sm<OUT_BF16, 2, BIAS>(ta, tb, td, p, stream)
+                                 : launch_2sm<OUT_F32, 2, BIAS>(ta, tb, td, p, stream);
+    if (pair)
+        return out == OUT_FP8    ? launch_2sm<OUT_FP8, 1, BIAS>(ta, tb, td, p, stream)
+               : out == OUT_BF16 ? launch_2sm<OUT_BF16, 1, BIAS>(ta, tb, td, p, stream)
+                                 : launch_2sm<OUT_F32, 1, BIAS>(ta, tb, td, p, stream);
+    return out == OUT_FP8    ? launch_1sm<OUT_FP8, BIAS>(ta, tb, td, p, stream)
+           : out == OUT_BF16 ? launch_1sm<OUT_BF16, BIAS>(ta, tb, td, p, stream)
+                             : launch_1sm<OUT_F32, BIAS>(ta, tb, td, p, stream);
+}
+
 }  // namespace
 
 size_t gemm_workspace_bytes() {
     static std::atomic<int> cached[64];
-    const int pairs = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached);
+    const int pairs = max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1, false>, Pair<1>::SMEM, cached);
     return WS_FLAG_BYTES + static_cast<size_t>(pairs) * 2 * WS_SLOT_FLOATS * sizeof(float);
 }
 
@@ -1829,7 +1876,7 @@ GemmPlan plan_gemm(int64_t m, int64_t n, int64_t k) {
     // pairs less well than the 256-row ones (e.g. 4096 x 8192: 256 tiles =
     // 3.46 waves of 74 pairs against 512 = 6.92 waves).
     g.m_sub = 1;
-    const int64_t cap = g.pair ? max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached_pairs) : 0;
+    const int64_t cap = g.pair ? max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1, false>, Pair<1>::SMEM, cached_pairs) : 0;
     const int64_t tn = (n + ACC_N - 1) / ACC_N;
     if (g.pair && m > 2 * S2_BM && k >= FP8DS_MSUB2_MIN_K) {
         const int64_t t1 = ((m + 2 * S2_BM - 1) / (2 * S2_BM)) * tn, t2 = ((m + 4 * S2_BM - 1) / (4 * S2_BM)) * tn;
@@ -1866,7 +1913,7 @@ void gemm_plan_info(int64_t m, int64_t n, int64_t k, int64_t info[5]) {
     info[1] = g.pair ? g.m_sub : 0;
     info[2] = g.tiles;
     info[3] = g.stream_k ? 1 : 0;
-    info[4] = g.pair ? max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1>, Pair<1>::SMEM, cached_pairs) : num_sms();
+    info[4] = g.pair ? max_pairs(fp8_gemm_2sm_kernel<OUT_BF16, 1, false>, Pair<1>::SMEM, cached_pairs) : num_sms();
 }
 
 fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_scale_inv, const uint8_t *b,
@@ -1946,20 +1993,8 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
         p.flags = static_cast<int32_t *>(workspace);
         p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + WS_FLAG_BYTES);
     }
-    cudaError_t e;
-    if (pair && m_sub == 2) {
-        e = out == OUT_FP8    ? launch_2sm<OUT_FP8, 2>(ta, tb, td, p, stream)
-            : out == OUT_BF16 ? launch_2sm<OUT_BF16, 2>(ta, tb, td, p, stream)
-                              : launch_2sm<OUT_F32, 2>(ta, tb, td, p, stream);
-    } else if (pair) {
-        e = out == OUT_FP8    ? launch_2sm<OUT_FP8, 1>(ta, tb, td, p, stream)
-            : out == OUT_BF16 ? launch_2sm<OUT_BF16, 1>(ta, tb, td, p, stream)
-                              : launch_2sm<OUT_F32, 1>(ta, tb, td, p, stream);
-    } else {
-        e = out == OUT_FP8    ? launch_1sm<OUT_FP8>(ta, tb, td, p, stream)
-            : out == OUT_BF16 ? launch_1sm<OUT_BF16>(ta, tb, td, p, stream)
-                              : launch_1sm<OUT_F32>(ta, tb, td, p, stream);
-    }
+    const cudaError_t e = p.bias_kind != 0 ? launch_any<true>(out, pair, m_sub, ta, tb, td, p, stream)
+                                           : launch_any<false>(out, pair, m_sub, ta, tb, td, p, stream);
     if (e != cudaSuccess) {
         set_error("fp8_gemm: launch failed: %s", cudaGetErrorString(e));
         return FP8DS_ERR_CUDA;
