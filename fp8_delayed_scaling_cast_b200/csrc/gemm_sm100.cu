@@ -1102,10 +1102,13 @@ __device__ __forceinline__ void epilogue_bf16_regs(uint32_t t_h, int lane, uint8
             if (lane == 0) mbar_arrive_cluster(empty_addr);
         }
         const float *bs = bias_s + half * (ACC_N / 2) + c * 32;
+        float bv[32];
+        if constexpr (BIAS) load_bias32(bs, bv);
         uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float4 b = bias4<BIAS>(bs + 4 * j);
+            const float4 b = BIAS ? make_float4(bv[4 * j], bv[4 * j + 1], bv[4 * j + 2], bv[4 * j + 3])
+                                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             const uint64_t v01 = scale_bias2(r[4 * j], r[4 * j + 1], sab2, b.x, b.y);
             const uint64_t v23 = scale_bias2(r[4 * j + 2], r[4 * j + 3], sab2, b.z, b.w);
             __nv_bfloat162 ha = __floats2bfloat162_rn(lo_f32(v01), hi_f32(v01));
