@@ -77,23 +77,12 @@ constexpr int TMEM_COLS = 512; // two accumulators
 #ifndef FP8DS_EPI_BOXES
 #define FP8DS_EPI_BOXES 1
 #endif
-// FP8DS_EPI_DIRECT: the epilogue stores D from registers with 32-byte
-// global stores (no shared-memory staging, no TMA store).
-#ifndef FP8DS_EPI_DIRECT
-#define FP8DS_EPI_DIRECT 0
-#endif
-constexpr bool EPI_DIRECT = FP8DS_EPI_DIRECT != 0;
 // FP8DS_EPI_EARLY: whole-tile bf16 and FP8 epilogues read the accumulator
 // into registers and release TMEM before they stage and store D.
 #ifndef FP8DS_EPI_EARLY
 #define FP8DS_EPI_EARLY 1
 #endif
-constexpr bool EPI_EARLY = FP8DS_EPI_EARLY != 0 && !EPI_DIRECT;
-// FP8DS_SPLIT_BF16: the 512-row tile with bf16 output also releases its two
-// M halves one at a time (always done for FP8 output).
-#ifndef FP8DS_SPLIT_BF16
-#define FP8DS_SPLIT_BF16 0
-#endif
+constexpr bool EPI_EARLY = FP8DS_EPI_EARLY != 0;
 constexpr int EPI_LD = FP8DS_EPI_LD;
 constexpr int EPI_NBOX = FP8DS_EPI_BOXES;
 static_assert(EPI_LD == 32 || EPI_LD == 64, "TMEM load width must be 32 or 64 columns");
@@ -260,6 +249,17 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint32_
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y)
+        : "memory");
+}
+
+// The same load with an L2 cache-policy hint (createpolicy), for the operand
+// that later waves of the launch read again.
+__device__ __forceinline__ void tma_load_2d_pair_hint(const CUtensorMap *map, uint32_t bar_cluster_addr, void *dst,
+                                                      int32_t x, int32_t y, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.cta_group::2.L2::cache_hint"
+        " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(bar_cluster_addr), "r"(x), "r"(y), "l"(policy)
         : "memory");
 }
 
@@ -432,6 +432,7 @@ struct Params {
     int32_t M, N, K;
     int32_t tiles_m, tiles_n, num_kb;
     int32_t group_m;      // row tiles per raster group (tile_coords)
+    int32_t l2_keep;      // operand loaded with an L2 evict_last hint: 0 none, 1 A, 2 B
     uint32_t idesc;
     int32_t a_mn, b_mn;   // 1: the operand is stored MN-major ([K, M] / [K, N] row-major)
     // stream-K (pair kernel only): 0 = whole tiles per cluster
@@ -449,8 +450,6 @@ struct Params {
     // error path only) whether split tiles withhold their publication
     unsigned long long partial_wait_ns;
     int32_t withhold_partials;
-    void *out;             // D (fp32 / bf16 output) for the direct-store epilogue
-    int32_t out_v8;        // D and its row pitch are 32-byte aligned (32-byte stores)
     uint8_t *out_d8t;      // [N, M] codes or NULL
     int32_t out_fmt;
 };
@@ -628,33 +627,6 @@ __device__ __forceinline__ float4 bias4(const float *bs) {
     return BIAS ? *reinterpret_cast<const float4 *>(bs) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 }
 
-__device__ __forceinline__ void st_global_v8(void *p, const uint32_t *w) {
-    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-                 : "memory");
-}
-
-// 32 columns of row m of D (bf16: 16 words, fp32: 32 words) from registers,
-// clipped at N (a multiple of 8 (bf16) or 4 (fp32): 16-byte granules are
-// wholly inside or outside).
-template <bool OUT_BF16>
-__device__ __forceinline__ void store_row_direct(void *out, int32_t m, int64_t n0, int32_t m_total, int32_t n_total,
-                                                 bool v8, const uint32_t *w) {
-    constexpr int WORDS = OUT_BF16 ? 16 : 32;
-    constexpr int COLS_PER_16B = OUT_BF16 ? 8 : 4;
-    if (m >= m_total || n0 >= n_total) return;
-    uint8_t *dst = static_cast<uint8_t *>(out) + (static_cast<int64_t>(m) * n_total + n0) * (OUT_BF16 ? 2 : 4);
-    if (v8 && n0 + 32 <= n_total) {
-#pragma unroll
-        for (int g = 0; g < WORDS / 8; ++g) st_global_v8(dst + 32 * g, w + 8 * g);
-    } else {
-#pragma unroll
-        for (int g = 0; g < WORDS / 4; ++g)
-            if (n0 + g * COLS_PER_16B < n_total)
-                *reinterpret_cast<uint4 *>(dst + 16 * g) = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
-    }
-}
-
 // Stream-K modes (bits): 1 = the segment does not end the tile's k-range at
 // its start (kb0 > 0), so it stores its raw partial sum for the tile's owner
 // instead of D; 2 = the tile's k-range goes on after the segment (kb1 <
@@ -669,9 +641,8 @@ template <bool OUT_BF16, bool BIAS>
 __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t *boxes, int &nbox, int half,
                                               const CUtensorMap *tmap_d, int64_t n_base, int32_t m_row0,
                                               float sab, const float *bias_s, uint32_t empty_bar_cluster,
-                                              bool arrive, int mode, const float *p_in, float *p_out, int h, int q,
-                                              void *out,
-                                              int32_t m_total, int32_t n_total, bool v8) {
+                                              bool arrive, int mode, const float *p_in, float *p_out, int h,
+                                              int q) {
     constexpr int SUBS_PER_BOX = OUT_BF16 ? 2 : 1;  // 32-column sub-blocks per staging box
     constexpr int CHUNKS = ACC_N / 2 / EPI_LD;      // TMEM loads per warp and row block
     constexpr int SUBS = EPI_LD / 32;               // 32-column sub-blocks per load
@@ -694,34 +665,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             const int hh = (col0 / 32) % SUBS_PER_BOX;
             const bool last_of_chunk = sb == SUBS - 1;
             if (mode != 0) partial_io(mode, rr, p_in, p_out, h, q, col0, lane);
-            if (EPI_DIRECT && !(mode & PART_OUT)) {
-                const float *bs = bias_s + col0;
-                if (OUT_BF16) {
-                    uint32_t packed[16];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const float4 b = bias4<BIAS>(bs + 4 * j);
-                        __nv_bfloat162 ha = __floats2bfloat162_rn(fmaf(__uint_as_float(rr[4 * j]), sab, b.x),
-                                                                  fmaf(__uint_as_float(rr[4 * j + 1]), sab, b.y));
-                        __nv_bfloat162 hb = __floats2bfloat162_rn(fmaf(__uint_as_float(rr[4 * j + 2]), sab, b.z),
-                                                                  fmaf(__uint_as_float(rr[4 * j + 3]), sab, b.w));
-                        packed[2 * j] = *reinterpret_cast<uint32_t *>(&ha);
-                        packed[2 * j + 1] = *reinterpret_cast<uint32_t *>(&hb);
-                    }
-                    store_row_direct<true>(out, m_row0 + lane, n_base + col0, m_total, n_total, v8, packed);
-                } else {
-                    uint32_t v[32];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const float4 b = bias4<BIAS>(bs + 4 * k);
-                        v[4 * k] = __float_as_uint(fmaf(__uint_as_float(rr[4 * k]), sab, b.x));
-                        v[4 * k + 1] = __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 1]), sab, b.y));
-                        v[4 * k + 2] = __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 2]), sab, b.z));
-                        v[4 * k + 3] = __float_as_uint(fmaf(__uint_as_float(rr[4 * k + 3]), sab, b.w));
-                    }
-                    store_row_direct<false>(out, m_row0 + lane, n_base + col0, m_total, n_total, v8, v);
-                }
-            } else if (!(mode & PART_OUT)) {
+            if (!(mode & PART_OUT)) {
                 uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
                 if (hh == 0) {
                     // Staging buffer reuse: the store issued from this box
@@ -766,7 +710,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t t_row, int lane, uint8_t 
             }
             // the registers of r are free: start the next chunk's TMEM load
             if (last_of_chunk && c + 1 < CHUNKS) tmem_ld(t_row + half * (ACC_N / 2) + (c + 1) * EPI_LD, r);
-            if (!EPI_DIRECT && !(mode & PART_OUT) && hh == SUBS_PER_BOX - 1) {
+            if (!(mode & PART_OUT) && hh == SUBS_PER_BOX - 1) {
                 uint8_t *box = boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES;
                 fence_async_smem();
                 __syncwarp();
@@ -834,7 +778,7 @@ __device__ __forceinline__ void epilogue_tile_fp8(uint32_t t_row, int lane, uint
     // Without the transpose the warp's 32 rows x 128 code bytes are one
     // 128-byte-swizzled staging box and one TMA store; with it, the codes go
     // out with plain stores beside the transposed ones (in box 0's memory).
-    const bool staged = !EPI_DIRECT && d8t == nullptr;
+    const bool staged = d8t == nullptr;
     uint8_t *box = staged ? boxes + (nbox % EPI_NBOX) * EPI_BOX_BYTES : boxes;
     if (staged && !(mode & PART_OUT)) {
         if (lane == 0) tma_store_wait_read<EPI_NBOX - 1>();
@@ -1332,12 +1276,10 @@ __device__ __forceinline__ void epilogue_loop(const Smem &sm, const CUtensorMap 
             } else {
                 if constexpr (BIAS)
                     epilogue_tile<OUT == OUT_BF16, true>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab, bias_s,
-                                                         empty_addr, release, mode, p_in, p_out, h, q, p.out, p.M, p.N,
-                                                         p.out_v8 != 0);
+                                                         empty_addr, release, mode, p_in, p_out, h, q);
                 else
                     epilogue_tile<OUT == OUT_BF16, false>(t_row, lane, boxes, nbox, half, tmap_d, n_base, m_row0, sab,
-                                                          bias_s, empty_addr, release, mode, p_in, p_out, h, q, p.out, p.M,
-                                                          p.N, p.out_v8 != 0);
+                                                          bias_s, empty_addr, release, mode, p_in, p_out, h, q);
             }
         }
         if (seg != 0) {
@@ -1531,7 +1473,7 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     // Half-by-half release of the 512-row tile's accumulator (FP8 output,
     // whose longer epilogue it hides best; measured neutral-to-negative with
     // bf16 and fp32 outputs).
-    constexpr bool SPLIT = M_SUB == 2 && (OUT == OUT_FP8 || (OUT == OUT_BF16 && FP8DS_SPLIT_BF16 != 0));
+    constexpr bool SPLIT = M_SUB == 2 && OUT == OUT_FP8;
     extern __shared__ uint8_t smem_raw[];
     const Smem sm = carve<STAGES, A_STAGE, S2_B_STAGE>(smem_raw);
     const int warp = threadIdx.x >> 5;
@@ -1580,6 +1522,9 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             bool ok = true;
             Sched sched(p, cluster_id, num_clusters);
             int tile, kb0, kb1;
+            uint64_t keep_policy;
+            asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep_policy));
+            const bool keep_a = p.l2_keep == 1, keep_b = p.l2_keep == 2;
             while (ok && sched.next(tile, kb0, kb1)) {
                 int m_blk, n_blk;
                 tile_coords(tile, p.tiles_m, p.tiles_n, p.group_m, m_blk, n_blk);
@@ -1597,15 +1542,19 @@ fp8_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
 #pragma unroll
                     for (int h = 0; h < M_SUB; ++h) {
                         uint8_t *a_dst = sm.a + stage * A_STAGE + h * S2_BM * BK;
-                        if (p.a_mn)
-                            tma_load_2d_pair(&tmap_a, full_leader, a_dst, a_row + h * 2 * S2_BM, kb * BK);
+                        const int32_t ax = p.a_mn ? a_row + h * 2 * S2_BM : kb * BK;
+                        const int32_t ay = p.a_mn ? kb * BK : a_row + h * 2 * S2_BM;
+                        if (keep_a)
+                            tma_load_2d_pair_hint(&tmap_a, full_leader, a_dst, ax, ay, keep_policy);
                         else
-                            tma_load_2d_pair(&tmap_a, full_leader, a_dst, kb * BK, a_row + h * 2 * S2_BM);
+                            tma_load_2d_pair(&tmap_a, full_leader, a_dst, ax, ay);
                     }
-                    if (p.b_mn)
-                        tma_load_2d_pair(&tmap_b, full_leader, sm.b + stage * S2_B_STAGE, b_row, kb * BK);
+                    uint8_t *b_dst = sm.b + stage * S2_B_STAGE;
+                    const int32_t bx = p.b_mn ? b_row : kb * BK, by = p.b_mn ? kb * BK : b_row;
+                    if (keep_b)
+                        tma_load_2d_pair_hint(&tmap_b, full_leader, b_dst, bx, by, keep_policy);
                     else
-                        tma_load_2d_pair(&tmap_b, full_leader, sm.b + stage * S2_B_STAGE, kb * BK, b_row);
+                        tma_load_2d_pair(&tmap_b, full_leader, b_dst, bx, by);
                     ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -1866,6 +1815,7 @@ struct GemmPlan {
     int m_sub;
     int64_t tiles;
     int group_m;     // raster group (tile_coords)
+    int l2_keep;     // Params::l2_keep
     bool stream_k;   // with a large enough workspace
 };
 
@@ -1896,6 +1846,16 @@ GemmPlan plan_gemm(int64_t m, int64_t n, int64_t k) {
     // each A row block (the larger operand) is streamed by one wave only and
     // the second wave re-reads only the smaller B.
     g.group_m = (g.pair && cap > 0 && g.tiles <= 2 * cap && tm > tn) ? 1 : GROUP_M;
+    // An operand that every wave streams whole (B under whole rows of tiles,
+    // A when all row tiles fit in one group) is read once per wave; with more
+    // than one wave it is loaded with an L2 evict_last hint, if it takes at
+    // most a quarter of the 126 MB L2, so that later waves find it there.
+    g.l2_keep = 0;
+    if (g.pair && cap > 0 && g.tiles > cap) {
+        const int64_t a_bytes = tm * tile_m * k, b_bytes = tn * ACC_N * k;
+        if (g.group_m == 1 && b_bytes <= (int64_t(32) << 20)) g.l2_keep = 2;
+        else if (g.group_m != 1 && tm <= g.group_m && a_bytes <= (int64_t(32) << 20)) g.l2_keep = 1;
+    }
     // Stream-K (given a workspace) when whole tiles would leave a ragged
     // last wave worth balancing: R = tiles mod pairs with pairs / 3 <= R <=
     // 7/8 pairs (a split tile then spans at most four clusters, and at
@@ -1962,6 +1922,7 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
     p.tiles_n = static_cast<int32_t>((n + ACC_N - 1) / ACC_N);
     p.num_kb = static_cast<int32_t>((k + BK - 1) / BK);
     p.group_m = plan.group_m;
+    p.l2_keep = pair ? plan.l2_keep : 0;
     p.idesc = make_idesc(a_fmt, b_fmt, pair ? 2 * S2_BM : S1_BM, ACC_N, a_mn, b_mn);
     p.a_mn = a_mn ? 1 : 0;
     p.b_mn = b_mn ? 1 : 0;
@@ -1983,8 +1944,6 @@ fp8ds_status launch_gemm(const uint8_t *a, fp8ds_format a_fmt, const float *a_sc
         const unsigned long long w = g_test_wait_ns.load(std::memory_order_relaxed);
         if (w != 0) p.partial_wait_ns = w;
     }
-    p.out = d;
-    p.out_v8 = (reinterpret_cast<uintptr_t>(d) % 32 == 0) && (n * (out == OUT_F32 ? 4 : 2)) % 32 == 0;
     if (plan.stream_k && workspace != nullptr && workspace_bytes >= gemm_workspace_bytes()) {
         static std::atomic<uint32_t> launches{0};
         uint32_t e = ++launches;
