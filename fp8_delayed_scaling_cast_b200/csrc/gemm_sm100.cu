@@ -197,6 +197,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test, letting the thread sleep until the phase completes or up to
+// `hint_ns` have passed (the suspend-time hint of mbarrier.try_wait), so that
+// a warp that waits a whole main loop issues almost nothing meanwhile.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t addr, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ void record_error(int32_t site) {
     atomicCAS(&g_device_error, 0, (site << 8) | FP8DS_ERR_TIMEOUT);
 }
@@ -209,9 +224,10 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
     if (mbar_try_wait(addr, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
+        // up to 32 x 20 us between looks at the abort flag and the clock
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(addr, parity)) return true;
+            if (mbar_try_wait_sleep(addr, parity, 20000u)) return true;
         if (*abort_flag) return false;
         if (globaltimer() - t0 > TIMEOUT_NS) {
             *abort_flag = 1;
